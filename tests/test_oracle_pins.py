@@ -1,0 +1,333 @@
+"""Pins of the oracle to things other than itself (library routines, closed forms,
+invariants, brute force).  CPU only."""
+import math
+
+import pytest
+import torch
+import torch.nn.functional as F
+
+import synth
+from oracle import (OracleDecoder, argmax_lowest, attention_decode, e4m3_decode_table,
+                    moe_route, rms_norm, rope_rotate, silu, swiglu_ffn)
+from synth.configs import DecoderConfig
+
+torch.manual_seed(0)
+
+
+# ------------------------------------------------------------------ RMSNorm
+
+def test_rmsnorm_matches_library():
+    x = torch.randn(5, 96)
+    g = torch.rand(96) + 0.5
+    ref = F.rms_norm(x, (96,), weight=g, eps=1e-5)
+    assert torch.allclose(rms_norm(x, g, 1e-5), ref, rtol=1e-6, atol=1e-6)
+
+
+def test_rmsnorm_closed_forms():
+    # constant vector c: every entry becomes c / sqrt(c^2 + eps)
+    for c in (0.25, -3.0):
+        x = torch.full((64,), c)
+        out = rms_norm(x, torch.ones(64), 1e-5)
+        assert torch.allclose(out, torch.full((64,), c / math.sqrt(c * c + 1e-5)), rtol=1e-6)
+    # unit gain gives unit RMS (eps negligible); scale invariance
+    x = torch.randn(256) * 7
+    y = rms_norm(x, torch.ones(256), 0.0)
+    assert abs(float(y.pow(2).mean().sqrt()) - 1.0) < 1e-6
+    assert torch.allclose(rms_norm(3.5 * x, torch.ones(256), 0.0), y, rtol=1e-5, atol=1e-6)
+
+
+# --------------------------------------------------------------------- RoPE
+
+def test_rope_matches_complex_rotation():
+    d, theta = 64, 1.0e4
+    x = torch.randn(3, d)
+    for pos in (0, 1, 17, 1000):
+        z = torch.complex(x[:, : d // 2].double(), x[:, d // 2:].double())
+        inv = theta ** (-2.0 * torch.arange(d // 2, dtype=torch.float64) / d)
+        rot = z * torch.polar(torch.ones(d // 2, dtype=torch.float64), pos * inv)
+        ref = torch.cat([rot.real, rot.imag], dim=-1).float()
+        assert torch.allclose(rope_rotate(x, pos, theta), ref, rtol=1e-5, atol=1e-5)
+
+
+def test_rope_invariants():
+    d = 128
+    q, k = torch.randn(d).double(), torch.randn(d).double()
+    assert torch.equal(rope_rotate(q.float(), 0, 1e4), q.float())            # R(0) = I
+    for m in (1, 50, 4097):
+        assert abs(float(rope_rotate(q.float(), m, 1e4).norm()) - float(q.norm())) < 1e-4
+    # relative position: <R(m) q, R(n) k> depends on m - n only
+    a = torch.dot(rope_rotate(q.float(), 7, 1e4), rope_rotate(k.float(), 3, 1e4))
+    b = torch.dot(rope_rotate(q.float(), 107, 1e4), rope_rotate(k.float(), 103, 1e4))
+    assert abs(float(a - b)) < 1e-3
+
+
+# ---------------------------------------------------------------- attention
+
+def _sdpa_gqa(q, K, V):
+    n_q, n_kv = q.shape[0], K.shape[0]
+    Ke = K.float().repeat_interleave(n_q // n_kv, dim=0)
+    Ve = V.float().repeat_interleave(n_q // n_kv, dim=0)
+    out = F.scaled_dot_product_attention(q[:, None, :], Ke, Ve)      # [n_q][1][d]
+    return out[:, 0]
+
+
+@pytest.mark.parametrize("n_q,n_kv,T,d", [(4, 2, 129, 64), (32, 8, 300, 128), (8, 8, 5, 64)])
+def test_attention_matches_library_sdpa(n_q, n_kv, T, d):
+    q = torch.randn(n_q, d) * 2
+    K = torch.randn(n_kv, T, d).to(torch.bfloat16)
+    V = torch.randn(n_kv, T, d).to(torch.bfloat16)
+    assert torch.allclose(attention_decode(q, K, V), _sdpa_gqa(q, K, V), rtol=1e-5, atol=1e-5)
+
+
+def test_attention_special_cases():
+    d = 64
+    q = torch.randn(4, d)
+    K = torch.randn(2, 1, d)
+    V = torch.randn(2, 1, d)
+    out = attention_decode(q, K, V)                                  # T = 1 -> output = v
+    assert torch.allclose(out[0], V[0, 0]) and torch.allclose(out[3], V[1, 0])
+    # one dominant score selects that V row; heads 0,1 read kv head 0, heads 2,3 kv head 1
+    K = torch.zeros(2, 6, d)
+    K[0, 4, 0] = 1.0
+    K[1, 2, 0] = 1.0
+    V = torch.randn(2, 6, d)
+    q = torch.zeros(4, d)
+    q[:, 0] = 1e4
+    out = attention_decode(q, K, V)
+    assert torch.allclose(out[1], V[0, 4], atol=1e-6)
+    assert torch.allclose(out[2], V[1, 2], atol=1e-6)
+
+
+def test_softmax_invariants_through_attention():
+    # uniform scores -> mean of V rows; adding a constant to all scores changes nothing
+    d = 64
+    V = torch.randn(1, 10, d)
+    out = attention_decode(torch.zeros(2, d), torch.randn(1, 10, d), V)
+    assert torch.allclose(out[0], V[0].mean(0), atol=1e-6)
+    q = torch.randn(1, d)
+    K = torch.randn(1, 10, d)
+    K2 = K + q / q.norm() ** 2 * 5.0 * math.sqrt(d)                  # shifts every score by 5
+    assert torch.allclose(attention_decode(q, K, V), attention_decode(q, K2, V), atol=1e-4)
+
+
+# ------------------------------------------------------------------- SwiGLU
+
+def test_silu_matches_library_and_closed_forms():
+    z = torch.linspace(-30, 30, 1001)
+    assert torch.allclose(silu(z), F.silu(z), rtol=1e-6, atol=1e-7)
+    assert float(silu(torch.tensor(0.0))) == 0.0
+    assert abs(float(silu(torch.tensor(1.0))) - 0.7310585786300049) < 1e-7
+    assert abs(float(silu(torch.tensor(40.0))) - 40.0) < 1e-5
+    assert abs(float(silu(torch.tensor(-40.0)))) < 1e-12
+
+
+def test_swiglu_structured():
+    # diagonal gate/up and a permutation down projection: closed form per index
+    n = 6
+    a, b = torch.randn(n), torch.randn(n)
+    sigma = [2, 0, 5, 1, 4, 3]
+    wd = torch.zeros(n, n)
+    for i, j in enumerate(sigma):
+        wd[i, j] = 1.0
+    xn = torch.randn(n)
+    out = swiglu_ffn(xn, torch.diag(a), torch.diag(b), wd)
+    for i, j in enumerate(sigma):
+        z = float(a[j] * xn[j])
+        assert abs(float(out[i]) - (z / (1 + math.exp(-z))) * float(b[j] * xn[j])) < 1e-5
+
+
+# ---------------------------------------------------------------------- MoE
+
+def test_moe_route_topk_vs_full_sort_and_ties():
+    logits = torch.randn(64)
+    ids, w, p = moe_route(logits, 8)
+    assert abs(float(p.sum()) - 1.0) < 1e-6
+    ref = torch.topk(torch.softmax(logits, 0), 8)
+    assert ids == ref.indices.tolist()
+    assert torch.allclose(torch.tensor(w), ref.values)
+    # ties go to the lower expert id
+    tied = torch.zeros(16)
+    tied[[3, 9, 12]] = 2.0
+    ids, _, _ = moe_route(tied, 2)
+    assert ids == [3, 9]
+    ids, _, _ = moe_route(torch.zeros(16), 4)
+    assert ids == [0, 1, 2, 3]
+
+
+def test_moe_single_expert_reduces_to_dense():
+    base = DecoderConfig(name="t", n_layers=1, hidden=128, n_q_heads=2, n_kv_heads=1, head_dim=64,
+                         ffn=256, vocab=300, kv_len=4, steps=2)
+    moe = base.with_(ffn=0, n_experts=1, top_k=1, n_shared_experts=0, expert_ffn=256)
+    wd = synth.make_weights(base)
+    wm = synth.make_weights(moe)
+    for k in ("w_gate", "w_up", "w_down"):
+        wm[f"layers.0.experts.0.{k}"] = wd[f"layers.0.{k}"]
+    dense, sparse = OracleDecoder(base, wd, 1), OracleDecoder(moe, wm, 1)
+    for t in (5, 17, 299):
+        ld, _ = dense.step([t])
+        ls, _ = sparse.step([t])
+        assert torch.allclose(ld, ls, rtol=1e-6, atol=1e-6)
+        assert sparse.last_experts[0] == [[0]]
+
+
+# ---------------------------------------------------------------------- FP8
+
+def test_e4m3_table_matches_library_and_format():
+    table = e4m3_decode_table()
+    lib = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float()
+    nan = torch.isnan(lib)
+    assert torch.equal(torch.isnan(table), nan)
+    assert nan.sum() == 2 and bool(nan[0x7F]) and bool(nan[0xFF])
+    assert torch.equal(table[~nan], lib[~nan])
+    assert float(table[0x38]) == 1.0 and float(table[0x7E]) == 448.0
+    assert float(table[0x01]) == 2.0 ** -9 and float(table[0xFE]) == -448.0
+    assert float(table[0x80]) == 0.0
+
+
+def test_fp8_quantisation_roundtrip_within_half_ulp():
+    w = synth.normal_bf16(0, "q", (256, 384), 0.02)
+    codes, scales = synth.quantize_fp8_blocks(w)
+    deq = (e4m3_decode_table()[codes.long()].view(2, 128, 3, 128) * scales[:, None, :, None]).view(256, 384)
+    rel = ((deq - w.float()).abs() / w.float().abs().clamp_min(1e-6))
+    full_scale = scales.repeat_interleave(128, 0).repeat_interleave(128, 1)
+    big = (w.float() / full_scale).abs() >= 2.0 ** -6                   # e4m3 normal range
+    assert float(rel[big].max()) <= 2.0 ** -4 + 1e-6                   # 3 mantissa bits: half ulp
+    assert float(codes.view(torch.float8_e4m3fn).float().abs().max()) == 448.0
+
+
+# ------------------------------------------------------------------- argmax
+
+def test_argmax_lowest_index_on_ties():
+    v = torch.tensor([1.0, 3.0, 2.0, 3.0, 3.0])
+    assert argmax_lowest(v) == 1
+    v = torch.randn(1000)
+    assert argmax_lowest(v) == int(torch.argmax(v))
+
+
+# ------------------------------------------------------------ whole model
+
+def _tiny(**kw):
+    return synth.get_config("tiny", **kw)
+
+
+def test_zero_layers_reduces_to_norm_and_lm_head():
+    cfg = _tiny(n_layers=0)
+    w = synth.make_weights(cfg, norm_std=0.1)
+    m = OracleDecoder(cfg, w, 1)
+    for t in (0, 7, 4095):
+        logits, hidden = m.step([t])
+        e = w["embed"][t].float()
+        ref = F.linear(F.rms_norm(e, (cfg.hidden,), w["final_norm"], cfg.rms_eps), w["lm_head"].float())
+        assert torch.allclose(hidden[0], e)
+        assert torch.allclose(logits[0], ref, rtol=1e-5, atol=1e-6)
+
+
+def test_structured_layer_closed_form():
+    """One layer whose projections select / permute entries (every matrix non-square).
+
+    Catches a transposed operand, a dropped residual, a wrong GQA group or a
+    norm taken from the wrong vector: the expected output is built by index
+    arithmetic only.
+    """
+    H, nq, nkv, d, Fw, V = 8, 2, 1, 2, 6, 16
+    cfg = DecoderConfig(name="s", n_layers=1, hidden=H, n_q_heads=nq, n_kv_heads=nkv, head_dim=d,
+                        ffn=Fw, vocab=V, kv_len=0, steps=3, rms_eps=1e-5)
+    w = synth.make_weights(cfg)
+    wq = torch.zeros(nq * d, H); wq[0, 0] = wq[1, 1] = wq[2, 2] = wq[3, 3] = 1.0
+    wk = torch.zeros(nkv * d, H); wk[0, 4] = wk[1, 5] = 1.0
+    wv = torch.zeros(nkv * d, H); wv[0, 6] = wv[1, 7] = 1.0
+    wo = torch.zeros(H, nq * d)
+    so = [3, 0, 2, 1, 0, 3, 1, 2]
+    for i, j in enumerate(so):
+        wo[i, j] = 1.0 if i < 4 else -1.0
+    wg = torch.zeros(Fw, H); wu = torch.zeros(Fw, H); wdn = torch.zeros(H, Fw)
+    sg, su = [1, 3, 5, 7, 0, 2], [2, 2, 4, 6, 1, 0]
+    for f in range(Fw):
+        wg[f, sg[f]] = 1.5
+        wu[f, su[f]] = -0.5
+    sd = [5, 4, 3, 2, 1, 0, 5, 4]
+    for i, f in enumerate(sd):
+        wdn[i, f] = 1.0
+    lm = torch.zeros(V, H)
+    for t in range(V):
+        lm[t, t % H] = 1.0 if t < H else -2.0
+    for name, t in (("wq", wq), ("wk", wk), ("wv", wv), ("wo", wo), ("w_gate", wg),
+                    ("w_up", wu), ("w_down", wdn)):
+        w[f"layers.0.{name}"] = t.to(torch.bfloat16)
+    w["lm_head"] = lm.to(torch.bfloat16)
+    m = OracleDecoder(cfg, w, 1, max_seq=4)
+
+    def norm(v):
+        r = 1.0 / math.sqrt(sum(a * a for a in v) / len(v) + 1e-5)
+        return [a * r for a in v]
+
+    def rot(p, pos):   # d = 2: one pair, theta_0 = 1
+        c, s = math.cos(pos), math.sin(pos)
+        return [p[0] * c - p[1] * s, p[0] * s + p[1] * c]
+
+    ks, vs = [], []
+    for pos, tok in enumerate([3, 11, 6]):
+        x = [float(a) for a in w["embed"][tok].float()]
+        xn = norm(x)
+        q = [rot(xn[0:2], pos), rot(xn[2:4], pos)]
+        ks.append([float(torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)) for a in rot(xn[4:6], pos)])
+        vs.append([float(torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)) for a in xn[6:8]])
+        o = []
+        for h in range(nq):               # both q heads read kv head 0
+            sc = [(q[h][0] * k[0] + q[h][1] * k[1]) / math.sqrt(d) for k in ks]
+            mx = max(sc)
+            e = [math.exp(s - mx) for s in sc]
+            o += [sum(e[t] * vs[t][i] for t in range(len(e))) / sum(e) for i in range(d)]
+        x1 = [x[i] + (o[so[i]] if i < 4 else -o[so[i]]) for i in range(H)]
+        x1n = norm(x1)
+        hmid = [(1.5 * x1n[sg[f]]) / (1 + math.exp(-1.5 * x1n[sg[f]])) * (-0.5 * x1n[su[f]])
+                for f in range(Fw)]
+        x2 = [x1[i] + hmid[sd[i]] for i in range(H)]
+        x2n = norm(x2)
+        ref = [x2n[t % H] * (1.0 if t < H else -2.0) for t in range(V)]
+        logits, hidden = m.step([tok])
+        assert torch.allclose(hidden[0], torch.tensor(x2), rtol=1e-5, atol=1e-5), pos
+        assert torch.allclose(logits[0], torch.tensor(ref), rtol=1e-5, atol=1e-5), pos
+        assert int(m.pos[0]) == pos + 1
+
+
+def test_incremental_decode_equals_full_recompute():
+    cfg = _tiny(n_layers=2)
+    w = synth.make_weights(cfg, norm_std=0.1)
+    toks = synth.make_prompt(cfg.with_(kv_len=12))                 # [1][13]
+    full = OracleDecoder(cfg, w, 1, max_seq=16)
+    ref = full.forward_sequence(toks)[0]                              # [13][V]
+    inc = OracleDecoder(cfg, w, 1, max_seq=16)
+    for t in range(toks.shape[1]):
+        logits, _ = inc.step([int(toks[0, t])])
+        assert torch.allclose(logits[0], ref[t], rtol=1e-4, atol=1e-5), t
+    T = toks.shape[1]
+    assert torch.equal(inc.K[:, :, :, :T], full.K[:, :, :, :T]) or \
+        float((inc.K[:, :, :, :T].float() - full.K[:, :, :, :T].float()).abs().max()) < 2e-2
+    assert torch.allclose(inc.V[:, :, :, :T].float(), full.V[:, :, :, :T].float(), atol=2e-2)
+
+
+def test_gqa_with_equal_heads_is_mha():
+    cfg = _tiny(n_layers=1, n_kv_heads=4)
+    w = synth.make_weights(cfg)
+    m = OracleDecoder(cfg, w, 1, max_seq=8)
+    q = torch.randn(4, 64)
+    K = torch.randn(4, 7, 64).to(torch.bfloat16)
+    V = torch.randn(4, 7, 64).to(torch.bfloat16)
+    ref = F.scaled_dot_product_attention(q[:, None], K.float(), V.float())[:, 0]
+    assert torch.allclose(attention_decode(q, K, V), ref, atol=1e-5)
+    logits, _ = m.step([1])
+    assert logits.shape == (1, cfg.vocab)
+
+
+def test_batch_sequences_are_independent():
+    cfg = _tiny(n_layers=1, batch=2)
+    w = synth.make_weights(cfg)
+    mb = OracleDecoder(cfg, w, 2, max_seq=8)
+    m0 = OracleDecoder(cfg, w, 1, max_seq=8)
+    m1 = OracleDecoder(cfg, w, 1, max_seq=8)
+    for a, b in ((3, 9), (100, 7)):
+        lb, _ = mb.step([a, b])
+        l0, _ = m0.step([a])
+        l1, _ = m1.step([b])
+        assert torch.equal(lb[0], l0[0]) and torch.equal(lb[1], l1[0])
