@@ -1,0 +1,199 @@
+/*
+ * xlpk.h - persistent single-kernel small-batch decode on one B200 (sm_100a).
+ *
+ * The whole greedy decode of N tokens runs as ONE cooperative kernel launch:
+ * every SM holds one resident CTA that walks a statically planned list of
+ * tile tasks (RMSNorm-folded QKV GEMV + RoPE + KV append, flash-decoding
+ * attention split over the sequence, O-projection + residual, gate/up +
+ * SwiGLU, down projection + residual, LM head + argmax) and orders them with
+ * device-side dependency counters instead of kernel launches.  This follows
+ * the "persistent Engine Kernel" and "tile-level pipeline" design described in
+ * "TileRT speed notes" (section "TileRT's direction: from discrete kernels to
+ * a resident execution pipeline") and in "Ultra-High Interactivity On NVIDIA
+ * GPUs? - TileRT InferenceX" (digest, "core views": the host launches once and
+ * the execution stays resident for the whole decode lifecycle).  The
+ * kernel-per-op baseline the pages compare against (launch, load, compute,
+ * store, synchronise per operator; "Persistent execution paradigm", section 1)
+ * is xlpk_decode_unfused, built from the same tiles.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are CUDA device pointers on the handle's device;
+ *    pointers named *_host are ordinary host memory.  Nothing is retained
+ *    past the call except where stated (weights/KV in xlpk_create).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Functions return XLPK_OK or a negative xlpk_status.  Argument errors are
+ *    detected on the host before anything is enqueued.  Device-side failures
+ *    of an enqueued decode (a dependency wait that exceeded its time limit)
+ *    are reported by xlpk_get_status after the work has finished.
+ *  - A handle is not thread-safe: calls on one handle must be serialised,
+ *    and its decodes must not overlap on the GPU.
+ *  - There is no CPU fallback: without a usable sm_100 device, xlpk_create
+ *    returns XLPK_ERR_UNSUPPORTED or XLPK_ERR_CUDA.
+ */
+#ifndef XLPK_H_
+#define XLPK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum xlpk_status {
+  XLPK_OK = 0,
+  XLPK_ERR_INVALID_ARG = -1,   /* bad pointer, size, shape or alignment */
+  XLPK_ERR_UNSUPPORTED = -2,   /* shape/dtype/batch this build does not handle, or no sm_100 GPU */
+  XLPK_ERR_CUDA = -3,          /* a CUDA runtime call failed (see xlpk_last_cuda_error) */
+  XLPK_ERR_OOM = -4,           /* device allocation failed */
+  XLPK_ERR_KV_FULL = -5,       /* n_steps would write past max_seq */
+  XLPK_ERR_TIMEOUT = -6,       /* a device-side dependency wait exceeded its limit */
+  XLPK_ERR_ABORTED = -7        /* the decode was abandoned after another CTA failed */
+} xlpk_status;
+
+typedef enum xlpk_dtype {
+  XLPK_DTYPE_BF16 = 0,         /* bf16 weights, row-major [N][K] */
+  XLPK_DTYPE_FP8_E4M3 = 1      /* e4m3 codes, row-major [N][K], + one fp32 scale per 128x128 block */
+} xlpk_dtype;
+
+/* Model and launch shape.  All widths are element counts.
+ * Dense models set n_experts = top_k = n_shared_experts = expert_ffn = 0. */
+typedef struct xlpk_config {
+  int32_t n_layers;
+  int32_t hidden;              /* H */
+  int32_t n_q_heads;           /* n_q */
+  int32_t n_kv_heads;          /* n_kv; n_q % n_kv == 0; query head h reads kv head h / (n_q / n_kv) */
+  int32_t head_dim;            /* d: 64 or 128 */
+  int32_t ffn;                 /* F, dense SwiGLU width */
+  int32_t vocab;               /* V */
+  int32_t n_experts;           /* E (MoE), else 0 */
+  int32_t top_k;               /* experts per token (MoE), else 0 */
+  int32_t n_shared_experts;    /* always-on experts (MoE), else 0 */
+  int32_t expert_ffn;          /* SwiGLU width of one expert (MoE), else 0 */
+  int32_t weight_dtype;        /* xlpk_dtype of every linear weight (embedding and router stay bf16) */
+  int32_t batch;               /* B sequences decoded together, 1..8 */
+  int32_t max_seq;             /* KV cache capacity per sequence (positions) */
+  float rope_theta;            /* RoPE base: pair (i, i + d/2) turns by pos * theta^(-2i/d) */
+  float rms_eps;               /* RMSNorm epsilon */
+  int32_t n_ctas;              /* persistent grid size; 0 = one CTA per SM */
+  int32_t spin_limit_us;       /* limit of every device-side wait; 0 = 200000 us */
+} xlpk_config;
+
+/* One linear weight: y = W x with W row-major [N][K] (PyTorch Linear layout).
+ * `scale` is NULL for bf16; for FP8 it is fp32 [N/128][K/128], row-major. */
+typedef struct xlpk_linear {
+  const void* w_dev;
+  const float* scale_dev;
+} xlpk_linear;
+
+typedef struct xlpk_layer_weights {
+  const float* attn_norm_dev;  /* fp32 [H] RMSNorm gain before attention */
+  xlpk_linear wq;              /* [n_q*d][H] */
+  xlpk_linear wk;              /* [n_kv*d][H] */
+  xlpk_linear wv;              /* [n_kv*d][H] */
+  xlpk_linear wo;              /* [H][n_q*d] */
+  const float* ffn_norm_dev;   /* fp32 [H] RMSNorm gain before the FFN */
+  xlpk_linear w_gate;          /* dense: [F][H] */
+  xlpk_linear w_up;            /* dense: [F][H] */
+  xlpk_linear w_down;          /* dense: [H][F] */
+  const void* router_dev;      /* MoE: bf16 [E][H] */
+  xlpk_linear we_gate;         /* MoE: [E][Fe][H], scale [E][Fe/128][H/128] */
+  xlpk_linear we_up;           /* MoE: [E][Fe][H] */
+  xlpk_linear we_down;         /* MoE: [E][H][Fe] */
+  xlpk_linear ws_gate;         /* MoE shared experts: [S][Fe][H] */
+  xlpk_linear ws_up;           /* MoE shared experts: [S][Fe][H] */
+  xlpk_linear ws_down;         /* MoE shared experts: [S][H][Fe] */
+} xlpk_layer_weights;
+
+typedef struct xlpk_weights {
+  const void* embed_dev;              /* bf16 [V][H] token embedding */
+  const float* final_norm_dev;        /* fp32 [H] */
+  xlpk_linear lm_head;                /* [V][H] */
+  const xlpk_layer_weights* layers;   /* HOST array of n_layers entries */
+} xlpk_weights;
+
+/* Caller-owned KV cache, bf16 [L][B][n_kv][max_seq][d] for K and V each,
+ * 16-byte aligned.  Entries are post-RoPE keys and values. */
+typedef struct xlpk_kv {
+  void* k_dev;
+  void* v_dev;
+} xlpk_kv;
+
+/* Optional per-step outputs and teacher forcing of one decode call.
+ * Every pointer may be NULL. */
+typedef struct xlpk_decode_io {
+  const int32_t* forced_tokens_dev;   /* [n_steps][B]: next input is forced[s][b] instead of the argmax */
+  float* logits_dev;                  /* [n_steps][B][V] fp32 logits of every step */
+  float* hidden_dev;                  /* [n_steps][B][H] fp32 residual after the last layer */
+  int32_t* experts_dev;               /* MoE: [n_steps][L][B][top_k] selected expert ids */
+} xlpk_decode_io;
+
+/* Facts about a created handle (for measurement and tests). */
+typedef struct xlpk_info {
+  int32_t n_ctas;               /* persistent grid size */
+  int32_t threads_per_cta;
+  int32_t smem_bytes;           /* dynamic shared memory per CTA */
+  int32_t ring_slots;           /* weight/KV staging slots per CTA */
+  int32_t slot_bytes;
+  int32_t kernels_per_step_unfused;
+  int64_t packed_weight_bytes;  /* library-owned packed copy of the weights */
+  int64_t workspace_bytes;
+  int64_t weight_bytes_per_step;  /* weights streamed per decode step (active experts for MoE at B=1) */
+} xlpk_info;
+
+typedef struct xlpk_engine* xlpk_handle;
+
+/* Validate `cfg`, pack the weights into a library-owned buffer laid out in
+ * the order the CTAs stream them, build the RoPE table, allocate the
+ * workspace and borrow the KV pointers for the handle's lifetime (the KV
+ * cache is written in place).  Weight buffers may be freed afterwards.
+ * Runs on the current device and synchronises it. */
+xlpk_status xlpk_create(const xlpk_config* cfg, const xlpk_weights* weights,
+                        const xlpk_kv* kv, xlpk_handle* out);
+
+/* Free everything the handle owns (not the caller's KV or weights). */
+xlpk_status xlpk_destroy(xlpk_handle h);
+
+/* Set the decode state: sequence b has seq_lens_host[b] positions already in
+ * the KV cache and pending input token tokens_host[b].  Enqueued on `stream`. */
+xlpk_status xlpk_set_state(xlpk_handle h, const int32_t* tokens_host,
+                           const int32_t* seq_lens_host, void* stream);
+
+/* Greedy-decode n_steps tokens per sequence as ONE persistent kernel launch.
+ * tokens_out_dev [n_steps][B] receives the argmax of every step.  Step s feeds
+ * the pending token at position seq_len + s, appends K/V there, and makes
+ * the argmax (or forced_tokens[s][b]) the next pending token.  Asynchronous
+ * on `stream`; XLPK_ERR_KV_FULL if seq_len + n_steps > max_seq. */
+xlpk_status xlpk_decode(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
+                        const xlpk_decode_io* io, void* stream);
+
+/* The same decode as one kernel launch per operator stage (5 per layer + 1
+ * per step), built from the same tiles: the kernel-per-op baseline. */
+xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
+                                const xlpk_decode_io* io, void* stream);
+
+/* End-to-end call with host buffers: uploads the state, decodes, downloads
+ * tokens_out_host [n_steps][B], and synchronises `stream`.  Returns the
+ * device status of the decode. */
+xlpk_status xlpk_generate(xlpk_handle h, const int32_t* tokens_host, const int32_t* seq_lens_host,
+                          int32_t n_steps, int32_t* tokens_out_host, void* stream);
+
+/* Synchronise the stream of the handle's last decode and return its device
+ * status (XLPK_OK, XLPK_ERR_TIMEOUT or XLPK_ERR_ABORTED).  After an error the
+ * handle's counters are reset; KV entries the failed call would have written
+ * are unspecified. */
+xlpk_status xlpk_get_status(xlpk_handle h);
+
+xlpk_status xlpk_get_info(xlpk_handle h, xlpk_info* out);
+
+/* Human-readable name of a status. */
+const char* xlpk_status_string(int32_t status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* xlpk_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XLPK_H_ */

@@ -1,0 +1,122 @@
+// Shared host/device description of one decode launch.
+//
+// The host planner (xlpk.cu) fills these at xlpk_create time; the kernels in
+// engine.cuh read them.  Everything a CTA needs to find its tiles is here or
+// derivable from (CTA index, grid size, step), so no per-task table has to be
+// fetched at run time: the "task list" of a CTA is the static partition of
+// every stage's rows (or attention chunks) by CTA index.
+#pragma once
+#include <stdint.h>
+
+namespace xlpk {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;      // + one producer warp
+constexpr int kSlotBytes = 32768;                     // one staging slot of the ring
+constexpr int kMaxSlots = 8;
+constexpr int kMaxBatch = 8;
+constexpr int kMaxGroup = 4;                          // query heads per kv head
+constexpr int kPairsPerTile = kConsumerWarps;         // one row pair per consumer warp
+constexpr int kMiscSmem = 4096;                       // barriers, flags, reduction scratch
+
+// Stages of one layer, in dependency order, then the LM head.
+enum StageKind : int {
+  ST_QKV = 0,     // RMSNorm(x) -> [q;k;v] GEMV, RoPE, KV append
+  ST_ATTN = 1,    // flash-decoding split over the sequence + last-arriver combine
+  ST_OPROJ = 2,   // x += Wo o   (layer 0: x = E[tok] + Wo o)
+  ST_GATEUP = 3,  // h = silu(Wg xn) * (Wu xn)
+  ST_DOWN = 4,    // x += Wd h
+  ST_LAYER = 5,   // stages per layer
+  ST_LM = 5       // logits = Wlm RMSNorm(x), argmax, next token
+};
+
+// Counter slots (unsigned, monotonic unless noted).
+//   cnt[l*ST_LAYER + kind]   arrivals of stage `kind` of layer l: G per step,
+//                            except ST_ATTN which counts finished (b, kv-head)
+//                            combines: B*n_kv per step.
+//   cnt[lm_arrive]           G per step
+//   cnt[step_done]           1 per step
+//   cnt[attn_arrive + ...]   per (layer, b, kv head) chunk arrivals, reset to 0
+//                            by the CTA that completes the head.
+struct CounterLayout {
+  int lm_arrive;
+  int step_done;
+  int attn_arrive;
+  int total;
+};
+
+// A packed GEMV operand: logical rows are grouped in pairs; the pairs are
+// split evenly over the CTAs; a CTA's pairs are cut into groups of up to 8
+// (one pair per consumer warp) and each group into k-chunks of KC columns.
+// Tile (group, chunk) holds [2*gp rows][KC cols] contiguously, and the tiles
+// of a CTA follow each other, so the CTA's whole span is one contiguous range
+// streamed front to back.
+struct Mat {
+  const uint8_t* packed;
+  const float* scales;   // FP8: per logical row, K/128 fp32 scales; else nullptr
+  int N;                 // logical rows (even)
+  int K;                 // columns
+  int KC;                // k-chunk (divides K)
+  int pad;
+};
+
+struct LayerParams {
+  Mat qkv;     // rows: q heads (RoPE pairs interleaved), k heads (interleaved), v heads
+  Mat o;
+  Mat gu;      // rows: gate_j, up_j interleaved
+  Mat down;
+  const float* attn_norm;
+  const float* ffn_norm;
+};
+
+struct Params {
+  // shape
+  int L, H, nq, nkv, d, F, V, B, max_seq;
+  int group;            // nq / nkv
+  int esz;              // weight bytes per element (2 bf16, 1 fp8)
+  float eps;
+  float qk_scale_log2;  // log2(e) / sqrt(d)
+  int G;                // CTAs
+  int nslot;            // ring slots in use
+  int act_bytes;        // activation / scratch region
+  int attn_pos_per_tile;
+  long long spin_limit_ns;
+  CounterLayout cl;
+
+  // weights
+  const uint16_t* embed;        // bf16 [V][H]
+  const float* final_norm;
+  Mat lm;
+  const LayerParams* layers;    // device array [L]
+
+  // KV cache (caller-owned), bf16 [L][B][nkv][max_seq][d]
+  uint16_t* kc;
+  uint16_t* vc;
+  const float2* rope;           // [max_seq][d/2] (cos, sin)
+
+  // workspace
+  float* x;          // [B][H] residual stream
+  float* q;          // [B][nq*d] rotated queries
+  float* o;          // [B][nq*d] attention output
+  float* h;          // [B][F] SwiGLU output
+  float* part_ml;    // [items][group][2] (running max in log2 units, sum)
+  float* part_o;     // [items][group][d]
+  float* lm_val;     // [G][B]
+  int* lm_idx;       // [G][B]
+  unsigned* cnt;
+  int* cur_tok;      // [B] pending input token
+  int* status;       // [0] error code, [1] where
+  int* abort_flag;
+
+  // per call
+  int n_steps;
+  int step_base;     // global index of this call's first step
+  int pos0[kMaxBatch];
+  int32_t* tokens_out;
+  const int32_t* forced;
+  float* logits_out;
+  float* hidden_out;
+};
+
+}  // namespace xlpk

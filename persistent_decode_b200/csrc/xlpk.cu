@@ -1,0 +1,626 @@
+// Host side of the C ABI (include/xlpk.h): validation, the ahead-of-time
+// planner (static partition of every stage over the CTAs, weight packing in
+// stream order, RoPE table, workspace), and the launches.
+//
+// The planner is the "AOT" half of the design the pages describe: the model is
+// unrolled ahead of time into a fixed schedule of tile tasks whose shapes,
+// placement and residency are decided before the first token ("Ultra-High
+// Interactivity On NVIDIA GPUs? - TileRT InferenceX", digest, core views: the
+// decode graph is statically compiled into one resident Engine Kernel; the
+// fixed temporary-tensor table of "Persistent execution paradigm", section
+// 5.3, becomes the static workspace arena below).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/xlpk.h"
+#include "engine.cuh"
+#include "params.h"
+
+using namespace xlpk;
+
+namespace {
+
+thread_local std::string g_cuda_err;
+
+xlpk_status cuda_fail(cudaError_t e, const char* what) {
+  g_cuda_err = std::string(what) + ": " + cudaGetErrorString(e);
+  return e == cudaErrorMemoryAllocation ? XLPK_ERR_OOM : XLPK_ERR_CUDA;
+}
+
+#define XLPK_CUDA(call)                               \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+struct PackJob {
+  const uint8_t* src;   // source row
+  long long dst;        // byte offset of the row's first chunk in the packed buffer
+  long long stride;     // bytes between consecutive chunks of this row
+};
+
+// One warp per packed row: chunk c of the row goes to dst + c*stride.
+__global__ void pack_rows_kernel(const PackJob* jobs, int njobs, uint8_t* out, int row_bytes,
+                                 int chunk_bytes) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= njobs) return;
+  const PackJob j = jobs[warp];
+  const int nvec = row_bytes >> 4, nvc = chunk_bytes >> 4;
+  const uint4* src = reinterpret_cast<const uint4*>(j.src);
+  for (int v = lane; v < nvec; v += 32) {
+    const int c = v / nvc, w = v - c * nvc;
+    *reinterpret_cast<uint4*>(out + j.dst + c * j.stride + static_cast<long long>(w) * 16) = src[v];
+  }
+}
+
+long long split_host(long long c, long long n, long long G) { return (c * n) / G; }
+
+int pick_kc(int K, int esz) {
+  const int vec = 16 / esz;
+  const int cap = kSlotBytes / (2 * kPairsPerTile * esz);
+  for (int kc = std::min(K, cap); kc >= vec; --kc)
+    if (K % kc == 0 && kc % vec == 0) return kc;
+  return 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+enum class MatKind { QKV, PLAIN, GATEUP };
+
+struct MatSrc {
+  MatKind kind;
+  const uint8_t* a;   // QKV: wq; GATEUP: gate; PLAIN: w
+  const uint8_t* b;   // QKV: wk; GATEUP: up
+  const uint8_t* c;   // QKV: wv
+};
+
+}  // namespace
+
+struct xlpk_engine {
+  xlpk_config cfg{};
+  int device = 0;
+  int G = 0;
+  int nslot = 0;
+  int smem = 0;
+  int act_bytes = 0;
+  int esz = 2;
+  int P = 0;
+  uint8_t* packed = nullptr;
+  size_t packed_bytes = 0;
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  LayerParams* d_layers = nullptr;
+  float2* rope = nullptr;
+  int32_t* tok_scratch = nullptr;
+  Params base{};
+  std::vector<int> pos;
+  int step_base = 0;
+  cudaStream_t last_stream = nullptr;
+  const void* kern_persistent = nullptr;
+  const void* kern_stage = nullptr;
+  void (*launch_stage)(const Params&, int, int, int, int, int, cudaStream_t) = nullptr;
+  int64_t weight_bytes_per_step = 0;
+};
+
+namespace {
+
+template <int B, int D>
+void launch_stage_impl(const Params& p, int kind, int layer, int step, int G, int smem,
+                       cudaStream_t st) {
+  engine_stage<B, D><<<G, kThreads, smem, st>>>(p, kind, layer, step);
+}
+
+template <int B, int D>
+void bind_kernels(xlpk_engine* e) {
+  e->kern_persistent = reinterpret_cast<const void*>(&engine_persistent<B, D>);
+  e->kern_stage = reinterpret_cast<const void*>(&engine_stage<B, D>);
+  e->launch_stage = &launch_stage_impl<B, D>;
+}
+
+bool bind_by_shape(xlpk_engine* e, int B, int D) {
+#define XLPK_BIND(b, d)          \
+  if (B == b && D == d) {        \
+    bind_kernels<b, d>(e);       \
+    return true;                 \
+  }
+  XLPK_BIND(1, 64)
+  XLPK_BIND(1, 128)
+  XLPK_BIND(2, 64)
+  XLPK_BIND(2, 128)
+  XLPK_BIND(4, 64)
+  XLPK_BIND(4, 128)
+  XLPK_BIND(8, 64)
+  XLPK_BIND(8, 128)
+#undef XLPK_BIND
+  return false;
+}
+
+// Logical row n of a packed matrix -> source row pointer.
+const uint8_t* source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_config& c) {
+  const long long row_bytes = static_cast<long long>(K) * esz;
+  const long long pr = n >> 1;
+  const int r = static_cast<int>(n & 1);
+  switch (ms.kind) {
+    case MatKind::PLAIN:
+      return ms.a + n * row_bytes;
+    case MatKind::GATEUP:
+      return (r == 0 ? ms.a : ms.b) + pr * row_bytes;
+    case MatKind::QKV: {
+      const long long half = c.head_dim / 2;
+      const long long hq = static_cast<long long>(c.n_q_heads) * half;
+      const long long hk = static_cast<long long>(c.n_kv_heads) * half;
+      if (pr < hq + hk) {
+        const bool isq = pr < hq;
+        const long long pp = isq ? pr : pr - hq;
+        const long long head = pp / half, i = pp % half;
+        const long long row = head * c.head_dim + i + r * half;
+        return (isq ? ms.a : ms.b) + row * row_bytes;
+      }
+      const long long pv = pr - hq - hk;
+      return ms.c + (2 * pv + r) * row_bytes;
+    }
+  }
+  return nullptr;
+}
+
+// Pack one matrix into `dst` (device) in stream order; returns the Mat view.
+xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t* dst, Mat* out,
+                        PackJob* d_jobs, size_t max_jobs, cudaStream_t st) {
+  const int esz = e->esz;
+  const int KC = pick_kc(K, esz);
+  if (KC == 0) return XLPK_ERR_UNSUPPORTED;
+  const long long NP = N / 2, G = e->G;
+  std::vector<PackJob> jobs;
+  jobs.reserve(static_cast<size_t>(N));
+  for (long long c = 0; c < G; ++c) {
+    const long long p0 = split_host(c, NP, G), p1 = split_host(c + 1, NP, G);
+    const long long npc = p1 - p0;
+    for (long long lp = 0; lp < npc; ++lp) {
+      const long long j = lp / kPairsPerTile, w = lp % kPairsPerTile;
+      const long long gp = std::min<long long>(kPairsPerTile, npc - kPairsPerTile * j);
+      const long long group_off =
+          (2 * p0 * K + 2LL * kPairsPerTile * j * K) * static_cast<long long>(esz);
+      for (int r = 0; r < 2; ++r) {
+        PackJob pj;
+        pj.src = source_row(ms, 2 * (p0 + lp) + r, K, esz, e->cfg);
+        pj.dst = group_off + (2 * w + r) * static_cast<long long>(KC) * esz;
+        pj.stride = 2 * gp * static_cast<long long>(KC) * esz;
+        jobs.push_back(pj);
+      }
+    }
+  }
+  const int row_bytes = K * esz, chunk_bytes = KC * esz;
+  for (size_t off = 0; off < jobs.size(); off += max_jobs) {
+    const size_t n = std::min(max_jobs, jobs.size() - off);
+    XLPK_CUDA(cudaMemcpyAsync(d_jobs, jobs.data() + off, n * sizeof(PackJob), cudaMemcpyHostToDevice, st));
+    const int threads = 256;
+    const int blocks = static_cast<int>((n * 32 + threads - 1) / threads);
+    pack_rows_kernel<<<blocks, threads, 0, st>>>(d_jobs, static_cast<int>(n), dst, row_bytes, chunk_bytes);
+    XLPK_CUDA(cudaGetLastError());
+    XLPK_CUDA(cudaStreamSynchronize(st));
+  }
+  out->packed = dst;
+  out->scales = nullptr;
+  out->N = N;
+  out->K = K;
+  out->KC = KC;
+  out->pad = 0;
+  return XLPK_OK;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+xlpk_status validate_config(const xlpk_config* c) {
+  if (!c) return XLPK_ERR_INVALID_ARG;
+  if (c->n_layers < 1 || c->n_layers > 1024 || c->hidden <= 0 || c->n_q_heads <= 0 ||
+      c->n_kv_heads <= 0 || c->head_dim <= 0 || c->vocab <= 1 || c->batch < 1 || c->max_seq < 1)
+    return XLPK_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads != 0) return XLPK_ERR_INVALID_ARG;
+  if (c->weight_dtype != XLPK_DTYPE_BF16 && c->weight_dtype != XLPK_DTYPE_FP8_E4M3)
+    return XLPK_ERR_INVALID_ARG;
+  if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return XLPK_ERR_INVALID_ARG;
+  if (c->n_ctas < 0 || c->spin_limit_us < 0) return XLPK_ERR_INVALID_ARG;
+  if (c->n_experts < 0 || c->top_k < 0 || c->n_shared_experts < 0 || c->expert_ffn < 0)
+    return XLPK_ERR_INVALID_ARG;
+  // shapes this build handles
+  if (c->head_dim != 64 && c->head_dim != 128) return XLPK_ERR_UNSUPPORTED;
+  if (c->n_q_heads / c->n_kv_heads > kMaxGroup) return XLPK_ERR_UNSUPPORTED;
+  if (c->batch != 1 && c->batch != 2 && c->batch != 4 && c->batch != 8) return XLPK_ERR_UNSUPPORTED;
+  if (c->weight_dtype != XLPK_DTYPE_BF16) return XLPK_ERR_UNSUPPORTED;
+  if (c->n_experts != 0) return XLPK_ERR_UNSUPPORTED;
+  if (c->ffn <= 0) return XLPK_ERR_INVALID_ARG;
+  if (c->hidden % 16 || c->ffn % 16 || (c->n_q_heads * c->head_dim) % 16 || c->vocab % 2)
+    return XLPK_ERR_UNSUPPORTED;
+  return XLPK_OK;
+}
+
+xlpk_status validate_weights(const xlpk_config* c, const xlpk_weights* w, const xlpk_kv* kv) {
+  if (!w || !kv || !w->layers || !w->embed_dev || !w->final_norm_dev || !w->lm_head.w_dev)
+    return XLPK_ERR_INVALID_ARG;
+  if (!kv->k_dev || !kv->v_dev || !aligned16(kv->k_dev) || !aligned16(kv->v_dev))
+    return XLPK_ERR_INVALID_ARG;
+  if (!aligned16(w->embed_dev) || !aligned16(w->lm_head.w_dev)) return XLPK_ERR_INVALID_ARG;
+  for (int l = 0; l < c->n_layers; ++l) {
+    const xlpk_layer_weights& L = w->layers[l];
+    const void* need[] = {L.attn_norm_dev, L.ffn_norm_dev, L.wq.w_dev, L.wk.w_dev, L.wv.w_dev,
+                          L.wo.w_dev, L.w_gate.w_dev, L.w_up.w_dev, L.w_down.w_dev};
+    for (const void* q : need)
+      if (!q || !aligned16(q)) return XLPK_ERR_INVALID_ARG;
+  }
+  return XLPK_OK;
+}
+
+void fill_rope(std::vector<float2>& t, int max_seq, int d, double theta) {
+  const int half = d / 2;
+  t.resize(static_cast<size_t>(max_seq) * half);
+  for (int pos = 0; pos < max_seq; ++pos)
+    for (int i = 0; i < half; ++i) {
+      const double inv = std::pow(theta, -2.0 * i / d);
+      const double a = static_cast<double>(pos) * inv;
+      t[static_cast<size_t>(pos) * half + i] =
+          make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
+    }
+}
+
+void free_engine(xlpk_engine* e) {
+  if (!e) return;
+  cudaFree(e->packed);
+  cudaFree(e->ws);
+  cudaFree(e->d_layers);
+  cudaFree(e->rope);
+  delete e;
+}
+
+xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlpk_kv* kv,
+                        xlpk_engine* e) {
+  const xlpk_config& c = *cfg;
+  e->cfg = c;
+  XLPK_CUDA(cudaGetDevice(&e->device));
+  cudaDeviceProp prop;
+  XLPK_CUDA(cudaGetDeviceProperties(&prop, e->device));
+  if (prop.major != 10) {
+    g_cuda_err = "device is not sm_100";
+    return XLPK_ERR_UNSUPPORTED;
+  }
+  if (!prop.cooperativeLaunch) return XLPK_ERR_UNSUPPORTED;
+  e->G = c.n_ctas > 0 ? c.n_ctas : prop.multiProcessorCount;
+  e->esz = c.weight_dtype == XLPK_DTYPE_FP8_E4M3 ? 1 : 2;
+  const int B = c.batch, H = c.hidden, d = c.head_dim, F = c.ffn;
+  const int qd = c.n_q_heads * d, kvd = c.n_kv_heads * d;
+  const int group = c.n_q_heads / c.n_kv_heads;
+  e->P = (kSlotBytes / 2) / (d * 2);
+
+  // shared memory: ring + activation/scratch + control
+  const int kmax = std::max(std::max(H, qd), F);
+  const int attn_scratch = (kConsumerWarps * kMaxGroup * 2 + kConsumerWarps * kMaxGroup * d) * 4;
+  e->act_bytes = static_cast<int>(align_up(std::max(B * kmax * 4, attn_scratch), 1024));
+  const int max_smem = static_cast<int>(prop.sharedMemPerBlockOptin);
+  e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - kMiscSmem) / kSlotBytes);
+  if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
+  e->smem = e->nslot * kSlotBytes + e->act_bytes + kMiscSmem;
+  if (!bind_by_shape(e, B, d)) return XLPK_ERR_UNSUPPORTED;
+
+  XLPK_CUDA(cudaFuncSetAttribute(e->kern_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, e->smem));
+  XLPK_CUDA(cudaFuncSetAttribute(e->kern_stage, cudaFuncAttributeMaxDynamicSharedMemorySize, e->smem));
+  int per_sm = 0;
+  XLPK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, e->kern_persistent, kThreads, e->smem));
+  if (per_sm < 1 || e->G > per_sm * prop.multiProcessorCount) {
+    g_cuda_err = "persistent grid does not fit co-resident";
+    return XLPK_ERR_UNSUPPORTED;
+  }
+
+  // packed weights: per layer qkv, o, gate/up, down; then the LM head
+  struct MatPlan {
+    MatSrc src;
+    int N, K;
+    size_t off;
+  };
+  std::vector<MatPlan> mats;
+  size_t total = 0;
+  auto add = [&](MatSrc s, int N, int K) {
+    mats.push_back({s, N, K, total});
+    total += align_up(static_cast<size_t>(N) * K * e->esz, 256);
+  };
+  for (int l = 0; l < c.n_layers; ++l) {
+    const xlpk_layer_weights& L = w->layers[l];
+    auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
+    add({MatKind::QKV, u8(L.wq.w_dev), u8(L.wk.w_dev), u8(L.wv.w_dev)}, qd + 2 * kvd, H);
+    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr}, H, qd);
+    add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr}, 2 * F, H);
+    add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, H, F);
+  }
+  add({MatKind::PLAIN, static_cast<const uint8_t*>(w->lm_head.w_dev), nullptr, nullptr}, c.vocab, H);
+  e->packed_bytes = total;
+  XLPK_CUDA(cudaMalloc(&e->packed, total));
+  e->weight_bytes_per_step = 0;
+  for (const MatPlan& m : mats) e->weight_bytes_per_step += static_cast<int64_t>(m.N) * m.K * e->esz;
+
+  cudaStream_t st;
+  XLPK_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+  const size_t max_jobs = 1 << 20;
+  PackJob* d_jobs = nullptr;
+  cudaError_t ce = cudaMalloc(&d_jobs, max_jobs * sizeof(PackJob));
+  if (ce != cudaSuccess) {
+    cudaStreamDestroy(st);
+    return cuda_fail(ce, "cudaMalloc(jobs)");
+  }
+  std::vector<LayerParams> lp(c.n_layers);
+  Mat lm{};
+  xlpk_status rc = XLPK_OK;
+  for (size_t i = 0; i < mats.size() && rc == XLPK_OK; ++i) {
+    Mat m{};
+    rc = pack_matrix(e, mats[i].src, mats[i].N, mats[i].K, e->packed + mats[i].off, &m, d_jobs, max_jobs, st);
+    if (rc != XLPK_OK) break;
+    if (i + 1 == mats.size()) {
+      lm = m;
+    } else {
+      LayerParams& L = lp[i / 4];
+      switch (i % 4) {
+        case 0: L.qkv = m; break;
+        case 1: L.o = m; break;
+        case 2: L.gu = m; break;
+        default: L.down = m; break;
+      }
+    }
+  }
+  cudaFree(d_jobs);
+  cudaStreamDestroy(st);
+  if (rc != XLPK_OK) return rc;
+  for (int l = 0; l < c.n_layers; ++l) {
+    lp[l].attn_norm = w->layers[l].attn_norm_dev;
+    lp[l].ffn_norm = w->layers[l].ffn_norm_dev;
+  }
+  XLPK_CUDA(cudaMalloc(&e->d_layers, sizeof(LayerParams) * c.n_layers));
+  XLPK_CUDA(cudaMemcpy(e->d_layers, lp.data(), sizeof(LayerParams) * c.n_layers, cudaMemcpyHostToDevice));
+
+  std::vector<float2> rope;
+  fill_rope(rope, c.max_seq, d, c.rope_theta);
+  XLPK_CUDA(cudaMalloc(&e->rope, rope.size() * sizeof(float2)));
+  XLPK_CUDA(cudaMemcpy(e->rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice));
+
+  // workspace arena with fixed offsets
+  const long long wmax = static_cast<long long>(B) * c.n_kv_heads * ((c.max_seq + e->P - 1) / e->P);
+  CounterLayout cl;
+  cl.lm_arrive = c.n_layers * ST_LAYER;
+  cl.step_done = cl.lm_arrive + 1;
+  cl.attn_arrive = cl.step_done + 1;
+  cl.total = cl.attn_arrive + c.n_layers * B * c.n_kv_heads;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_x = take(sizeof(float) * B * H);
+  const size_t o_q = take(sizeof(float) * B * qd);
+  const size_t o_o = take(sizeof(float) * B * qd);
+  const size_t o_h = take(sizeof(float) * B * F);
+  const size_t o_pml = take(sizeof(float) * wmax * group * 2);
+  const size_t o_po = take(sizeof(float) * wmax * group * d);
+  const size_t o_lv = take(sizeof(float) * e->G * B);
+  const size_t o_li = take(sizeof(int) * e->G * B);
+  const size_t o_cnt = take(sizeof(unsigned) * cl.total);
+  const size_t o_tok = take(sizeof(int) * B);
+  const size_t o_st = take(sizeof(int) * 4);
+  const size_t o_ab = take(sizeof(int));
+  const size_t o_ts = take(sizeof(int) * static_cast<size_t>(c.max_seq) * B);
+  e->ws_bytes = off;
+  XLPK_CUDA(cudaMalloc(&e->ws, e->ws_bytes));
+  XLPK_CUDA(cudaMemset(e->ws, 0, e->ws_bytes));
+
+  Params& p = e->base;
+  p.L = c.n_layers;
+  p.H = H;
+  p.nq = c.n_q_heads;
+  p.nkv = c.n_kv_heads;
+  p.d = d;
+  p.F = F;
+  p.V = c.vocab;
+  p.B = B;
+  p.max_seq = c.max_seq;
+  p.group = group;
+  p.esz = e->esz;
+  p.eps = c.rms_eps;
+  p.qk_scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  p.G = e->G;
+  p.nslot = e->nslot;
+  p.act_bytes = e->act_bytes;
+  p.attn_pos_per_tile = e->P;
+  p.spin_limit_ns = 1000LL * (c.spin_limit_us > 0 ? c.spin_limit_us : 200000);
+  p.cl = cl;
+  p.embed = static_cast<const uint16_t*>(w->embed_dev);
+  p.final_norm = w->final_norm_dev;
+  p.lm = lm;
+  p.layers = e->d_layers;
+  p.kc = static_cast<uint16_t*>(kv->k_dev);
+  p.vc = static_cast<uint16_t*>(kv->v_dev);
+  p.rope = e->rope;
+  p.x = reinterpret_cast<float*>(e->ws + o_x);
+  p.q = reinterpret_cast<float*>(e->ws + o_q);
+  p.o = reinterpret_cast<float*>(e->ws + o_o);
+  p.h = reinterpret_cast<float*>(e->ws + o_h);
+  p.part_ml = reinterpret_cast<float*>(e->ws + o_pml);
+  p.part_o = reinterpret_cast<float*>(e->ws + o_po);
+  p.lm_val = reinterpret_cast<float*>(e->ws + o_lv);
+  p.lm_idx = reinterpret_cast<int*>(e->ws + o_li);
+  p.cnt = reinterpret_cast<unsigned*>(e->ws + o_cnt);
+  p.cur_tok = reinterpret_cast<int*>(e->ws + o_tok);
+  p.status = reinterpret_cast<int*>(e->ws + o_st);
+  p.abort_flag = reinterpret_cast<int*>(e->ws + o_ab);
+  e->tok_scratch = reinterpret_cast<int32_t*>(e->ws + o_ts);
+  e->pos.assign(B, 0);
+  XLPK_CUDA(cudaDeviceSynchronize());
+  return XLPK_OK;
+}
+
+xlpk_status check_decode_args(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out) {
+  if (!h || n_steps < 0) return XLPK_ERR_INVALID_ARG;
+  if (n_steps > 0 && !tokens_out) return XLPK_ERR_INVALID_ARG;
+  for (int b = 0; b < h->cfg.batch; ++b)
+    if (static_cast<long long>(h->pos[b]) + n_steps > h->cfg.max_seq) return XLPK_ERR_KV_FULL;
+  return XLPK_OK;
+}
+
+Params call_params(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out, const xlpk_decode_io* io) {
+  Params p = h->base;
+  p.n_steps = n_steps;
+  p.step_base = h->step_base;
+  for (int b = 0; b < kMaxBatch; ++b) p.pos0[b] = b < h->cfg.batch ? h->pos[b] : 0;
+  p.tokens_out = tokens_out;
+  p.forced = io ? io->forced_tokens_dev : nullptr;
+  p.logits_out = io ? io->logits_dev : nullptr;
+  p.hidden_out = io ? io->hidden_dev : nullptr;
+  return p;
+}
+
+void advance(xlpk_engine* h, int32_t n_steps, cudaStream_t st) {
+  for (int b = 0; b < h->cfg.batch; ++b) h->pos[b] += n_steps;
+  h->step_base += n_steps;
+  h->last_stream = st;
+}
+
+}  // namespace
+
+extern "C" {
+
+xlpk_status xlpk_create(const xlpk_config* cfg, const xlpk_weights* weights, const xlpk_kv* kv,
+                        xlpk_handle* out) {
+  if (!out) return XLPK_ERR_INVALID_ARG;
+  *out = nullptr;
+  xlpk_status rc = validate_config(cfg);
+  if (rc != XLPK_OK) return rc;
+  rc = validate_weights(cfg, weights, kv);
+  if (rc != XLPK_OK) return rc;
+  xlpk_engine* e = new xlpk_engine();
+  rc = create_impl(cfg, weights, kv, e);
+  if (rc != XLPK_OK) {
+    free_engine(e);
+    return rc;
+  }
+  *out = e;
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_destroy(xlpk_handle h) {
+  if (!h) return XLPK_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  free_engine(h);
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_set_state(xlpk_handle h, const int32_t* tokens_host, const int32_t* seq_lens_host,
+                           void* stream) {
+  if (!h || !tokens_host || !seq_lens_host) return XLPK_ERR_INVALID_ARG;
+  for (int b = 0; b < h->cfg.batch; ++b) {
+    if (tokens_host[b] < 0 || tokens_host[b] >= h->cfg.vocab) return XLPK_ERR_INVALID_ARG;
+    if (seq_lens_host[b] < 0 || seq_lens_host[b] >= h->cfg.max_seq) return XLPK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  XLPK_CUDA(cudaMemcpyAsync(h->base.cur_tok, tokens_host, sizeof(int32_t) * h->cfg.batch,
+                            cudaMemcpyHostToDevice, st));
+  for (int b = 0; b < h->cfg.batch; ++b) h->pos[b] = seq_lens_host[b];
+  h->last_stream = st;
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_decode(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
+                        const xlpk_decode_io* io, void* stream) {
+  xlpk_status rc = check_decode_args(h, n_steps, tokens_out_dev);
+  if (rc != XLPK_OK || n_steps == 0) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = call_params(h, n_steps, tokens_out_dev, io);
+  void* args[] = {&p};
+  XLPK_CUDA(cudaLaunchCooperativeKernel(h->kern_persistent, dim3(h->G), dim3(kThreads), args,
+                                        static_cast<size_t>(h->smem), st));
+  advance(h, n_steps, st);
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
+                                const xlpk_decode_io* io, void* stream) {
+  xlpk_status rc = check_decode_args(h, n_steps, tokens_out_dev);
+  if (rc != XLPK_OK || n_steps == 0) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = call_params(h, n_steps, tokens_out_dev, io);
+  for (int s = 0; s < n_steps; ++s) {
+    for (int l = 0; l < h->cfg.n_layers; ++l)
+      for (int k = 0; k < ST_LAYER; ++k) h->launch_stage(p, k, l, s, h->G, h->smem, st);
+    h->launch_stage(p, ST_LM, 0, s, h->G, h->smem, st);
+  }
+  XLPK_CUDA(cudaGetLastError());
+  advance(h, n_steps, st);
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_generate(xlpk_handle h, const int32_t* tokens_host, const int32_t* seq_lens_host,
+                          int32_t n_steps, int32_t* tokens_out_host, void* stream) {
+  if (!h || !tokens_out_host) return XLPK_ERR_INVALID_ARG;
+  if (n_steps < 0 || n_steps > h->cfg.max_seq) return XLPK_ERR_INVALID_ARG;
+  xlpk_status rc = xlpk_set_state(h, tokens_host, seq_lens_host, stream);
+  if (rc != XLPK_OK) return rc;
+  rc = xlpk_decode(h, n_steps, h->tok_scratch, nullptr, stream);
+  if (rc != XLPK_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  XLPK_CUDA(cudaMemcpyAsync(tokens_out_host, h->tok_scratch,
+                            sizeof(int32_t) * static_cast<size_t>(n_steps) * h->cfg.batch,
+                            cudaMemcpyDeviceToHost, st));
+  return xlpk_get_status(h);
+}
+
+xlpk_status xlpk_get_status(xlpk_handle h) {
+  if (!h) return XLPK_ERR_INVALID_ARG;
+  XLPK_CUDA(cudaStreamSynchronize(h->last_stream));
+  int st[4] = {0, 0, 0, 0};
+  XLPK_CUDA(cudaMemcpy(st, h->base.status, sizeof(st), cudaMemcpyDeviceToHost));
+  if (st[0] == 0) return XLPK_OK;
+  // reset the device-side ordering state so the handle is usable again
+  XLPK_CUDA(cudaMemset(h->base.cnt, 0, sizeof(unsigned) * h->base.cl.total));
+  XLPK_CUDA(cudaMemset(h->base.status, 0, sizeof(int) * 4));
+  XLPK_CUDA(cudaMemset(h->base.abort_flag, 0, sizeof(int)));
+  XLPK_CUDA(cudaDeviceSynchronize());
+  h->step_base = 0;
+  char buf[128];
+  std::snprintf(buf, sizeof(buf), "device wait failed: stage %d layer %d step %d cta %d", st[1] & 0xff,
+                (st[1] >> 8) & 0xff, (st[1] >> 16) & 0x7fff, st[2]);
+  g_cuda_err = buf;
+  return static_cast<xlpk_status>(st[0]);
+}
+
+xlpk_status xlpk_get_info(xlpk_handle h, xlpk_info* out) {
+  if (!h || !out) return XLPK_ERR_INVALID_ARG;
+  out->n_ctas = h->G;
+  out->threads_per_cta = kThreads;
+  out->smem_bytes = h->smem;
+  out->ring_slots = h->nslot;
+  out->slot_bytes = kSlotBytes;
+  out->kernels_per_step_unfused = h->cfg.n_layers * ST_LAYER + 1;
+  out->packed_weight_bytes = static_cast<int64_t>(h->packed_bytes);
+  out->workspace_bytes = static_cast<int64_t>(h->ws_bytes);
+  out->weight_bytes_per_step = h->weight_bytes_per_step;
+  return XLPK_OK;
+}
+
+const char* xlpk_status_string(int32_t s) {
+  switch (s) {
+    case XLPK_OK: return "XLPK_OK";
+    case XLPK_ERR_INVALID_ARG: return "XLPK_ERR_INVALID_ARG";
+    case XLPK_ERR_UNSUPPORTED: return "XLPK_ERR_UNSUPPORTED";
+    case XLPK_ERR_CUDA: return "XLPK_ERR_CUDA";
+    case XLPK_ERR_OOM: return "XLPK_ERR_OOM";
+    case XLPK_ERR_KV_FULL: return "XLPK_ERR_KV_FULL";
+    case XLPK_ERR_TIMEOUT: return "XLPK_ERR_TIMEOUT";
+    case XLPK_ERR_ABORTED: return "XLPK_ERR_ABORTED";
+    default: return "XLPK_ERR_UNKNOWN";
+  }
+}
+
+const char* xlpk_last_cuda_error(void) { return g_cuda_err.c_str(); }
+
+}  // extern "C"

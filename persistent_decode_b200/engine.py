@@ -1,0 +1,158 @@
+"""Python handle over the C ABI: argument marshalling only.
+
+Every step of the decode runs in libxlpk.so's kernels; torch is used here only
+to hold device memory and to name the CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from typing import Dict, Optional
+
+from . import _abi
+
+_LIB = None
+
+
+def get_lib():
+    """The loaded libxlpk.so (raises ImportError if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _abi.load()
+    return _LIB
+
+
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(get_lib(), name)
+
+
+lib = _LazyLib()
+
+
+class XlpkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        msg = lib.xlpk_status_string(status).decode()
+        detail = lib.xlpk_last_cuda_error().decode()
+        super().__init__(f"{what}: {msg}" + (f" ({detail})" if detail else ""))
+        self.status = status
+
+
+def _check(status: int, what: str) -> None:
+    if status != _abi.XLPK_OK:
+        raise XlpkError(status, what)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) or None
+
+
+def make_config(cfg, n_ctas: int = 0, spin_limit_us: int = 0, batch: Optional[int] = None,
+                max_seq: Optional[int] = None) -> _abi.xlpk_config:
+    c = _abi.xlpk_config()
+    for f in ("n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
+              "n_experts", "top_k", "n_shared_experts", "expert_ffn"):
+        setattr(c, f, int(getattr(cfg, f)))
+    c.weight_dtype = _abi.XLPK_DTYPE_FP8_E4M3 if cfg.weight_dtype == "fp8_e4m3" else _abi.XLPK_DTYPE_BF16
+    c.batch = int(batch if batch is not None else cfg.batch)
+    c.max_seq = int(max_seq if max_seq is not None else cfg.max_seq)
+    c.rope_theta = float(cfg.rope_theta)
+    c.rms_eps = float(cfg.rms_eps)
+    c.n_ctas = int(n_ctas)
+    c.spin_limit_us = int(spin_limit_us)
+    return c
+
+
+class Engine:
+    """One xlpk handle.
+
+    `weights` maps names ("embed", "lm_head", "final_norm", "layers.{l}.wq", ...,
+    with ".scale" companions for FP8) to CUDA tensors in row-major [out][in]
+    layout; `k_cache`/`v_cache` are bf16 CUDA tensors [L][B][n_kv][max_seq][d]
+    that the engine writes in place.
+    """
+
+    def __init__(self, cfg, weights: Dict[str, "object"], k_cache, v_cache, n_ctas: int = 0,
+                 spin_limit_us: int = 0):
+        self.cfg = cfg
+        self.B = int(k_cache.shape[1])
+        self.max_seq = int(k_cache.shape[3])
+        self._c = make_config(cfg, n_ctas, spin_limit_us, batch=self.B, max_seq=self.max_seq)
+        L = cfg.n_layers
+        self._layers = (_abi.xlpk_layer_weights * max(L, 1))()
+
+        def lin(name):
+            return _abi.xlpk_linear(_ptr(weights[name]), _ptr(weights.get(name + ".scale")))
+
+        for l in range(L):
+            p = f"layers.{l}."
+            lw = self._layers[l]
+            lw.attn_norm_dev = _ptr(weights[p + "attn_norm"])
+            lw.ffn_norm_dev = _ptr(weights[p + "ffn_norm"])
+            lw.wq, lw.wk, lw.wv, lw.wo = lin(p + "wq"), lin(p + "wk"), lin(p + "wv"), lin(p + "wo")
+            if getattr(cfg, "n_experts", 0):
+                lw.router_dev = _ptr(weights[p + "router"])
+            else:
+                lw.w_gate, lw.w_up, lw.w_down = lin(p + "w_gate"), lin(p + "w_up"), lin(p + "w_down")
+        self._w = _abi.xlpk_weights(_ptr(weights["embed"]), _ptr(weights["final_norm"]),
+                                    lin("lm_head"), self._layers)
+        self._kv = _abi.xlpk_kv(_ptr(k_cache), _ptr(v_cache))
+        self._refs = (weights, k_cache, v_cache)
+        h = C.c_void_p()
+        _check(lib.xlpk_create(C.byref(self._c), C.byref(self._w), C.byref(self._kv), C.byref(h)),
+               "xlpk_create")
+        self.h = h
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            lib.xlpk_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def info(self) -> _abi.xlpk_info:
+        out = _abi.xlpk_info()
+        _check(lib.xlpk_get_info(self.h, C.byref(out)), "xlpk_get_info")
+        return out
+
+    def set_state(self, tokens, seq_lens, stream=None) -> None:
+        t = (C.c_int32 * self.B)(*[int(v) for v in tokens])
+        s = (C.c_int32 * self.B)(*[int(v) for v in seq_lens])
+        _check(lib.xlpk_set_state(self.h, t, s, _stream_handle(stream)), "xlpk_set_state")
+
+    @staticmethod
+    def _io(forced=None, logits=None, hidden=None, experts=None):
+        if forced is None and logits is None and hidden is None and experts is None:
+            return None
+        return _abi.xlpk_decode_io(_ptr(forced), _ptr(logits), _ptr(hidden), _ptr(experts))
+
+    def decode(self, n_steps: int, tokens_out, forced=None, logits=None, hidden=None, experts=None,
+               stream=None, unfused: bool = False) -> None:
+        io = self._io(forced, logits, hidden, experts)
+        fn = lib.xlpk_decode_unfused if unfused else lib.xlpk_decode
+        _check(fn(self.h, int(n_steps), _ptr(tokens_out), C.byref(io) if io is not None else None,
+                  _stream_handle(stream)), "xlpk_decode_unfused" if unfused else "xlpk_decode")
+
+    def status(self) -> int:
+        return int(lib.xlpk_get_status(self.h))
+
+    def check(self) -> None:
+        _check(lib.xlpk_get_status(self.h), "device status")
+
+    def generate(self, tokens, seq_lens, n_steps: int, out_host, stream=None) -> None:
+        """End-to-end call with host buffers; `out_host` is a pinned int32 CPU tensor [n_steps][B]."""
+        t = (C.c_int32 * self.B)(*[int(v) for v in tokens])
+        s = (C.c_int32 * self.B)(*[int(v) for v in seq_lens])
+        _check(lib.xlpk_generate(self.h, t, s, int(n_steps),
+                                 C.cast(C.c_void_p(out_host.data_ptr()), C.POINTER(C.c_int32)),
+                                 _stream_handle(stream)), "xlpk_generate")

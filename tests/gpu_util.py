@@ -1,0 +1,87 @@
+"""Helpers for the GPU parity tests: run the engine through the C ABI and replay
+the same steps in the oracle (teacher-forced on the engine's emitted tokens)."""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import torch
+
+import synth
+from oracle import OracleDecoder
+from persistent_decode_b200 import workload
+
+REL_L2_BF16 = 1e-2      # hidden-state and logit relative L2 tolerance (bf16 weights)
+REL_L2_FP8 = 3e-2       # FP8 weights
+ARGMAX_MARGIN = 1e-2    # argmax must agree where the oracle's top-2 gap exceeds this
+
+
+@dataclasses.dataclass
+class Run:
+    tokens: torch.Tensor   # [n][B] int32 (host)
+    logits: torch.Tensor   # [n][B][V] fp32 (host)
+    hidden: torch.Tensor   # [n][B][H] fp32 (host)
+
+
+def run_engine(m: workload.GpuModel, n_steps: int, unfused: bool = False, keep_logits: bool = True) -> Run:
+    cfg, dev = m.cfg, m.k.device
+    B = cfg.batch
+    workload.reset_state(m)
+    tok = torch.empty(n_steps, B, dtype=torch.int32, device=dev)
+    lg = torch.empty(n_steps, B, cfg.vocab, dtype=torch.float32, device=dev) if keep_logits else None
+    hd = torch.empty(n_steps, B, cfg.hidden, dtype=torch.float32, device=dev)
+    m.engine.decode(n_steps, tok, logits=lg, hidden=hd, unfused=unfused)
+    m.engine.check()
+    return Run(tok.cpu(), lg.cpu() if lg is not None else None, hd.cpu())
+
+
+def oracle_for(m: workload.GpuModel, max_seq: Optional[int] = None) -> OracleDecoder:
+    """An oracle at the same decode start state as the engine.
+
+    Weights are the generator's tensors copied to the host.  Prompt workloads
+    are prefilled by the oracle's own full causal recompute; synthetic-KV
+    workloads get the generator's cache contents (regenerated, not read back
+    from the engine's cache).
+    """
+    cfg = m.cfg
+    w = {k: v.cpu() for k, v in m.weights.items()}
+    o = OracleDecoder(cfg, w, cfg.batch, max_seq=max_seq or m.k.shape[3])
+    if cfg.prefill:
+        o.forward_sequence(m.prompt[:, : cfg.kv_len])
+    else:
+        dev = m.k.device
+        for l in range(cfg.n_layers):
+            kl, vl = synth.make_synthetic_kv(cfg, l, device=dev)
+            o.load_kv(l, kl.cpu(), vl.cpu())
+        o.pos = [cfg.kv_len] * cfg.batch
+    return o
+
+
+def rel_l2(a: torch.Tensor, b: torch.Tensor) -> float:
+    return float((a.double() - b.double()).norm() / b.double().norm().clamp_min(1e-30))
+
+
+def compare_with_oracle(m: workload.GpuModel, run: Run, o: OracleDecoder, n_check: int,
+                        tol: float = REL_L2_BF16) -> List[dict]:
+    """Teacher-forced replay of the first n_check steps; asserts the acceptance rules."""
+    cfg = m.cfg
+    report = []
+    for s in range(n_check):
+        inp = m.start_tokens.tolist() if s == 0 else run.tokens[s - 1].tolist()
+        lg, hd = o.step(inp)
+        for b in range(cfg.batch):
+            e_h = rel_l2(run.hidden[s, b], hd[b])
+            e_l = rel_l2(run.logits[s, b], lg[b]) if run.logits is not None else 0.0
+            top2 = torch.topk(lg[b], 2)
+            margin = float(top2.values[0] - top2.values[1])
+            want = int(top2.indices[0])
+            got = int(run.tokens[s, b])
+            report.append(dict(step=s, b=b, hidden=e_h, logits=e_l, margin=margin, want=want, got=got))
+            assert e_h <= tol, f"step {s} seq {b}: hidden rel L2 {e_h:.3e} > {tol}"
+            assert e_l <= tol, f"step {s} seq {b}: logits rel L2 {e_l:.3e} > {tol}"
+            if margin > ARGMAX_MARGIN:
+                assert got == want, f"step {s} seq {b}: argmax {got} != oracle {want} (margin {margin:.3e})"
+            else:
+                # near-tie: the engine's token must be one of the oracle's top values within the margin
+                assert float(lg[b, got]) >= float(top2.values[0]) - ARGMAX_MARGIN, (s, b, got)
+    return report

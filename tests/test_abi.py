@@ -1,0 +1,81 @@
+"""The C-ABI library loads, exports every entry point include/xlpk.h declares, and
+rejects bad arguments on the host before touching a GPU.  CPU only."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from persistent_decode_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "xlpk.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(xlpk_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from persistent_decode_b200.build import build
+    build()
+    return _abi.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "xlpk_create" in names and "xlpk_decode" in names and "xlpk_decode_unfused" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(_abi.SIGNATURES), set(names) - set(_abi.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert lib.xlpk_status_string(0) == b"XLPK_OK"
+    assert lib.xlpk_status_string(-5) == b"XLPK_ERR_KV_FULL"
+    assert lib.xlpk_status_string(-6) == b"XLPK_ERR_TIMEOUT"
+    assert lib.xlpk_status_string(123) == b"XLPK_ERR_UNKNOWN"
+
+
+def _tiny_cfg(**kw):
+    c = _abi.xlpk_config(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=1024,
+                         vocab=4096, batch=1, max_seq=160, rope_theta=1e4, rms_eps=1e-5)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_host_side_argument_checks(lib):
+    h = C.c_void_p()
+    w = _abi.xlpk_weights()
+    kv = _abi.xlpk_kv()
+    assert lib.xlpk_create(None, C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_INVALID_ARG
+    # bad shapes are rejected before any CUDA call
+    for bad in (dict(n_layers=0), dict(n_q_heads=3), dict(batch=0), dict(max_seq=0), dict(vocab=1),
+                dict(weight_dtype=7), dict(rope_theta=0.0)):
+        c = _tiny_cfg(**bad)
+        assert lib.xlpk_create(C.byref(c), C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_INVALID_ARG, bad
+    for unsup in (dict(head_dim=96), dict(batch=3), dict(n_q_heads=16, n_kv_heads=2)):
+        c = _tiny_cfg(**unsup)
+        assert lib.xlpk_create(C.byref(c), C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_UNSUPPORTED, unsup
+    # a valid shape with missing weight pointers
+    c = _tiny_cfg()
+    assert lib.xlpk_create(C.byref(c), C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_INVALID_ARG
+    # calls on a NULL handle
+    assert lib.xlpk_decode(None, 1, None, None, None) == _abi.XLPK_ERR_INVALID_ARG
+    assert lib.xlpk_decode_unfused(None, 1, None, None, None) == _abi.XLPK_ERR_INVALID_ARG
+    assert lib.xlpk_get_status(None) == _abi.XLPK_ERR_INVALID_ARG
+    assert lib.xlpk_destroy(None) == _abi.XLPK_ERR_INVALID_ARG
+    info = _abi.xlpk_info()
+    assert lib.xlpk_get_info(None, C.byref(info)) == _abi.XLPK_ERR_INVALID_ARG
+
+
+def test_struct_layout_matches_header(lib):
+    # 18 four-byte fields in xlpk_config; pointer-sized members elsewhere
+    assert C.sizeof(_abi.xlpk_config) == 18 * 4
+    assert C.sizeof(_abi.xlpk_linear) == 16
+    assert C.sizeof(_abi.xlpk_layer_weights) == 8 + 4 * 16 + 8 + 3 * 16 + 8 + 6 * 16
+    assert C.sizeof(_abi.xlpk_decode_io) == 32
+    assert C.sizeof(_abi.xlpk_info) == 6 * 4 + 3 * 8

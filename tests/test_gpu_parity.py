@@ -1,0 +1,109 @@
+"""Engine vs oracle, element by element, through the C ABI on a B200."""
+import pytest
+import torch
+
+import synth
+from persistent_decode_b200 import workload
+
+from tests.gpu_util import compare_with_oracle, oracle_for, rel_l2, run_engine
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tiny(cuda_device):
+    return workload.build(synth.get_config("tiny"), device=cuda_device)
+
+
+def test_generator_device_matches_host(cuda_device):
+    w_gpu = synth.normal_bf16(0, "layers.0.wq", (256, 256), 0.02, device=cuda_device).cpu()
+    w_cpu = synth.normal_bf16(0, "layers.0.wq", (256, 256), 0.02, device="cpu")
+    assert torch.equal(w_gpu.view(torch.int16), w_cpu.view(torch.int16))
+    t_gpu = synth.uniform_tokens(1, "prompt", (1000,), 32000, device=cuda_device).cpu()
+    assert torch.equal(t_gpu, synth.uniform_tokens(1, "prompt", (1000,), 32000))
+
+
+def test_tiny_prefill_cache_matches_oracle(tiny):
+    o = oracle_for(tiny)
+    T = tiny.cfg.kv_len
+    k_gpu = tiny.k[:, :, :, :T].float().cpu()
+    v_gpu = tiny.v[:, :, :, :T].float().cpu()
+    assert rel_l2(k_gpu, o.K[:, :, :, :T].float()) < 1e-2
+    assert rel_l2(v_gpu, o.V[:, :, :, :T].float()) < 1e-2
+    # positions beyond the prompt were never written
+    assert int(tiny.k[:, :, :, T:].abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("unfused", [False, True], ids=["persistent", "kernel_per_op"])
+def test_tiny_decode_matches_oracle(tiny, unfused):
+    run = run_engine(tiny, tiny.cfg.steps, unfused=unfused)
+    o = oracle_for(tiny)
+    compare_with_oracle(tiny, run, o, tiny.cfg.steps)
+
+
+def test_tiny_persistent_equals_kernel_per_op_bitwise(tiny):
+    a = run_engine(tiny, tiny.cfg.steps, unfused=False)
+    b = run_engine(tiny, tiny.cfg.steps, unfused=True)
+    assert torch.equal(a.tokens, b.tokens)
+    assert torch.equal(a.logits, b.logits)
+    assert torch.equal(a.hidden, b.hidden)
+
+
+def test_tiny_decode_is_deterministic_and_resumable(tiny):
+    a = run_engine(tiny, 16)
+    # the same 16 steps as two calls of 8 (state carried in the handle)
+    workload.reset_state(tiny)
+    dev = tiny.k.device
+    t1 = torch.empty(8, 1, dtype=torch.int32, device=dev)
+    t2 = torch.empty(8, 1, dtype=torch.int32, device=dev)
+    tiny.engine.decode(8, t1)
+    tiny.engine.decode(8, t2)
+    tiny.engine.check()
+    assert torch.equal(torch.cat([t1, t2]).cpu(), a.tokens)
+
+
+def test_tiny_kv_append_positions_exact(tiny):
+    cfg = tiny.cfg
+    T, n = cfg.kv_len, cfg.steps
+    before = tiny.k[:, :, :, :T].clone()
+    run = run_engine(tiny, n)
+    # the prompt's entries are untouched, each step wrote exactly its position
+    assert torch.equal(tiny.k[:, :, :, :T], before)
+    written = tiny.k[:, :, :, T:T + n].float().abs().sum(dim=-1)
+    assert bool((written > 0).all())
+    o = oracle_for(tiny)
+    compare_with_oracle(tiny, run, o, n)
+    assert rel_l2(tiny.k[:, :, :, T:T + n].float().cpu(), o.K[:, :, :, T:T + n].float()) < 1e-2
+    assert rel_l2(tiny.v[:, :, :, T:T + n].float().cpu(), o.V[:, :, :, T:T + n].float()) < 1e-2
+
+
+@pytest.mark.parametrize("batch", [2, 4])
+def test_tiny_batched_with_gains(cuda_device, batch):
+    cfg = synth.get_config("tiny", batch=batch, steps=12)
+    m = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    run = run_engine(m, cfg.steps)
+    compare_with_oracle(m, run, oracle_for(m), cfg.steps)
+
+
+def test_tiny_ragged_grid(cuda_device):
+    # a grid size that divides nothing evenly: every stage gets ragged CTA spans
+    cfg = synth.get_config("tiny", steps=6)
+    m = workload.build(cfg, device=cuda_device, n_ctas=37)
+    run = run_engine(m, cfg.steps)
+    compare_with_oracle(m, run, oracle_for(m), cfg.steps)
+
+
+def test_generate_with_host_buffers(tiny):
+    ref = run_engine(tiny, 8)
+    out = torch.empty(8, 1, dtype=torch.int32).pin_memory()
+    tiny.engine.generate(tiny.start_tokens.tolist(), [tiny.cfg.kv_len], 8, out)
+    assert torch.equal(out, ref.tokens)
+
+
+def test_kv_full_is_rejected(tiny):
+    from persistent_decode_b200 import XlpkError
+    workload.reset_state(tiny)
+    tok = torch.empty(tiny.cfg.steps + 1, 1, dtype=torch.int32, device=tiny.k.device)
+    with pytest.raises(XlpkError) as e:
+        tiny.engine.decode(tiny.cfg.steps + 1, tok)
+    assert e.value.status == -5
