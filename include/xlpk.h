@@ -126,6 +126,12 @@ typedef struct xlpk_decode_io {
   float* logits_dev;                  /* [n_steps][B][V] fp32 logits of every step */
   float* hidden_dev;                  /* [n_steps][B][H] fp32 residual after the last layer */
   int32_t* experts_dev;               /* MoE: [n_steps][L][B][top_k] selected expert ids */
+  uint64_t* trace_dev;                /* [n_steps][n_stages][n_ctas][8] globaltimer stamps (ns) per
+                                         stage and CTA: consumer entry, dependency met, activation
+                                         staged, consumer done, producer first copy, producer last
+                                         copy; attention stages also record the total ns spent
+                                         waiting for KV chunks [6] and merging partials [7];
+                                         n_stages = 5 * n_layers + 1 */
 } xlpk_decode_io;
 
 /* Facts about a created handle (for measurement and tests). */

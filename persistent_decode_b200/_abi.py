@@ -52,7 +52,7 @@ class xlpk_kv(C.Structure):
 
 class xlpk_decode_io(C.Structure):
     _fields_ = [("forced_tokens_dev", C.c_void_p), ("logits_dev", C.c_void_p),
-                ("hidden_dev", C.c_void_p), ("experts_dev", C.c_void_p)]
+                ("hidden_dev", C.c_void_p), ("experts_dev", C.c_void_p), ("trace_dev", C.c_void_p)]
 
 
 class xlpk_info(C.Structure):

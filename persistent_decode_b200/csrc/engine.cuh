@@ -65,6 +65,100 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread is parked by the hardware
+// until the phase completes or about `ns` nanoseconds pass, instead of
+// re-issuing the test (which would steal issue slots from the warps that
+// share its scheduler).
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Explicit shared-state-space loads.  The stage bodies are separate
+// (non-inlined) functions, where the compiler cannot prove that a pointer into
+// the ring or the activation buffer addresses shared memory; generic loads
+// would take the slower L1TEX path.  Volatile: ring slots are rewritten by
+// bulk copies between mbarrier phases.
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_u2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u1(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a));
+  return v;
+}
+// 2-D tiled TMA load (box of the tensor map at column x, row y) into this
+// CTA's shared memory, completing its bytes on `bar`.  x * 2 bytes is a
+// multiple of 16 (x is 0 or 64).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+// D += A * B for one 16x8x16 tile: bf16 operands, fp32 accumulate (warp-wide).
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+      " {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// Two-term bf16 split of an fp32 pair: x = hi + lo with hi = bf16(x) and
+// lo = bf16(x - hi), so hi*k + lo*k carries ~16 significant bits of x into a
+// bf16 tensor-core product with an exact bf16 k (K and V entries).
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+// Shared address of element (row r, dim d) of a K or V chunk of P rows as the
+// 128-byte-swizzled TMA boxes lay it out: box d/64 holds [P][64 dims]; the
+// 16-byte unit u of row r sits at unit u ^ (r % 8).
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int P, int r, int d) {
+  return base + (d >> 6) * (P * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4) + ((d & 7) << 1);
+}
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -131,6 +225,7 @@ __device__ __forceinline__ int split_owner(int i, int n, int G) {
 struct alignas(16) SmemCtl {
   uint64_t full[kMaxSlots];
   uint64_t empty[kMaxSlots];
+  uint64_t act_bar;      // completion of the activation bulk copy
   volatile int abort;
   int flag;
   int pad[2];
@@ -158,6 +253,7 @@ struct Ctx {
   int warp;
   int lane;
   int tid;
+  uint32_t act_phase;   // parity of the next activation-copy phase (consumers)
 };
 
 enum ErrCode : int { kErrNone = 0, kErrTimeout = -6, kErrAborted = -7 };
@@ -174,24 +270,33 @@ __device__ __forceinline__ int where_code(int kind, int layer, int step) {
   return (step << 16) | ((layer & 0xff) << 8) | (kind & 0xff);
 }
 
+// Optional stage trace: stamp k of (step s, stage index si) for this CTA.
+__device__ __forceinline__ void trace_stamp(const Params& p, int s, int si, int k) {
+  if (p.trace) {
+    const size_t n_st = static_cast<size_t>(p.L) * ST_LAYER + 1;
+    p.trace[((static_cast<size_t>(s) * n_st + si) * p.G + blockIdx.x) * 8 + k] = globaltimer();
+  }
+}
+__device__ __forceinline__ int stage_index(const Params& p, int kind, int l) {
+  return kind == ST_LM ? p.L * ST_LAYER : l * ST_LAYER + kind;
+}
+
 // Bounded wait on a ring barrier phase.  Returns false (and marks the CTA
 // aborted) if the global abort flag is raised or the time limit passes.
 __device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint32_t bar,
                                             uint32_t parity, int where) {
   const uint64_t t0 = globaltimer();
-  for (unsigned it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
     if (ctl->abort) return false;
-    if ((it & 31u) == 0) {
-      if (ld_volatile(p.abort_flag)) {
-        ctl->abort = 1;
-        return false;
-      }
-      if (static_cast<long long>(globaltimer() - t0) > p.spin_limit_ns) {
-        raise_error(p, kErrTimeout, where);
-        ctl->abort = 1;
-        return false;
-      }
+    if (ld_volatile(p.abort_flag)) {
+      ctl->abort = 1;
+      return false;
+    }
+    if (static_cast<long long>(globaltimer() - t0) > p.spin_limit_ns) {
+      raise_error(p, kErrTimeout, where);
+      ctl->abort = 1;
+      return false;
     }
   }
 }
@@ -206,7 +311,10 @@ __device__ __forceinline__ bool ring_wait(const Params& p, SmemCtl* ctl, uint32_
 __device__ __noinline__ bool counter_wait_slow(const Params& p, SmemCtl* ctl, const unsigned* cnt,
                                                unsigned target, int where) {
   const uint64_t t0 = globaltimer();
+  unsigned nap = 16;
   for (unsigned it = 1;; ++it) {
+    __nanosleep(nap);               // back off: each poll is an L2 round trip
+    if (nap < 128) nap <<= 1;
     if (static_cast<int>(ld_acquire(cnt) - target) >= 0) return true;
     if (ctl->abort) return false;
     if ((it & 15u) == 0) {
@@ -232,8 +340,11 @@ __device__ __forceinline__ bool counter_wait(const Params& p, SmemCtl* ctl, cons
 // Consumers: thread 0 waits, everyone learns the outcome.  Returns false if aborted.
 __device__ __forceinline__ bool stage_wait(const Params& p, Ctx& cx, const unsigned* cnt,
                                            unsigned target, int where, bool fused) {
-  if (fused && cx.tid == 0) {
-    if (!counter_wait(p, cx.ctl, cnt, target, where)) cx.ctl->abort = 1;
+  if (cx.tid == 0) {
+    const int s = where >> 16, kind = where & 0xff, l = (where >> 8) & 0xff;
+    trace_stamp(p, s, stage_index(p, kind, l), 0);
+    if (fused && !counter_wait(p, cx.ctl, cnt, target, where)) cx.ctl->abort = 1;
+    trace_stamp(p, s, stage_index(p, kind, l), 1);
   }
   consumer_sync();
   return !cx.ctl->abort;
@@ -277,65 +388,108 @@ __device__ __forceinline__ void argmax_merge(float& v, int& i, float v2, int i2)
 
 // ------------------------------------------------------------------ activations
 
-// Activation vector [B][K] staged in shared memory as two fp32 planes so that
-// lane-consecutive 16-byte reads of 8-element weight vectors are conflict-free:
-//   plane 0: float4 [B][K/8] = elements 8v..8v+3,  plane 1: elements 8v+4..8v+7.
-__device__ __forceinline__ int act_index(int b, int k, int B, int nvK) {
-  const int v = k >> 3, e = k & 7;
-  return ((((e >> 2) * B + b) * nvK + v) << 2) + (e & 3);
+// Activation vectors [B][K] (the residual x, the attention output o, the
+// SwiGLU output h) are kept in global memory and in shared memory in the same
+// "two-plane" fp32 layout, so a stage's input moves as ONE bulk copy and
+// lane-consecutive 16-byte reads of 8-element weight vectors are
+// conflict-free:  plane 0 holds float4 [B][K/8] = elements 8v..8v+3,
+// plane 1 holds elements 8v+4..8v+7.
+__host__ __device__ __forceinline__ size_t plane_index(int b, int k, int B, int K) {
+  return ((static_cast<size_t>((k >> 2) & 1) * B + b) * (K >> 3) + (k >> 3)) * 4 + (k & 3);
 }
 
 enum ActSrc : int { SRC_RESID = 0, SRC_EMBED = 1, SRC_PLAIN = 2 };
 
-// Load the stage input into shared memory.  With `gain`, apply RMSNorm:
-// v * rsqrt(mean(v^2) + eps) * gain.  `hidden_dbg` (LM stage, CTA 0) receives
-// the raw residual.
+// Stage the input vector in shared memory.  A residual / plain source (two-plane
+// layout in global memory, written by other CTAs in an earlier stage) arrives
+// as one bulk copy issued right after the dependency wait; the embedding row
+// of layer 0 (bf16) is converted by the threads.  With `gain`, RMSNorm is
+// applied in place: v * rsqrt(mean(v^2) + eps) * gain.  `hidden_dbg` (LM
+// stage, CTA 0) receives the raw residual in natural [B][K] order.
 template <int B>
-__device__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const float* gsrc,
-                         const float* gain, float* hidden_dbg) {
+__device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const float* gsrc,
+                                      const float* gain, float* hidden_dbg, int where) {
   const int nvK = K >> 3;
-  float ss[B];
-  int tok[B];
+  const int n4 = K >> 2;
+  float4* act4 = reinterpret_cast<float4*>(cx.act);
+  if (src == SRC_EMBED) {
+    int tok[B];
 #pragma unroll
-  for (int b = 0; b < B; ++b) {
-    ss[b] = 0.f;
-    tok[b] = (src == SRC_EMBED) ? __ldcg(p.cur_tok + b) : 0;
-  }
-  for (int k = cx.tid; k < K; k += kConsumerThreads) {
+    for (int b = 0; b < B; ++b) tok[b] = __ldcg(p.cur_tok + b);
+    for (int q0 = cx.tid; q0 < n4; q0 += kConsumerThreads * 4) {
+      uint2 e[4][B];
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
-      float v;
-      if (src == SRC_EMBED) {
-        v = __uint_as_float(static_cast<uint32_t>(p.embed[static_cast<size_t>(tok[b]) * K + k]) << 16);
-      } else {
-        v = __ldcg(gsrc + static_cast<size_t>(b) * K + k);
-      }
-      if (hidden_dbg) hidden_dbg[static_cast<size_t>(b) * K + k] = v;
-      ss[b] = fmaf(v, v, ss[b]);
-      cx.act[act_index(b, k, B, nvK)] = v;
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int q = q0 + u * kConsumerThreads;
+          if (q < n4) e[u][b] = __ldg(reinterpret_cast<const uint2*>(p.embed + static_cast<size_t>(tok[b]) * K) + q);
+        }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int q = q0 + u * kConsumerThreads;
+          if (q < n4)
+            act4[((q & 1) * B + b) * nvK + (q >> 1)] =
+                make_float4(bf16_lo(e[u][b].x), bf16_hi(e[u][b].x), bf16_lo(e[u][b].y), bf16_hi(e[u][b].y));
+        }
     }
+  } else {
+    const uint32_t bar = smem_addr(&cx.ctl->act_bar);
+    if (gain) {   // warm this SM's L1 with the gains while the copy is in flight
+      for (int q = cx.tid; q < n4; q += kConsumerThreads)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(gain + 4 * q));
+    }
+    if (cx.tid == 0) {
+      // order the other CTAs' global writes (acquired) and this CTA's earlier
+      // shared-memory accesses before the async-proxy copy
+      asm volatile("fence.proxy.async;" ::: "memory");
+      const uint32_t bytes = static_cast<uint32_t>(B) * K * 4u;
+      mbar_expect_tx(bar, bytes);
+      bulk_g2s_nohint(smem_addr(cx.act), gsrc, bytes, bar);
+    }
+    if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+    cx.act_phase ^= 1u;
+  }
+  if (hidden_dbg) {
+    if (src == SRC_EMBED) consumer_sync();
+    for (int k = cx.tid; k < K; k += kConsumerThreads)
+#pragma unroll
+      for (int b = 0; b < B; ++b) hidden_dbg[static_cast<size_t>(b) * K + k] = cx.act[plane_index(b, k, B, K)];
   }
   if (gain) {
+    if (src == SRC_EMBED) consumer_sync();
+    float ss[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) ss[b] = 0.f;
+    for (int q = cx.tid; q < n4; q += kConsumerThreads)
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float4 x = act4[((q & 1) * B + b) * nvK + (q >> 1)];
+        ss[b] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ss[b]))));
+      }
 #pragma unroll
     for (int b = 0; b < B; ++b) {
-      const float s = warp_sum(ss[b]);
-      if (cx.lane == 0) cx.ctl->red[cx.warp][b] = s;
+      const float t = warp_sum(ss[b]);
+      if (cx.lane == 0) cx.ctl->red[cx.warp][b] = t;
     }
     consumer_sync();
     float r[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) {
-      float s = 0.f;
+      float t = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) s += cx.ctl->red[w][b];
-      r[b] = rsqrtf(s / static_cast<float>(K) + p.eps);
+      for (int w = 0; w < kConsumerWarps; ++w) t += cx.ctl->red[w][b];
+      r[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
     }
-    for (int k = cx.tid; k < K; k += kConsumerThreads) {
-      const float g = __ldg(gain + k);
+    for (int q = cx.tid; q < n4; q += kConsumerThreads) {
+      const float4 g4 = __ldg(reinterpret_cast<const float4*>(gain) + q);
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        float& a = cx.act[act_index(b, k, B, nvK)];
-        a = a * r[b] * g;
+        float4& a = act4[((q & 1) * B + b) * nvK + (q >> 1)];
+        const float rb = r[b];
+        a = make_float4(a.x * rb * g4.x, a.y * rb * g4.y, a.z * rb * g4.z, a.w * rb * g4.w);
       }
     }
   }
@@ -344,42 +498,19 @@ __device__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const floa
 
 // ------------------------------------------------------------------ GEMV stages
 
-// Producer side of one GEMV stage: the CTA's span, tile by tile.
-__device__ bool produce_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, uint64_t pol,
-                             int where) {
-  const int NP = m.N >> 1;
-  const int p0 = split_point(cx.c, NP, p.G), p1 = split_point(cx.c + 1, NP, p.G);
-  const int nkc = m.K / m.KC;
-  const uint8_t* src = m.packed + static_cast<size_t>(2) * p0 * m.K * p.esz;
-  for (int g0 = p0; g0 < p1; g0 += kPairsPerTile) {
-    const int gp = min(kPairsPerTile, p1 - g0);
-    const uint32_t bytes = 2u * gp * m.KC * p.esz;
-    for (int kc = 0; kc < nkc; ++kc) {
-      const uint32_t eb = smem_addr(&cx.ctl->empty[rp.slot]);
-      if (!ring_wait(p, cx.ctl, eb, rp.phase ^ 1u, where)) return false;
-      const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
-      mbar_expect_tx(fb, bytes);
-      bulk_g2s(smem_addr(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes), src, bytes, fb, pol);
-      src += bytes;
-      rp.next(p.nslot);
-    }
-  }
-  return true;
-}
-
 // Consumer side: each warp owns one row pair of every tile of a group and
 // accumulates it over the group's k-chunks; `epi(pair, acc0, acc1)` runs on
 // the reduced sums (identical in every lane).
 template <int B, class Epi>
-__device__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where,
-                             Epi& epi) {
+__device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp,
+                                          int where, Epi& epi) {
   const int NP = m.N >> 1;
   const int p0 = split_point(cx.c, NP, p.G), p1 = split_point(cx.c + 1, NP, p.G);
   const int nkc = m.K / m.KC;
   const int nv = m.KC >> 3;   // 16-byte vectors per row chunk
   const int nvK = m.K >> 3;
-  const float4* act_lo = reinterpret_cast<const float4*>(cx.act);
-  const float4* act_hi = act_lo + B * nvK;
+  const uint32_t act_lo_s = smem_addr(cx.act);
+  const uint32_t act_hi_s = act_lo_s + B * nvK * 16;
   for (int g0 = p0; g0 < p1; g0 += kPairsPerTile) {
     const int gp = min(kPairsPerTile, p1 - g0);
     float a0[B], a1[B];
@@ -389,19 +520,18 @@ __device__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp
       const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
       const bool ok = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
       if (ok && cx.warp < gp) {
-        const uint4* r0 =
-            reinterpret_cast<const uint4*>(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes) +
-            (2 * cx.warp) * nv;
-        const uint4* r1 = r0 + nv;
-        const int vb = kc * nv;
+        const uint32_t r0 = smem_addr(cx.ring) + rp.slot * kSlotBytes + (2 * cx.warp) * nv * 16;
+        const uint32_t r1 = r0 + nv * 16;
+        const uint32_t alo = act_lo_s + (kc * nv) * 16;
+        const uint32_t ahi = act_hi_s + (kc * nv) * 16;
 #pragma unroll 4
         for (int v = cx.lane; v < nv; v += 32) {
-          const uint4 w0 = r0[v];
-          const uint4 w1 = r1[v];
+          const uint4 w0 = lds_u4(r0 + v * 16);
+          const uint4 w1 = lds_u4(r1 + v * 16);
 #pragma unroll
           for (int b = 0; b < B; ++b) {
-            const float4 lo = act_lo[b * nvK + vb + v];
-            const float4 hi = act_hi[b * nvK + vb + v];
+            const float4 lo = lds_f4(alo + (b * nvK + v) * 16);
+            const float4 hi = lds_f4(ahi + (b * nvK + v) * 16);
             a0[b] = dot8_bf16(w0, lo, hi, a0[b]);
             a1[b] = dot8_bf16(w1, lo, hi, a1[b]);
           }
@@ -473,7 +603,7 @@ struct EpiResid {
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       if (lane != b) continue;
-      float2* xp = reinterpret_cast<float2*>(p.x + static_cast<size_t>(b) * p.H) + pg;
+      float2* xp = reinterpret_cast<float2*>(p.x + plane_index(b, 2 * pg, p.B, p.H));
       float2 base;
       if (from_embed) {
         const int tok = __ldcg(p.cur_tok + b);
@@ -496,7 +626,7 @@ struct EpiSwiGLU {
     for (int b = 0; b < B; ++b) {
       if (lane != b) continue;
       const float g = a0[b];
-      p.h[static_cast<size_t>(b) * p.F + pg] = g / (1.f + expf(-g)) * a1[b];
+      p.h[plane_index(b, pg, p.B, p.F)] = g / (1.f + expf(-g)) * a1[b];
     }
   }
 };
@@ -526,16 +656,21 @@ struct EpiLM {
 
 // ------------------------------------------------------------------ attention
 
+// The attention work of one step: items (b, g, chunk j) in that order, chunk j
+// covering positions [j*P, (j+1)*P) of sequence b's T = pos0[b] + s + 1.
+template <int B>
 struct AttnPlan {
-  int nch[kMaxBatch];
-  int base[kMaxBatch];
+  int nch[B];
+  int base[B];
   int W;
 };
 
-__device__ __forceinline__ void attn_plan(const Params& p, int s, AttnPlan& ap) {
+template <int B>
+__device__ __forceinline__ void attn_plan(const Params& p, int s, AttnPlan<B>& ap) {
   const int P = p.attn_pos_per_tile;
   int w = 0;
-  for (int b = 0; b < p.B; ++b) {
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
     const int T = p.pos0[b] + s + 1;
     ap.nch[b] = (T + P - 1) / P;
     ap.base[b] = w;
@@ -544,274 +679,244 @@ __device__ __forceinline__ void attn_plan(const Params& p, int s, AttnPlan& ap) 
   ap.W = w;
 }
 
-__device__ __forceinline__ void attn_item(const Params& p, const AttnPlan& ap, int i, int& b, int& g,
-                                          int& j) {
+template <int B>
+__device__ __forceinline__ void attn_item(const Params& p, const AttnPlan<B>& ap, int i, int& b,
+                                          int& g, int& j, int& nch, int& base) {
   b = 0;
-  while (b + 1 < p.B && ap.base[b + 1] <= i) ++b;
-  const int r = i - ap.base[b];
-  g = r / ap.nch[b];
-  j = r - g * ap.nch[b];
+  nch = ap.nch[0];
+  base = ap.base[0];
+#pragma unroll
+  for (int bb = 1; bb < B; ++bb)
+    if (ap.base[bb] <= i) {
+      b = bb;
+      nch = ap.nch[bb];
+      base = ap.base[bb];
+    }
+  const int r = i - base;
+  g = r / nch;
+  j = r - g * nch;
 }
 
 __device__ __forceinline__ size_t kv_row(const Params& p, int l, int b, int g, int t) {
   return (((static_cast<size_t>(l) * p.B + b) * p.nkv + g) * p.max_seq + t) * p.d;
 }
 
-__device__ bool produce_attn(const Params& p, Ctx& cx, int l, int s, RingPos& rp, uint64_t pol,
-                             bool fused) {
-  AttnPlan ap;
-  attn_plan(p, s, ap);
-  const int i0 = split_point(cx.c, ap.W, p.G), i1 = split_point(cx.c + 1, ap.W, p.G);
-  if (i0 >= i1) return true;
-  const int where = where_code(ST_ATTN, l, s) | (1 << 15);
-  // Cache rows up to pos-1 were written by this layer's QKV stage of earlier
-  // steps (or before the launch).  Make sure the previous step's write is done
-  // before reading it through the async proxy.
-  if (fused) {
-    const unsigned target = static_cast<unsigned>(p.G) * static_cast<unsigned>(p.step_base + s);
-    if (!counter_wait(p, cx.ctl, p.cnt + l * ST_LAYER + ST_QKV, target, where)) return false;
-  }
-  fence_proxy_async_global();
-  const int P = p.attn_pos_per_tile;
-  const uint32_t vhalf = kSlotBytes / 2;
-  for (int i = i0; i < i1; ++i) {
-    int b, g, j;
-    attn_item(p, ap, i, b, g, j);
-    const int T = p.pos0[b] + s + 1;
-    const int t_lo = j * P;
-    const int n_old = min(t_lo + P, T - 1) - t_lo;
-    if (n_old <= 0) continue;
-    const uint32_t bytes = static_cast<uint32_t>(n_old) * p.d * 2u;
-    const uint32_t eb = smem_addr(&cx.ctl->empty[rp.slot]);
-    if (!ring_wait(p, cx.ctl, eb, rp.phase ^ 1u, where)) return false;
-    const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
-    mbar_expect_tx(fb, 2u * bytes);
-    const uint32_t dst = smem_addr(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes);
-    const size_t off = kv_row(p, l, b, g, t_lo);
-    bulk_g2s(dst, p.kc + off, bytes, fb, pol);
-    bulk_g2s(dst + vhalf, p.vc + off, bytes, fb, pol);
-    rp.next(p.nslot);
-  }
-  return true;
+// Attention scratch in the activation region (the attention stage stages no
+// activation vector).  Sizes are in floats.
+__host__ __device__ constexpr int attn_scratch_floats(int D, int G) {
+  return kConsumerWarps * 16 * kMaxGroup        // p of each warp's positions
+         + kConsumerWarps * kMaxGroup * 2       // per-warp (m, l)
+         + kConsumerWarps * kMaxGroup * D       // per-warp o
+         + 3 * G * kMaxGroup + 2 * kMaxGroup;   // combine: (M, L, weight) per contributor, M*, L*
 }
 
-// Flash-decoding over this CTA's chunks.  Lanes: grp = lane>>3 picks one of
-// 4 positions per warp-round, li = lane&7 owns D/8 of its dims for q.k;
-// for p.V each lane owns D/32 consecutive dims.
+// Flash-decoding over this CTA's chunks of the (sequence, kv head) space on
+// warp-level tensor cores.  A chunk is P = 64 (d=128) or 128 (d=64) positions
+// whose K and V rows arrive as 128-byte-swizzled TMA boxes.  Warp w takes the
+// 16 positions of group pg = w % (P/16) and, for p.V, the dims of half
+// ds = w / (P/16) (d=128) or all of them (d=64).  The GQA group's query heads
+// fill rows 0..3 of the m16n8k16 A operand, so S = Q K^T for 16 positions is
+// 2 n-tiles x d/16 k-steps of mma, the scores stay in the accumulator
+// registers for a warp-level online softmax (one row max / sum per head over
+// the 16 positions: 2 shuffles each), and P is reused in registers as the A
+// operand of O += P V (the accumulator-to-A register reuse of FlashAttention-2).
+// The new token's K/V row (written by this step's QKV stage) is patched into
+// the chunk in shared memory.
 template <int B, int D>
-__device__ void consume_attn(const Params& p, Ctx& cx, int l, int s, RingPos& rp, bool fused) {
-  constexpr int NCH = D / 64;   // 8-dim chunks per lane for q.k
-  constexpr int DV = D / 32;    // dims per lane for p.V
-  AttnPlan ap;
-  attn_plan(p, s, ap);
+__device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s, RingPos& rp,
+                                         bool fused) {
+  static_assert(kMaxGroup == 4, "query heads per kv head fill at most rows 0..3 of the A tile");
+  constexpr int P = (kSlotBytes / 2) / (D * 2);               // positions per chunk
+  constexpr int NPG = P / 16;                                 // position groups per chunk
+  constexpr int NDS = kConsumerWarps / NPG;                   // p.V dim splits
+  constexpr int DW = D / NDS;                                 // p.V dims per warp
+  constexpr int NT = DW / 8;                                  // p.V n-tiles per warp
+  constexpr int KS = D / 16;                                  // q.k k-steps
+  constexpr int DV = D / 32;                                  // new-row dims per lane
+  static_assert(NPG * NDS == kConsumerWarps && NT % 2 == 0, "chunk shape");
+  AttnPlan<B> ap;
+  attn_plan<B>(p, s, ap);
   const int i0 = split_point(cx.c, ap.W, p.G), i1 = split_point(cx.c + 1, ap.W, p.G);
   const int where = where_code(ST_ATTN, l, s);
   const unsigned S1 = static_cast<unsigned>(p.step_base + s + 1);
   if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_QKV, static_cast<unsigned>(p.G) * S1, where, fused))
     return;
+  if (cx.tid == 0) trace_stamp(p, s, stage_index(p, ST_ATTN, l), 2);
   if (i0 >= i1) return;
-  const int P = p.attn_pos_per_tile;
   const int GQ = p.group;
-  const int grp = cx.lane >> 3, li = cx.lane & 7;
-  float* sm_ml = cx.act;                                       // [8][kMaxGroup][2]
-  float* sm_o = cx.act + kConsumerWarps * kMaxGroup * 2;       // [8][kMaxGroup][D]
+  const int pg = cx.warp % NPG, ds = cx.warp / NPG;
+  const int gid = cx.lane >> 2, tig = cx.lane & 3;
+  const int mi = cx.lane >> 3, rr = cx.lane & 7;             // ldmatrix: matrix / row of this lane
+  float* sm_ml = cx.act;                                      // [8 warps][4 heads][2]
+  float* sm_o = sm_ml + kConsumerWarps * kMaxGroup * 2;       // [8 warps][4 heads][DW]
+  float* cb = sm_o + kConsumerWarps * kMaxGroup * DW;         // combine scratch
+  const uint32_t ring_s = smem_addr(cx.ring);
 
-  float qr[kMaxGroup][NCH * 8];
-  float m[kMaxGroup], ls[kMaxGroup], oa[kMaxGroup][DV];
-  int seg_b = -1, seg_g = -1, seg_first = 0, seg_items = 0;
+  uint32_t qa0[KS], qa2[KS], qb0[KS], qb2[KS];   // q as bf16 hi (a) + lo (b) parts
+  float o[NT][4];
+  float m_h = -INFINITY, l_h = 0.f;                          // softmax state of head gid
+  int seg_b = -1, seg_g = -1, seg_items = 0, seg_nch = 0, seg_base = 0;
+  unsigned long long t_wait = 0, t_merge = 0;                 // trace only (thread 0)
 
   for (int i = i0; i < i1; ++i) {
-    int b, g, j;
-    attn_item(p, ap, i, b, g, j);
+    int b, g, j, nch, base;
+    attn_item<B>(p, ap, i, b, g, j, nch, base);
     if (b != seg_b || g != seg_g) {
       seg_b = b;
       seg_g = g;
-      seg_first = i;
       seg_items = 0;
+      seg_nch = nch;
+      seg_base = base;
+      m_h = -INFINITY;
+      l_h = 0.f;
 #pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        m[h] = -INFINITY;
-        ls[h] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+      if (gid < GQ) {
+        const float* qs = p.q + (static_cast<size_t>(b) * p.nq + g * GQ + gid) * D;
+        const float sc = p.qk_scale_log2;
 #pragma unroll
-        for (int e = 0; e < DV; ++e) oa[h][e] = 0.f;
-        if (h < GQ) {
-          const float* qs = p.q + (static_cast<size_t>(b) * p.nq + g * GQ + h) * D;
-#pragma unroll
-          for (int ch = 0; ch < NCH; ++ch) {
-            const float4 u = __ldcg(reinterpret_cast<const float4*>(qs + ch * 64 + li * 8));
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(qs + ch * 64 + li * 8 + 4));
-            qr[h][ch * 8 + 0] = u.x * p.qk_scale_log2;
-            qr[h][ch * 8 + 1] = u.y * p.qk_scale_log2;
-            qr[h][ch * 8 + 2] = u.z * p.qk_scale_log2;
-            qr[h][ch * 8 + 3] = u.w * p.qk_scale_log2;
-            qr[h][ch * 8 + 4] = v.x * p.qk_scale_log2;
-            qr[h][ch * 8 + 5] = v.y * p.qk_scale_log2;
-            qr[h][ch * 8 + 6] = v.z * p.qk_scale_log2;
-            qr[h][ch * 8 + 7] = v.w * p.qk_scale_log2;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < NCH * 8; ++e) qr[h][e] = 0.f;
+        for (int ks = 0; ks < KS; ++ks) {
+          const float2 u = __ldcg(reinterpret_cast<const float2*>(qs + ks * 16 + tig * 2));
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(qs + ks * 16 + 8 + tig * 2));
+          split_bf16x2(u.x * sc, u.y * sc, qa0[ks], qb0[ks]);
+          split_bf16x2(v.x * sc, v.y * sc, qa2[ks], qb2[ks]);
         }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) qa0[ks] = qa2[ks] = qb0[ks] = qb2[ks] = 0u;
       }
     }
     ++seg_items;
     const int T = p.pos0[b] + s + 1;
     const int t_lo = j * P;
-    const int npos = min(t_lo + P, T) - t_lo;
-    const int n_old = min(t_lo + P, T - 1) - t_lo;
-    const uint16_t* sK = nullptr;
-    const uint16_t* sV = nullptr;
-    bool have_tile = false;
-    if (n_old > 0) {
-      const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
-      have_tile = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
-      sK = reinterpret_cast<const uint16_t*>(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes);
-      sV = sK + kSlotBytes / 4;
-    }
-    const uint16_t* gK = p.kc + kv_row(p, l, b, g, T - 1);
-    const uint16_t* gV = p.vc + kv_row(p, l, b, g, T - 1);
-    for (int r0 = 0; r0 < npos; r0 += 4 * kConsumerWarps) {
-      const int r = r0 + cx.warp * 4 + grp;
-      const bool valid = r < npos && (r >= n_old || have_tile);
-      // q . k for this lane group's position
-      float sc[kMaxGroup];
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) sc[h] = 0.f;
-      if (valid) {
-        const uint16_t* krow = (r < n_old) ? sK + static_cast<size_t>(r) * D : gK;
-#pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) {
-          uint4 kv;
-          if (r < n_old) {
-            kv = *reinterpret_cast<const uint4*>(krow + ch * 64 + li * 8);
-          } else {
-            kv = __ldcg(reinterpret_cast<const uint4*>(krow + ch * 64 + li * 8));
-          }
-          const float k0 = bf16_lo(kv.x), k1 = bf16_hi(kv.x), k2 = bf16_lo(kv.y), k3 = bf16_hi(kv.y);
-          const float k4 = bf16_lo(kv.z), k5 = bf16_hi(kv.z), k6 = bf16_lo(kv.w), k7 = bf16_hi(kv.w);
-#pragma unroll
-          for (int h = 0; h < kMaxGroup; ++h) {
-            float a = sc[h];
-            a = fmaf(qr[h][ch * 8 + 0], k0, a);
-            a = fmaf(qr[h][ch * 8 + 1], k1, a);
-            a = fmaf(qr[h][ch * 8 + 2], k2, a);
-            a = fmaf(qr[h][ch * 8 + 3], k3, a);
-            a = fmaf(qr[h][ch * 8 + 4], k4, a);
-            a = fmaf(qr[h][ch * 8 + 5], k5, a);
-            a = fmaf(qr[h][ch * 8 + 6], k6, a);
-            a = fmaf(qr[h][ch * 8 + 7], k7, a);
-            sc[h] = a;
-          }
+    const int npos = min(t_lo + P, T) - t_lo;      // positions of this chunk (incl. the new token)
+    const int n_old = min(t_lo + P, T - 1) - t_lo; // positions already in the cache before this step
+    const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
+    const unsigned long long tw0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+    const bool have_tile = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
+    if (p.trace && cx.tid == 0) t_wait += globaltimer() - tw0;
+    const uint32_t kt = ring_s + rp.slot * kSlotBytes;
+    const uint32_t vt = kt + kSlotBytes / 2;
+    if (have_tile && pg * 16 < npos) {   // warp-uniform
+      if (npos > n_old && (n_old >> 4) == pg) {
+        // this step's K/V entry of the head, from the cache (written by the QKV stage)
+        const size_t row = kv_row(p, l, b, g, T - 1);
+        const uint32_t ka = sw128_addr(kt, P, n_old, cx.lane * DV);
+        const uint32_t va = sw128_addr(vt, P, n_old, cx.lane * DV);
+        if (DV == 4) {
+          const uint2 kk = __ldcg(reinterpret_cast<const uint2*>(p.kc + row + cx.lane * DV));
+          const uint2 vv = __ldcg(reinterpret_cast<const uint2*>(p.vc + row + cx.lane * DV));
+          asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(ka), "r"(kk.x), "r"(kk.y) : "memory");
+          asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(va), "r"(vv.x), "r"(vv.y) : "memory");
+        } else {
+          const unsigned kk = __ldcg(reinterpret_cast<const unsigned*>(p.kc + row + cx.lane * DV));
+          const unsigned vv = __ldcg(reinterpret_cast<const unsigned*>(p.vc + row + cx.lane * DV));
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(ka), "r"(kk) : "memory");
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(va), "r"(vv) : "memory");
         }
+        // the slot is refilled by the async proxy later
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
       }
-      float pw[kMaxGroup];
+      // ---- S = Q K^T for positions pg*16 .. pg*16+15
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      const int kr = pg * 16 + ((mi >> 1) << 3) + rr;
 #pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        float v = sc[h];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        const float sv = valid ? v : -INFINITY;
-        float mr = fmaxf(sv, __shfl_xor_sync(0xffffffffu, sv, 8));
-        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 16));
-        const float mn = fmaxf(m[h], mr);
-        const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
-        const float pv = valid ? exp2f(sv - mn) : 0.f;
-        float ps = pv + __shfl_xor_sync(0xffffffffu, pv, 8);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-        ls[h] = ls[h] * alpha + ps;
-        m[h] = mn;
-#pragma unroll
-        for (int e = 0; e < DV; ++e) oa[h][e] *= alpha;
-        pw[h] = pv;
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4(sw128_addr(kt, P, kr, ks * 16 + ((mi & 1) << 3)), b00, b01, b10, b11);
+        mma_16816(s0, qa0[ks], 0u, qa2[ks], 0u, b00, b01);
+        mma_16816(s1, qa0[ks], 0u, qa2[ks], 0u, b10, b11);
+        mma_16816(s0, qb0[ks], 0u, qb2[ks], 0u, b00, b01);
+        mma_16816(s1, qb0[ks], 0u, qb2[ks], 0u, b10, b11);
       }
-      // p . V: every lane accumulates its DV dims over the 4 positions
+      // ---- online softmax of head gid over the 16 positions (4 per lane)
+      const int pa = pg * 16 + tig * 2;
+      const float v0 = pa < npos ? s0[0] : -INFINITY;
+      const float v1 = pa + 1 < npos ? s0[1] : -INFINITY;
+      const float v2 = pa + 8 < npos ? s1[0] : -INFINITY;
+      const float v3 = pa + 9 < npos ? s1[1] : -INFINITY;
+      float mr = fmaxf(fmaxf(v0, v1), fmaxf(v2, v3));
+      mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 1));
+      mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 2));
+      const float mn = fmaxf(m_h, mr);
+      const float alpha = (mn == -INFINITY) ? 1.f : exp2f(m_h - mn);
+      const float p0 = v0 == -INFINITY ? 0.f : exp2f(v0 - mn);
+      const float p1 = v1 == -INFINITY ? 0.f : exp2f(v1 - mn);
+      const float p2 = v2 == -INFINITY ? 0.f : exp2f(v2 - mn);
+      const float p3 = v3 == -INFINITY ? 0.f : exp2f(v3 - mn);
+      float rs = (p0 + p1) + (p2 + p3);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+      l_h = l_h * alpha + rs;
+      m_h = mn;
 #pragma unroll
-      for (int gq = 0; gq < 4; ++gq) {
-        const int rr = r0 + cx.warp * 4 + gq;
-        const bool vv = rr < npos && (rr >= n_old || have_tile);
-        float pg[kMaxGroup];
+      for (int nt = 0; nt < NT; ++nt) {
+        o[nt][0] *= alpha;
+        o[nt][1] *= alpha;
+      }
+      uint32_t pa0, pa2, pb0, pb2;
+      split_bf16x2(p0, p1, pa0, pb0);
+      split_bf16x2(p2, p3, pa2, pb2);
+      // ---- O += P V for this warp's dims
+      const int vr = pg * 16 + ((mi & 1) << 3) + rr;
 #pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) pg[h] = __shfl_sync(0xffffffffu, pw[h], gq * 8);
-        if (vv) {
-          float vf[DV];
-          if (rr < n_old) {
-            const uint16_t* vrow = sV + static_cast<size_t>(rr) * D + cx.lane * DV;
-            if (DV == 4) {
-              const uint2 u = *reinterpret_cast<const uint2*>(vrow);
-              vf[0] = bf16_lo(u.x);
-              vf[1] = bf16_hi(u.x);
-              vf[2] = bf16_lo(u.y);
-              vf[3] = bf16_hi(u.y);
-            } else {
-              const uint32_t u = *reinterpret_cast<const uint32_t*>(vrow);
-              vf[0] = bf16_lo(u);
-              vf[1] = bf16_hi(u);
-            }
-          } else {
-            const uint16_t* vrow = gV + cx.lane * DV;
-            if (DV == 4) {
-              const uint2 u = __ldcg(reinterpret_cast<const uint2*>(vrow));
-              vf[0] = bf16_lo(u.x);
-              vf[1] = bf16_hi(u.x);
-              vf[2] = bf16_lo(u.y);
-              vf[3] = bf16_hi(u.y);
-            } else {
-              const uint32_t u = __ldcg(reinterpret_cast<const unsigned int*>(vrow));
-              vf[0] = bf16_lo(u);
-              vf[1] = bf16_hi(u);
-            }
-          }
-#pragma unroll
-          for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-            for (int e = 0; e < DV; ++e) oa[h][e] = fmaf(pg[h], vf[e], oa[h][e]);
-        }
+      for (int n2 = 0; n2 < NT / 2; ++n2) {
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4_t(sw128_addr(vt, P, vr, ds * DW + n2 * 16 + ((mi >> 1) << 3)), b00, b01, b10, b11);
+        mma_16816(o[2 * n2], pa0, 0u, pa2, 0u, b00, b01);
+        mma_16816(o[2 * n2 + 1], pa0, 0u, pa2, 0u, b10, b11);
+        mma_16816(o[2 * n2], pb0, 0u, pb2, 0u, b00, b01);
+        mma_16816(o[2 * n2 + 1], pb0, 0u, pb2, 0u, b10, b11);
       }
     }
-    if (n_old > 0) {
-      __syncwarp();
-      if (cx.lane == 0) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
-      rp.next(p.nslot);
+    __syncwarp();
+    if (cx.lane == 0) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
+    rp.next(p.nslot);
+    // end of a (b, g) segment: merge the 8 warps into this CTA's partial, and
+    // let the CTA that completes the head combine every contributor's partial.
+    const int ib = seg_base + seg_g * seg_nch;
+    const int ie = ib + seg_nch;
+    if (i + 1 < i1 && i + 1 < ie) continue;   // the segment goes on
+    const unsigned long long tm0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+
+    const int c_first = split_owner(ib, ap.W, p.G);
+    const size_t head_row = (static_cast<size_t>(seg_b) * p.nkv + seg_g) * p.G;   // partial rows of this head
+    if (tig == 0 && gid < kMaxGroup) {   // lanes 4h hold head h's state
+      sm_ml[(cx.warp * kMaxGroup + gid) * 2 + 0] = m_h;
+      sm_ml[(cx.warp * kMaxGroup + gid) * 2 + 1] = l_h;
     }
-    // end of a (b, g) segment: merge the 8 warps, publish the partial, and
-    // let the CTA that completes the head combine all partials.
-    bool seg_end = (i + 1 == i1);
-    if (!seg_end) {
-      int b2, g2, j2;
-      attn_item(p, ap, i + 1, b2, g2, j2);
-      seg_end = (b2 != seg_b || g2 != seg_g);
-    }
-    if (!seg_end) continue;
+    if (gid < kMaxGroup) {
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      if (cx.lane == 0) {
-        sm_ml[(cx.warp * kMaxGroup + h) * 2 + 0] = m[h];
-        sm_ml[(cx.warp * kMaxGroup + h) * 2 + 1] = ls[h];
+      for (int nt = 0; nt < NT; ++nt) {
+        sm_o[(cx.warp * kMaxGroup + gid) * DW + nt * 8 + tig * 2 + 0] = o[nt][0];
+        sm_o[(cx.warp * kMaxGroup + gid) * DW + nt * 8 + tig * 2 + 1] = o[nt][1];
       }
-#pragma unroll
-      for (int e = 0; e < DV; ++e) sm_o[(cx.warp * kMaxGroup + h) * D + cx.lane * DV + e] = oa[h][e];
     }
     consumer_sync();
-    for (int idx = cx.tid; idx < GQ * D; idx += kConsumerThreads) {
-      const int h = idx / D, dd = idx - h * D;
-      float M = -INFINITY;
+    {
+      // merge the position groups: dims of half ds come from warps pg + ds*NPG
+      const size_t row = head_row + (cx.c - c_first);
+      for (int idx = cx.tid; idx < GQ * D; idx += kConsumerThreads) {
+        const int h = idx / D, dd = idx - h * D;
+        const int dsd = dd / DW, dl = dd - dsd * DW;
+        float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_ml[(w * kMaxGroup + h) * 2]);
-      float Ls = 0.f, Os = 0.f;
+        for (int q = 0; q < NPG; ++q) M = fmaxf(M, sm_ml[((q + dsd * NPG) * kMaxGroup + h) * 2]);
+        float Ls = 0.f, Os = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float mw = sm_ml[(w * kMaxGroup + h) * 2];
-        if (mw == -INFINITY) continue;
-        const float f = exp2f(mw - M);
-        Ls = fmaf(sm_ml[(w * kMaxGroup + h) * 2 + 1], f, Ls);
-        Os = fmaf(sm_o[(w * kMaxGroup + h) * D + dd], f, Os);
-      }
-      p.part_o[(static_cast<size_t>(seg_first) * GQ + h) * D + dd] = Os;
-      if (dd == 0) {
-        p.part_ml[(static_cast<size_t>(seg_first) * GQ + h) * 2 + 0] = M;
-        p.part_ml[(static_cast<size_t>(seg_first) * GQ + h) * 2 + 1] = Ls;
+        for (int q = 0; q < NPG; ++q) {
+          const int w = q + dsd * NPG;
+          const float mw = sm_ml[(w * kMaxGroup + h) * 2];
+          const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+          Ls = fmaf(sm_ml[(w * kMaxGroup + h) * 2 + 1], f, Ls);
+          Os = fmaf(sm_o[(w * kMaxGroup + h) * DW + dl], f, Os);
+        }
+        p.part_o[(row * GQ + h) * D + dd] = Os;
+        if (dd == 0) {
+          p.part_ml[(row * GQ + h) * 2 + 0] = M;
+          p.part_ml[(row * GQ + h) * 2 + 1] = Ls;
+        }
       }
     }
     consumer_sync();
@@ -819,42 +924,87 @@ __device__ void consume_attn(const Params& p, Ctx& cx, int l, int s, RingPos& rp
     if (cx.tid == 0) {
       const unsigned old = release_add(arrive, static_cast<unsigned>(seg_items));
       __threadfence();
-      cx.ctl->flag = (old + seg_items == static_cast<unsigned>(ap.nch[seg_b])) ? 1 : 0;
+      cx.ctl->flag = (old + seg_items == static_cast<unsigned>(seg_nch)) ? 1 : 0;
     }
     consumer_sync();
-    if (cx.ctl->flag) {
-      const int ib = ap.base[seg_b] + seg_g * ap.nch[seg_b];
-      const int ie = ib + ap.nch[seg_b];
-      for (int idx = cx.tid; idx < GQ * D; idx += kConsumerThreads) {
-        const int h = idx / D, dd = idx - h * D;
-        float M = -INFINITY, Ls = 0.f, Os = 0.f;
-        int st = ib;
-        while (st < ie) {
-          const int cc = split_owner(st, ap.W, p.G);
-          const int en = min(ie, split_point(cc + 1, ap.W, p.G));
-          const float ms = __ldcg(p.part_ml + (static_cast<size_t>(st) * GQ + h) * 2);
-          const float lsg = __ldcg(p.part_ml + (static_cast<size_t>(st) * GQ + h) * 2 + 1);
-          const float os = __ldcg(p.part_o + (static_cast<size_t>(st) * GQ + h) * D + dd);
-          if (ms > M) {
-            const float f = exp2f(M - ms);
-            Ls = fmaf(Ls, f, lsg);
-            Os = fmaf(Os, f, os);
-            M = ms;
-          } else if (ms != -INFINITY) {
-            const float f = exp2f(ms - M);
-            Ls = fmaf(lsg, f, Ls);
-            Os = fmaf(os, f, Os);
-          }
-          st = en;
-        }
-        p.o[(static_cast<size_t>(seg_b) * p.nq + seg_g * GQ + h) * D + dd] = Os / Ls;
-      }
-      consumer_sync();
-      if (cx.tid == 0) {
-        atomicExch(arrive, 0u);
-        release_add(p.cnt + l * ST_LAYER + ST_ATTN, 1u);
-      }
+    if (!cx.ctl->flag) {
+      if (p.trace && cx.tid == 0) t_merge += globaltimer() - tm0;
+      continue;
     }
+    // ---- combine: contributors are CTAs c_first .. c_last (rows 0..ncov-1);
+    // a CTA in that range with no chunk of this head contributes nothing.
+    const int c_last = split_owner(ie - 1, ap.W, p.G);
+    const int ncov = c_last - c_first + 1;
+    float* cM = cb;                       // [ncov][GQ]
+    float* cL = cM + p.G * kMaxGroup;     // [ncov][GQ]
+    float* cW = cL + p.G * kMaxGroup;     // [ncov][GQ]
+    float* cS = cW + p.G * kMaxGroup;     // M*[GQ], L*[GQ]
+    for (int idx = cx.tid; idx < ncov * GQ; idx += kConsumerThreads) {
+      const int t = idx / GQ, h = idx - t * GQ;
+      const int cc = c_first + t;
+      const int lo = max(ib, split_point(cc, ap.W, p.G)), hi = min(ie, split_point(cc + 1, ap.W, p.G));
+      float M = -INFINITY, Lv = 0.f;
+      if (lo < hi) {
+        M = __ldcg(p.part_ml + ((head_row + t) * GQ + h) * 2);
+        Lv = __ldcg(p.part_ml + ((head_row + t) * GQ + h) * 2 + 1);
+      }
+      cM[t * kMaxGroup + h] = M;
+      cL[t * kMaxGroup + h] = Lv;
+    }
+    consumer_sync();
+    if (cx.warp < GQ) {
+      const int h = cx.warp;
+      float M = -INFINITY;
+      for (int t = cx.lane; t < ncov; t += 32) M = fmaxf(M, cM[t * kMaxGroup + h]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float Lsum = 0.f;
+      for (int t = cx.lane; t < ncov; t += 32) {
+        const float mt = cM[t * kMaxGroup + h];
+        const float wgt = (mt == -INFINITY) ? 0.f : exp2f(mt - M);
+        cW[t * kMaxGroup + h] = wgt;
+        Lsum = fmaf(wgt, cL[t * kMaxGroup + h], Lsum);
+      }
+      Lsum = warp_sum(Lsum);
+      if (cx.lane == 0) cS[kMaxGroup + h] = Lsum;
+    }
+    consumer_sync();
+    for (int idx = cx.tid; idx < GQ * D; idx += kConsumerThreads) {
+      const int h = idx / D, dd = idx - h * D;
+      const float* src = p.part_o + (head_row * GQ + h) * D + dd;
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+      int t = 0;
+      for (; t + 4 <= ncov; t += 4) {
+        const float w0 = cW[(t + 0) * kMaxGroup + h], w1 = cW[(t + 1) * kMaxGroup + h];
+        const float w2 = cW[(t + 2) * kMaxGroup + h], w3 = cW[(t + 3) * kMaxGroup + h];
+        const float o0 = w0 != 0.f ? __ldcg(src + static_cast<size_t>(t + 0) * GQ * D) : 0.f;
+        const float o1 = w1 != 0.f ? __ldcg(src + static_cast<size_t>(t + 1) * GQ * D) : 0.f;
+        const float o2 = w2 != 0.f ? __ldcg(src + static_cast<size_t>(t + 2) * GQ * D) : 0.f;
+        const float o3 = w3 != 0.f ? __ldcg(src + static_cast<size_t>(t + 3) * GQ * D) : 0.f;
+        acc0 = fmaf(w0, o0, acc0);
+        acc1 = fmaf(w1, o1, acc1);
+        acc2 = fmaf(w2, o2, acc2);
+        acc3 = fmaf(w3, o3, acc3);
+      }
+      for (; t < ncov; ++t) {
+        const float w0 = cW[t * kMaxGroup + h];
+        if (w0 != 0.f) acc0 = fmaf(w0, __ldcg(src + static_cast<size_t>(t) * GQ * D), acc0);
+      }
+      p.o[plane_index(seg_b, (seg_g * GQ + h) * D + dd, p.B, p.nq * D)] =
+          ((acc0 + acc1) + (acc2 + acc3)) / cS[kMaxGroup + h];
+    }
+    consumer_sync();
+    if (cx.tid == 0) {
+      atomicExch(arrive, 0u);
+      release_add(p.cnt + l * ST_LAYER + ST_ATTN, 1u);
+      if (p.trace) t_merge += globaltimer() - tm0;
+    }
+  }
+  if (p.trace && cx.tid == 0) {
+    const size_t n_st = static_cast<size_t>(p.L) * ST_LAYER + 1;
+    unsigned long long* e = p.trace + ((static_cast<size_t>(s) * n_st + stage_index(p, ST_ATTN, l)) * p.G + blockIdx.x) * 8;
+    e[6] = t_wait;
+    e[7] = t_merge;
   }
 }
 
@@ -864,33 +1014,24 @@ __device__ __forceinline__ const Mat& stage_mat(const LayerParams& L, int kind) 
   return kind == ST_QKV ? L.qkv : kind == ST_OPROJ ? L.o : kind == ST_GATEUP ? L.gu : L.down;
 }
 
-// Producer: the stream of one stage.
-template <int D>
-__device__ bool produce_stage(const Params& p, Ctx& cx, int kind, int l, int s, RingPos& rp,
-                              uint64_t pol, bool fused) {
-  const int where = where_code(kind, l, s) | (1 << 15);
-  if (kind == ST_LM) return produce_gemv(p, cx, p.lm, rp, pol, where);
-  if (kind == ST_ATTN) return produce_attn(p, cx, l, s, rp, pol, fused);
-  const LayerParams& L = p.layers[l];
-  return produce_gemv(p, cx, stage_mat(L, kind), rp, pol, where);
-}
-
 // Consumers: one stage.  Returns false once the CTA is aborting.
 template <int B, int D>
-__device__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s, RingPos& rp,
-                              bool fused) {
+__device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s,
+                                           RingPos& rp, bool fused) {
   const unsigned G = static_cast<unsigned>(p.G);
   const unsigned S1 = static_cast<unsigned>(p.step_base + s + 1);
   const int where = where_code(kind, l, s);
   if (kind == ST_ATTN) {
     consume_attn<B, D>(p, cx, l, s, rp, fused);
     consumer_sync();
+    if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
     return !cx.ctl->abort;
   }
   if (kind == ST_LM) {
     if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused)) return false;
     float* hid = (p.hidden_out && cx.c == 0) ? p.hidden_out + static_cast<size_t>(s) * p.B * p.H : nullptr;
-    load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid);
+    load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, where);
+    if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     EpiLM<B> epi{p, s, &bv, &bi};
@@ -944,6 +1085,7 @@ __device__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s, 
       if (cx.tid == 0) release_add(p.cnt + p.cl.step_done, 1u);
     }
     consumer_sync();
+    if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
     return !cx.ctl->abort;
   }
   const LayerParams& L = p.layers[l];
@@ -953,11 +1095,13 @@ __device__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s, 
       if (l == 0) {
         ok = stage_wait(p, cx, p.cnt + p.cl.step_done, S1 - 1u, where, fused);
         if (!ok) return false;
-        load_act<B>(p, cx, p.H, SRC_EMBED, nullptr, L.attn_norm, nullptr);
+        load_act<B>(p, cx, p.H, SRC_EMBED, nullptr, L.attn_norm, nullptr, where);
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       } else {
         ok = stage_wait(p, cx, p.cnt + (l - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused);
         if (!ok) return false;
-        load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.attn_norm, nullptr);
+        load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.attn_norm, nullptr, where);
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       }
       EpiQKV<B> epi{p, l, s};
       consume_gemv<B>(p, cx, L.qkv, rp, where, epi);
@@ -966,21 +1110,24 @@ __device__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s, 
     case ST_OPROJ: {
       const unsigned tgt = static_cast<unsigned>(p.B * p.nkv) * S1;
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_ATTN, tgt, where, fused)) return false;
-      load_act<B>(p, cx, p.nq * p.d, SRC_PLAIN, p.o, nullptr, nullptr);
+      load_act<B>(p, cx, p.nq * p.d, SRC_PLAIN, p.o, nullptr, nullptr, where);
+      if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiResid<B> epi{p, l == 0};
       consume_gemv<B>(p, cx, L.o, rp, where, epi);
       break;
     }
     case ST_GATEUP: {
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_OPROJ, G * S1, where, fused)) return false;
-      load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr);
+      load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr, where);
+      if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiSwiGLU<B> epi{p};
       consume_gemv<B>(p, cx, L.gu, rp, where, epi);
       break;
     }
     default: {  // ST_DOWN
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_GATEUP, G * S1, where, fused)) return false;
-      load_act<B>(p, cx, p.F, SRC_PLAIN, p.h, nullptr, nullptr);
+      load_act<B>(p, cx, p.F, SRC_PLAIN, p.h, nullptr, nullptr, where);
+      if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiResid<B> epi{p, false};
       consume_gemv<B>(p, cx, L.down, rp, where, epi);
       break;
@@ -990,7 +1137,10 @@ __device__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s, 
   // the async proxy (bulk copies): order this thread's generic writes first.
   if (kind == ST_QKV) fence_proxy_async_global();
   consumer_sync();
-  if (cx.tid == 0) release_add(p.cnt + l * ST_LAYER + kind, 1u);
+  if (cx.tid == 0) {
+    trace_stamp(p, s, stage_index(p, kind, l), 3);
+    release_add(p.cnt + l * ST_LAYER + kind, 1u);
+  }
   return !cx.ctl->abort;
 }
 
@@ -1005,6 +1155,7 @@ __device__ __forceinline__ Ctx make_ctx(uint8_t* smem, const Params& p) {
   cx.tid = threadIdx.x;
   cx.warp = threadIdx.x >> 5;
   cx.lane = threadIdx.x & 31;
+  cx.act_phase = 0;
   return cx;
 }
 
@@ -1014,6 +1165,7 @@ __device__ __forceinline__ void init_ring(const Params& p, Ctx& cx) {
       mbar_init(smem_addr(&cx.ctl->full[i]), 1);
       mbar_init(smem_addr(&cx.ctl->empty[i]), kConsumerWarps);
     }
+    mbar_init(smem_addr(&cx.ctl->act_bar), 1);
     cx.ctl->abort = 0;
     cx.ctl->flag = 0;
     fence_barrier_init();
@@ -1041,26 +1193,184 @@ __device__ void drain_ring(const Params& p, Ctx& cx, const RingPos& rp, int issu
     // 2 s, independent of the dependency-wait limit) only guards against a
     // device that stopped making progress.
     const long long limit = p.spin_limit_ns > 2000000000LL ? p.spin_limit_ns : 2000000000LL;
-    while (!mbar_try_wait(fb, q.phase)) {
+    while (!mbar_try_wait_suspend(fb, q.phase, 20000u)) {
       if (static_cast<long long>(globaltimer() - t0) > limit) break;
     }
   }
 }
 
-template <int D>
+// ------------------------------------------------------------------ producer
+
+// One tile of the CTA's stream: one contiguous global range (a packed weight
+// tile) or two (the K rows and V rows of an attention chunk, the V rows landing
+// at the slot's second half).
+struct Tile {
+  const uint8_t* src;   // GEMV: packed tile
+  int y;                // attention: first cache row of the chunk (tensor-map row)
+  uint32_t bytes;       // bytes landing in the slot
+  bool attn;
+  int stage;            // stage_index
+  int layer;
+  int step;
+};
+
+// A position in the CTA's static schedule: steps x (layers x 5 stages + LM).
+// The producer runs two: the copy cursor (tiles into the ring) and, ahead of
+// it, the prefetch cursor (the same tiles into L2).
+template <int B>
+struct Cursor {
+  int s, l, kind;
+  bool open;           // the current stage's range has been set up
+  bool one_stage;      // kernel-per-op launch: only one stage
+  bool done;
+  int a, a_end;        // GEMV: next pair of the CTA's span / span end; attention: item range
+  int kc, nkc, KC;
+  const uint8_t* src;  // GEMV: next tile
+  AttnPlan<B> ap;
+};
+
+template <int B>
+__device__ __forceinline__ void cursor_start(Cursor<B>& cu, int s, int l, int kind, bool one) {
+  cu.s = s;
+  cu.l = l;
+  cu.kind = kind;
+  cu.open = false;
+  cu.one_stage = one;
+  cu.done = false;
+}
+
+template <int B>
+__device__ __forceinline__ void cursor_next_stage(const Params& p, Cursor<B>& cu) {
+  cu.open = false;
+  if (cu.one_stage) {
+    cu.done = true;
+  } else if (cu.kind == ST_LM) {
+    cu.kind = 0;
+    cu.l = 0;
+    if (++cu.s >= p.n_steps) cu.done = true;
+  } else if (++cu.kind == ST_LAYER) {
+    cu.kind = 0;
+    if (++cu.l == p.L) {
+      cu.kind = ST_LM;
+      cu.l = 0;
+    }
+  }
+}
+
+template <int B>
+__device__ bool cursor_next(const Params& p, int c, Cursor<B>& cu, Tile& t) {
+  while (!cu.done) {
+    if (!cu.open) {
+      cu.open = true;
+      if (cu.kind == ST_ATTN) {
+        attn_plan<B>(p, cu.s, cu.ap);
+        cu.a = split_point(c, cu.ap.W, p.G);
+        cu.a_end = split_point(c + 1, cu.ap.W, p.G);
+      } else {
+        const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
+        const int NP = m.N >> 1;
+        cu.a = split_point(c, NP, p.G);
+        cu.a_end = split_point(c + 1, NP, p.G);
+        cu.kc = 0;
+        cu.nkc = m.K / m.KC;
+        cu.KC = m.KC;
+        cu.src = m.packed + static_cast<size_t>(2) * cu.a * m.K * p.esz;
+      }
+    }
+    t.stage = stage_index(p, cu.kind, cu.l);
+    t.layer = cu.l;
+    t.step = cu.s;
+    if (cu.kind == ST_ATTN) {
+      if (cu.a < cu.a_end) {   // every chunk is one tile (K and V boxes)
+        int b, g, j, nch, base;
+        attn_item<B>(p, cu.ap, cu.a, b, g, j, nch, base);
+        ++cu.a;
+        t.y = static_cast<int>(kv_row(p, cu.l, b, g, j * p.attn_pos_per_tile) / p.d);
+        t.src = nullptr;
+        t.bytes = kSlotBytes;
+        t.attn = true;
+        return true;
+      }
+    } else if (cu.a < cu.a_end) {
+      const int gp = min(kPairsPerTile, cu.a_end - cu.a);
+      t.bytes = 2u * gp * cu.KC * p.esz;
+      t.src = cu.src;
+      t.attn = false;
+      cu.src += t.bytes;
+      if (++cu.kc == cu.nkc) {
+        cu.kc = 0;
+        cu.a += kPairsPerTile;
+      }
+      return true;
+    }
+    cursor_next_stage<B>(p, cu);
+  }
+  return false;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// The producer (one thread): copy cursor -> ring, prefetch cursor -> L2,
+// `p.l2_prefetch_bytes` ahead.  Weights do not depend on activations, so both
+// run ahead of the consumers across stage boundaries; only attention chunks
+// wait for the previous step's KV write of their layer.
+template <int B>
 __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
   RingPos rp;
   const uint64_t pol = evict_first_policy();
-  bool ok = true;
-  if (fused) {
-    for (int s = 0; s < p.n_steps && ok; ++s) {
-      for (int l = 0; l < p.L && ok; ++l)
-        for (int k = 0; k < ST_LAYER && ok; ++k) ok = produce_stage<D>(p, cx, k, l, s, rp, pol, true);
-      if (ok) ok = produce_stage<D>(p, cx, ST_LM, 0, s, rp, pol, true);
+  Cursor<B> cc, pc;
+  cursor_start<B>(cc, s0, l0, kind0, !fused);
+  cursor_start<B>(pc, s0, l0, kind0, !fused);
+  long long ahead = 0;
+  bool pc_live = true;
+  int cur_stage = -1, cur_step = -1;
+  Tile t, tp;
+  while (cursor_next<B>(p, cx.c, cc, t)) {
+    const uint32_t tb = t.bytes;
+    ahead -= tb;
+    while (pc_live && ahead < p.l2_prefetch_bytes) {
+      pc_live = cursor_next<B>(p, cx.c, pc, tp);
+      if (!pc_live) break;
+      if (!tp.attn) prefetch_l2(tp.src, tp.bytes);
+      ahead += tp.bytes;
     }
-  } else {
-    ok = produce_stage<D>(p, cx, kind0, l0, s0, rp, pol, false);
+    if (t.stage != cur_stage || t.step != cur_step) {
+      if (cur_stage >= 0) trace_stamp(p, cur_step, cur_stage, 5);
+      cur_stage = t.stage;
+      cur_step = t.step;
+      trace_stamp(p, t.step, t.stage, 4);
+      if (t.attn) {
+        // KV rows up to pos-1 were written by this layer's QKV stage of earlier
+        // steps (or before the launch); make sure the previous step's write is
+        // complete before reading it through the async proxy.
+        if (fused) {
+          const unsigned target = static_cast<unsigned>(p.G) * static_cast<unsigned>(p.step_base + t.step);
+          const int where = where_code(ST_ATTN, t.layer, t.step) | (1 << 15);
+          if (!counter_wait(p, cx.ctl, p.cnt + t.layer * ST_LAYER + ST_QKV, target, where)) break;
+        }
+        fence_proxy_async_global();
+      }
+    }
+    const int where = where_code(t.stage % ST_LAYER, t.layer, t.step) | (1 << 15);
+    const uint32_t eb = smem_addr(&cx.ctl->empty[rp.slot]);
+    if (!ring_wait(p, cx.ctl, eb, rp.phase ^ 1u, where)) break;
+    const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
+    mbar_expect_tx(fb, tb);
+    const uint32_t dst = smem_addr(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes);
+    if (t.attn) {
+      const int box = p.attn_pos_per_tile * 128;
+      for (int x = 0; x < p.d; x += 64) {
+        tma_load_2d(dst + (x >> 6) * box, &p.tmap_k, x, t.y, fb, pol);
+        tma_load_2d(dst + kSlotBytes / 2 + (x >> 6) * box, &p.tmap_v, x, t.y, fb, pol);
+      }
+    } else {
+      bulk_g2s(dst, t.src, t.bytes, fb, pol);
+    }
+    rp.next(p.nslot);
   }
+  if (cur_stage >= 0) trace_stamp(p, cur_step, cur_stage, 5);
   // Every slot's most recent copy must have landed before the CTA may exit.
   drain_ring(p, cx, rp, p.nslot);
 }
@@ -1087,7 +1397,7 @@ __global__ void __launch_bounds__(kThreads, 1) engine_persistent(const __grid_co
   Ctx cx = make_ctx(smem, p);
   init_ring(p, cx);
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<D>(p, cx, 0, 0, 0, true);
+    if (cx.lane == 0) producer_main<B>(p, cx, 0, 0, 0, true);
     __syncwarp();
   } else {
     consumer_main<B, D>(p, cx, 0, 0, 0, true);
@@ -1102,7 +1412,7 @@ __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constan
   Ctx cx = make_ctx(smem, p);
   init_ring(p, cx);
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<D>(p, cx, kind, layer, step, false);
+    if (cx.lane == 0) producer_main<B>(p, cx, kind, layer, step, false);
     __syncwarp();
   } else {
     consumer_main<B, D>(p, cx, kind, layer, step, false);

@@ -6,6 +6,7 @@
 // fetched at run time: the "task list" of a CTA is the static partition of
 // every stage's rows (or attention chunks) by CTA index.
 #pragma once
+#include <cuda.h>   // CUtensorMap (type only; the library does not link libcuda)
 #include <stdint.h>
 
 namespace xlpk {
@@ -82,6 +83,7 @@ struct Params {
   int act_bytes;        // activation / scratch region
   int attn_pos_per_tile;
   long long spin_limit_ns;
+  long long l2_prefetch_bytes;  // how far the producer's L2-prefetch cursor runs ahead
   CounterLayout cl;
 
   // weights
@@ -90,7 +92,11 @@ struct Params {
   Mat lm;
   const LayerParams* layers;    // device array [L]
 
-  // KV cache (caller-owned), bf16 [L][B][nkv][max_seq][d]
+  // KV cache (caller-owned), bf16 [L][B][nkv][max_seq][d]; the tensor maps view
+  // each as a 2-D [L*B*nkv*max_seq rows][d] array read in 64-column boxes of
+  // attn_pos_per_tile rows with 128-byte swizzle
+  CUtensorMap tmap_k;
+  CUtensorMap tmap_v;
   uint16_t* kc;
   uint16_t* vc;
   const float2* rope;           // [max_seq][d/2] (cos, sin)
@@ -100,8 +106,8 @@ struct Params {
   float* q;          // [B][nq*d] rotated queries
   float* o;          // [B][nq*d] attention output
   float* h;          // [B][F] SwiGLU output
-  float* part_ml;    // [items][group][2] (running max in log2 units, sum)
-  float* part_o;     // [items][group][d]
+  float* part_ml;    // [B][nkv][G][group][2] per contributing CTA: (max in log2 units, sum)
+  float* part_o;     // [B][nkv][G][group][d] unnormalised attention output
   float* lm_val;     // [G][B]
   int* lm_idx;       // [G][B]
   unsigned* cnt;
@@ -117,6 +123,7 @@ struct Params {
   const int32_t* forced;
   float* logits_out;
   float* hidden_out;
+  unsigned long long* trace;   // optional stage timestamps
 };
 
 }  // namespace xlpk

@@ -9,11 +9,14 @@
 // decode graph is statically compiled into one resident Engine Kernel; the
 // fixed temporary-tensor table of "Persistent execution paradigm", section
 // 5.3, becomes the static workspace arena below).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -217,6 +220,37 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Tensor map of one KV cache viewed as a 2-D [rows][d] bf16 array, read in
+// boxes of 64 columns x P rows with 128-byte swizzle (the layout the attention
+// tile's ldmatrix addressing expects).  The encoder is the driver's
+// cuTensorMapEncodeTiled, reached through the runtime's entry-point query so
+// the library does not link libcuda.
+xlpk_status encode_kv_map(CUtensorMap* map, void* base, unsigned long long rows, int d, int P) {
+  static PFN_cuTensorMapEncodeTiled encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+      g_cuda_err = "cuTensorMapEncodeTiled unavailable";
+      return XLPK_ERR_CUDA;
+    }
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+  }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(P)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_cuda_err = "cuTensorMapEncodeTiled failed (" + std::to_string(static_cast<int>(r)) + ")";
+    return XLPK_ERR_CUDA;
+  }
+  return XLPK_OK;
+}
+
 xlpk_status validate_config(const xlpk_config* c) {
   if (!c) return XLPK_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->n_layers > 1024 || c->hidden <= 0 || c->n_q_heads <= 0 ||
@@ -299,7 +333,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
 
   // shared memory: ring + activation/scratch + control
   const int kmax = std::max(std::max(H, qd), F);
-  const int attn_scratch = (kConsumerWarps * kMaxGroup * 2 + kConsumerWarps * kMaxGroup * d) * 4;
+  const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
   e->act_bytes = static_cast<int>(align_up(std::max(B * kmax * 4, attn_scratch), 1024));
   const int max_smem = static_cast<int>(prop.sharedMemPerBlockOptin);
   e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - kMiscSmem) / kSlotBytes);
@@ -307,8 +341,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->smem = e->nslot * kSlotBytes + e->act_bytes + kMiscSmem;
   if (!bind_by_shape(e, B, d)) return XLPK_ERR_UNSUPPORTED;
 
-  XLPK_CUDA(cudaFuncSetAttribute(e->kern_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, e->smem));
-  XLPK_CUDA(cudaFuncSetAttribute(e->kern_stage, cudaFuncAttributeMaxDynamicSharedMemorySize, e->smem));
+  // The attribute is per kernel function, shared by every handle that uses the
+  // same instantiation: allow the device maximum rather than this handle's size.
+  XLPK_CUDA(cudaFuncSetAttribute(e->kern_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem));
+  XLPK_CUDA(cudaFuncSetAttribute(e->kern_stage, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem));
   int per_sm = 0;
   XLPK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, e->kern_persistent, kThreads, e->smem));
   if (per_sm < 1 || e->G > per_sm * prop.multiProcessorCount) {
@@ -337,6 +373,12 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, H, F);
   }
   add({MatKind::PLAIN, static_cast<const uint8_t*>(w->lm_head.w_dev), nullptr, nullptr}, c.vocab, H);
+  // library-owned copies of the embedding table and the norm gains, so the
+  // caller may free every weight buffer after create
+  const size_t off_embed = total;
+  total += align_up(static_cast<size_t>(c.vocab) * H * 2, 256);
+  const size_t off_norms = total;
+  total += align_up(sizeof(float) * H * (2 * static_cast<size_t>(c.n_layers) + 1), 256);
   e->packed_bytes = total;
   XLPK_CUDA(cudaMalloc(&e->packed, total));
   e->weight_bytes_per_step = 0;
@@ -373,10 +415,19 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   cudaFree(d_jobs);
   cudaStreamDestroy(st);
   if (rc != XLPK_OK) return rc;
+  uint16_t* embed_copy = reinterpret_cast<uint16_t*>(e->packed + off_embed);
+  float* norms = reinterpret_cast<float*>(e->packed + off_norms);
+  XLPK_CUDA(cudaMemcpy(embed_copy, w->embed_dev, static_cast<size_t>(c.vocab) * H * 2, cudaMemcpyDeviceToDevice));
   for (int l = 0; l < c.n_layers; ++l) {
-    lp[l].attn_norm = w->layers[l].attn_norm_dev;
-    lp[l].ffn_norm = w->layers[l].ffn_norm_dev;
+    float* an = norms + static_cast<size_t>(2 * l) * H;
+    float* fn = an + H;
+    XLPK_CUDA(cudaMemcpy(an, w->layers[l].attn_norm_dev, sizeof(float) * H, cudaMemcpyDeviceToDevice));
+    XLPK_CUDA(cudaMemcpy(fn, w->layers[l].ffn_norm_dev, sizeof(float) * H, cudaMemcpyDeviceToDevice));
+    lp[l].attn_norm = an;
+    lp[l].ffn_norm = fn;
   }
+  float* final_norm_copy = norms + static_cast<size_t>(2 * c.n_layers) * H;
+  XLPK_CUDA(cudaMemcpy(final_norm_copy, w->final_norm_dev, sizeof(float) * H, cudaMemcpyDeviceToDevice));
   XLPK_CUDA(cudaMalloc(&e->d_layers, sizeof(LayerParams) * c.n_layers));
   XLPK_CUDA(cudaMemcpy(e->d_layers, lp.data(), sizeof(LayerParams) * c.n_layers, cudaMemcpyHostToDevice));
 
@@ -386,7 +437,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   XLPK_CUDA(cudaMemcpy(e->rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice));
 
   // workspace arena with fixed offsets
-  const long long wmax = static_cast<long long>(B) * c.n_kv_heads * ((c.max_seq + e->P - 1) / e->P);
+  // attention partials: one row per (sequence, kv head, contributing CTA)
+  const long long prow = static_cast<long long>(B) * c.n_kv_heads * e->G;
   CounterLayout cl;
   cl.lm_arrive = c.n_layers * ST_LAYER;
   cl.step_done = cl.lm_arrive + 1;
@@ -402,8 +454,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const size_t o_q = take(sizeof(float) * B * qd);
   const size_t o_o = take(sizeof(float) * B * qd);
   const size_t o_h = take(sizeof(float) * B * F);
-  const size_t o_pml = take(sizeof(float) * wmax * group * 2);
-  const size_t o_po = take(sizeof(float) * wmax * group * d);
+  const size_t o_pml = take(sizeof(float) * prow * group * 2);
+  const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * e->G * B);
   const size_t o_li = take(sizeof(int) * e->G * B);
   const size_t o_cnt = take(sizeof(unsigned) * cl.total);
@@ -434,13 +486,27 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.act_bytes = e->act_bytes;
   p.attn_pos_per_tile = e->P;
   p.spin_limit_ns = 1000LL * (c.spin_limit_us > 0 ? c.spin_limit_us : 200000);
+  {
+    // L2 prefetch distance per CTA (tuning knob; 0 disables)
+    long long kb = 256;
+    if (const char* env = std::getenv("XLPK_L2_PREFETCH_KB")) kb = std::atoll(env);
+    p.l2_prefetch_bytes = kb * 1024;
+  }
   p.cl = cl;
-  p.embed = static_cast<const uint16_t*>(w->embed_dev);
-  p.final_norm = w->final_norm_dev;
+  p.embed = embed_copy;
+  p.final_norm = final_norm_copy;
   p.lm = lm;
   p.layers = e->d_layers;
   p.kc = static_cast<uint16_t*>(kv->k_dev);
   p.vc = static_cast<uint16_t*>(kv->v_dev);
+  {
+    const unsigned long long rows =
+        static_cast<unsigned long long>(c.n_layers) * B * c.n_kv_heads * static_cast<unsigned long long>(c.max_seq);
+    xlpk_status st = encode_kv_map(&p.tmap_k, kv->k_dev, rows, d, e->P);
+    if (st != XLPK_OK) return st;
+    st = encode_kv_map(&p.tmap_v, kv->v_dev, rows, d, e->P);
+    if (st != XLPK_OK) return st;
+  }
   p.rope = e->rope;
   p.x = reinterpret_cast<float*>(e->ws + o_x);
   p.q = reinterpret_cast<float*>(e->ws + o_q);
@@ -477,6 +543,7 @@ Params call_params(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out, const x
   p.forced = io ? io->forced_tokens_dev : nullptr;
   p.logits_out = io ? io->logits_dev : nullptr;
   p.hidden_out = io ? io->hidden_dev : nullptr;
+  p.trace = io ? reinterpret_cast<unsigned long long*>(io->trace_dev) : nullptr;
   return p;
 }
 

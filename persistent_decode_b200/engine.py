@@ -131,14 +131,14 @@ class Engine:
         _check(lib.xlpk_set_state(self.h, t, s, _stream_handle(stream)), "xlpk_set_state")
 
     @staticmethod
-    def _io(forced=None, logits=None, hidden=None, experts=None):
-        if forced is None and logits is None and hidden is None and experts is None:
+    def _io(forced=None, logits=None, hidden=None, experts=None, trace=None):
+        if all(t is None for t in (forced, logits, hidden, experts, trace)):
             return None
-        return _abi.xlpk_decode_io(_ptr(forced), _ptr(logits), _ptr(hidden), _ptr(experts))
+        return _abi.xlpk_decode_io(_ptr(forced), _ptr(logits), _ptr(hidden), _ptr(experts), _ptr(trace))
 
     def decode(self, n_steps: int, tokens_out, forced=None, logits=None, hidden=None, experts=None,
-               stream=None, unfused: bool = False) -> None:
-        io = self._io(forced, logits, hidden, experts)
+               trace=None, stream=None, unfused: bool = False) -> None:
+        io = self._io(forced, logits, hidden, experts, trace)
         fn = lib.xlpk_decode_unfused if unfused else lib.xlpk_decode
         _check(fn(self.h, int(n_steps), _ptr(tokens_out), C.byref(io) if io is not None else None,
                   _stream_handle(stream)), "xlpk_decode_unfused" if unfused else "xlpk_decode")

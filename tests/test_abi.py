@@ -77,5 +77,5 @@ def test_struct_layout_matches_header(lib):
     assert C.sizeof(_abi.xlpk_config) == 18 * 4
     assert C.sizeof(_abi.xlpk_linear) == 16
     assert C.sizeof(_abi.xlpk_layer_weights) == 8 + 4 * 16 + 8 + 3 * 16 + 8 + 6 * 16
-    assert C.sizeof(_abi.xlpk_decode_io) == 32
+    assert C.sizeof(_abi.xlpk_decode_io) == 40
     assert C.sizeof(_abi.xlpk_info) == 6 * 4 + 3 * 8

@@ -107,3 +107,62 @@ def test_kv_full_is_rejected(tiny):
     with pytest.raises(XlpkError) as e:
         tiny.engine.decode(tiny.cfg.steps + 1, tok)
     assert e.value.status == -5
+
+
+def test_weights_may_be_freed_after_create(tiny, cuda_device):
+    """The engine keeps its own copies (packed weights, embedding, norm gains)."""
+    from persistent_decode_b200 import Engine
+    ref = run_engine(tiny, 8)
+    w2 = {k: v.clone() for k, v in tiny.weights.items()}
+    k2, v2 = tiny.k.clone(), tiny.v.clone()
+    eng = Engine(tiny.cfg, w2, k2, v2)
+    del w2
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    junk = torch.full((64 << 20,), 7, dtype=torch.int32, device=cuda_device)   # reuse the freed memory
+    eng.set_state(tiny.start_tokens.tolist(), [tiny.cfg.kv_len])
+    tok = torch.empty(8, 1, dtype=torch.int32, device=cuda_device)
+    eng.decode(8, tok)
+    eng.check()
+    assert torch.equal(tok.cpu(), ref.tokens)
+    del junk
+    eng.close()
+
+
+def test_head_dim_128_group_4_multi_chunk(cuda_device):
+    # d = 128 and 4 query heads per kv head (the 8B/MoE attention shape) at a
+    # size the oracle finishes quickly; KV 200 spans several 64-position chunks
+    # with a ragged tail, and n_ctas 148 leaves CTAs without attention work.
+    cfg = synth.get_config("tiny", hidden=512, n_q_heads=4, n_kv_heads=1, head_dim=128,
+                           ffn=1024, kv_len=200, steps=10)
+    m = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    for unfused in (False, True):
+        run = run_engine(m, cfg.steps, unfused=unfused)
+        compare_with_oracle(m, run, oracle_for(m), cfg.steps)
+
+
+def test_llama1b_full_size_prefix(cuda_device):
+    # the 1B shape at its full size (KV 1024 from a 1024-token prompt prefilled
+    # through the engine, the whole grid): the oracle replays the first steps.
+    cfg = synth.get_config("llama1b")
+    m = workload.build(cfg, device=cuda_device)
+    run = run_engine(m, 24)
+    o = oracle_for(m)
+    T = cfg.kv_len
+    assert rel_l2(m.k[:, :, :, :T].float().cpu(), o.K[:, :, :, :T].float()) < 1e-2
+    compare_with_oracle(m, run, o, 3)
+    assert int(run.tokens.min()) >= 0 and int(run.tokens.max()) < cfg.vocab
+
+
+def test_llama8b_full_size_prefix(cuda_device):
+    # the 8B shape with its 8192-entry synthetic cache, in the launch
+    # configuration the bench times (one CTA per SM, one launch per call)
+    cfg = synth.get_config("llama8b")
+    m = workload.build(cfg, device=cuda_device)
+    run = run_engine(m, 16)
+    o = oracle_for(m)
+    compare_with_oracle(m, run, o, 2)
+    T = cfg.kv_len
+    # steps wrote exactly positions T .. T+15
+    assert bool((m.k[:, :, :, T:T + 16].float().abs().sum(-1) > 0).all())
+    assert int(m.k[:, :, :, T + 16:].float().abs().sum().item()) == 0
