@@ -178,6 +178,31 @@ xlpk_status xlpk_decode(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
 xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                                 const xlpk_decode_io* io, void* stream);
 
+/* Allocation-free decode.  The pages have no counterpart to this entry point;
+ * it exists for callers that must not allocate device memory while they
+ * decode: code that records the decode into a CUDA graph during stream capture,
+ * threads that must never enter the CUDA allocator, or processes whose device
+ * memory is entirely owned by another framework's caching allocator.  It runs
+ * the same persistent kernel as xlpk_decode, with the same arguments and
+ * results, but every per-call scratch buffer of the kernel (activation vectors,
+ * attention and LM-head partials, dependency counters) lives in one array
+ * compiled into the library: XLPK_NOALLOC_SCRATCH_BYTES bytes of file-scope
+ * __device__ memory that every GPU which loads the library holds until the
+ * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Returns XLPK_ERR_UNSUPPORTED (with a message in xlpk_last_cuda_error) if
+ *    the handle's scratch would exceed the array.
+ *  - The counters in the array are cleared on `stream` at the start of each
+ *    call; every other scratch byte is written before it is read.
+ *  - All calls share the one array: calls whose executions overlap on the GPU
+ *    (different streams, handles or threads) race.  Serialise them.
+ *  - Device-side status is reported by xlpk_get_status(h) as for xlpk_decode. */
+#define XLPK_NOALLOC_SCRATCH_BYTES (8u << 20)
+xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
+                                const xlpk_decode_io* io, void* stream);
+
 /* End-to-end call with host buffers: uploads the state, decodes, downloads
  * tokens_out_host [n_steps][B], and synchronises `stream`.  Returns the
  * device status of the decode. */

@@ -16,6 +16,8 @@ XLPK_ERR_KV_FULL = -5
 XLPK_ERR_TIMEOUT = -6
 XLPK_ERR_ABORTED = -7
 
+XLPK_NOALLOC_SCRATCH_BYTES = 8 << 20
+
 XLPK_DTYPE_BF16 = 0
 XLPK_DTYPE_FP8_E4M3 = 1
 
@@ -70,6 +72,8 @@ SIGNATURES = {
     "xlpk_set_state": (C.c_int32, [C.c_void_p, C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.c_void_p]),
     "xlpk_decode": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p, C.POINTER(xlpk_decode_io), C.c_void_p]),
     "xlpk_decode_unfused": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p,
+                                        C.POINTER(xlpk_decode_io), C.c_void_p]),
+    "xlpk_decode_noalloc": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p,
                                         C.POINTER(xlpk_decode_io), C.c_void_p]),
     "xlpk_generate": (C.c_int32, [C.c_void_p, C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.c_int32,
                                   C.POINTER(C.c_int32), C.c_void_p]),

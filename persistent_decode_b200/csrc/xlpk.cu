@@ -18,6 +18,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -555,6 +556,34 @@ void advance(xlpk_engine* h, int32_t n_steps, cudaStream_t st) {
 
 }  // namespace
 
+// ------------------------------------------------------------------ allocation-free decode
+// Scratch of xlpk_decode_noalloc: one library-wide array on every device that
+// loads the library.  Host code must not use the symbol's host address; the
+// device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[XLPK_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the array on `dev` (which must be the current device).
+xlpk_status noalloc_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= kMaxDevices) return XLPK_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    g_noalloc_addr[dev] = static_cast<unsigned char*>(ptr);
+  }
+  *out = g_noalloc_addr[dev];
+  return XLPK_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 xlpk_status xlpk_create(const xlpk_config* cfg, const xlpk_weights* weights, const xlpk_kv* kv,
@@ -623,6 +652,64 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   }
   XLPK_CUDA(cudaGetLastError());
   advance(h, n_steps, st);
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
+                                const xlpk_decode_io* io, void* stream) {
+  xlpk_status rc = check_decode_args(h, n_steps, tokens_out_dev);
+  if (rc != XLPK_OK || n_steps == 0) return rc;
+  int dev = -1;
+  XLPK_CUDA(cudaGetDevice(&dev));
+  if (dev != h->device) return XLPK_ERR_INVALID_ARG;
+  unsigned char* sc = nullptr;
+  rc = noalloc_scratch(dev, &sc);
+  if (rc != XLPK_OK) return rc;
+  const xlpk_config& c = h->cfg;
+  const int B = c.batch, H = c.hidden, d = c.head_dim, F = c.ffn;
+  const int qd = c.n_q_heads * d, group = c.n_q_heads / c.n_kv_heads;
+  const size_t prow = static_cast<size_t>(B) * c.n_kv_heads * h->G;
+  // counters first, so one memset clears everything that must start at zero
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_cnt = take(sizeof(unsigned) * h->base.cl.total);
+  const size_t cnt_bytes = off;
+  const size_t o_x = take(sizeof(float) * B * H);
+  const size_t o_q = take(sizeof(float) * B * qd);
+  const size_t o_o = take(sizeof(float) * B * qd);
+  const size_t o_h = take(sizeof(float) * B * F);
+  const size_t o_pml = take(sizeof(float) * prow * group * 2);
+  const size_t o_po = take(sizeof(float) * prow * group * d);
+  const size_t o_lv = take(sizeof(float) * h->G * B);
+  const size_t o_li = take(sizeof(int) * h->G * B);
+  if (off > XLPK_NOALLOC_SCRATCH_BYTES) {
+    g_cuda_err = "xlpk_decode_noalloc: this handle needs " + std::to_string(off) +
+                 " bytes of scratch, more than the " + std::to_string(XLPK_NOALLOC_SCRATCH_BYTES) +
+                 "-byte static array";
+    return XLPK_ERR_UNSUPPORTED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = call_params(h, n_steps, tokens_out_dev, io);
+  p.step_base = 0;   // fresh counters
+  p.cnt = reinterpret_cast<unsigned*>(sc + o_cnt);
+  p.x = reinterpret_cast<float*>(sc + o_x);
+  p.q = reinterpret_cast<float*>(sc + o_q);
+  p.o = reinterpret_cast<float*>(sc + o_o);
+  p.h = reinterpret_cast<float*>(sc + o_h);
+  p.part_ml = reinterpret_cast<float*>(sc + o_pml);
+  p.part_o = reinterpret_cast<float*>(sc + o_po);
+  p.lm_val = reinterpret_cast<float*>(sc + o_lv);
+  p.lm_idx = reinterpret_cast<int*>(sc + o_li);
+  XLPK_CUDA(cudaMemsetAsync(sc, 0, cnt_bytes, st));
+  void* args[] = {&p};
+  XLPK_CUDA(cudaLaunchCooperativeKernel(h->kern_persistent, dim3(h->G), dim3(kThreads), args,
+                                        static_cast<size_t>(h->smem), st));
+  for (int b = 0; b < B; ++b) h->pos[b] += n_steps;
+  h->last_stream = st;
   return XLPK_OK;
 }
 

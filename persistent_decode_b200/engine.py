@@ -143,6 +143,14 @@ class Engine:
         _check(fn(self.h, int(n_steps), _ptr(tokens_out), C.byref(io) if io is not None else None,
                   _stream_handle(stream)), "xlpk_decode_unfused" if unfused else "xlpk_decode")
 
+    def decode_noalloc(self, n_steps: int, tokens_out, forced=None, logits=None, hidden=None,
+                       stream=None) -> None:
+        """xlpk_decode_noalloc: the same decode with its scratch in the library's static array."""
+        io = self._io(forced, logits, hidden, None, None)
+        _check(lib.xlpk_decode_noalloc(self.h, int(n_steps), _ptr(tokens_out),
+                                       C.byref(io) if io is not None else None, _stream_handle(stream)),
+               "xlpk_decode_noalloc")
+
     def status(self) -> int:
         return int(lib.xlpk_get_status(self.h))
 
