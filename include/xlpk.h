@@ -153,7 +153,9 @@ typedef struct xlpk_engine* xlpk_handle;
  * the order the CTAs stream them, build the RoPE table, allocate the
  * workspace and borrow the KV pointers for the handle's lifetime (the KV
  * cache is written in place).  Weight buffers may be freed afterwards.
- * Runs on the current device and synchronises it. */
+ * Runs on the current device and synchronises it first, so weights still
+ * being written by work enqueued on any stream are complete before they are
+ * packed. */
 xlpk_status xlpk_create(const xlpk_config* cfg, const xlpk_weights* weights,
                         const xlpk_kv* kv, xlpk_handle* out);
 

@@ -205,6 +205,24 @@ __device__ __forceinline__ int ld_volatile(const int* p) {
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
+// Consumer barrier that also ORs `v` over the consumer threads, so that every
+// consumer gets the same answer.  Any decision of the consumers to leave the
+// stage loop must be taken this way: the CTA's abort word can be raised at any
+// moment (by the producer or by a consumer whose wait gave up), and consumers
+// that read it at different moments would otherwise split, some leaving while
+// the rest wait forever at the next consumer barrier.
+__device__ __forceinline__ bool consumer_sync_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, o;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.or.pred o, 1, %2, a;\n\t"
+      "selp.u32 %0, 1, 0, o;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kConsumerThreads)
+      : "memory");
+  return r != 0;
+}
 // Release all prior writes of this CTA (ordered by a preceding consumer_sync)
 // and add `v` to a gpu-scope counter.
 __device__ __forceinline__ unsigned release_add(unsigned* p, unsigned v) {
@@ -301,6 +319,18 @@ __device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint3
   }
 }
 
+// Wait for a bulk copy's barrier phase regardless of the abort state.  Copies
+// only read device memory and always complete; the bound (at least 2 s,
+// independent of the dependency-wait limit) only guards against a device that
+// stopped making progress.
+__device__ __noinline__ void copy_wait(const Params& p, uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  const long long limit = p.spin_limit_ns > 2000000000LL ? p.spin_limit_ns : 2000000000LL;
+  while (!mbar_try_wait_suspend(bar, parity, 20000u)) {
+    if (static_cast<long long>(globaltimer() - t0) > limit) break;
+  }
+}
+
 __device__ __forceinline__ bool ring_wait(const Params& p, SmemCtl* ctl, uint32_t bar,
                                           uint32_t parity, int where) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -346,8 +376,7 @@ __device__ __forceinline__ bool stage_wait(const Params& p, Ctx& cx, const unsig
     if (fused && !counter_wait(p, cx.ctl, cnt, target, where)) cx.ctl->abort = 1;
     trace_stamp(p, s, stage_index(p, kind, l), 1);
   }
-  consumer_sync();
-  return !cx.ctl->abort;
+  return !consumer_sync_any(cx.ctl->abort != 0);
 }
 
 // ------------------------------------------------------------------ math
@@ -450,6 +479,8 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
       bulk_g2s_nohint(smem_addr(cx.act), gsrc, bytes, bar);
     }
     if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+    // even when aborting, the copy must land before the CTA may exit
+    if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
     cx.act_phase ^= 1u;
   }
   if (hidden_dbg) {
@@ -538,7 +569,10 @@ __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m
         }
       }
       __syncwarp();
-      if (cx.lane == 0) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
+      // Release the slot only after its copy landed: an aborting consumer
+      // stops releasing, so the producer never refills a slot whose copy may
+      // still be in flight (it notices the abort at its next wait).
+      if (cx.lane == 0 && ok) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
       rp.next(p.nslot);
     }
     if (cx.warp < gp) {
@@ -793,7 +827,9 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     const int n_old = min(t_lo + P, T - 1) - t_lo; // positions already in the cache before this step
     const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
     const unsigned long long tw0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
-    const bool have_tile = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
+    // warp-uniform: the tile body below is warp-collective (ldmatrix, mma, shuffles)
+    const bool have_tile =
+        __all_sync(0xffffffffu, cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where));
     if (p.trace && cx.tid == 0) t_wait += globaltimer() - tw0;
     const uint32_t kt = ring_s + rp.slot * kSlotBytes;
     const uint32_t vt = kt + kSlotBytes / 2;
@@ -815,6 +851,22 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
           asm volatile("st.shared.u32 [%0], %1;" ::"r"(va), "r"(vv) : "memory");
         }
         // the slot is refilled by the async proxy later
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
+      if (npos < pg * 16 + 16) {
+        // Rows past the sequence end hold whatever the cache has there; their
+        // softmax weight is 0, but 0 * (inf or NaN) is not, so zero this warp's
+        // share of those V rows before they enter P V.
+        constexpr int UPR = DW / 8;                       // 16-byte units per row of this warp's dims
+        const int r0 = npos;
+        for (int u = cx.lane; u < 16 * UPR; u += 32) {
+          const int r = pg * 16 + u / UPR;
+          if (r >= r0) {
+            const uint32_t a = sw128_addr(vt, P, r, ds * DW + (u % UPR) * 8);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+          }
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
       }
@@ -871,7 +923,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       }
     }
     __syncwarp();
-    if (cx.lane == 0) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
+    if (cx.lane == 0 && have_tile) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
     rp.next(p.nslot);
     // end of a (b, g) segment: merge the 8 warps into this CTA's partial, and
     // let the CTA that completes the head combine every contributor's partial.
@@ -1023,9 +1075,9 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   const int where = where_code(kind, l, s);
   if (kind == ST_ATTN) {
     consume_attn<B, D>(p, cx, l, s, rp, fused);
-    consumer_sync();
+    const bool ab = consumer_sync_any(cx.ctl->abort != 0);
     if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
-    return !cx.ctl->abort;
+    return !ab;
   }
   if (kind == ST_LM) {
     if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused)) return false;
@@ -1084,9 +1136,9 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       consumer_sync();
       if (cx.tid == 0) release_add(p.cnt + p.cl.step_done, 1u);
     }
-    consumer_sync();
+    const bool ab = consumer_sync_any(cx.ctl->abort != 0);
     if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
-    return !cx.ctl->abort;
+    return !ab;
   }
   const LayerParams& L = p.layers[l];
   bool ok = true;
@@ -1136,12 +1188,13 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   // KV entries written by the QKV epilogue are read by later steps through
   // the async proxy (bulk copies): order this thread's generic writes first.
   if (kind == ST_QKV) fence_proxy_async_global();
-  consumer_sync();
+  const bool ab = consumer_sync_any(cx.ctl->abort != 0);
   if (cx.tid == 0) {
     trace_stamp(p, s, stage_index(p, kind, l), 3);
-    release_add(p.cnt + l * ST_LAYER + kind, 1u);
+    const bool dropped = p.fault_drop_stage == stage_index(p, kind, l) && cx.c == 0 && s == 0;
+    if (!dropped) release_add(p.cnt + l * ST_LAYER + kind, 1u);
   }
-  return !cx.ctl->abort;
+  return !ab;
 }
 
 // ------------------------------------------------------------------ kernels
@@ -1160,6 +1213,16 @@ __device__ __forceinline__ Ctx make_ctx(uint8_t* smem, const Params& p) {
 }
 
 __device__ __forceinline__ void init_ring(const Params& p, Ctx& cx) {
+#ifdef XLPK_DEBUG_POISON
+  // Debug build: fill the ring and the activation region with NaN bit
+  // patterns so that a read of shared memory nobody wrote shows up as NaN.
+  {
+    uint32_t* w = reinterpret_cast<uint32_t*>(cx.ring);
+    const int n = (p.nslot * kSlotBytes + p.act_bytes) >> 2;
+    for (int i = cx.tid; i < n; i += kThreads) w[i] = 0xffffffffu;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+#endif
   if (cx.tid == 0) {
     for (int i = 0; i < p.nslot; ++i) {
       mbar_init(smem_addr(&cx.ctl->full[i]), 1);
@@ -1187,15 +1250,7 @@ __device__ void drain_ring(const Params& p, Ctx& cx, const RingPos& rp, int issu
     } else {
       --q.slot;
     }
-    const uint32_t fb = smem_addr(&cx.ctl->full[q.slot]);
-    const uint64_t t0 = globaltimer();
-    // Copies only read device memory and always complete; the bound (at least
-    // 2 s, independent of the dependency-wait limit) only guards against a
-    // device that stopped making progress.
-    const long long limit = p.spin_limit_ns > 2000000000LL ? p.spin_limit_ns : 2000000000LL;
-    while (!mbar_try_wait_suspend(fb, q.phase, 20000u)) {
-      if (static_cast<long long>(globaltimer() - t0) > limit) break;
-    }
+    copy_wait(p, smem_addr(&cx.ctl->full[q.slot]), q.phase);
   }
 }
 
@@ -1207,6 +1262,7 @@ __device__ void drain_ring(const Params& p, Ctx& cx, const RingPos& rp, int issu
 struct Tile {
   const uint8_t* src;   // GEMV: packed tile
   int y;                // attention: first cache row of the chunk (tensor-map row)
+  int rows;             // attention: positions of the chunk that exist (<= chunk size)
   uint32_t bytes;       // bytes landing in the slot
   bool attn;
   int stage;            // stage_index
@@ -1286,6 +1342,7 @@ __device__ bool cursor_next(const Params& p, int c, Cursor<B>& cu, Tile& t) {
         attn_item<B>(p, cu.ap, cu.a, b, g, j, nch, base);
         ++cu.a;
         t.y = static_cast<int>(kv_row(p, cu.l, b, g, j * p.attn_pos_per_tile) / p.d);
+        t.rows = min(p.attn_pos_per_tile, p.pos0[b] + cu.s + 1 - j * p.attn_pos_per_tile);
         t.src = nullptr;
         t.bytes = kSlotBytes;
         t.attn = true;
@@ -1333,7 +1390,16 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
     while (pc_live && ahead < p.l2_prefetch_bytes) {
       pc_live = cursor_next<B>(p, cx.c, pc, tp);
       if (!pc_live) break;
-      if (!tp.attn) prefetch_l2(tp.src, tp.bytes);
+      if (!tp.attn) {
+        prefetch_l2(tp.src, tp.bytes);
+      } else {
+        // the chunk's existing K and V rows (contiguous, 16-byte multiples);
+        // L2 is the coherence point, so a row rewritten later is still read fresh
+        const size_t off = static_cast<size_t>(tp.y) * p.d;
+        const uint32_t nb = static_cast<uint32_t>(tp.rows) * p.d * 2u;
+        prefetch_l2(p.kc + off, nb);
+        prefetch_l2(p.vc + off, nb);
+      }
       ahead += tp.bytes;
     }
     if (t.stage != cur_stage || t.step != cur_step) {

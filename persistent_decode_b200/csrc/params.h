@@ -124,6 +124,8 @@ struct Params {
   float* logits_out;
   float* hidden_out;
   unsigned long long* trace;   // optional stage timestamps
+  int fault_drop_stage;        // failure-detection tests: CTA 0 withholds its release of this
+                               // stage index at the call's first step (-1: never)
 };
 
 }  // namespace xlpk

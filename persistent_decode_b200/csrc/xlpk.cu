@@ -318,6 +318,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const xlpk_config& c = *cfg;
   e->cfg = c;
   XLPK_CUDA(cudaGetDevice(&e->device));
+  // The weights may still be in flight on any stream of the caller (the
+  // packing below runs on a stream of its own that does not wait for them):
+  // finish all enqueued work on the device first.
+  XLPK_CUDA(cudaDeviceSynchronize());
   cudaDeviceProp prop;
   XLPK_CUDA(cudaGetDeviceProperties(&prop, e->device));
   if (prop.major != 10) {
@@ -382,6 +386,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   total += align_up(sizeof(float) * H * (2 * static_cast<size_t>(c.n_layers) + 1), 256);
   e->packed_bytes = total;
   XLPK_CUDA(cudaMalloc(&e->packed, total));
+#ifdef XLPK_DEBUG_POISON
+  XLPK_CUDA(cudaMemset(e->packed, 0xff, total));   // debug build: unwritten bytes read as NaN
+#endif
   e->weight_bytes_per_step = 0;
   for (const MatPlan& m : mats) e->weight_bytes_per_step += static_cast<int64_t>(m.N) * m.K * e->esz;
 
@@ -467,6 +474,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->ws_bytes = off;
   XLPK_CUDA(cudaMalloc(&e->ws, e->ws_bytes));
   XLPK_CUDA(cudaMemset(e->ws, 0, e->ws_bytes));
+#ifdef XLPK_DEBUG_POISON
+  // debug build: scratch that every step must write before reading it holds NaN
+  XLPK_CUDA(cudaMemset(e->ws + o_x, 0xff, o_lv - o_x));
+#endif
 
   Params& p = e->base;
   p.L = c.n_layers;
@@ -487,12 +498,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.act_bytes = e->act_bytes;
   p.attn_pos_per_tile = e->P;
   p.spin_limit_ns = 1000LL * (c.spin_limit_us > 0 ? c.spin_limit_us : 200000);
-  {
-    // L2 prefetch distance per CTA (tuning knob; 0 disables)
-    long long kb = 256;
-    if (const char* env = std::getenv("XLPK_L2_PREFETCH_KB")) kb = std::atoll(env);
-    p.l2_prefetch_bytes = kb * 1024;
-  }
+  p.l2_prefetch_bytes = 256 * 1024;
   p.cl = cl;
   p.embed = embed_copy;
   p.final_norm = final_norm_copy;
@@ -545,6 +551,13 @@ Params call_params(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out, const x
   p.logits_out = io ? io->logits_dev : nullptr;
   p.hidden_out = io ? io->hidden_dev : nullptr;
   p.trace = io ? reinterpret_cast<unsigned long long*>(io->trace_dev) : nullptr;
+  // L2 prefetch distance per CTA: a tuning knob read at each call (0 disables)
+  if (const char* env = std::getenv("XLPK_L2_PREFETCH_KB")) p.l2_prefetch_bytes = std::atoll(env) * 1024;
+  // Failure-detection tests: make one dependency wait run out (a release that
+  // never happens) so the time limit, the abort path and the status report
+  // are exercised without faulting anything.
+  p.fault_drop_stage = -1;
+  if (const char* env = std::getenv("XLPK_FAULT_DROP_RELEASE")) p.fault_drop_stage = std::atoi(env);
   return p;
 }
 

@@ -85,6 +85,20 @@ def test_tiny_batched_with_gains(cuda_device, batch):
     compare_with_oracle(m, run, oracle_for(m), cfg.steps)
 
 
+def test_cache_tail_garbage_is_ignored(cuda_device):
+    # positions at and beyond the current length are not part of the sequence:
+    # fill them with NaN (what an uninitialised cache may hold) and the decode
+    # must be unaffected, since each step writes its position before reading it
+    cfg = synth.get_config("tiny", steps=10)
+    m = workload.build(cfg, device=cuda_device)
+    T = cfg.kv_len
+    m.k[:, :, :, T:] = float("nan")
+    m.v[:, :, :, T:] = float("nan")
+    run = run_engine(m, cfg.steps)
+    assert bool(torch.isfinite(run.hidden).all())
+    compare_with_oracle(m, run, oracle_for(m), cfg.steps)
+
+
 def test_tiny_ragged_grid(cuda_device):
     # a grid size that divides nothing evenly: every stage gets ragged CTA spans
     cfg = synth.get_config("tiny", steps=6)
