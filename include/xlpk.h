@@ -126,11 +126,14 @@ typedef struct xlpk_decode_io {
   float* logits_dev;                  /* [n_steps][B][V] fp32 logits of every step */
   float* hidden_dev;                  /* [n_steps][B][H] fp32 residual after the last layer */
   int32_t* experts_dev;               /* MoE: [n_steps][L][B][top_k] selected expert ids */
-  uint64_t* trace_dev;                /* [n_steps][n_stages][n_ctas][8] globaltimer stamps (ns) per
-                                         stage and CTA: consumer entry, dependency met, activation
-                                         staged, consumer done, producer first copy, producer last
-                                         copy; attention stages also record the total ns spent
-                                         waiting for KV chunks [6] and merging partials [7];
+  uint64_t* trace_dev;                /* [n_steps][n_stages][n_ctas][16] globaltimer stamps (ns) per
+                                         stage and CTA: [0] consumer entry, [1] dependency met,
+                                         [2] inputs staged, [3] consumer done, [4] producer first
+                                         copy, [5] producer last copy.  Attention stages also record
+                                         totals of thread 0: [6] ns waiting for KV chunks, [7] ns
+                                         from the end of the chunks to leaving (merge, arrive,
+                                         combine), [8] q loads, [9] chunk math, [10] merge,
+                                         [11] arrive, [12] combine, [13] chunks processed.
                                          n_stages = 5 * n_layers + 1 */
 } xlpk_decode_io;
 

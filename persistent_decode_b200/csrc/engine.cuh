@@ -247,8 +247,10 @@ struct alignas(16) SmemCtl {
   volatile int abort;
   int flag;
   int pad[2];
-  float red[kConsumerWarps][kMaxBatch];
-  int redi[kConsumerWarps][kMaxBatch];
+  float red[kConsumerWarps][kMaxBatch];    // RMSNorm partial sums
+  float redv[kConsumerWarps][kMaxBatch];   // LM-head argmax values
+  int redi[kConsumerWarps][kMaxBatch];     // LM-head argmax indices
+  unsigned long long tacc[8];              // attention trace totals (thread 0)
 };
 static_assert(sizeof(SmemCtl) <= kMiscSmem, "control block too large");
 
@@ -266,6 +268,7 @@ struct RingPos {
 struct Ctx {
   uint8_t* ring;
   float* act;
+  uint8_t* side;       // epilogue side data (RoPE rows, residual / embedding slices)
   SmemCtl* ctl;
   int c;
   int warp;
@@ -292,7 +295,7 @@ __device__ __forceinline__ int where_code(int kind, int layer, int step) {
 __device__ __forceinline__ void trace_stamp(const Params& p, int s, int si, int k) {
   if (p.trace) {
     const size_t n_st = static_cast<size_t>(p.L) * ST_LAYER + 1;
-    p.trace[((static_cast<size_t>(s) * n_st + si) * p.G + blockIdx.x) * 8 + k] = globaltimer();
+    p.trace[((static_cast<size_t>(s) * n_st + si) * p.G + blockIdx.x) * kTraceSlots + k] = globaltimer();
   }
 }
 __device__ __forceinline__ int stage_index(const Params& p, int kind, int l) {
@@ -302,16 +305,18 @@ __device__ __forceinline__ int stage_index(const Params& p, int kind, int l) {
 // Bounded wait on a ring barrier phase.  Returns false (and marks the CTA
 // aborted) if the global abort flag is raised or the time limit passes.
 __device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint32_t bar,
-                                            uint32_t parity, int where) {
+                                            uint32_t parity, int where, int limit_mult = 1) {
   const uint64_t t0 = globaltimer();
+  const long long limit = p.spin_limit_ns * limit_mult;
   for (;;) {
-    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    if (p.wait_hint_ns ? mbar_try_wait_suspend(bar, parity, p.wait_hint_ns) : mbar_try_wait(bar, parity))
+      return true;
     if (ctl->abort) return false;
     if (ld_volatile(p.abort_flag)) {
       ctl->abort = 1;
       return false;
     }
-    if (static_cast<long long>(globaltimer() - t0) > p.spin_limit_ns) {
+    if (static_cast<long long>(globaltimer() - t0) > limit) {
       raise_error(p, kErrTimeout, where);
       ctl->abort = 1;
       return false;
@@ -326,7 +331,7 @@ __device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint3
 __device__ __noinline__ void copy_wait(const Params& p, uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   const long long limit = p.spin_limit_ns > 2000000000LL ? p.spin_limit_ns : 2000000000LL;
-  while (!mbar_try_wait_suspend(bar, parity, 20000u)) {
+  while (!(p.wait_hint_ns ? mbar_try_wait_suspend(bar, parity, p.wait_hint_ns) : mbar_try_wait(bar, parity))) {
     if (static_cast<long long>(globaltimer() - t0) > limit) break;
   }
 }
@@ -429,18 +434,82 @@ __host__ __device__ __forceinline__ size_t plane_index(int b, int k, int B, int 
 
 enum ActSrc : int { SRC_RESID = 0, SRC_EMBED = 1, SRC_PLAIN = 2 };
 
-// Stage the input vector in shared memory.  A residual / plain source (two-plane
-// layout in global memory, written by other CTAs in an earlier stage) arrives
-// as one bulk copy issued right after the dependency wait; the embedding row
-// of layer 0 (bf16) is converted by the threads.  With `gain`, RMSNorm is
-// applied in place: v * rsqrt(mean(v^2) + eps) * gain.  `hidden_dbg` (LM
-// stage, CTA 0) receives the raw residual in natural [B][K] order.
+// What the stage's epilogue reads besides its GEMV sums, staged in the CTA's
+// side region by the same bulk-copy phase as the input vector, so that no
+// epilogue waits on a global load of its own:
+//   SIDE_ROPE   cos/sin of this step's position per sequence (QKV)
+//   SIDE_RESID  this CTA's rows of the residual x (O-projection, down)
+//   SIDE_EMBED  this CTA's rows of the pending tokens' embeddings (layer-0 O-projection)
+enum SideKind : int { SIDE_NONE = 0, SIDE_ROPE = 1, SIDE_RESID = 2, SIDE_EMBED = 3 };
+
+// Row range [r0, r1) of this CTA in a stage whose matrix has H logical rows.
+__device__ __forceinline__ void resid_rows(const Params& p, int c, int& r0, int& r1) {
+  r0 = 2 * split_point(c, p.H >> 1, p.G);
+  r1 = 2 * split_point(c + 1, p.H >> 1, p.G);
+}
+
+// Stage the input vector and the epilogue's side data in shared memory.  A
+// residual / plain source (two-plane layout in global memory, written by other
+// CTAs in an earlier stage), the RMSNorm gains and the side data arrive by
+// bulk copies on one barrier phase issued right after the dependency wait; the
+// embedding rows of layer 0 (bf16) are converted by the threads meanwhile.
+// With `gain`, RMSNorm is split: one pass forms v * gain in place and the sum
+// of squares; rn[b] = rsqrt(mean(v^2) + eps) is applied to the GEMV sums
+// (W (g v) r = W (r g v)), so the stage needs a single consumer barrier.
+// `hidden_dbg` (LM stage, CTA 0) receives the raw residual in natural [B][K] order.
 template <int B>
 __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const float* gsrc,
-                                      const float* gain, float* hidden_dbg, int where) {
+                                      const float* gain, float* hidden_dbg, int side, int s,
+                                      float (&rn)[B], int where) {
   const int nvK = K >> 3;
   const int n4 = K >> 2;
   float4* act4 = reinterpret_cast<float4*>(cx.act);
+  const uint32_t bar = smem_addr(&cx.ctl->act_bar);
+  const uint32_t gain_s = smem_addr(cx.act + static_cast<size_t>(B) * K);
+  if (cx.tid == 0) {
+    // order the other CTAs' global writes (acquired) and this CTA's earlier
+    // shared-memory accesses before the async-proxy copies
+    asm volatile("fence.proxy.async;" ::: "memory");
+    const uint32_t side_s = smem_addr(cx.side);
+    int r0 = 0, r1 = 0;
+    if (side == SIDE_RESID || side == SIDE_EMBED) resid_rows(p, cx.c, r0, r1);
+    int tok[B];
+    if (side == SIDE_EMBED)
+#pragma unroll
+      for (int b = 0; b < B; ++b) tok[b] = __ldcg(p.cur_tok + b);
+    // total bytes of this phase
+    uint32_t total = 0;
+    if (src != SRC_EMBED) total += static_cast<uint32_t>(B) * K * 4u;
+    if (gain) total += static_cast<uint32_t>(K) * 4u;
+    const uint32_t rope_bytes = static_cast<uint32_t>(p.d) * 4u;   // d/2 (cos, sin) pairs
+    const int v0 = r0 >> 3, nv = r1 > r0 ? ((r1 - 1) >> 3) - v0 + 1 : 0;
+    const int e0 = r0 & ~7, e1 = (r1 + 7) & ~7;
+    if (side == SIDE_ROPE) total += B * rope_bytes;
+    if (side == SIDE_RESID) total += static_cast<uint32_t>(B) * 2u * nv * 16u;
+    if (side == SIDE_EMBED && r1 > r0) total += static_cast<uint32_t>(B) * (e1 - e0) * 2u;
+    mbar_expect_tx(bar, total);
+    if (src != SRC_EMBED) bulk_g2s_nohint(smem_addr(cx.act), gsrc, static_cast<uint32_t>(B) * K * 4u, bar);
+    if (gain) bulk_g2s_nohint(gain_s, gain, static_cast<uint32_t>(K) * 4u, bar);
+    if (side == SIDE_ROPE) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        bulk_g2s_nohint(side_s + p.side_rope + b * rope_bytes,
+                        p.rope + static_cast<size_t>(p.pos0[b] + s) * (p.d >> 1), rope_bytes, bar);
+    } else if (side == SIDE_RESID && nv > 0) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        for (int pl = 0; pl < 2; ++pl)
+          bulk_g2s_nohint(side_s + p.side_resid + ((b * 2 + pl) * p.nvr) * 16,
+                          p.x + ((static_cast<size_t>(pl) * p.B + b) * (p.H >> 3) + v0) * 4,
+                          static_cast<uint32_t>(nv) * 16u, bar);
+    } else if (side == SIDE_EMBED && r1 > r0) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        bulk_g2s_nohint(side_s + p.side_embed + b * p.evb,
+                        p.embed + static_cast<size_t>(tok[b]) * p.H + e0,
+                        static_cast<uint32_t>(e1 - e0) * 2u, bar);
+    }
+  }
   if (src == SRC_EMBED) {
     int tok[B];
 #pragma unroll
@@ -464,67 +533,52 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
                 make_float4(bf16_lo(e[u][b].x), bf16_hi(e[u][b].x), bf16_lo(e[u][b].y), bf16_hi(e[u][b].y));
         }
     }
-  } else {
-    const uint32_t bar = smem_addr(&cx.ctl->act_bar);
-    if (gain) {   // warm this SM's L1 with the gains while the copy is in flight
-      for (int q = cx.tid; q < n4; q += kConsumerThreads)
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(gain + 4 * q));
-    }
-    if (cx.tid == 0) {
-      // order the other CTAs' global writes (acquired) and this CTA's earlier
-      // shared-memory accesses before the async-proxy copy
-      asm volatile("fence.proxy.async;" ::: "memory");
-      const uint32_t bytes = static_cast<uint32_t>(B) * K * 4u;
-      mbar_expect_tx(bar, bytes);
-      bulk_g2s_nohint(smem_addr(cx.act), gsrc, bytes, bar);
-    }
-    if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
-    // even when aborting, the copy must land before the CTA may exit
-    if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
-    cx.act_phase ^= 1u;
   }
+  if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+  // even when aborting, the copies must land before the CTA may exit
+  if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
+  cx.act_phase ^= 1u;
   if (hidden_dbg) {
     if (src == SRC_EMBED) consumer_sync();
     for (int k = cx.tid; k < K; k += kConsumerThreads)
 #pragma unroll
       for (int b = 0; b < B; ++b) hidden_dbg[static_cast<size_t>(b) * K + k] = cx.act[plane_index(b, k, B, K)];
+    consumer_sync();   // the pass below rewrites the vector in place
   }
+#pragma unroll
+  for (int b = 0; b < B; ++b) rn[b] = 1.f;
   if (gain) {
-    if (src == SRC_EMBED) consumer_sync();
+    // each thread rewrites exactly the float4s it converted above (same q), so
+    // the embedding path needs no barrier before this pass
     float ss[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) ss[b] = 0.f;
-    for (int q = cx.tid; q < n4; q += kConsumerThreads)
+    for (int q = cx.tid; q < n4; q += kConsumerThreads) {
+      const float4 g4 = lds_f4(gain_s + q * 16);
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        const float4 x = act4[((q & 1) * B + b) * nvK + (q >> 1)];
+        float4& a = act4[((q & 1) * B + b) * nvK + (q >> 1)];
+        const float4 x = a;
         ss[b] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ss[b]))));
+        a = make_float4(x.x * g4.x, x.y * g4.y, x.z * g4.z, x.w * g4.w);
       }
+    }
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       const float t = warp_sum(ss[b]);
       if (cx.lane == 0) cx.ctl->red[cx.warp][b] = t;
     }
     consumer_sync();
-    float r[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       float t = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) t += cx.ctl->red[w][b];
-      r[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
+      rn[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
     }
-    for (int q = cx.tid; q < n4; q += kConsumerThreads) {
-      const float4 g4 = __ldg(reinterpret_cast<const float4*>(gain) + q);
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        float4& a = act4[((q & 1) * B + b) * nvK + (q >> 1)];
-        const float rb = r[b];
-        a = make_float4(a.x * rb * g4.x, a.y * rb * g4.y, a.z * rb * g4.z, a.w * rb * g4.w);
-      }
-    }
+  } else if (src == SRC_EMBED) {
+    consumer_sync();
   }
-  consumer_sync();
 }
 
 // ------------------------------------------------------------------ GEMV stages
@@ -534,7 +588,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
 // the reduced sums (identical in every lane).
 template <int B, class Epi>
 __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp,
-                                          int where, Epi& epi) {
+                                          int where, const float (&rn)[B], Epi& epi) {
   const int NP = m.N >> 1;
   const int p0 = split_point(cx.c, NP, p.G), p1 = split_point(cx.c + 1, NP, p.G);
   const int nkc = m.K / m.KC;
@@ -578,8 +632,8 @@ __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m
     if (cx.warp < gp) {
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        a0[b] = warp_sum(a0[b]);
-        a1[b] = warp_sum(a1[b]);
+        a0[b] = warp_sum(a0[b]) * rn[b];
+        a1[b] = warp_sum(a1[b]) * rn[b];
       }
       epi(g0 + cx.warp, a0, a1, cx.lane);
     }
@@ -587,10 +641,12 @@ __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m
 }
 
 // QKV epilogue: RoPE on q/k pairs, q -> workspace, bf16 k/v -> cache at pos.
+// The step's cos/sin rows were staged in shared memory (SIDE_ROPE).
 template <int B>
 struct EpiQKV {
   const Params& p;
   int l, s;
+  const float2* rope_s;   // [B][d/2]
   __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
     const int half = p.d >> 1;
     const int hq = p.nq * half, hk = p.nkv * half;
@@ -603,7 +659,7 @@ struct EpiQKV {
         const bool isq = pg < hq;
         const int pp = isq ? pg : pg - hq;
         const int head = pp / half, i = pp - head * half;
-        const float2 cs = __ldg(p.rope + static_cast<size_t>(pos) * half + i);
+        const float2 cs = rope_s[b * half + i];
         const float y0 = r0 * cs.x - r1 * cs.y;
         const float y1 = r0 * cs.y + r1 * cs.x;
         if (isq) {
@@ -628,23 +684,30 @@ struct EpiQKV {
   }
 };
 
-// Residual epilogue: x[b][2pg..2pg+1] += (r0, r1); with `embed_base`, x = E[tok] + r.
+// Residual epilogue: x[b][2pg..2pg+1] += (r0, r1); with `from_embed`, x = E[tok] + r.
+// The CTA's rows of x (SIDE_RESID) or of the embedding rows (SIDE_EMBED) were
+// staged in shared memory: vectors from v0 of each plane, embedding elements
+// from e0.
 template <int B>
 struct EpiResid {
   const Params& p;
   bool from_embed;
+  const uint8_t* side;
+  int v0, e0;
   __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       if (lane != b) continue;
-      float2* xp = reinterpret_cast<float2*>(p.x + plane_index(b, 2 * pg, p.B, p.H));
+      const int r = 2 * pg;
+      float2* xp = reinterpret_cast<float2*>(p.x + plane_index(b, r, p.B, p.H));
       float2 base;
       if (from_embed) {
-        const int tok = __ldcg(p.cur_tok + b);
-        const uint32_t e = *reinterpret_cast<const uint32_t*>(p.embed + static_cast<size_t>(tok) * p.H + 2 * pg);
+        const uint32_t e =
+            *reinterpret_cast<const uint32_t*>(side + p.side_embed + b * p.evb + (r - e0) * 2);
         base = make_float2(bf16_lo(e), bf16_hi(e));
       } else {
-        base = __ldcg(xp);
+        const float* rs = reinterpret_cast<const float*>(side + p.side_resid);
+        base = *reinterpret_cast<const float2*>(rs + ((b * 2 + ((r >> 2) & 1)) * p.nvr + (r >> 3) - v0) * 4 + (r & 3));
       }
       *xp = make_float2(base.x + a0[b], base.y + a1[b]);
     }
@@ -713,6 +776,47 @@ __device__ __forceinline__ void attn_plan(const Params& p, int s, AttnPlan<B>& a
   ap.W = w;
 }
 
+// Which CTAs work on which chunks.  With at least one CTA per (sequence, kv
+// head), each head gets its own contiguous range of CTAs (head h: CTAs
+// [h*G/NH, (h+1)*G/NH)) and its chunks are split evenly over them, so no CTA
+// straddles two heads: each CTA loads one q, merges once and arrives once.
+// With fewer CTAs than heads the chunks of all heads are split evenly over
+// the CTAs in (b, g, j) order, and a CTA may span several heads.
+__device__ __forceinline__ bool attn_aligned(const Params& p) { return p.G >= p.B * p.nkv; }
+
+// CTA range [c0, c0 + nc) of head (b, g) in the aligned split.
+__device__ __forceinline__ void attn_head_ctas(const Params& p, int b, int g, int& c0, int& nc) {
+  const int NH = p.B * p.nkv, h = b * p.nkv + g;
+  c0 = split_point(h, p.G, NH);
+  nc = split_point(h + 1, p.G, NH) - c0;
+}
+
+// Item range [i0, i1) of CTA c (items numbered (b, g, j) in that order).
+template <int B>
+__device__ __forceinline__ void attn_cta_items(const Params& p, const AttnPlan<B>& ap, int c, int& i0,
+                                               int& i1) {
+  if (!attn_aligned(p)) {
+    i0 = split_point(c, ap.W, p.G);
+    i1 = split_point(c + 1, ap.W, p.G);
+    return;
+  }
+  const int NH = p.B * p.nkv;
+  const int h = split_owner(c, p.G, NH);   // the head whose CTA range holds c
+  const int b = h / p.nkv, g = h - b * p.nkv;
+  int c0, nc;
+  attn_head_ctas(p, b, g, c0, nc);
+  int nch = ap.nch[0], base = ap.base[0];
+#pragma unroll
+  for (int bb = 1; bb < B; ++bb)
+    if (bb == b) {
+      nch = ap.nch[bb];
+      base = ap.base[bb];
+    }
+  const int hb = base + g * nch;
+  i0 = hb + split_point(c - c0, nch, nc);
+  i1 = hb + split_point(c - c0 + 1, nch, nc);
+}
+
 template <int B>
 __device__ __forceinline__ void attn_item(const Params& p, const AttnPlan<B>& ap, int i, int& b,
                                           int& g, int& j, int& nch, int& base) {
@@ -770,7 +874,8 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
   static_assert(NPG * NDS == kConsumerWarps && NT % 2 == 0, "chunk shape");
   AttnPlan<B> ap;
   attn_plan<B>(p, s, ap);
-  const int i0 = split_point(cx.c, ap.W, p.G), i1 = split_point(cx.c + 1, ap.W, p.G);
+  int i0, i1;
+  attn_cta_items<B>(p, ap, cx.c, i0, i1);
   const int where = where_code(ST_ATTN, l, s);
   const unsigned S1 = static_cast<unsigned>(p.step_base + s + 1);
   if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_QKV, static_cast<unsigned>(p.G) * S1, where, fused))
@@ -783,14 +888,18 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
   const int mi = cx.lane >> 3, rr = cx.lane & 7;             // ldmatrix: matrix / row of this lane
   float* sm_ml = cx.act;                                      // [8 warps][4 heads][2]
   float* sm_o = sm_ml + kConsumerWarps * kMaxGroup * 2;       // [8 warps][4 heads][DW]
-  float* cb = sm_o + kConsumerWarps * kMaxGroup * DW;         // combine scratch
   const uint32_t ring_s = smem_addr(cx.ring);
 
   uint32_t qa0[KS], qa2[KS], qb0[KS], qb2[KS];   // q as bf16 hi (a) + lo (b) parts
   float o[NT][4];
   float m_h = -INFINITY, l_h = 0.f;                          // softmax state of head gid
   int seg_b = -1, seg_g = -1, seg_items = 0, seg_nch = 0, seg_base = 0;
-  unsigned long long t_wait = 0, t_merge = 0;                 // trace only (thread 0)
+  // trace only (thread 0, kept in shared memory to spare registers): ns in
+  // ring waits, from the end of the chunks to leaving, q loads, chunk math,
+  // merge, arrive, combine; chunks processed
+  unsigned long long* ta = cx.ctl->tacc;
+  if (p.trace && cx.tid == 0)
+    for (int k = 0; k < 8; ++k) ta[k] = 0;
 
   for (int i = i0; i < i1; ++i) {
     int b, g, j, nch, base;
@@ -805,6 +914,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       l_h = 0.f;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+      const unsigned long long tq0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
       if (gid < GQ) {
         const float* qs = p.q + (static_cast<size_t>(b) * p.nq + g * GQ + gid) * D;
         const float sc = p.qk_scale_log2;
@@ -819,6 +929,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) qa0[ks] = qa2[ks] = qb0[ks] = qb2[ks] = 0u;
       }
+      if (p.trace && cx.tid == 0) ta[2] += globaltimer() - tq0;
     }
     ++seg_items;
     const int T = p.pos0[b] + s + 1;
@@ -830,7 +941,11 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     // warp-uniform: the tile body below is warp-collective (ldmatrix, mma, shuffles)
     const bool have_tile =
         __all_sync(0xffffffffu, cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where));
-    if (p.trace && cx.tid == 0) t_wait += globaltimer() - tw0;
+    if (p.trace && cx.tid == 0) {
+      ta[0] += globaltimer() - tw0;
+      ++ta[7];
+    }
+    const unsigned long long tc0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
     const uint32_t kt = ring_s + rp.slot * kSlotBytes;
     const uint32_t vt = kt + kSlotBytes / 2;
     if (have_tile && pg * 16 < npos) {   // warp-uniform
@@ -871,6 +986,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
         __syncwarp();
       }
       // ---- S = Q K^T for positions pg*16 .. pg*16+15
+      // (two accumulator chains: splitting them further measured slower)
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       const int kr = pg * 16 + ((mi >> 1) << 3) + rr;
 #pragma unroll
@@ -923,6 +1039,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       }
     }
     __syncwarp();
+    if (p.trace && cx.tid == 0) ta[3] += globaltimer() - tc0;
     if (cx.lane == 0 && have_tile) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
     rp.next(p.nslot);
     // end of a (b, g) segment: merge the 8 warps into this CTA's partial, and
@@ -932,7 +1049,14 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     if (i + 1 < i1 && i + 1 < ie) continue;   // the segment goes on
     const unsigned long long tm0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
 
-    const int c_first = split_owner(ib, ap.W, p.G);
+    // contributors of this head: CTAs c_first .. c_first + ncov - 1 (partial rows 0 .. ncov-1)
+    int c_first, ncov;
+    if (attn_aligned(p)) {
+      attn_head_ctas(p, seg_b, seg_g, c_first, ncov);
+    } else {
+      c_first = split_owner(ib, ap.W, p.G);
+      ncov = split_owner(ie - 1, ap.W, p.G) - c_first + 1;
+    }
     const size_t head_row = (static_cast<size_t>(seg_b) * p.nkv + seg_g) * p.G;   // partial rows of this head
     if (tig == 0 && gid < kMaxGroup) {   // lanes 4h hold head h's state
       sm_ml[(cx.warp * kMaxGroup + gid) * 2 + 0] = m_h;
@@ -970,8 +1094,11 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
           p.part_ml[(row * GQ + h) * 2 + 1] = Ls;
         }
       }
+      fence_proxy_async_global();   // the combiner may read the partials by bulk copy
     }
     consumer_sync();
+    const unsigned long long ta0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+    if (p.trace && cx.tid == 0) ta[4] += ta0 - tm0;
     unsigned* arrive = p.cnt + p.cl.attn_arrive + (l * p.B + seg_b) * p.nkv + seg_g;
     if (cx.tid == 0) {
       const unsigned old = release_add(arrive, static_cast<unsigned>(seg_items));
@@ -979,84 +1106,117 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       cx.ctl->flag = (old + seg_items == static_cast<unsigned>(seg_nch)) ? 1 : 0;
     }
     consumer_sync();
+    const unsigned long long tb0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+    if (p.trace && cx.tid == 0) ta[5] += tb0 - ta0;
     if (!cx.ctl->flag) {
-      if (p.trace && cx.tid == 0) t_merge += globaltimer() - tm0;
+      if (p.trace && cx.tid == 0) ta[1] += globaltimer() - tm0;
       continue;
     }
-    // ---- combine: contributors are CTAs c_first .. c_last (rows 0..ncov-1);
-    // a CTA in that range with no chunk of this head contributes nothing.
-    const int c_last = split_owner(ie - 1, ap.W, p.G);
-    const int ncov = c_last - c_first + 1;
-    float* cM = cb;                       // [ncov][GQ]
-    float* cL = cM + p.G * kMaxGroup;     // [ncov][GQ]
-    float* cW = cL + p.G * kMaxGroup;     // [ncov][GQ]
-    float* cS = cW + p.G * kMaxGroup;     // M*[GQ], L*[GQ]
-    for (int idx = cx.tid; idx < ncov * GQ; idx += kConsumerThreads) {
-      const int t = idx / GQ, h = idx - t * GQ;
-      const int cc = c_first + t;
-      const int lo = max(ib, split_point(cc, ap.W, p.G)), hi = min(ie, split_point(cc + 1, ap.W, p.G));
-      float M = -INFINITY, Lv = 0.f;
-      if (lo < hi) {
-        M = __ldcg(p.part_ml + ((head_row + t) * GQ + h) * 2);
-        Lv = __ldcg(p.part_ml + ((head_row + t) * GQ + h) * 2 + 1);
-      }
-      cM[t * kMaxGroup + h] = M;
-      cL[t * kMaxGroup + h] = Lv;
-    }
-    consumer_sync();
-    if (cx.warp < GQ) {
-      const int h = cx.warp;
-      float M = -INFINITY;
-      for (int t = cx.lane; t < ncov; t += 32) M = fmaxf(M, cM[t * kMaxGroup + h]);
+    // ---- combine: contributors are CTAs c_first .. c_first + ncov - 1 (rows
+    // 0..ncov-1); a CTA in that range with no chunk of this head contributes
+    // nothing.  Each thread owns 4 consecutive output dims of one query head
+    // and reads what it needs straight from L2 with independent loads: all
+    // contributors' maxima (one round trip), then their (max, sum) and output
+    // vectors (a second round trip); no shared scratch and no barrier.
+    // which of the ncov CTAs hold chunks of this head (32-bit arithmetic: the
+    // 64-bit division of split_point is far too slow for a per-contributor loop)
+    // (each lane decides for contributors lane, lane+32, ...; a ballot shares it)
+    uint32_t has_mask[(kMaxCtas + 31) / 32];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      float Lsum = 0.f;
-      for (int t = cx.lane; t < ncov; t += 32) {
-        const float mt = cM[t * kMaxGroup + h];
-        const float wgt = (mt == -INFINITY) ? 0.f : exp2f(mt - M);
-        cW[t * kMaxGroup + h] = wgt;
-        Lsum = fmaf(wgt, cL[t * kMaxGroup + h], Lsum);
+    for (int w = 0; w < (kMaxCtas + 31) / 32; ++w) {
+      const int t = w * 32 + cx.lane;
+      bool has = false;
+      if (t < ncov) {
+        if (attn_aligned(p)) {
+          has = seg_nch >= ncov || ((t + 1) * seg_nch) / ncov > (t * seg_nch) / ncov;
+        } else {
+          const int cc = c_first + t;
+          has = max(ib, (cc * ap.W) / p.G) < min(ie, ((cc + 1) * ap.W) / p.G);
+        }
       }
-      Lsum = warp_sum(Lsum);
-      if (cx.lane == 0) cS[kMaxGroup + h] = Lsum;
+      has_mask[w] = __ballot_sync(0xffffffffu, has);
     }
-    consumer_sync();
-    for (int idx = cx.tid; idx < GQ * D; idx += kConsumerThreads) {
-      const int h = idx / D, dd = idx - h * D;
-      const float* src = p.part_o + (head_row * GQ + h) * D + dd;
-      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-      int t = 0;
-      for (; t + 4 <= ncov; t += 4) {
-        const float w0 = cW[(t + 0) * kMaxGroup + h], w1 = cW[(t + 1) * kMaxGroup + h];
-        const float w2 = cW[(t + 2) * kMaxGroup + h], w3 = cW[(t + 3) * kMaxGroup + h];
-        const float o0 = w0 != 0.f ? __ldcg(src + static_cast<size_t>(t + 0) * GQ * D) : 0.f;
-        const float o1 = w1 != 0.f ? __ldcg(src + static_cast<size_t>(t + 1) * GQ * D) : 0.f;
-        const float o2 = w2 != 0.f ? __ldcg(src + static_cast<size_t>(t + 2) * GQ * D) : 0.f;
-        const float o3 = w3 != 0.f ? __ldcg(src + static_cast<size_t>(t + 3) * GQ * D) : 0.f;
-        acc0 = fmaf(w0, o0, acc0);
-        acc1 = fmaf(w1, o1, acc1);
-        acc2 = fmaf(w2, o2, acc2);
-        acc3 = fmaf(w3, o3, acc3);
+    // The head's partial rows are contiguous in the workspace: when they fit
+    // the scratch behind the merge buffers, one bulk copy brings them all in
+    // (one round trip); otherwise every thread reads its own from L2.
+    float* cp_ml = sm_o + kConsumerWarps * kMaxGroup * DW;     // [ncov][GQ][2]
+    float* cp_o = cp_ml + ncov * GQ * 2;                         // [ncov][GQ][D]
+    const uint32_t ml_bytes = static_cast<uint32_t>(ncov) * GQ * 2 * 4;
+    const uint32_t o_bytes = static_cast<uint32_t>(ncov) * GQ * D * 4;
+    // bulk copies need 16-byte aligned addresses and sizes: the (max, sum)
+    // block starts at head_row*GQ*8 bytes and is ncov*GQ*8 long
+    const bool staged = (cp_o - cx.act) * 4 + o_bytes <= static_cast<uint32_t>(p.act_bytes) &&
+                        ((ncov * GQ) & 1) == 0 && ((head_row * GQ) & 1) == 0;
+    const float* mlsrc = p.part_ml + head_row * GQ * 2;
+    const float* osrc = p.part_o + head_row * GQ * D;
+    if (staged) {
+      const uint32_t bar = smem_addr(&cx.ctl->act_bar);
+      if (cx.tid == 0) {
+        asm volatile("fence.proxy.async;" ::: "memory");
+        mbar_expect_tx(bar, ml_bytes + o_bytes);
+        bulk_g2s_nohint(smem_addr(cp_ml), mlsrc, ml_bytes, bar);
+        bulk_g2s_nohint(smem_addr(cp_o), osrc, o_bytes, bar);
       }
-      for (; t < ncov; ++t) {
-        const float w0 = cW[t * kMaxGroup + h];
-        if (w0 != 0.f) acc0 = fmaf(w0, __ldcg(src + static_cast<size_t>(t) * GQ * D), acc0);
-      }
-      p.o[plane_index(seg_b, (seg_g * GQ + h) * D + dd, p.B, p.nq * D)] =
-          ((acc0 + acc1) + (acc2 + acc3)) / cS[kMaxGroup + h];
+      if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+      if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
+      cx.act_phase ^= 1u;
+      mlsrc = cp_ml;
+      osrc = cp_o;
     }
+    for (int o4 = cx.tid; o4 < GQ * D / 4; o4 += kConsumerThreads) {
+      const int h = (o4 * 4) / D, dd = o4 * 4 - h * D;
+      const float* mlh = mlsrc + h * 2;
+      const float* oh = osrc + h * D + dd;
+      float M = -INFINITY;
+      for (int t = 0; t < ncov; ++t) {
+        const float mt = staged ? mlh[t * GQ * 2] : __ldcg(mlh + static_cast<size_t>(t) * GQ * 2);
+        if ((has_mask[t >> 5] >> (t & 31)) & 1u) M = fmaxf(M, mt);
+      }
+      float Ls = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int t = 0; t < ncov; ++t) {
+        float2 ml;
+        float4 ov;
+        if (staged) {
+          ml = *reinterpret_cast<const float2*>(mlh + t * GQ * 2);
+          ov = *reinterpret_cast<const float4*>(oh + t * GQ * D);
+        } else {
+          ml = __ldcg(reinterpret_cast<const float2*>(mlh + static_cast<size_t>(t) * GQ * 2));
+          ov = __ldcg(reinterpret_cast<const float4*>(oh + static_cast<size_t>(t) * GQ * D));
+        }
+        if (((has_mask[t >> 5] >> (t & 31)) & 1u) && ml.x != -INFINITY) {
+          const float w = exp2f(ml.x - M);
+          Ls = fmaf(w, ml.y, Ls);
+          acc.x = fmaf(w, ov.x, acc.x);
+          acc.y = fmaf(w, ov.y, acc.y);
+          acc.z = fmaf(w, ov.z, acc.z);
+          acc.w = fmaf(w, ov.w, acc.w);
+        }
+      }
+      const float inv = 1.f / Ls;
+      *reinterpret_cast<float4*>(p.o + plane_index(seg_b, (seg_g * GQ + h) * D + dd, p.B, p.nq * D)) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    fence_proxy_async_global();   // o is read by bulk copies
     consumer_sync();
     if (cx.tid == 0) {
-      atomicExch(arrive, 0u);
+      // reset the arrival count for the next step (ordered before the
+      // release below, which the next step's contributors wait behind)
+      *reinterpret_cast<volatile unsigned*>(arrive) = 0u;
       release_add(p.cnt + l * ST_LAYER + ST_ATTN, 1u);
-      if (p.trace) t_merge += globaltimer() - tm0;
+      if (p.trace) {
+        const unsigned long long te = globaltimer();
+        ta[1] += te - tm0;
+        ta[6] += te - tb0;
+      }
     }
   }
   if (p.trace && cx.tid == 0) {
     const size_t n_st = static_cast<size_t>(p.L) * ST_LAYER + 1;
-    unsigned long long* e = p.trace + ((static_cast<size_t>(s) * n_st + stage_index(p, ST_ATTN, l)) * p.G + blockIdx.x) * 8;
-    e[6] = t_wait;
-    e[7] = t_merge;
+    unsigned long long* e =
+        p.trace + ((static_cast<size_t>(s) * n_st + stage_index(p, ST_ATTN, l)) * p.G + blockIdx.x) * kTraceSlots;
+    for (int k = 0; k < 8; ++k) e[6 + k] = ta[k];
   }
 }
 
@@ -1082,21 +1242,22 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   if (kind == ST_LM) {
     if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused)) return false;
     float* hid = (p.hidden_out && cx.c == 0) ? p.hidden_out + static_cast<size_t>(s) * p.B * p.H : nullptr;
-    load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, where);
+    float rn[B];
+    load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, SIDE_NONE, s, rn, where);
     if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     EpiLM<B> epi{p, s, &bv, &bi};
-    consume_gemv<B>(p, cx, p.lm, rp, where, epi);
+    consume_gemv<B>(p, cx, p.lm, rp, where, rn, epi);
     if (cx.lane < B) {
-      cx.ctl->red[cx.warp][cx.lane] = bv;
+      cx.ctl->redv[cx.warp][cx.lane] = bv;
       cx.ctl->redi[cx.warp][cx.lane] = bi;
     }
     consumer_sync();
     if (cx.tid < B) {
       float v = -INFINITY;
       int ix = 0x7fffffff;
-      for (int w = 0; w < kConsumerWarps; ++w) argmax_merge(v, ix, cx.ctl->red[w][cx.tid], cx.ctl->redi[w][cx.tid]);
+      for (int w = 0; w < kConsumerWarps; ++w) argmax_merge(v, ix, cx.ctl->redv[w][cx.tid], cx.ctl->redi[w][cx.tid]);
       p.lm_val[cx.c * p.B + cx.tid] = v;
       p.lm_idx[cx.c * p.B + cx.tid] = ix;
     }
@@ -1142,52 +1303,57 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   }
   const LayerParams& L = p.layers[l];
   bool ok = true;
+  float rn[B];
+  int r0, r1;
+  resid_rows(p, cx.c, r0, r1);
   switch (kind) {
     case ST_QKV: {
       if (l == 0) {
         ok = stage_wait(p, cx, p.cnt + p.cl.step_done, S1 - 1u, where, fused);
         if (!ok) return false;
-        load_act<B>(p, cx, p.H, SRC_EMBED, nullptr, L.attn_norm, nullptr, where);
+        load_act<B>(p, cx, p.H, SRC_EMBED, nullptr, L.attn_norm, nullptr, SIDE_ROPE, s, rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       } else {
         ok = stage_wait(p, cx, p.cnt + (l - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused);
         if (!ok) return false;
-        load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.attn_norm, nullptr, where);
+        load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.attn_norm, nullptr, SIDE_ROPE, s, rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       }
-      EpiQKV<B> epi{p, l, s};
-      consume_gemv<B>(p, cx, L.qkv, rp, where, epi);
+      EpiQKV<B> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
+      consume_gemv<B>(p, cx, L.qkv, rp, where, rn, epi);
       break;
     }
     case ST_OPROJ: {
       const unsigned tgt = static_cast<unsigned>(p.B * p.nkv) * S1;
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_ATTN, tgt, where, fused)) return false;
-      load_act<B>(p, cx, p.nq * p.d, SRC_PLAIN, p.o, nullptr, nullptr, where);
+      load_act<B>(p, cx, p.nq * p.d, SRC_PLAIN, p.o, nullptr, nullptr, l == 0 ? SIDE_EMBED : SIDE_RESID, s,
+                  rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      EpiResid<B> epi{p, l == 0};
-      consume_gemv<B>(p, cx, L.o, rp, where, epi);
+      EpiResid<B> epi{p, l == 0, cx.side, r0 >> 3, r0 & ~7};
+      consume_gemv<B>(p, cx, L.o, rp, where, rn, epi);
       break;
     }
     case ST_GATEUP: {
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_OPROJ, G * S1, where, fused)) return false;
-      load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr, where);
+      load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr, SIDE_NONE, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiSwiGLU<B> epi{p};
-      consume_gemv<B>(p, cx, L.gu, rp, where, epi);
+      consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
       break;
     }
     default: {  // ST_DOWN
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_GATEUP, G * S1, where, fused)) return false;
-      load_act<B>(p, cx, p.F, SRC_PLAIN, p.h, nullptr, nullptr, where);
+      load_act<B>(p, cx, p.F, SRC_PLAIN, p.h, nullptr, nullptr, SIDE_RESID, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      EpiResid<B> epi{p, false};
-      consume_gemv<B>(p, cx, L.down, rp, where, epi);
+      EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
+      consume_gemv<B>(p, cx, L.down, rp, where, rn, epi);
       break;
     }
   }
-  // KV entries written by the QKV epilogue are read by later steps through
-  // the async proxy (bulk copies): order this thread's generic writes first.
-  if (kind == ST_QKV) fence_proxy_async_global();
+  // Every stage's outputs (KV entries, q, x, h) are read later through the
+  // async proxy (bulk copies, here or in other CTAs): order this thread's
+  // generic writes first.
+  fence_proxy_async_global();
   const bool ab = consumer_sync_any(cx.ctl->abort != 0);
   if (cx.tid == 0) {
     trace_stamp(p, s, stage_index(p, kind, l), 3);
@@ -1203,7 +1369,8 @@ __device__ __forceinline__ Ctx make_ctx(uint8_t* smem, const Params& p) {
   Ctx cx;
   cx.ring = smem;
   cx.act = reinterpret_cast<float*>(smem + static_cast<size_t>(p.nslot) * kSlotBytes);
-  cx.ctl = reinterpret_cast<SmemCtl*>(smem + static_cast<size_t>(p.nslot) * kSlotBytes + p.act_bytes);
+  cx.side = smem + static_cast<size_t>(p.nslot) * kSlotBytes + p.act_bytes;
+  cx.ctl = reinterpret_cast<SmemCtl*>(cx.side + p.side_bytes);
   cx.c = blockIdx.x;
   cx.tid = threadIdx.x;
   cx.warp = threadIdx.x >> 5;
@@ -1320,8 +1487,7 @@ __device__ bool cursor_next(const Params& p, int c, Cursor<B>& cu, Tile& t) {
       cu.open = true;
       if (cu.kind == ST_ATTN) {
         attn_plan<B>(p, cu.s, cu.ap);
-        cu.a = split_point(c, cu.ap.W, p.G);
-        cu.a_end = split_point(c + 1, cu.ap.W, p.G);
+        attn_cta_items<B>(p, cu.ap, c, cu.a, cu.a_end);
       } else {
         const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
         const int NP = m.N >> 1;
@@ -1421,7 +1587,10 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
     }
     const int where = where_code(t.stage % ST_LAYER, t.layer, t.step) | (1 << 15);
     const uint32_t eb = smem_addr(&cx.ctl->empty[rp.slot]);
-    if (!ring_wait(p, cx.ctl, eb, rp.phase ^ 1u, where)) break;
+    // A full ring only means the consumers are waiting on a dependency; give
+    // their own (bounded) wait the chance to time out first, so the reported
+    // failure names the dependency rather than this stall.
+    if (!mbar_try_wait(eb, rp.phase ^ 1u) && !ring_wait_slow(p, cx.ctl, eb, rp.phase ^ 1u, where, 2)) break;
     const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
     mbar_expect_tx(fb, tb);
     const uint32_t dst = smem_addr(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes);

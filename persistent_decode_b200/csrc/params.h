@@ -20,6 +20,8 @@ constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 4;                          // query heads per kv head
 constexpr int kPairsPerTile = kConsumerWarps;         // one row pair per consumer warp
 constexpr int kMiscSmem = 4096;                       // barriers, flags, reduction scratch
+constexpr int kMaxCtas = 160;                        // persistent grid limit (one CTA per SM; B200 has 148)
+constexpr int kTraceSlots = 16;                       // u64 stamps per (step, stage, CTA) in a trace
 
 // Stages of one layer, in dependency order, then the LM head.
 enum StageKind : int {
@@ -81,8 +83,15 @@ struct Params {
   int G;                // CTAs
   int nslot;            // ring slots in use
   int act_bytes;        // activation / scratch region
+  int side_bytes;       // epilogue side region (after the activation region)
+  int side_rope;        //   byte offset of the RoPE rows [B][d/2] float2
+  int side_resid;       //   byte offset of the residual slice [B][2 planes][nvr] float4
+  int side_embed;       //   byte offset of the embedding slice [B][evb bytes]
+  int nvr;              //   float4 vectors per (sequence, plane) of the residual slice
+  int evb;              //   bytes per sequence of the embedding slice
   int attn_pos_per_tile;
   long long spin_limit_ns;
+  unsigned wait_hint_ns;  // suspend-time hint of mbarrier waits (0: plain polling)
   long long l2_prefetch_bytes;  // how far the producer's L2-prefetch cursor runs ahead
   CounterLayout cl;
 

@@ -94,6 +94,7 @@ struct xlpk_engine {
   int nslot = 0;
   int smem = 0;
   int act_bytes = 0;
+  int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, evb = 0;
   int esz = 2;
   int P = 0;
   uint8_t* packed = nullptr;
@@ -330,6 +331,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   }
   if (!prop.cooperativeLaunch) return XLPK_ERR_UNSUPPORTED;
   e->G = c.n_ctas > 0 ? c.n_ctas : prop.multiProcessorCount;
+  if (e->G > kMaxCtas) {
+    g_cuda_err = "persistent grid larger than " + std::to_string(kMaxCtas) + " CTAs";
+    return XLPK_ERR_UNSUPPORTED;
+  }
   e->esz = c.weight_dtype == XLPK_DTYPE_FP8_E4M3 ? 1 : 2;
   const int B = c.batch, H = c.hidden, d = c.head_dim, F = c.ffn;
   const int qd = c.n_q_heads * d, kvd = c.n_kv_heads * d;
@@ -339,11 +344,25 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   // shared memory: ring + activation/scratch + control
   const int kmax = std::max(std::max(H, qd), F);
   const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
-  e->act_bytes = static_cast<int>(align_up(std::max(B * kmax * 4, attn_scratch), 1024));
+  const int norm_stage = (B + 1) * H * 4;   // normed input vector + its RMSNorm gains
+  e->act_bytes = static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
+  // epilogue side region: RoPE rows, then this CTA's rows of the residual (two
+  // planes of float4) and of the embedding (bf16, 8-aligned) for the stages
+  // with H output rows
+  {
+    const int maxp = (H / 2 + e->G - 1) / e->G;
+    const int rows_max = 2 * maxp;
+    e->side_rope = 0;
+    e->side_resid = static_cast<int>(align_up(static_cast<size_t>(B) * d * 4, 16));
+    e->nvr = rows_max / 8 + 2;
+    e->side_embed = e->side_resid + B * 2 * e->nvr * 16;
+    e->evb = static_cast<int>(align_up(static_cast<size_t>(rows_max + 16) * 2, 16));
+    e->side_bytes = static_cast<int>(align_up(static_cast<size_t>(e->side_embed) + B * e->evb, 128));
+  }
   const int max_smem = static_cast<int>(prop.sharedMemPerBlockOptin);
-  e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - kMiscSmem) / kSlotBytes);
+  e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
-  e->smem = e->nslot * kSlotBytes + e->act_bytes + kMiscSmem;
+  e->smem = e->nslot * kSlotBytes + e->act_bytes + e->side_bytes + kMiscSmem;
   if (!bind_by_shape(e, B, d)) return XLPK_ERR_UNSUPPORTED;
 
   // The attribute is per kernel function, shared by every handle that uses the
@@ -496,9 +515,16 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.G = e->G;
   p.nslot = e->nslot;
   p.act_bytes = e->act_bytes;
+  p.side_bytes = e->side_bytes;
+  p.side_rope = e->side_rope;
+  p.side_resid = e->side_resid;
+  p.side_embed = e->side_embed;
+  p.nvr = e->nvr;
+  p.evb = e->evb;
   p.attn_pos_per_tile = e->P;
   p.spin_limit_ns = 1000LL * (c.spin_limit_us > 0 ? c.spin_limit_us : 200000);
   p.l2_prefetch_bytes = 256 * 1024;
+  p.wait_hint_ns = 20000;
   p.cl = cl;
   p.embed = embed_copy;
   p.final_norm = final_norm_copy;
@@ -553,6 +579,8 @@ Params call_params(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out, const x
   p.trace = io ? reinterpret_cast<unsigned long long*>(io->trace_dev) : nullptr;
   // L2 prefetch distance per CTA: a tuning knob read at each call (0 disables)
   if (const char* env = std::getenv("XLPK_L2_PREFETCH_KB")) p.l2_prefetch_bytes = std::atoll(env) * 1024;
+  // suspend-time hint of the mbarrier waits (tuning knob; 0 polls)
+  if (const char* env = std::getenv("XLPK_WAIT_HINT_NS")) p.wait_hint_ns = static_cast<unsigned>(std::atoll(env));
   // Failure-detection tests: make one dependency wait run out (a release that
   // never happens) so the time limit, the abort path and the status report
   // are exercised without faulting anything.
