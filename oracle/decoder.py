@@ -155,7 +155,8 @@ class OracleDecoder:
         p = f"layers.{l}."
         if not cfg.is_moe:
             return swiglu_ffn(xn, self.W(p + "w_gate"), self.W(p + "w_up"), self.W(p + "w_down")), []
-        ids, gates, _ = moe_route(self.W(p + "router") @ xn, cfg.top_k)
+        ids, gates, probs = moe_route(self.W(p + "router") @ xn, cfg.top_k)
+        self._router_probs.append(probs)
         out = torch.zeros(cfg.hidden, dtype=torch.float32)
         for e, ge in zip(ids, gates):
             q = f"{p}experts.{e}."
@@ -176,6 +177,7 @@ class OracleDecoder:
         logits = torch.empty(self.B, cfg.vocab, dtype=torch.float32)
         hidden = torch.empty(self.B, cfg.hidden, dtype=torch.float32)
         experts: List[List[int]] = []
+        self._router_probs: List[torch.Tensor] = []
         for b in range(self.B):
             pos = self.pos[b]
             assert pos < self.max_seq
@@ -200,6 +202,9 @@ class OracleDecoder:
             logits[b] = self.W("lm_head") @ rms_norm(x, self.w["final_norm"], cfg.rms_eps)
             self.pos[b] = pos + 1
         self.last_experts = [experts[b * cfg.n_layers:(b + 1) * cfg.n_layers] for b in range(self.B)]
+        # the router probabilities behind each selection (records only)
+        self.last_router_probs = [self._router_probs[b * cfg.n_layers:(b + 1) * cfg.n_layers]
+                                  for b in range(self.B)] if cfg.is_moe else []
         return logits, hidden
 
     # ---------------------------------------------------------------- prefill
@@ -218,6 +223,7 @@ class OracleDecoder:
         grp = nq // nkv
         Bn, T = tokens.shape
         out = torch.empty(Bn, T, cfg.vocab, dtype=torch.float32)
+        self._router_probs = []
         for b in range(Bn):
             x = self.w["embed"][tokens[b].long()].float()          # [T][H]
             for l in range(cfg.n_layers):

@@ -251,6 +251,12 @@ struct alignas(16) SmemCtl {
   float redv[kConsumerWarps][kMaxBatch];   // LM-head argmax values
   int redi[kConsumerWarps][kMaxBatch];     // LM-head argmax indices
   unsigned long long tacc[8];              // attention trace totals (thread 0)
+  // MoE routing of the current layer, computed by this CTA's consumers and
+  // read by its producer: route_seq = step * L + layer + 1 once the table is set
+  volatile int route_seq;
+  int route_exp[kMaxMoeSlots];
+  float route_w[kMaxMoeSlots];
+  float logits[kMaxExperts];
 };
 static_assert(sizeof(SmemCtl) <= kMiscSmem, "control block too large");
 
@@ -286,6 +292,10 @@ __device__ __forceinline__ void raise_error(const Params& p, int code, int where
   }
   atomicExch(p.abort_flag, 1);
 }
+
+// Value of the control block's route_seq once the MoE routing of (step s,
+// layer l) is in its table.
+__device__ __forceinline__ int route_want(const Params& p, int s, int l) { return s * p.L + l + 1; }
 
 __device__ __forceinline__ int where_code(int kind, int layer, int step) {
   return (step << 16) | ((layer & 0xff) << 8) | (kind & 0xff);
@@ -586,11 +596,14 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
 // Consumer side: each warp owns one row pair of every tile of a group and
 // accumulates it over the group's k-chunks; `epi(pair, acc0, acc1)` runs on
 // the reduced sums (identical in every lane).
+// [q0, q1) overrides the CTA's pair range (default: the even split of m's pairs).
 template <int B, class Epi>
 __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp,
-                                          int where, const float (&rn)[B], Epi& epi) {
+                                          int where, const float (&rn)[B], Epi& epi, int q0 = -1,
+                                          int q1 = -1) {
   const int NP = m.N >> 1;
-  const int p0 = split_point(cx.c, NP, p.G), p1 = split_point(cx.c + 1, NP, p.G);
+  const int p0 = q0 >= 0 ? q0 : split_point(cx.c, NP, p.G);
+  const int p1 = q0 >= 0 ? q1 : split_point(cx.c + 1, NP, p.G);
   const int nkc = m.K / m.KC;
   const int nv = m.KC >> 3;   // 16-byte vectors per row chunk
   const int nvK = m.K >> 3;
@@ -750,6 +763,97 @@ struct EpiLM {
     }
   }
 };
+
+// MoE router epilogue: the expert logits of this CTA's copy of the router, to
+// shared memory (every CTA computes all of them).
+template <int B>
+struct EpiRouter {
+  float* logits;
+  __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
+    if (lane == 0) {
+      logits[2 * pg] = a0[0];
+      logits[2 * pg + 1] = a1[0];
+    }
+  }
+};
+
+// MoE gate/up epilogue over the virtual [slot][pair] space: h = w_slot * silu(gate) * up.
+template <int B>
+struct EpiMoeGU {
+  const Params& p;
+  const float* route_w;
+  __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
+    if (lane == 0) {
+      const float g = a0[0];
+      p.h[plane_index(0, pg, 1, p.S * p.Fe)] = route_w[pg / p.Fe] * (g / (1.f + expf(-g)) * a1[0]);
+    }
+  }
+};
+
+// MoE routing of one token (warp 0 of the consumers): softmax over the E
+// router logits, the top_k most probable experts (ties -> lower id) with their
+// probabilities as weights (not renormalised), shared experts first with
+// weight 1.  Writes this CTA's routing table; CTA 0 also records it globally
+// (for the kernel-per-op down launch and the caller's experts output).
+__device__ __noinline__ void moe_route(const Params& p, Ctx& cx, int l, int s) {
+  constexpr int PER = kMaxExperts / 32;
+  float v[PER];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = cx.lane + 32 * i;
+    v[i] = e < p.E ? cx.ctl->logits[e] : -INFINITY;
+    mx = fmaxf(mx, v[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    v[i] = (cx.lane + 32 * i < p.E) ? expf(v[i] - mx) : 0.f;
+    sum += v[i];
+  }
+  sum = warp_sum(sum);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = (cx.lane + 32 * i < p.E) ? v[i] / sum : -1.f;
+  for (int k = 0; k < p.topk; ++k) {
+    float bv = -2.f;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) argmax_merge(bv, bi, v[i], cx.lane + 32 * i);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+      argmax_merge(bv, bi, v2, i2);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (cx.lane + 32 * i == bi) v[i] = -1.f;   // taken
+    if (cx.lane == 0) {
+      cx.ctl->route_exp[p.nsh + k] = bi;
+      cx.ctl->route_w[p.nsh + k] = bv;
+      if (cx.c == 0) {
+        p.route_exp[l * p.S + p.nsh + k] = bi;
+        p.route_w[l * p.S + p.nsh + k] = bv;
+        if (p.experts_out) p.experts_out[(static_cast<size_t>(s) * p.L + l) * p.topk + k] = bi;
+      }
+    }
+  }
+  if (cx.lane < p.nsh) {
+    cx.ctl->route_exp[cx.lane] = p.E + cx.lane;
+    cx.ctl->route_w[cx.lane] = 1.f;
+    if (cx.c == 0) {
+      p.route_exp[l * p.S + cx.lane] = p.E + cx.lane;
+      p.route_w[l * p.S + cx.lane] = 1.f;
+    }
+  }
+  __syncwarp();
+  if (cx.lane == 0) {
+    __threadfence_block();
+    cx.ctl->route_seq = route_want(p, s, l);   // the producer may stream the experts now
+  }
+}
 
 // ------------------------------------------------------------------ attention
 
@@ -1337,16 +1441,42 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_OPROJ, G * S1, where, fused)) return false;
       load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr, SIDE_NONE, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      EpiSwiGLU<B> epi{p};
-      consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
+      if (p.E > 0) {
+        if constexpr (B == 1) {
+          // router (all E logits in every CTA), routing, then this CTA's groups
+          // of the virtual [slot][pair] gate/up space
+          EpiRouter<B> er{cx.ctl->logits};
+          consume_gemv<B>(p, cx, L.router, rp, where, rn, er, 0, L.router.N >> 1);
+          consumer_sync();
+          if (cx.warp == 0) moe_route(p, cx, l, s);
+          consumer_sync();
+          const int ng = p.S * (p.Fe >> 3);
+          Mat v = L.egu;
+          v.N = 2 * p.S * p.Fe;
+          EpiMoeGU<B> eg{p, cx.ctl->route_w};
+          consume_gemv<B>(p, cx, v, rp, where, rn, eg, 8 * split_point(cx.c, ng, p.G),
+                          8 * split_point(cx.c + 1, ng, p.G));
+        }
+      } else {
+        EpiSwiGLU<B> epi{p};
+        consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
+      }
       break;
     }
     default: {  // ST_DOWN
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_GATEUP, G * S1, where, fused)) return false;
-      load_act<B>(p, cx, p.F, SRC_PLAIN, p.h, nullptr, nullptr, SIDE_RESID, s, rn, where);
+      const int K = p.E > 0 ? p.S * p.Fe : p.F;
+      load_act<B>(p, cx, K, SRC_PLAIN, p.h, nullptr, nullptr, SIDE_RESID, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
-      consume_gemv<B>(p, cx, L.down, rp, where, rn, epi);
+      if (p.E > 0) {
+        // K runs over [slot][expert column]: the producer streams each slot's expert
+        Mat v = L.edown;
+        v.K = K;
+        consume_gemv<B>(p, cx, v, rp, where, rn, epi);
+      } else {
+        consume_gemv<B>(p, cx, L.down, rp, where, rn, epi);
+      }
       break;
     }
   }
@@ -1398,6 +1528,7 @@ __device__ __forceinline__ void init_ring(const Params& p, Ctx& cx) {
     mbar_init(smem_addr(&cx.ctl->act_bar), 1);
     cx.ctl->abort = 0;
     cx.ctl->flag = 0;
+    cx.ctl->route_seq = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -1446,9 +1577,13 @@ struct Cursor {
   bool open;           // the current stage's range has been set up
   bool one_stage;      // kernel-per-op launch: only one stage
   bool done;
-  int a, a_end;        // GEMV: next pair of the CTA's span / span end; attention: item range
+  int a, a_end;        // GEMV: next pair of the CTA's span / span end; attention: item range;
+                       // MoE gate/up experts: next virtual group / end
   int kc, nkc, KC;
+  int esz;             // bytes per weight element of the current matrix
   const uint8_t* src;  // GEMV: next tile
+  int phase;           // MoE gate/up: 0 router, 1 experts
+  int slot, grp;       // MoE down: slot of the next tile, group index within the CTA's span
   AttnPlan<B> ap;
 };
 
@@ -1480,14 +1615,39 @@ __device__ __forceinline__ void cursor_next_stage(const Params& p, Cursor<B>& cu
   }
 }
 
+enum CursorResult : int { CUR_DONE = 0, CUR_TILE = 1, CUR_BLOCKED = 2 };
+
 template <int B>
-__device__ bool cursor_next(const Params& p, int c, Cursor<B>& cu, Tile& t) {
+__device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>& cu, Tile& t) {
   while (!cu.done) {
+    const bool moe = p.E > 0 && (cu.kind == ST_GATEUP || cu.kind == ST_DOWN);
     if (!cu.open) {
       cu.open = true;
+      cu.esz = p.esz;
       if (cu.kind == ST_ATTN) {
         attn_plan<B>(p, cu.s, cu.ap);
         attn_cta_items<B>(p, cu.ap, c, cu.a, cu.a_end);
+      } else if (moe && cu.kind == ST_GATEUP) {
+        // the router first (every CTA streams all of it), then the CTA's groups
+        // of the virtual [slot][pair] space
+        const Mat& r = p.layers[cu.l].router;
+        cu.phase = 0;
+        cu.a = 0;
+        cu.a_end = r.N >> 1;
+        cu.kc = 0;
+        cu.nkc = r.K / r.KC;
+        cu.KC = r.KC;
+        cu.esz = 2;
+        cu.src = r.packed;
+      } else if (moe) {   // MoE down: the CTA's output rows, every slot's expert in turn
+        const Mat& m = p.layers[cu.l].edown;
+        cu.a = split_point(c, p.H >> 1, p.G);
+        cu.a_end = split_point(c + 1, p.H >> 1, p.G);
+        cu.kc = 0;
+        cu.nkc = m.K / m.KC;
+        cu.KC = m.KC;
+        cu.slot = 0;
+        cu.grp = 0;
       } else {
         const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
         const int NP = m.N >> 1;
@@ -1502,6 +1662,7 @@ __device__ bool cursor_next(const Params& p, int c, Cursor<B>& cu, Tile& t) {
     t.stage = stage_index(p, cu.kind, cu.l);
     t.layer = cu.l;
     t.step = cu.s;
+    t.attn = false;
     if (cu.kind == ST_ATTN) {
       if (cu.a < cu.a_end) {   // every chunk is one tile (K and V boxes)
         int b, g, j, nch, base;
@@ -1512,27 +1673,96 @@ __device__ bool cursor_next(const Params& p, int c, Cursor<B>& cu, Tile& t) {
         t.src = nullptr;
         t.bytes = kSlotBytes;
         t.attn = true;
-        return true;
+        return CUR_TILE;
+      }
+    } else if (moe && cu.kind == ST_GATEUP && cu.phase == 1) {
+      if (cu.a < cu.a_end) {
+        const LayerParams& L = p.layers[cu.l];
+        const int gpe = p.Fe >> 3;                     // groups of 8 pairs per expert
+        const int slot = cu.a / gpe, grp = cu.a - slot * gpe;
+        if (slot >= p.nsh && ctl->route_seq != route_want(p, cu.s, cu.l)) return CUR_BLOCKED;
+        const int ex = slot < p.nsh ? p.E + slot : ctl->route_exp[slot];
+        const uint32_t tb = 2u * kPairsPerTile * cu.KC * cu.esz;
+        t.bytes = tb;
+        t.src = L.egu.packed + ex * L.egu_stride + (static_cast<size_t>(grp) * cu.nkc + cu.kc) * tb;
+        if (++cu.kc == cu.nkc) {
+          cu.kc = 0;
+          ++cu.a;
+        }
+        return CUR_TILE;
+      }
+    } else if (moe && cu.kind == ST_DOWN) {
+      if (cu.a < cu.a_end) {
+        if (ctl->route_seq != route_want(p, cu.s, cu.l)) return CUR_BLOCKED;
+        const LayerParams& L = p.layers[cu.l];
+        const int gp = min(kPairsPerTile, cu.a_end - cu.a);
+        const int ex = ctl->route_exp[cu.slot];
+        const int a0 = split_point(c, p.H >> 1, p.G);
+        t.bytes = 2u * gp * cu.KC * cu.esz;
+        t.src = L.edown.packed + ex * L.edown_stride +
+                (static_cast<size_t>(2) * a0 * p.Fe + static_cast<size_t>(cu.grp) * 2 * kPairsPerTile * p.Fe) *
+                    cu.esz +
+                static_cast<size_t>(cu.kc) * t.bytes;
+        if (++cu.kc == cu.nkc) {
+          cu.kc = 0;
+          if (++cu.slot == p.S) {
+            cu.slot = 0;
+            ++cu.grp;
+            cu.a += kPairsPerTile;
+          }
+        }
+        return CUR_TILE;
       }
     } else if (cu.a < cu.a_end) {
       const int gp = min(kPairsPerTile, cu.a_end - cu.a);
-      t.bytes = 2u * gp * cu.KC * p.esz;
+      t.bytes = 2u * gp * cu.KC * cu.esz;
       t.src = cu.src;
-      t.attn = false;
       cu.src += t.bytes;
       if (++cu.kc == cu.nkc) {
         cu.kc = 0;
         cu.a += kPairsPerTile;
       }
-      return true;
+      return CUR_TILE;
+    } else if (moe && cu.kind == ST_GATEUP && cu.phase == 0) {
+      // router done: the experts' gate/up groups of this CTA
+      const Mat& m = p.layers[cu.l].egu;
+      const int ng = p.S * (p.Fe >> 3);
+      cu.phase = 1;
+      cu.a = split_point(c, ng, p.G);
+      cu.a_end = split_point(c + 1, ng, p.G);
+      cu.kc = 0;
+      cu.nkc = m.K / m.KC;
+      cu.KC = m.KC;
+      cu.esz = p.esz;
+      continue;
     }
     cursor_next_stage<B>(p, cu);
   }
-  return false;
+  return CUR_DONE;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Bounded wait of the producer for its CTA's routing of (step, layer).
+__device__ __noinline__ bool route_wait(const Params& p, SmemCtl* ctl, int want, int where) {
+  const uint64_t t0 = globaltimer();
+  while (ctl->route_seq != want) {
+    if (ctl->abort) return false;
+    if (ld_volatile(p.abort_flag)) {
+      ctl->abort = 1;
+      return false;
+    }
+    if (static_cast<long long>(globaltimer() - t0) > 2 * p.spin_limit_ns) {
+      raise_error(p, kErrTimeout, where);
+      ctl->abort = 1;
+      return false;
+    }
+    __nanosleep(32);
+  }
+  __threadfence_block();   // the table was written before route_seq
+  return true;
 }
 
 // The producer (one thread): copy cursor -> ring, prefetch cursor -> L2,
@@ -1550,11 +1780,21 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
   bool pc_live = true;
   int cur_stage = -1, cur_step = -1;
   Tile t, tp;
-  while (cursor_next<B>(p, cx.c, cc, t)) {
+  for (;;) {
+    int r = cursor_next<B>(p, cx.c, cx.ctl, cc, t);
+    if (r == CUR_BLOCKED) {
+      // the next tile is an expert chosen by this CTA's own consumers: wait
+      // (bounded) until they publish the layer's routing
+      if (!route_wait(p, cx.ctl, route_want(p, cc.s, cc.l), where_code(cc.kind, cc.l, cc.s) | (1 << 15))) break;
+      r = cursor_next<B>(p, cx.c, cx.ctl, cc, t);
+    }
+    if (r != CUR_TILE) break;
     const uint32_t tb = t.bytes;
     ahead -= tb;
     while (pc_live && ahead < p.l2_prefetch_bytes) {
-      pc_live = cursor_next<B>(p, cx.c, pc, tp);
+      const int pr = cursor_next<B>(p, cx.c, cx.ctl, pc, tp);
+      if (pr == CUR_BLOCKED) break;   // resume once the routing is known
+      pc_live = pr == CUR_TILE;
       if (!pc_live) break;
       if (!tp.attn) {
         prefetch_l2(tp.src, tp.bytes);
@@ -1645,7 +1885,16 @@ __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constan
                                                             int layer, int step) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctx cx = make_ctx(smem, p);
+  if (p.E > 0 && kind == ST_DOWN && cx.tid < p.S) {
+    // the routing was computed by the gate/up launch: take CTA 0's record
+    cx.ctl->route_exp[cx.tid] = p.route_exp[layer * p.S + cx.tid];
+    cx.ctl->route_w[cx.tid] = p.route_w[layer * p.S + cx.tid];
+  }
   init_ring(p, cx);
+  if (p.E > 0 && kind == ST_DOWN) {
+    if (cx.tid == 0) cx.ctl->route_seq = route_want(p, step, layer);
+    __syncthreads();
+  }
   if (cx.warp == kConsumerWarps) {
     if (cx.lane == 0) producer_main<B>(p, cx, kind, layer, step, false);
     __syncwarp();

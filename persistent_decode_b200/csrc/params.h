@@ -20,6 +20,8 @@ constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 4;                          // query heads per kv head
 constexpr int kPairsPerTile = kConsumerWarps;         // one row pair per consumer warp
 constexpr int kMiscSmem = 4096;                       // barriers, flags, reduction scratch
+constexpr int kMaxExperts = 256;                      // routed experts per MoE layer
+constexpr int kMaxMoeSlots = 16;                      // shared + selected experts per token
 constexpr int kMaxCtas = 160;                        // persistent grid limit (one CTA per SM; B200 has 148)
 constexpr int kTraceSlots = 16;                       // u64 stamps per (step, stage, CTA) in a trace
 
@@ -67,15 +69,27 @@ struct Mat {
 struct LayerParams {
   Mat qkv;     // rows: q heads (RoPE pairs interleaved), k heads (interleaved), v heads
   Mat o;
-  Mat gu;      // rows: gate_j, up_j interleaved
-  Mat down;
+  Mat gu;      // rows: gate_j, up_j interleaved (dense layers)
+  Mat down;    // dense layers
   const float* attn_norm;
   const float* ffn_norm;
+  // MoE layers.  Experts are numbered 0..E-1 (routed) then E..E+S_sh-1
+  // (shared).  The router and every expert's gate/up are packed as one
+  // block streamed whole (groups of 8 row pairs in order, not split over the
+  // CTAs); every expert's down projection is packed like a dense matrix
+  // (rows split over the CTAs).  egu / edown describe expert 0; expert e's
+  // block starts e * egu_stride (edown_stride) bytes further.
+  Mat router;
+  Mat egu;
+  Mat edown;
+  long long egu_stride;
+  long long edown_stride;
 };
 
 struct Params {
   // shape
   int L, H, nq, nkv, d, F, V, B, max_seq;
+  int E, topk, nsh, S, Fe;  // MoE: routed experts, selected per token, shared, slots (nsh + topk), expert width
   int group;            // nq / nkv
   int esz;              // weight bytes per element (2 bf16, 1 fp8)
   float eps;
@@ -114,7 +128,9 @@ struct Params {
   float* x;          // [B][H] residual stream
   float* q;          // [B][nq*d] rotated queries
   float* o;          // [B][nq*d] attention output
-  float* h;          // [B][F] SwiGLU output
+  float* h;          // [B][F] SwiGLU output (MoE: [B][S*Fe], slot-major, gate-weighted)
+  int* route_exp;    // MoE: [L][S] expert of each slot (written by CTA 0)
+  float* route_w;    // MoE: [L][S] weight of each slot
   float* part_ml;    // [B][nkv][G][group][2] per contributing CTA: (max in log2 units, sum)
   float* part_o;     // [B][nkv][G][group][d] unnormalised attention output
   float* lm_val;     // [G][B]
@@ -132,6 +148,7 @@ struct Params {
   const int32_t* forced;
   float* logits_out;
   float* hidden_out;
+  int32_t* experts_out;        // MoE: [n_steps][L][B][topk] selected experts (may be null)
   unsigned long long* trace;   // optional stage timestamps
   int fault_drop_stage;        // failure-detection tests: CTA 0 withholds its release of this
                                // stage index at the call's first step (-1: never)

@@ -176,12 +176,14 @@ const uint8_t* source_row(const MatSrc& ms, long long n, int K, int esz, const x
 }
 
 // Pack one matrix into `dst` (device) in stream order; returns the Mat view.
+// `split` CTAs share the rows (1: the whole matrix is one block streamed by
+// every CTA that needs it, e.g. the MoE router and expert gate/up blocks).
 xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t* dst, Mat* out,
-                        PackJob* d_jobs, size_t max_jobs, cudaStream_t st) {
+                        PackJob* d_jobs, size_t max_jobs, cudaStream_t st, int split) {
   const int esz = e->esz;
   const int KC = pick_kc(K, esz);
   if (KC == 0) return XLPK_ERR_UNSUPPORTED;
-  const long long NP = N / 2, G = e->G;
+  const long long NP = N / 2, G = split;
   std::vector<PackJob> jobs;
   jobs.reserve(static_cast<size_t>(N));
   for (long long c = 0; c < G; ++c) {
@@ -270,10 +272,18 @@ xlpk_status validate_config(const xlpk_config* c) {
   if (c->n_q_heads / c->n_kv_heads > kMaxGroup) return XLPK_ERR_UNSUPPORTED;
   if (c->batch != 1 && c->batch != 2 && c->batch != 4 && c->batch != 8) return XLPK_ERR_UNSUPPORTED;
   if (c->weight_dtype != XLPK_DTYPE_BF16) return XLPK_ERR_UNSUPPORTED;
-  if (c->n_experts != 0) return XLPK_ERR_UNSUPPORTED;
-  if (c->ffn <= 0) return XLPK_ERR_INVALID_ARG;
-  if (c->hidden % 16 || c->ffn % 16 || (c->n_q_heads * c->head_dim) % 16 || c->vocab % 2)
-    return XLPK_ERR_UNSUPPORTED;
+  if (c->n_experts > 0) {
+    if (c->top_k < 1 || c->top_k > c->n_experts || c->expert_ffn <= 0) return XLPK_ERR_INVALID_ARG;
+    if (c->n_experts > kMaxExperts || c->top_k + c->n_shared_experts > kMaxMoeSlots || c->n_experts % 2)
+      return XLPK_ERR_UNSUPPORTED;
+    if (c->expert_ffn % 16) return XLPK_ERR_UNSUPPORTED;
+    if (c->batch != 1) return XLPK_ERR_UNSUPPORTED;   // per-sequence routing at B > 1 is not built
+  } else {
+    if (c->top_k != 0 || c->n_shared_experts != 0) return XLPK_ERR_INVALID_ARG;
+    if (c->ffn <= 0) return XLPK_ERR_INVALID_ARG;
+    if (c->ffn % 16) return XLPK_ERR_UNSUPPORTED;
+  }
+  if (c->hidden % 16 || (c->n_q_heads * c->head_dim) % 16 || c->vocab % 2) return XLPK_ERR_UNSUPPORTED;
   return XLPK_OK;
 }
 
@@ -286,9 +296,23 @@ xlpk_status validate_weights(const xlpk_config* c, const xlpk_weights* w, const 
   for (int l = 0; l < c->n_layers; ++l) {
     const xlpk_layer_weights& L = w->layers[l];
     const void* need[] = {L.attn_norm_dev, L.ffn_norm_dev, L.wq.w_dev, L.wk.w_dev, L.wv.w_dev,
-                          L.wo.w_dev, L.w_gate.w_dev, L.w_up.w_dev, L.w_down.w_dev};
+                          L.wo.w_dev};
     for (const void* q : need)
       if (!q || !aligned16(q)) return XLPK_ERR_INVALID_ARG;
+    if (c->n_experts > 0) {
+      const void* moe[] = {L.router_dev, L.we_gate.w_dev, L.we_up.w_dev, L.we_down.w_dev};
+      for (const void* q : moe)
+        if (!q || !aligned16(q)) return XLPK_ERR_INVALID_ARG;
+      if (c->n_shared_experts > 0) {
+        const void* sh[] = {L.ws_gate.w_dev, L.ws_up.w_dev, L.ws_down.w_dev};
+        for (const void* q : sh)
+          if (!q || !aligned16(q)) return XLPK_ERR_INVALID_ARG;
+      }
+    } else {
+      const void* ffn[] = {L.w_gate.w_dev, L.w_up.w_dev, L.w_down.w_dev};
+      for (const void* q : ffn)
+        if (!q || !aligned16(q)) return XLPK_ERR_INVALID_ARG;
+    }
   }
   return XLPK_OK;
 }
@@ -342,7 +366,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->P = (kSlotBytes / 2) / (d * 2);
 
   // shared memory: ring + activation/scratch + control
-  const int kmax = std::max(std::max(H, qd), F);
+  const int S_moe = c.n_experts > 0 ? c.top_k + c.n_shared_experts : 0;
+  const int kmax = std::max(std::max(H, qd), std::max(F, S_moe * c.expert_ffn));
   const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
   const int norm_stage = (B + 1) * H * 4;   // normed input vector + its RMSNorm gains
   e->act_bytes = static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
@@ -376,27 +401,51 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     return XLPK_ERR_UNSUPPORTED;
   }
 
-  // packed weights: per layer qkv, o, gate/up, down; then the LM head
+  // packed weights: per layer qkv, o, then gate/up + down (dense) or the
+  // router + every expert's gate/up and down (MoE); then the LM head
+  enum Role { R_QKV, R_O, R_GU, R_DOWN, R_ROUTER, R_EGU, R_EDOWN, R_LM };
   struct MatPlan {
     MatSrc src;
     int N, K;
     size_t off;
+    int layer, role, split;
   };
+  const bool moe = c.n_experts > 0;
+  const int Fe = c.expert_ffn, nE = c.n_experts + c.n_shared_experts;
   std::vector<MatPlan> mats;
   size_t total = 0;
-  auto add = [&](MatSrc s, int N, int K) {
-    mats.push_back({s, N, K, total});
+  auto add = [&](MatSrc s, int N, int K, int layer, int role, int split) {
+    mats.push_back({s, N, K, total, layer, role, split});
     total += align_up(static_cast<size_t>(N) * K * e->esz, 256);
   };
+  auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
+  const size_t eg_bytes = static_cast<size_t>(Fe) * H * e->esz;   // one expert's gate (or up, or down)
   for (int l = 0; l < c.n_layers; ++l) {
     const xlpk_layer_weights& L = w->layers[l];
-    auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
-    add({MatKind::QKV, u8(L.wq.w_dev), u8(L.wk.w_dev), u8(L.wv.w_dev)}, qd + 2 * kvd, H);
-    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr}, H, qd);
-    add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr}, 2 * F, H);
-    add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, H, F);
+    add({MatKind::QKV, u8(L.wq.w_dev), u8(L.wk.w_dev), u8(L.wv.w_dev)}, qd + 2 * kvd, H, l, R_QKV, e->G);
+    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr}, H, qd, l, R_O, e->G);
+    if (!moe) {
+      add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr}, 2 * F, H, l, R_GU, e->G);
+      add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, H, F, l, R_DOWN, e->G);
+    } else {
+      // router logits are bf16 whatever the weight dtype
+      add({MatKind::PLAIN, u8(L.router_dev), nullptr, nullptr}, c.n_experts, H, l, R_ROUTER, 1);
+      for (int x = 0; x < nE; ++x) {
+        const bool sh = x >= c.n_experts;
+        const int xi = sh ? x - c.n_experts : x;
+        const uint8_t* g = u8(sh ? L.ws_gate.w_dev : L.we_gate.w_dev) + xi * eg_bytes;
+        const uint8_t* u = u8(sh ? L.ws_up.w_dev : L.we_up.w_dev) + xi * eg_bytes;
+        add({MatKind::GATEUP, g, u, nullptr}, 2 * Fe, H, l, R_EGU, 1);
+      }
+      for (int x = 0; x < nE; ++x) {
+        const bool sh = x >= c.n_experts;
+        const int xi = sh ? x - c.n_experts : x;
+        const uint8_t* dn = u8(sh ? L.ws_down.w_dev : L.we_down.w_dev) + xi * eg_bytes;
+        add({MatKind::PLAIN, dn, nullptr, nullptr}, H, Fe, l, R_EDOWN, e->G);
+      }
+    }
   }
-  add({MatKind::PLAIN, static_cast<const uint8_t*>(w->lm_head.w_dev), nullptr, nullptr}, c.vocab, H);
+  add({MatKind::PLAIN, u8(w->lm_head.w_dev), nullptr, nullptr}, c.vocab, H, -1, R_LM, e->G);
   // library-owned copies of the embedding table and the norm gains, so the
   // caller may free every weight buffer after create
   const size_t off_embed = total;
@@ -408,8 +457,16 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
 #ifdef XLPK_DEBUG_POISON
   XLPK_CUDA(cudaMemset(e->packed, 0xff, total));   // debug build: unwritten bytes read as NaN
 #endif
+  // weights streamed per step: every dense matrix; for MoE the router and the
+  // shared + top_k experts of each layer
   e->weight_bytes_per_step = 0;
-  for (const MatPlan& m : mats) e->weight_bytes_per_step += static_cast<int64_t>(m.N) * m.K * e->esz;
+  for (const MatPlan& m : mats) {
+    if (m.role == R_EGU || m.role == R_EDOWN) continue;
+    e->weight_bytes_per_step += static_cast<int64_t>(m.N) * m.K * (m.role == R_ROUTER ? 2 : e->esz);
+  }
+  if (moe)
+    e->weight_bytes_per_step += static_cast<int64_t>(c.n_layers) * (c.top_k + c.n_shared_experts) * 3 *
+                                static_cast<int64_t>(eg_bytes);
 
   cudaStream_t st;
   XLPK_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
@@ -423,20 +480,30 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   std::vector<LayerParams> lp(c.n_layers);
   Mat lm{};
   xlpk_status rc = XLPK_OK;
+  const int esz_saved = e->esz;
   for (size_t i = 0; i < mats.size() && rc == XLPK_OK; ++i) {
+    const MatPlan& mp = mats[i];
     Mat m{};
-    rc = pack_matrix(e, mats[i].src, mats[i].N, mats[i].K, e->packed + mats[i].off, &m, d_jobs, max_jobs, st);
+    e->esz = mp.role == R_ROUTER ? 2 : esz_saved;
+    rc = pack_matrix(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, d_jobs, max_jobs, st, mp.split);
+    e->esz = esz_saved;
     if (rc != XLPK_OK) break;
-    if (i + 1 == mats.size()) {
-      lm = m;
-    } else {
-      LayerParams& L = lp[i / 4];
-      switch (i % 4) {
-        case 0: L.qkv = m; break;
-        case 1: L.o = m; break;
-        case 2: L.gu = m; break;
-        default: L.down = m; break;
-      }
+    LayerParams* L = mp.layer >= 0 ? &lp[mp.layer] : nullptr;
+    switch (mp.role) {
+      case R_QKV: L->qkv = m; break;
+      case R_O: L->o = m; break;
+      case R_GU: L->gu = m; break;
+      case R_DOWN: L->down = m; break;
+      case R_ROUTER: L->router = m; break;
+      case R_EGU:
+        if (!L->egu.packed) L->egu = m;
+        L->egu_stride = static_cast<long long>(align_up(2 * eg_bytes, 256));
+        break;
+      case R_EDOWN:
+        if (!L->edown.packed) L->edown = m;
+        L->edown_stride = static_cast<long long>(align_up(eg_bytes, 256));
+        break;
+      default: lm = m; break;
     }
   }
   cudaFree(d_jobs);
@@ -480,11 +547,13 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const size_t o_x = take(sizeof(float) * B * H);
   const size_t o_q = take(sizeof(float) * B * qd);
   const size_t o_o = take(sizeof(float) * B * qd);
-  const size_t o_h = take(sizeof(float) * B * F);
+  const size_t o_h = take(sizeof(float) * B * std::max(F, S_moe * c.expert_ffn));
   const size_t o_pml = take(sizeof(float) * prow * group * 2);
   const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * e->G * B);
   const size_t o_li = take(sizeof(int) * e->G * B);
+  const size_t o_rte = take(sizeof(int) * c.n_layers * std::max(S_moe, 1));
+  const size_t o_rtw = take(sizeof(float) * c.n_layers * std::max(S_moe, 1));
   const size_t o_cnt = take(sizeof(unsigned) * cl.total);
   const size_t o_tok = take(sizeof(int) * B);
   const size_t o_st = take(sizeof(int) * 4);
@@ -545,6 +614,13 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.q = reinterpret_cast<float*>(e->ws + o_q);
   p.o = reinterpret_cast<float*>(e->ws + o_o);
   p.h = reinterpret_cast<float*>(e->ws + o_h);
+  p.route_exp = reinterpret_cast<int*>(e->ws + o_rte);
+  p.route_w = reinterpret_cast<float*>(e->ws + o_rtw);
+  p.E = c.n_experts;
+  p.topk = c.top_k;
+  p.nsh = c.n_shared_experts;
+  p.S = S_moe;
+  p.Fe = c.expert_ffn;
   p.part_ml = reinterpret_cast<float*>(e->ws + o_pml);
   p.part_o = reinterpret_cast<float*>(e->ws + o_po);
   p.lm_val = reinterpret_cast<float*>(e->ws + o_lv);
@@ -576,6 +652,7 @@ Params call_params(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out, const x
   p.forced = io ? io->forced_tokens_dev : nullptr;
   p.logits_out = io ? io->logits_dev : nullptr;
   p.hidden_out = io ? io->hidden_dev : nullptr;
+  p.experts_out = io ? io->experts_dev : nullptr;
   p.trace = io ? reinterpret_cast<unsigned long long*>(io->trace_dev) : nullptr;
   // L2 prefetch distance per CTA: a tuning knob read at each call (0 disables)
   if (const char* env = std::getenv("XLPK_L2_PREFETCH_KB")) p.l2_prefetch_bytes = std::atoll(env) * 1024;
@@ -722,11 +799,14 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   const size_t o_x = take(sizeof(float) * B * H);
   const size_t o_q = take(sizeof(float) * B * qd);
   const size_t o_o = take(sizeof(float) * B * qd);
-  const size_t o_h = take(sizeof(float) * B * F);
+  const int S_moe = h->base.S;
+  const size_t o_h = take(sizeof(float) * B * std::max(F, S_moe * c.expert_ffn));
   const size_t o_pml = take(sizeof(float) * prow * group * 2);
   const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * h->G * B);
   const size_t o_li = take(sizeof(int) * h->G * B);
+  const size_t o_rte = take(sizeof(int) * c.n_layers * std::max(S_moe, 1));
+  const size_t o_rtw = take(sizeof(float) * c.n_layers * std::max(S_moe, 1));
   if (off > XLPK_NOALLOC_SCRATCH_BYTES) {
     g_cuda_err = "xlpk_decode_noalloc: this handle needs " + std::to_string(off) +
                  " bytes of scratch, more than the " + std::to_string(XLPK_NOALLOC_SCRATCH_BYTES) +
@@ -741,6 +821,8 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   p.q = reinterpret_cast<float*>(sc + o_q);
   p.o = reinterpret_cast<float*>(sc + o_o);
   p.h = reinterpret_cast<float*>(sc + o_h);
+  p.route_exp = reinterpret_cast<int*>(sc + o_rte);
+  p.route_w = reinterpret_cast<float*>(sc + o_rtw);
   p.part_ml = reinterpret_cast<float*>(sc + o_pml);
   p.part_o = reinterpret_cast<float*>(sc + o_po);
   p.lm_val = reinterpret_cast<float*>(sc + o_lv);

@@ -90,6 +90,20 @@ class Engine:
         def lin(name):
             return _abi.xlpk_linear(_ptr(weights[name]), _ptr(weights.get(name + ".scale")))
 
+        import torch
+
+        # MoE: the C ABI takes each layer's experts as one [E][...] array per
+        # projection; per-expert tensors are stacked here (kept alive until
+        # create has packed them)
+        stacks = []
+
+        def stacked(prefix, n, proj):
+            if n == 0:
+                return _abi.xlpk_linear(0, 0)
+            t = torch.stack([weights[f"{prefix}{i}.{proj}"] for i in range(n)]).contiguous()
+            stacks.append(t)
+            return _abi.xlpk_linear(_ptr(t), 0)
+
         for l in range(L):
             p = f"layers.{l}."
             lw = self._layers[l]
@@ -98,6 +112,13 @@ class Engine:
             lw.wq, lw.wk, lw.wv, lw.wo = lin(p + "wq"), lin(p + "wk"), lin(p + "wv"), lin(p + "wo")
             if getattr(cfg, "n_experts", 0):
                 lw.router_dev = _ptr(weights[p + "router"])
+                E, S = cfg.n_experts, cfg.n_shared_experts
+                lw.we_gate = stacked(p + "experts.", E, "w_gate")
+                lw.we_up = stacked(p + "experts.", E, "w_up")
+                lw.we_down = stacked(p + "experts.", E, "w_down")
+                lw.ws_gate = stacked(p + "shared.", S, "w_gate")
+                lw.ws_up = stacked(p + "shared.", S, "w_up")
+                lw.ws_down = stacked(p + "shared.", S, "w_down")
             else:
                 lw.w_gate, lw.w_up, lw.w_down = lin(p + "w_gate"), lin(p + "w_up"), lin(p + "w_down")
         self._w = _abi.xlpk_weights(_ptr(weights["embed"]), _ptr(weights["final_norm"]),
@@ -108,6 +129,7 @@ class Engine:
         _check(lib.xlpk_create(C.byref(self._c), C.byref(self._w), C.byref(self._kv), C.byref(h)),
                "xlpk_create")
         self.h = h
+        del stacks   # packed into the library's own buffer
 
     def close(self) -> None:
         if getattr(self, "h", None):

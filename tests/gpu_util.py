@@ -21,6 +21,10 @@ class Run:
     tokens: torch.Tensor   # [n][B] int32 (host)
     logits: torch.Tensor   # [n][B][V] fp32 (host)
     hidden: torch.Tensor   # [n][B][H] fp32 (host)
+    experts: Optional[torch.Tensor] = None   # MoE: [n][L][B][top_k] int32 (host)
+
+
+ROUTER_GAP = 1e-6       # expert selections must match where the router probabilities differ by more
 
 
 def run_engine(m: workload.GpuModel, n_steps: int, unfused: bool = False, keep_logits: bool = True) -> Run:
@@ -30,9 +34,29 @@ def run_engine(m: workload.GpuModel, n_steps: int, unfused: bool = False, keep_l
     tok = torch.empty(n_steps, B, dtype=torch.int32, device=dev)
     lg = torch.empty(n_steps, B, cfg.vocab, dtype=torch.float32, device=dev) if keep_logits else None
     hd = torch.empty(n_steps, B, cfg.hidden, dtype=torch.float32, device=dev)
-    m.engine.decode(n_steps, tok, logits=lg, hidden=hd, unfused=unfused)
+    ex = torch.full((n_steps, cfg.n_layers, B, max(cfg.top_k, 1)), -1, dtype=torch.int32, device=dev) \
+        if cfg.is_moe else None
+    m.engine.decode(n_steps, tok, logits=lg, hidden=hd, experts=ex, unfused=unfused)
     m.engine.check()
-    return Run(tok.cpu(), lg.cpu() if lg is not None else None, hd.cpu())
+    return Run(tok.cpu(), lg.cpu() if lg is not None else None, hd.cpu(), ex.cpu() if ex is not None else None)
+
+
+def check_experts(run: Run, o: OracleDecoder, s: int, b: int) -> None:
+    """Engine's expert choice at step s vs the oracle's last step: the selected set
+    must agree wherever the k-th and (k+1)-th router probabilities differ by more
+    than ROUTER_GAP, and the order wherever adjacent selected ones do."""
+    cfg = o.cfg
+    k = cfg.top_k
+    for l in range(cfg.n_layers):
+        probs = o.last_router_probs[b][l]
+        ps = torch.sort(probs, descending=True).values
+        got = [int(v) for v in run.experts[s, l, b, :k]]
+        want = o.last_experts[b][l]
+        boundary = float(ps[k - 1] - ps[k]) if k < probs.numel() else 1.0
+        if boundary > ROUTER_GAP:
+            assert sorted(got) == sorted(want), f"step {s} layer {l}: experts {got} != oracle {want}"
+            if all(float(ps[i] - ps[i + 1]) > ROUTER_GAP for i in range(k - 1)):
+                assert got == want, f"step {s} layer {l}: expert order {got} != oracle {want}"
 
 
 def oracle_for(m: workload.GpuModel, max_seq: Optional[int] = None) -> OracleDecoder:
@@ -77,6 +101,8 @@ def compare_with_oracle(m: workload.GpuModel, run: Run, o: OracleDecoder, n_chec
             want = int(top2.indices[0])
             got = int(run.tokens[s, b])
             report.append(dict(step=s, b=b, hidden=e_h, logits=e_l, margin=margin, want=want, got=got))
+            if run.experts is not None:
+                check_experts(run, o, s, b)
             assert e_h <= tol, f"step {s} seq {b}: hidden rel L2 {e_h:.3e} > {tol}"
             assert e_l <= tol, f"step {s} seq {b}: logits rel L2 {e_l:.3e} > {tol}"
             if margin > ARGMAX_MARGIN:
