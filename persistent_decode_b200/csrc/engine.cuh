@@ -33,6 +33,8 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "params.h"
@@ -412,6 +414,30 @@ __device__ __forceinline__ float dot8_bf16(const uint4 w, const float4 lo, const
   return acc;
 }
 
+// Two e4m3 codes (low byte first) -> two floats, through the CUDA fp8
+// conversion to half precision (every e4m3 value is exact in fp16 and fp32).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Sum over 16 e4m3 codes (one 16-byte vector) times 16 fp32 activations
+// x0 = elements 0..3, x1 = 4..7, x2 = 8..11, x3 = 12..15.
+__device__ __forceinline__ float dot16_e4m3(const uint4 w, const float4 x0, const float4 x1, const float4 x2,
+                                            const float4 x3) {
+  float acc = 0.f;
+  float2 f;
+  f = e4m3x2_to_float2(w.x & 0xffffu);  acc = fmaf(f.x, x0.x, fmaf(f.y, x0.y, acc));
+  f = e4m3x2_to_float2(w.x >> 16);      acc = fmaf(f.x, x0.z, fmaf(f.y, x0.w, acc));
+  f = e4m3x2_to_float2(w.y & 0xffffu);  acc = fmaf(f.x, x1.x, fmaf(f.y, x1.y, acc));
+  f = e4m3x2_to_float2(w.y >> 16);      acc = fmaf(f.x, x1.z, fmaf(f.y, x1.w, acc));
+  f = e4m3x2_to_float2(w.z & 0xffffu);  acc = fmaf(f.x, x2.x, fmaf(f.y, x2.y, acc));
+  f = e4m3x2_to_float2(w.z >> 16);      acc = fmaf(f.x, x2.z, fmaf(f.y, x2.w, acc));
+  f = e4m3x2_to_float2(w.w & 0xffffu);  acc = fmaf(f.x, x3.x, fmaf(f.y, x3.y, acc));
+  f = e4m3x2_to_float2(w.w >> 16);      acc = fmaf(f.x, x3.z, fmaf(f.y, x3.w, acc));
+  return acc;
+}
+
 __device__ __forceinline__ uint16_t f2bf(float v) {
   __nv_bfloat16 h = __float2bfloat16_rn(v);
   return *reinterpret_cast<uint16_t*>(&h);
@@ -597,15 +623,15 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
 // accumulates it over the group's k-chunks; `epi(pair, acc0, acc1)` runs on
 // the reduced sums (identical in every lane).
 // [q0, q1) overrides the CTA's pair range (default: the even split of m's pairs).
-template <int B, class Epi>
-__device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp,
-                                          int where, const float (&rn)[B], Epi& epi, int q0 = -1,
-                                          int q1 = -1) {
+template <int B, bool FP8, class Epi>
+__device__ __noinline__ void consume_gemv_t(const Params& p, Ctx& cx, const Mat& m, RingPos& rp,
+                                            int where, const float (&rn)[B], Epi& epi, int q0, int q1) {
   const int NP = m.N >> 1;
   const int p0 = q0 >= 0 ? q0 : split_point(cx.c, NP, p.G);
   const int p1 = q0 >= 0 ? q1 : split_point(cx.c + 1, NP, p.G);
-  const int nkc = m.K / m.KC;
-  const int nv = m.KC >> 3;   // 16-byte vectors per row chunk
+  const int KC = m.KC;
+  const int nkc = m.K / KC;
+  const int nv = KC >> 3;     // 16-byte vectors per row chunk (bf16)
   const int nvK = m.K >> 3;
   const uint32_t act_lo_s = smem_addr(cx.act);
   const uint32_t act_hi_s = act_lo_s + B * nvK * 16;
@@ -617,7 +643,36 @@ __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m
     for (int kc = 0; kc < nkc; ++kc) {
       const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
       const bool ok = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
-      if (ok && cx.warp < gp) {
+      if constexpr (FP8) {
+        if (ok && cx.warp < gp) {
+        // e4m3 tile: lane vectors of 16 codes, each inside one 128-column
+        // scale block; the block's sum is scaled once
+        const int nv8 = KC >> 4;
+        const uint32_t base = smem_addr(cx.ring) + rp.slot * kSlotBytes;
+        const uint32_t r0 = base + (2 * cx.warp) * KC;
+        const uint32_t r1 = r0 + KC;
+        const uint32_t s0 = base + 2 * gp * KC + (2 * cx.warp) * (KC >> 5);
+        const uint32_t s1 = s0 + (KC >> 5);
+        const uint32_t alo = act_lo_s + ((kc * KC) >> 3) * 16;
+        const uint32_t ahi = act_hi_s + ((kc * KC) >> 3) * 16;
+#pragma unroll 2
+        for (int v = cx.lane; v < nv8; v += 32) {
+          const uint4 w0 = lds_u4(r0 + v * 16);
+          const uint4 w1 = lds_u4(r1 + v * 16);
+          const float sc0 = __uint_as_float(lds_u1(s0 + (v >> 3) * 4));
+          const float sc1 = __uint_as_float(lds_u1(s1 + (v >> 3) * 4));
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            const float4 x0 = lds_f4(alo + (b * nvK + 2 * v) * 16);
+            const float4 x1 = lds_f4(ahi + (b * nvK + 2 * v) * 16);
+            const float4 x2 = lds_f4(alo + (b * nvK + 2 * v + 1) * 16);
+            const float4 x3 = lds_f4(ahi + (b * nvK + 2 * v + 1) * 16);
+            a0[b] = fmaf(sc0, dot16_e4m3(w0, x0, x1, x2, x3), a0[b]);
+            a1[b] = fmaf(sc1, dot16_e4m3(w1, x0, x1, x2, x3), a1[b]);
+          }
+        }
+        }
+      } else if (ok && cx.warp < gp) {
         const uint32_t r0 = smem_addr(cx.ring) + rp.slot * kSlotBytes + (2 * cx.warp) * nv * 16;
         const uint32_t r1 = r0 + nv * 16;
         const uint32_t alo = act_lo_s + (kc * nv) * 16;
@@ -651,6 +706,17 @@ __device__ __noinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m
       epi(g0 + cx.warp, a0, a1, cx.lane);
     }
   }
+}
+
+// e4m3 and bf16 tiles are separate instantiations, so neither inner loop
+// carries the other's code.
+template <int B, class Epi>
+__device__ __forceinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where,
+                                             const float (&rn)[B], Epi& epi, int q0 = -1, int q1 = -1) {
+  if (m.fp8)
+    consume_gemv_t<B, true>(p, cx, m, rp, where, rn, epi, q0, q1);
+  else
+    consume_gemv_t<B, false>(p, cx, m, rp, where, rn, epi, q0, q1);
 }
 
 // QKV epilogue: RoPE on q/k pairs, q -> workspace, bf16 k/v -> cache at pos.
@@ -968,7 +1034,7 @@ template <int B, int D>
 __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s, RingPos& rp,
                                          bool fused) {
   static_assert(kMaxGroup == 4, "query heads per kv head fill at most rows 0..3 of the A tile");
-  constexpr int P = (kSlotBytes / 2) / (D * 2);               // positions per chunk
+  constexpr int P = (kTileBytes / 2) / (D * 2);               // positions per chunk
   constexpr int NPG = P / 16;                                 // position groups per chunk
   constexpr int NDS = kConsumerWarps / NPG;                   // p.V dim splits
   constexpr int DW = D / NDS;                                 // p.V dims per warp
@@ -1051,7 +1117,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     }
     const unsigned long long tc0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
     const uint32_t kt = ring_s + rp.slot * kSlotBytes;
-    const uint32_t vt = kt + kSlotBytes / 2;
+    const uint32_t vt = kt + kTileBytes / 2;
     if (have_tile && pg * 16 < npos) {   // warp-uniform
       if (npos > n_old && (n_old >> 4) == pg) {
         // this step's K/V entry of the head, from the cache (written by the QKV stage)
@@ -1331,7 +1397,7 @@ __device__ __forceinline__ const Mat& stage_mat(const LayerParams& L, int kind) 
 }
 
 // Consumers: one stage.  Returns false once the CTA is aborting.
-template <int B, int D>
+template <int B, int D, bool MOE>
 __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s,
                                            RingPos& rp, bool fused) {
   const unsigned G = static_cast<unsigned>(p.G);
@@ -1441,7 +1507,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_OPROJ, G * S1, where, fused)) return false;
       load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr, SIDE_NONE, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      if (p.E > 0) {
+      if constexpr (MOE) {
         if constexpr (B == 1) {
           // router (all E logits in every CTA), routing, then this CTA's groups
           // of the virtual [slot][pair] gate/up space
@@ -1465,11 +1531,11 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
     }
     default: {  // ST_DOWN
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_GATEUP, G * S1, where, fused)) return false;
-      const int K = p.E > 0 ? p.S * p.Fe : p.F;
+      const int K = MOE ? p.S * p.Fe : p.F;
       load_act<B>(p, cx, K, SRC_PLAIN, p.h, nullptr, nullptr, SIDE_RESID, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
-      if (p.E > 0) {
+      if constexpr (MOE) {
         // K runs over [slot][expert column]: the producer streams each slot's expert
         Mat v = L.edown;
         v.K = K;
@@ -1581,6 +1647,7 @@ struct Cursor {
                        // MoE gate/up experts: next virtual group / end
   int kc, nkc, KC;
   int esz;             // bytes per weight element of the current matrix
+  int trow;            // packed bytes per row of one tile (codes/values + FP8 scales)
   const uint8_t* src;  // GEMV: next tile
   int phase;           // MoE gate/up: 0 router, 1 experts
   int slot, grp;       // MoE down: slot of the next tile, group index within the CTA's span
@@ -1615,12 +1682,22 @@ __device__ __forceinline__ void cursor_next_stage(const Params& p, Cursor<B>& cu
   }
 }
 
-enum CursorResult : int { CUR_DONE = 0, CUR_TILE = 1, CUR_BLOCKED = 2 };
+enum CursorResult : int { CUR_DONE = 0, CUR_TILE = 1, CUR_BLOCKED = 2, CUR_RUN = 3 };
 
-template <int B>
-__device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>& cu, Tile& t) {
+// A dense GEMV stage of one CTA is one contiguous byte range: n1 tiles of b1
+// bytes (full groups of 8 row pairs), then n2 tiles of b2 bytes (the last,
+// partial group).  The producer drains it from registers.
+struct Run {
+  const uint8_t* src;
+  int n1, n2;
+  uint32_t b1, b2;
+  int stage, layer, step;
+};
+
+template <int B, bool MOE>
+__device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>& cu, Tile& t, Run* run) {
   while (!cu.done) {
-    const bool moe = p.E > 0 && (cu.kind == ST_GATEUP || cu.kind == ST_DOWN);
+    const bool moe = MOE && (cu.kind == ST_GATEUP || cu.kind == ST_DOWN);
     if (!cu.open) {
       cu.open = true;
       cu.esz = p.esz;
@@ -1638,6 +1715,7 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         cu.nkc = r.K / r.KC;
         cu.KC = r.KC;
         cu.esz = 2;
+        cu.trow = packed_row_bytes(r, r.KC);
         cu.src = r.packed;
       } else if (moe) {   // MoE down: the CTA's output rows, every slot's expert in turn
         const Mat& m = p.layers[cu.l].edown;
@@ -1656,7 +1734,8 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         cu.kc = 0;
         cu.nkc = m.K / m.KC;
         cu.KC = m.KC;
-        cu.src = m.packed + static_cast<size_t>(2) * cu.a * m.K * p.esz;
+        cu.trow = packed_row_bytes(m, m.KC);
+        cu.src = m.packed + static_cast<size_t>(2) * cu.a * packed_row_bytes(m, m.K);
       }
     }
     t.stage = stage_index(p, cu.kind, cu.l);
@@ -1671,7 +1750,7 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         t.y = static_cast<int>(kv_row(p, cu.l, b, g, j * p.attn_pos_per_tile) / p.d);
         t.rows = min(p.attn_pos_per_tile, p.pos0[b] + cu.s + 1 - j * p.attn_pos_per_tile);
         t.src = nullptr;
-        t.bytes = kSlotBytes;
+        t.bytes = kTileBytes;
         t.attn = true;
         return CUR_TILE;
       }
@@ -1713,9 +1792,22 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         }
         return CUR_TILE;
       }
+    } else if (cu.a < cu.a_end && !(moe && cu.kind == ST_GATEUP) && cu.kc == 0) {
+      // a whole dense stage (the MoE router goes tile by tile)
+      const int np = cu.a_end - cu.a;
+      run->src = cu.src;
+      run->n1 = (np / kPairsPerTile) * cu.nkc;
+      run->b1 = 2u * kPairsPerTile * cu.trow;
+      run->n2 = (np % kPairsPerTile) ? cu.nkc : 0;
+      run->b2 = 2u * (np % kPairsPerTile) * cu.trow;
+      run->stage = t.stage;
+      run->layer = t.layer;
+      run->step = t.step;
+      cu.a = cu.a_end;
+      return CUR_RUN;
     } else if (cu.a < cu.a_end) {
       const int gp = min(kPairsPerTile, cu.a_end - cu.a);
-      t.bytes = 2u * gp * cu.KC * cu.esz;
+      t.bytes = 2u * gp * cu.trow;
       t.src = cu.src;
       cu.src += t.bytes;
       if (++cu.kc == cu.nkc) {
@@ -1769,7 +1861,7 @@ __device__ __noinline__ bool route_wait(const Params& p, SmemCtl* ctl, int want,
 // `p.l2_prefetch_bytes` ahead.  Weights do not depend on activations, so both
 // run ahead of the consumers across stage boundaries; only attention chunks
 // wait for the previous step's KV write of their layer.
-template <int B>
+template <int B, bool MOE>
 __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
   RingPos rp;
   const uint64_t pol = evict_first_policy();
@@ -1779,21 +1871,77 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
   long long ahead = 0;
   bool pc_live = true;
   int cur_stage = -1, cur_step = -1;
+  // The copy cursor's current tile and dense run live in scalars (registers);
+  // only the slow path (stage changes, attention, MoE) goes through the
+  // memory-resident Cursor/Tile/Run structures.
   Tile t, tp;
+  Run nr, prun;
+  const uint8_t* r_src = nullptr;
+  int r_n1 = 0, r_n2 = 0;
+  uint32_t r_b1 = 0, r_b2 = 0;
+  int r_stage = 0, r_layer = 0, r_step = 0;
+  const uint8_t* pf_src = nullptr;   // the prefetch cursor's current dense range
+  long long pf_left = 0;
   for (;;) {
-    int r = cursor_next<B>(p, cx.c, cx.ctl, cc, t);
-    if (r == CUR_BLOCKED) {
-      // the next tile is an expert chosen by this CTA's own consumers: wait
-      // (bounded) until they publish the layer's routing
-      if (!route_wait(p, cx.ctl, route_want(p, cc.s, cc.l), where_code(cc.kind, cc.l, cc.s) | (1 << 15))) break;
-      r = cursor_next<B>(p, cx.c, cx.ctl, cc, t);
+    const uint8_t* t_src;
+    uint32_t tb;
+    bool t_attn = false;
+    int t_stage, t_layer, t_step, t_y = 0;
+    if (r_n1 + r_n2 == 0) {
+      int r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+      if (r == CUR_BLOCKED) {
+        // the next tile is an expert chosen by this CTA's own consumers: wait
+        // (bounded) until they publish the layer's routing
+        if (!route_wait(p, cx.ctl, route_want(p, cc.s, cc.l), where_code(cc.kind, cc.l, cc.s) | (1 << 15))) break;
+        r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+      }
+      if (r == CUR_RUN) {
+        r_src = nr.src;
+        r_n1 = nr.n1;
+        r_n2 = nr.n2;
+        r_b1 = nr.b1;
+        r_b2 = nr.b2;
+        r_stage = nr.stage;
+        r_layer = nr.layer;
+        r_step = nr.step;
+      } else if (r != CUR_TILE) {
+        break;
+      }
     }
-    if (r != CUR_TILE) break;
-    const uint32_t tb = t.bytes;
+    if (r_n1 + r_n2 > 0) {   // next tile of the dense run
+      t_src = r_src;
+      tb = r_n1 ? r_b1 : r_b2;
+      if (r_n1) --r_n1; else --r_n2;
+      r_src += tb;
+      t_stage = r_stage;
+      t_layer = r_layer;
+      t_step = r_step;
+    } else {
+      t_src = t.src;
+      tb = t.bytes;
+      t_attn = t.attn;
+      t_stage = t.stage;
+      t_layer = t.layer;
+      t_step = t.step;
+      t_y = t.y;
+    }
     ahead -= tb;
     while (pc_live && ahead < p.l2_prefetch_bytes) {
-      const int pr = cursor_next<B>(p, cx.c, cx.ctl, pc, tp);
+      if (pf_left > 0) {   // dense range: prefetch in tile-sized pieces
+        const uint32_t nb = static_cast<uint32_t>(min(pf_left, static_cast<long long>(kTileBytes)));
+        prefetch_l2(pf_src, nb);
+        pf_src += nb;
+        pf_left -= nb;
+        ahead += nb;
+        continue;
+      }
+      const int pr = cursor_next<B, MOE>(p, cx.c, cx.ctl, pc, tp, &prun);
       if (pr == CUR_BLOCKED) break;   // resume once the routing is known
+      if (pr == CUR_RUN) {
+        pf_src = prun.src;
+        pf_left = static_cast<long long>(prun.n1) * prun.b1 + static_cast<long long>(prun.n2) * prun.b2;
+        continue;
+      }
       pc_live = pr == CUR_TILE;
       if (!pc_live) break;
       if (!tp.attn) {
@@ -1808,40 +1956,41 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
       }
       ahead += tp.bytes;
     }
-    if (t.stage != cur_stage || t.step != cur_step) {
+    if (t_stage != cur_stage || t_step != cur_step) {
       if (cur_stage >= 0) trace_stamp(p, cur_step, cur_stage, 5);
-      cur_stage = t.stage;
-      cur_step = t.step;
-      trace_stamp(p, t.step, t.stage, 4);
-      if (t.attn) {
+      cur_stage = t_stage;
+      cur_step = t_step;
+      trace_stamp(p, t_step, t_stage, 4);
+      if (t_attn) {
         // KV rows up to pos-1 were written by this layer's QKV stage of earlier
         // steps (or before the launch); make sure the previous step's write is
         // complete before reading it through the async proxy.
         if (fused) {
-          const unsigned target = static_cast<unsigned>(p.G) * static_cast<unsigned>(p.step_base + t.step);
-          const int where = where_code(ST_ATTN, t.layer, t.step) | (1 << 15);
-          if (!counter_wait(p, cx.ctl, p.cnt + t.layer * ST_LAYER + ST_QKV, target, where)) break;
+          const unsigned target = static_cast<unsigned>(p.G) * static_cast<unsigned>(p.step_base + t_step);
+          const int where = where_code(ST_ATTN, t_layer, t_step) | (1 << 15);
+          if (!counter_wait(p, cx.ctl, p.cnt + t_layer * ST_LAYER + ST_QKV, target, where)) break;
         }
         fence_proxy_async_global();
       }
     }
-    const int where = where_code(t.stage % ST_LAYER, t.layer, t.step) | (1 << 15);
     const uint32_t eb = smem_addr(&cx.ctl->empty[rp.slot]);
     // A full ring only means the consumers are waiting on a dependency; give
     // their own (bounded) wait the chance to time out first, so the reported
     // failure names the dependency rather than this stall.
-    if (!mbar_try_wait(eb, rp.phase ^ 1u) && !ring_wait_slow(p, cx.ctl, eb, rp.phase ^ 1u, where, 2)) break;
+    if (!mbar_try_wait(eb, rp.phase ^ 1u) &&
+        !ring_wait_slow(p, cx.ctl, eb, rp.phase ^ 1u, where_code(t_stage % ST_LAYER, t_layer, t_step) | (1 << 15), 2))
+      break;
     const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
     mbar_expect_tx(fb, tb);
     const uint32_t dst = smem_addr(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes);
-    if (t.attn) {
+    if (t_attn) {
       const int box = p.attn_pos_per_tile * 128;
       for (int x = 0; x < p.d; x += 64) {
-        tma_load_2d(dst + (x >> 6) * box, &p.tmap_k, x, t.y, fb, pol);
-        tma_load_2d(dst + kSlotBytes / 2 + (x >> 6) * box, &p.tmap_v, x, t.y, fb, pol);
+        tma_load_2d(dst + (x >> 6) * box, &p.tmap_k, x, t_y, fb, pol);
+        tma_load_2d(dst + kTileBytes / 2 + (x >> 6) * box, &p.tmap_v, x, t_y, fb, pol);
       }
     } else {
-      bulk_g2s(dst, t.src, t.bytes, fb, pol);
+      bulk_g2s(dst, t_src, tb, fb, pol);
     }
     rp.next(p.nslot);
   }
@@ -1850,56 +1999,56 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
   drain_ring(p, cx, rp, p.nslot);
 }
 
-template <int B, int D>
+template <int B, int D, bool MOE>
 __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
   RingPos rp;
   if (fused) {
     for (int s = 0; s < p.n_steps; ++s) {
       for (int l = 0; l < p.L; ++l)
         for (int k = 0; k < ST_LAYER; ++k)
-          if (!consume_stage<B, D>(p, cx, k, l, s, rp, true)) return;
-      if (!consume_stage<B, D>(p, cx, ST_LM, 0, s, rp, true)) return;
+          if (!consume_stage<B, D, MOE>(p, cx, k, l, s, rp, true)) return;
+      if (!consume_stage<B, D, MOE>(p, cx, ST_LM, 0, s, rp, true)) return;
     }
   } else {
-    consume_stage<B, D>(p, cx, kind0, l0, s0, rp, false);
+    consume_stage<B, D, MOE>(p, cx, kind0, l0, s0, rp, false);
   }
 }
 
 // The persistent engine: one launch decodes p.n_steps tokens.
-template <int B, int D>
+template <int B, int D, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) engine_persistent(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctx cx = make_ctx(smem, p);
   init_ring(p, cx);
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<B>(p, cx, 0, 0, 0, true);
+    if (cx.lane == 0) producer_main<B, MOE>(p, cx, 0, 0, 0, true);
     __syncwarp();
   } else {
-    consumer_main<B, D>(p, cx, 0, 0, 0, true);
+    consumer_main<B, D, MOE>(p, cx, 0, 0, 0, true);
   }
 }
 
 // Kernel-per-op baseline: one launch runs one stage (same tiles, no waits).
-template <int B, int D>
+template <int B, int D, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constant__ Params p, int kind,
                                                             int layer, int step) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctx cx = make_ctx(smem, p);
-  if (p.E > 0 && kind == ST_DOWN && cx.tid < p.S) {
+  if (MOE && kind == ST_DOWN && cx.tid < p.S) {
     // the routing was computed by the gate/up launch: take CTA 0's record
     cx.ctl->route_exp[cx.tid] = p.route_exp[layer * p.S + cx.tid];
     cx.ctl->route_w[cx.tid] = p.route_w[layer * p.S + cx.tid];
   }
   init_ring(p, cx);
-  if (p.E > 0 && kind == ST_DOWN) {
+  if (MOE && kind == ST_DOWN) {
     if (cx.tid == 0) cx.ctl->route_seq = route_want(p, step, layer);
     __syncthreads();
   }
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<B>(p, cx, kind, layer, step, false);
+    if (cx.lane == 0) producer_main<B, MOE>(p, cx, kind, layer, step, false);
     __syncwarp();
   } else {
-    consumer_main<B, D>(p, cx, kind, layer, step, false);
+    consumer_main<B, D, MOE>(p, cx, kind, layer, step, false);
   }
 }
 

@@ -14,7 +14,8 @@ namespace xlpk {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;      // + one producer warp
-constexpr int kSlotBytes = 32768;                     // one staging slot of the ring
+constexpr int kTileBytes = 32768;                     // data of one tile: weights, or a K and a V chunk
+constexpr int kSlotBytes = kTileBytes + 1024;         // ring slot stride: + FP8 tiles' per-row block scales
 constexpr int kMaxSlots = 8;
 constexpr int kMaxBatch = 8;
 constexpr int kMaxGroup = 4;                          // query heads per kv head
@@ -57,14 +58,24 @@ struct CounterLayout {
 // Tile (group, chunk) holds [2*gp rows][KC cols] contiguously, and the tiles
 // of a CTA follow each other, so the CTA's whole span is one contiguous range
 // streamed front to back.
+//
+// FP8 (e4m3) matrices: each tile's [2*gp rows][KC codes] is followed by the
+// rows' block scales [2*gp rows][KC/128] fp32 (the scale of the row's 128x128
+// block for each 128 columns of the chunk), so a tile still arrives as one
+// bulk copy; a packed row then takes K + K/32 bytes.
 struct Mat {
   const uint8_t* packed;
-  const float* scales;   // FP8: per logical row, K/128 fp32 scales; else nullptr
+  const float* scales;   // unused (FP8 scales travel inside the tiles)
   int N;                 // logical rows (even)
   int K;                 // columns
   int KC;                // k-chunk (divides K)
-  int pad;
+  int fp8;               // 1: e4m3 codes + in-tile block scales; 0: bf16
 };
+
+// Bytes of one packed row over `k` columns (codes or bf16 values, plus FP8 scales).
+__host__ __device__ __forceinline__ int packed_row_bytes(const Mat& m, int k) {
+  return m.fp8 ? k + k / 32 : 2 * k;
+}
 
 struct LayerParams {
   Mat qkv;     // rows: q heads (RoPE pairs interleaved), k heads (interleaved), v heads

@@ -47,7 +47,19 @@ struct PackJob {
   const uint8_t* src;   // source row
   long long dst;        // byte offset of the row's first chunk in the packed buffer
   long long stride;     // bytes between consecutive chunks of this row
+  const float* scale;   // FP8: the row's block-scale row ([K/128] fp32), else null
+  long long sdst;       // FP8: byte offset of the row's scales in its first tile
 };
+
+// FP8: one thread per (row, chunk): the chunk's KC/128 block scales of the row.
+__global__ void pack_scales_kernel(const PackJob* jobs, int njobs, uint8_t* out, int nchunk, int kb_per_chunk) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<long long>(njobs) * nchunk) return;
+  const int jb = static_cast<int>(t / nchunk), c = static_cast<int>(t - static_cast<long long>(jb) * nchunk);
+  const PackJob j = jobs[jb];
+  float* d = reinterpret_cast<float*>(out + j.sdst + c * j.stride);
+  for (int k = 0; k < kb_per_chunk; ++k) d[k] = j.scale[c * kb_per_chunk + k];
+}
 
 // One warp per packed row: chunk c of the row goes to dst + c*stride.
 __global__ void pack_rows_kernel(const PackJob* jobs, int njobs, uint8_t* out, int row_bytes,
@@ -66,9 +78,11 @@ __global__ void pack_rows_kernel(const PackJob* jobs, int njobs, uint8_t* out, i
 
 long long split_host(long long c, long long n, long long G) { return (c * n) / G; }
 
+// Largest k-chunk dividing K whose tile of 8 row pairs fits kTileBytes (FP8:
+// also a whole number of 128-column scale blocks).
 int pick_kc(int K, int esz) {
-  const int vec = 16 / esz;
-  const int cap = kSlotBytes / (2 * kPairsPerTile * esz);
+  const int vec = esz == 1 ? 128 : 16 / esz;
+  const int cap = kTileBytes / (2 * kPairsPerTile * esz);
   for (int kc = std::min(K, cap); kc >= vec; --kc)
     if (K % kc == 0 && kc % vec == 0) return kc;
   return 0;
@@ -83,6 +97,14 @@ struct MatSrc {
   const uint8_t* a;   // QKV: wq; GATEUP: gate; PLAIN: w
   const uint8_t* b;   // QKV: wk; GATEUP: up
   const uint8_t* c;   // QKV: wv
+  const float* sa = nullptr;   // FP8 block scales [rows/128][K/128] of a, b, c
+  const float* sb = nullptr;
+  const float* sc = nullptr;
+};
+
+struct SrcRow {
+  const uint8_t* w;
+  const float* s;   // FP8: the row's block-scale row
 };
 
 }  // namespace
@@ -116,20 +138,27 @@ struct xlpk_engine {
 
 namespace {
 
-template <int B, int D>
+template <int B, int D, bool MOE>
 void launch_stage_impl(const Params& p, int kind, int layer, int step, int G, int smem,
                        cudaStream_t st) {
-  engine_stage<B, D><<<G, kThreads, smem, st>>>(p, kind, layer, step);
+  engine_stage<B, D, MOE><<<G, kThreads, smem, st>>>(p, kind, layer, step);
 }
 
-template <int B, int D>
+// Dense and MoE models use separate kernel instantiations, so the dense
+// kernels carry none of the routing code.
+template <int B, int D, bool MOE = false>
 void bind_kernels(xlpk_engine* e) {
-  e->kern_persistent = reinterpret_cast<const void*>(&engine_persistent<B, D>);
-  e->kern_stage = reinterpret_cast<const void*>(&engine_stage<B, D>);
-  e->launch_stage = &launch_stage_impl<B, D>;
+  e->kern_persistent = reinterpret_cast<const void*>(&engine_persistent<B, D, MOE>);
+  e->kern_stage = reinterpret_cast<const void*>(&engine_stage<B, D, MOE>);
+  e->launch_stage = &launch_stage_impl<B, D, MOE>;
 }
 
-bool bind_by_shape(xlpk_engine* e, int B, int D) {
+bool bind_by_shape(xlpk_engine* e, int B, int D, bool moe) {
+  if (moe) {   // MoE is built for batch 1
+    if (B == 1 && D == 64) return bind_kernels<1, 64, true>(e), true;
+    if (B == 1 && D == 128) return bind_kernels<1, 128, true>(e), true;
+    return false;
+  }
 #define XLPK_BIND(b, d)          \
   if (B == b && D == d) {        \
     bind_kernels<b, d>(e);       \
@@ -147,16 +176,21 @@ bool bind_by_shape(xlpk_engine* e, int B, int D) {
   return false;
 }
 
-// Logical row n of a packed matrix -> source row pointer.
-const uint8_t* source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_config& c) {
+// Logical row n of a packed matrix -> source row (and its FP8 block-scale row).
+SrcRow source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_config& c) {
   const long long row_bytes = static_cast<long long>(K) * esz;
   const long long pr = n >> 1;
   const int r = static_cast<int>(n & 1);
+  const uint8_t* base = nullptr;
+  const float* sbase = nullptr;
+  long long row = 0;
   switch (ms.kind) {
     case MatKind::PLAIN:
-      return ms.a + n * row_bytes;
+      base = ms.a, sbase = ms.sa, row = n;
+      break;
     case MatKind::GATEUP:
-      return (r == 0 ? ms.a : ms.b) + pr * row_bytes;
+      base = r == 0 ? ms.a : ms.b, sbase = r == 0 ? ms.sa : ms.sb, row = pr;
+      break;
     case MatKind::QKV: {
       const long long half = c.head_dim / 2;
       const long long hq = static_cast<long long>(c.n_q_heads) * half;
@@ -165,14 +199,19 @@ const uint8_t* source_row(const MatSrc& ms, long long n, int K, int esz, const x
         const bool isq = pr < hq;
         const long long pp = isq ? pr : pr - hq;
         const long long head = pp / half, i = pp % half;
-        const long long row = head * c.head_dim + i + r * half;
-        return (isq ? ms.a : ms.b) + row * row_bytes;
+        row = head * c.head_dim + i + r * half;
+        base = isq ? ms.a : ms.b, sbase = isq ? ms.sa : ms.sb;
+      } else {
+        row = 2 * (pr - hq - hk) + r;
+        base = ms.c, sbase = ms.sc;
       }
-      const long long pv = pr - hq - hk;
-      return ms.c + (2 * pv + r) * row_bytes;
+      break;
     }
   }
-  return nullptr;
+  SrcRow out;
+  out.w = base + row * row_bytes;
+  out.s = sbase ? sbase + (row / 128) * (K / 128) : nullptr;
+  return out;
 }
 
 // Pack one matrix into `dst` (device) in stream order; returns the Mat view.
@@ -183,6 +222,12 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
   const int esz = e->esz;
   const int KC = pick_kc(K, esz);
   if (KC == 0) return XLPK_ERR_UNSUPPORTED;
+  const bool fp8 = esz == 1;
+  if (fp8 && (!ms.sa || (ms.kind != MatKind::PLAIN && !ms.sb) || (ms.kind == MatKind::QKV && !ms.sc)))
+    return XLPK_ERR_INVALID_ARG;
+  // bytes per packed row over a chunk / over K (codes + FP8 block scales)
+  const long long tile_row = static_cast<long long>(KC) * esz + (fp8 ? KC / 32 : 0);
+  const long long full_row = static_cast<long long>(K) * esz + (fp8 ? K / 32 : 0);
   const long long NP = N / 2, G = split;
   std::vector<PackJob> jobs;
   jobs.reserve(static_cast<size_t>(N));
@@ -192,13 +237,15 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
     for (long long lp = 0; lp < npc; ++lp) {
       const long long j = lp / kPairsPerTile, w = lp % kPairsPerTile;
       const long long gp = std::min<long long>(kPairsPerTile, npc - kPairsPerTile * j);
-      const long long group_off =
-          (2 * p0 * K + 2LL * kPairsPerTile * j * K) * static_cast<long long>(esz);
+      const long long group_off = (2 * p0 + 2LL * kPairsPerTile * j) * full_row;
       for (int r = 0; r < 2; ++r) {
+        const SrcRow sr = source_row(ms, 2 * (p0 + lp) + r, K, esz, e->cfg);
         PackJob pj;
-        pj.src = source_row(ms, 2 * (p0 + lp) + r, K, esz, e->cfg);
+        pj.src = sr.w;
         pj.dst = group_off + (2 * w + r) * static_cast<long long>(KC) * esz;
-        pj.stride = 2 * gp * static_cast<long long>(KC) * esz;
+        pj.stride = 2 * gp * tile_row;
+        pj.scale = sr.s;
+        pj.sdst = group_off + 2 * gp * static_cast<long long>(KC) * esz + (2 * w + r) * (KC / 32);
         jobs.push_back(pj);
       }
     }
@@ -211,6 +258,12 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
     const int blocks = static_cast<int>((n * 32 + threads - 1) / threads);
     pack_rows_kernel<<<blocks, threads, 0, st>>>(d_jobs, static_cast<int>(n), dst, row_bytes, chunk_bytes);
     XLPK_CUDA(cudaGetLastError());
+    if (fp8) {
+      const long long nt = static_cast<long long>(n) * (K / KC);
+      pack_scales_kernel<<<static_cast<int>((nt + threads - 1) / threads), threads, 0, st>>>(
+          d_jobs, static_cast<int>(n), dst, K / KC, KC / 128);
+      XLPK_CUDA(cudaGetLastError());
+    }
     XLPK_CUDA(cudaStreamSynchronize(st));
   }
   out->packed = dst;
@@ -218,7 +271,7 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
   out->N = N;
   out->K = K;
   out->KC = KC;
-  out->pad = 0;
+  out->fp8 = fp8 ? 1 : 0;
   return XLPK_OK;
 }
 
@@ -271,7 +324,12 @@ xlpk_status validate_config(const xlpk_config* c) {
   if (c->head_dim != 64 && c->head_dim != 128) return XLPK_ERR_UNSUPPORTED;
   if (c->n_q_heads / c->n_kv_heads > kMaxGroup) return XLPK_ERR_UNSUPPORTED;
   if (c->batch != 1 && c->batch != 2 && c->batch != 4 && c->batch != 8) return XLPK_ERR_UNSUPPORTED;
-  if (c->weight_dtype != XLPK_DTYPE_BF16) return XLPK_ERR_UNSUPPORTED;
+  if (c->weight_dtype == XLPK_DTYPE_FP8_E4M3) {
+    // 128x128 scale blocks tile every matrix exactly
+    const int qd = c->n_q_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
+    if (c->n_experts > 0) return XLPK_ERR_UNSUPPORTED;
+    if (c->hidden % 128 || qd % 128 || kvd % 128 || c->ffn % 128 || c->vocab % 128) return XLPK_ERR_UNSUPPORTED;
+  }
   if (c->n_experts > 0) {
     if (c->top_k < 1 || c->top_k > c->n_experts || c->expert_ffn <= 0) return XLPK_ERR_INVALID_ARG;
     if (c->n_experts > kMaxExperts || c->top_k + c->n_shared_experts > kMaxMoeSlots || c->n_experts % 2)
@@ -293,6 +351,16 @@ xlpk_status validate_weights(const xlpk_config* c, const xlpk_weights* w, const 
   if (!kv->k_dev || !kv->v_dev || !aligned16(kv->k_dev) || !aligned16(kv->v_dev))
     return XLPK_ERR_INVALID_ARG;
   if (!aligned16(w->embed_dev) || !aligned16(w->lm_head.w_dev)) return XLPK_ERR_INVALID_ARG;
+  if (c->weight_dtype == XLPK_DTYPE_FP8_E4M3) {
+    // every linear weight carries its block scales
+    if (!w->lm_head.scale_dev) return XLPK_ERR_INVALID_ARG;
+    for (int l = 0; l < c->n_layers; ++l) {
+      const xlpk_layer_weights& L = w->layers[l];
+      const xlpk_linear* lin[] = {&L.wq, &L.wk, &L.wv, &L.wo, &L.w_gate, &L.w_up, &L.w_down};
+      for (const xlpk_linear* x : lin)
+        if (!x->scale_dev || (reinterpret_cast<uintptr_t>(x->scale_dev) & 3u)) return XLPK_ERR_INVALID_ARG;
+    }
+  }
   for (int l = 0; l < c->n_layers; ++l) {
     const xlpk_layer_weights& L = w->layers[l];
     const void* need[] = {L.attn_norm_dev, L.ffn_norm_dev, L.wq.w_dev, L.wk.w_dev, L.wv.w_dev,
@@ -363,7 +431,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const int B = c.batch, H = c.hidden, d = c.head_dim, F = c.ffn;
   const int qd = c.n_q_heads * d, kvd = c.n_kv_heads * d;
   const int group = c.n_q_heads / c.n_kv_heads;
-  e->P = (kSlotBytes / 2) / (d * 2);
+  e->P = (kTileBytes / 2) / (d * 2);
 
   // shared memory: ring + activation/scratch + control
   const int S_moe = c.n_experts > 0 ? c.top_k + c.n_shared_experts : 0;
@@ -388,7 +456,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
   e->smem = e->nslot * kSlotBytes + e->act_bytes + e->side_bytes + kMiscSmem;
-  if (!bind_by_shape(e, B, d)) return XLPK_ERR_UNSUPPORTED;
+  if (!bind_by_shape(e, B, d, c.n_experts > 0)) return XLPK_ERR_UNSUPPORTED;
 
   // The attribute is per kernel function, shared by every handle that uses the
   // same instantiation: allow the device maximum rather than this handle's size.
@@ -416,17 +484,21 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   size_t total = 0;
   auto add = [&](MatSrc s, int N, int K, int layer, int role, int split) {
     mats.push_back({s, N, K, total, layer, role, split});
-    total += align_up(static_cast<size_t>(N) * K * e->esz, 256);
+    const size_t esz_m = role == R_ROUTER ? 2 : e->esz;
+    total += align_up(static_cast<size_t>(N) * K * esz_m + (esz_m == 1 ? static_cast<size_t>(N) * K / 32 : 0), 256);
   };
   auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
   const size_t eg_bytes = static_cast<size_t>(Fe) * H * e->esz;   // one expert's gate (or up, or down)
   for (int l = 0; l < c.n_layers; ++l) {
     const xlpk_layer_weights& L = w->layers[l];
-    add({MatKind::QKV, u8(L.wq.w_dev), u8(L.wk.w_dev), u8(L.wv.w_dev)}, qd + 2 * kvd, H, l, R_QKV, e->G);
-    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr}, H, qd, l, R_O, e->G);
+    add({MatKind::QKV, u8(L.wq.w_dev), u8(L.wk.w_dev), u8(L.wv.w_dev), L.wq.scale_dev, L.wk.scale_dev,
+         L.wv.scale_dev},
+        qd + 2 * kvd, H, l, R_QKV, e->G);
+    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr, L.wo.scale_dev}, H, qd, l, R_O, e->G);
     if (!moe) {
-      add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr}, 2 * F, H, l, R_GU, e->G);
-      add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, H, F, l, R_DOWN, e->G);
+      add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr, L.w_gate.scale_dev, L.w_up.scale_dev},
+          2 * F, H, l, R_GU, e->G);
+      add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev}, H, F, l, R_DOWN, e->G);
     } else {
       // router logits are bf16 whatever the weight dtype
       add({MatKind::PLAIN, u8(L.router_dev), nullptr, nullptr}, c.n_experts, H, l, R_ROUTER, 1);
@@ -445,7 +517,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       }
     }
   }
-  add({MatKind::PLAIN, u8(w->lm_head.w_dev), nullptr, nullptr}, c.vocab, H, -1, R_LM, e->G);
+  add({MatKind::PLAIN, u8(w->lm_head.w_dev), nullptr, nullptr, w->lm_head.scale_dev}, c.vocab, H, -1, R_LM, e->G);
   // library-owned copies of the embedding table and the norm gains, so the
   // caller may free every weight buffer after create
   const size_t off_embed = total;
@@ -462,7 +534,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->weight_bytes_per_step = 0;
   for (const MatPlan& m : mats) {
     if (m.role == R_EGU || m.role == R_EDOWN) continue;
-    e->weight_bytes_per_step += static_cast<int64_t>(m.N) * m.K * (m.role == R_ROUTER ? 2 : e->esz);
+    const int64_t nk = static_cast<int64_t>(m.N) * m.K;
+    e->weight_bytes_per_step += m.role == R_ROUTER ? 2 * nk : e->esz == 1 ? nk + nk / 32 : 2 * nk;
   }
   if (moe)
     e->weight_bytes_per_step += static_cast<int64_t>(c.n_layers) * (c.top_k + c.n_shared_experts) * 3 *
