@@ -318,7 +318,7 @@ def main():
     extra = {}
     if not args.no_baselines:
         # kernel-per-op baseline, same tiles, one launch per stage
-        un_steps = min(n, 32)
+        un_steps = min(n, 16)
         workload.reset_state(m)
         m.engine.decode(un_steps, tok, unfused=True)
         torch.cuda.synchronize(dev)
