@@ -773,6 +773,7 @@ struct EpiResid {
   bool from_embed;
   const uint8_t* side;
   int v0, e0;
+  float* also = nullptr;   // fused FFN (O-projection): the same sum also to y
   __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
 #pragma unroll
     for (int b = 0; b < B; ++b) {
@@ -788,7 +789,9 @@ struct EpiResid {
         const float* rs = reinterpret_cast<const float*>(side + p.side_resid);
         base = *reinterpret_cast<const float2*>(rs + ((b * 2 + ((r >> 2) & 1)) * p.nvr + (r >> 3) - v0) * 4 + (r & 3));
       }
-      *xp = make_float2(base.x + a0[b], base.y + a1[b]);
+      const float2 v = make_float2(base.x + a0[b], base.y + a1[b]);
+      *xp = v;
+      if (also) *reinterpret_cast<float2*>(also + plane_index(b, r, p.B, p.H)) = v;
     }
   }
 };
@@ -806,6 +809,84 @@ struct EpiSwiGLU {
     }
   }
 };
+
+// Fused FFN gate/up epilogue: h = silu(gate) * up into this CTA's own slice
+// (shared memory, [B][hloc]), pair pg at index pg - p0.
+template <int B>
+struct EpiSwiGLULocal {
+  float* hl;
+  int hloc, p0;
+  __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      if (lane != b) continue;
+      const float g = a0[b];
+      hl[b * hloc + (pg - p0)] = g / (1.f + expf(-g)) * a1[b];
+    }
+  }
+};
+
+// Fused FFN, second half: this CTA's columns [j0, j1) of W_down times its own
+// h slice, for all H output rows (split-K over the CTAs), added into x with
+// vector float atomics.  Tiles are jt rows of W_down^T (= W_down columns), H
+// bf16 each; thread t owns the 8-row vectors t, t + 256, ... of the output.
+template <int B>
+__device__ __noinline__ void consume_downT(const Params& p, Ctx& cx, RingPos& rp, int where, int j0, int j1,
+                                           const float* hl) {
+  constexpr int NV = 2;                        // 8-row vectors per thread (H <= 4096)
+  const int V8 = p.H >> 3;
+  float acc[NV][8][B];
+#pragma unroll
+  for (int q = 0; q < NV; ++q)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+#pragma unroll
+      for (int b = 0; b < B; ++b) acc[q][e][b] = 0.f;
+  const int nj = j1 - j0;
+  for (int t0 = 0; t0 < nj; t0 += p.jt) {
+    const int ncol = min(p.jt, nj - t0);
+    const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
+    const bool ok = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
+    if (ok) {
+      const uint32_t base = smem_addr(cx.ring) + rp.slot * kSlotBytes;
+      for (int jj = 0; jj < ncol; ++jj) {
+        float hv[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) hv[b] = hl[b * p.hloc + t0 + jj];
+        const uint32_t col = base + jj * p.H * 2;
+#pragma unroll
+        for (int q = 0; q < NV; ++q) {
+          const int v = cx.tid + q * kConsumerThreads;
+          if (v < V8) {
+            const uint4 w = lds_u4(col + v * 16);
+            const float wf[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                 bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+#pragma unroll
+              for (int b = 0; b < B; ++b) acc[q][e][b] = fmaf(wf[e], hv[b], acc[q][e][b]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (cx.lane == 0 && ok) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));   // this warp is done with it
+    rp.next(p.nslot);
+  }
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    const int v = cx.tid + q * kConsumerThreads;
+    if (v < V8) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float4* x0 = reinterpret_cast<float4*>(p.x + plane_index(b, 8 * v, p.B, p.H));
+        float4* x1 = reinterpret_cast<float4*>(p.x + plane_index(b, 8 * v + 4, p.B, p.H));
+        atomicAdd(x0, make_float4(acc[q][0][b], acc[q][1][b], acc[q][2][b], acc[q][3][b]));
+        atomicAdd(x1, make_float4(acc[q][4][b], acc[q][5][b], acc[q][6][b], acc[q][7][b]));
+      }
+    }
+  }
+}
 
 // LM-head epilogue: running (max, lowest index) per sequence in lane b.
 template <int B>
@@ -1409,8 +1490,10 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
     if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
     return !ab;
   }
+  const int ffn_done = p.ffn_fused ? ST_GATEUP : ST_DOWN;   // the stage that completes a layer
+  if (kind == ST_DOWN && p.ffn_fused) return true;         // done inside the fused gate/up stage
   if (kind == ST_LM) {
-    if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused)) return false;
+    if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ffn_done, G * S1, where, fused)) return false;
     float* hid = (p.hidden_out && cx.c == 0) ? p.hidden_out + static_cast<size_t>(s) * p.B * p.H : nullptr;
     float rn[B];
     load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, SIDE_NONE, s, rn, where);
@@ -1484,7 +1567,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         load_act<B>(p, cx, p.H, SRC_EMBED, nullptr, L.attn_norm, nullptr, SIDE_ROPE, s, rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       } else {
-        ok = stage_wait(p, cx, p.cnt + (l - 1) * ST_LAYER + ST_DOWN, G * S1, where, fused);
+        ok = stage_wait(p, cx, p.cnt + (l - 1) * ST_LAYER + ffn_done, G * S1, where, fused);
         if (!ok) return false;
         load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.attn_norm, nullptr, SIDE_ROPE, s, rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
@@ -1499,13 +1582,13 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       load_act<B>(p, cx, p.nq * p.d, SRC_PLAIN, p.o, nullptr, nullptr, l == 0 ? SIDE_EMBED : SIDE_RESID, s,
                   rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      EpiResid<B> epi{p, l == 0, cx.side, r0 >> 3, r0 & ~7};
+      EpiResid<B> epi{p, l == 0, cx.side, r0 >> 3, r0 & ~7, p.ffn_fused ? p.y : nullptr};
       consume_gemv<B>(p, cx, L.o, rp, where, rn, epi);
       break;
     }
     case ST_GATEUP: {
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_OPROJ, G * S1, where, fused)) return false;
-      load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.ffn_norm, nullptr, SIDE_NONE, s, rn, where);
+      load_act<B>(p, cx, p.H, SRC_RESID, p.ffn_fused ? p.y : p.x, L.ffn_norm, nullptr, SIDE_NONE, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       if constexpr (MOE) {
         if constexpr (B == 1) {
@@ -1523,6 +1606,14 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
           consume_gemv<B>(p, cx, v, rp, where, rn, eg, 8 * split_point(cx.c, ng, p.G),
                           8 * split_point(cx.c + 1, ng, p.G));
         }
+      } else if (p.ffn_fused) {
+        // gate/up into this CTA's h slice, then its columns of W_down, added into x
+        const int q0 = split_point(cx.c, p.F, p.G), q1 = split_point(cx.c + 1, p.F, p.G);
+        float* hl = reinterpret_cast<float*>(cx.side + p.side_hloc);
+        EpiSwiGLULocal<B> epi{hl, p.hloc, q0};
+        consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
+        consumer_sync();
+        consume_downT<B>(p, cx, rp, where, q0, q1, hl);
       } else {
         EpiSwiGLU<B> epi{p};
         consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
@@ -1673,11 +1764,15 @@ __device__ __forceinline__ void cursor_next_stage(const Params& p, Cursor<B>& cu
     cu.kind = 0;
     cu.l = 0;
     if (++cu.s >= p.n_steps) cu.done = true;
-  } else if (++cu.kind == ST_LAYER) {
-    cu.kind = 0;
-    if (++cu.l == p.L) {
-      cu.kind = ST_LM;
-      cu.l = 0;
+  } else {
+    ++cu.kind;
+    if (cu.kind == ST_DOWN && p.ffn_fused) ++cu.kind;   // done inside the fused gate/up stage
+    if (cu.kind == ST_LAYER) {
+      cu.kind = 0;
+      if (++cu.l == p.L) {
+        cu.kind = ST_LM;
+        cu.l = 0;
+      }
     }
   }
 }
@@ -1736,6 +1831,7 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         cu.KC = m.KC;
         cu.trow = packed_row_bytes(m, m.KC);
         cu.src = m.packed + static_cast<size_t>(2) * cu.a * packed_row_bytes(m, m.K);
+        cu.phase = 0;
       }
     }
     t.stage = stage_index(p, cu.kind, cu.l);
@@ -1815,6 +1911,24 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         cu.a += kPairsPerTile;
       }
       return CUR_TILE;
+    } else if (!MOE && p.ffn_fused && cu.kind == ST_GATEUP && cu.phase == 0) {
+      // fused FFN: after the gate/up run, this CTA's rows of W_down^T (one run)
+      const int j0 = split_point(c, p.F, p.G), j1 = split_point(c + 1, p.F, p.G);
+      const int nj = j1 - j0;
+      cu.phase = 1;
+      if (nj > 0) {
+        const uint32_t colb = static_cast<uint32_t>(p.H) * 2u;
+        run->src = p.layers[cu.l].downT.packed + static_cast<size_t>(j0) * colb;
+        run->n1 = nj / p.jt;
+        run->b1 = static_cast<uint32_t>(p.jt) * colb;
+        run->n2 = (nj % p.jt) ? 1 : 0;
+        run->b2 = static_cast<uint32_t>(nj % p.jt) * colb;
+        run->stage = t.stage;
+        run->layer = t.layer;
+        run->step = t.step;
+        return CUR_RUN;
+      }
+      continue;
     } else if (moe && cu.kind == ST_GATEUP && cu.phase == 0) {
       // router done: the experts' gate/up groups of this CTA
       const Mat& m = p.layers[cu.l].egu;

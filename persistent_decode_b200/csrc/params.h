@@ -90,6 +90,10 @@ struct LayerParams {
   // CTAs); every expert's down projection is packed like a dense matrix
   // (rows split over the CTAs).  egu / edown describe expert 0; expert e's
   // block starts e * egu_stride (edown_stride) bytes further.
+  // Dense layers with the fused FFN stage: W_down transposed, bf16 [F][H]
+  // row-major; a CTA streams the rows (= W_down columns) matching its own
+  // gate/up pairs.
+  Mat downT;
   Mat router;
   Mat egu;
   Mat edown;
@@ -140,6 +144,12 @@ struct Params {
   float* q;          // [B][nq*d] rotated queries
   float* o;          // [B][nq*d] attention output
   float* h;          // [B][F] SwiGLU output (MoE: [B][S*Fe], slot-major, gate-weighted)
+  float* y;          // fused FFN: [B][H] residual after attention (the FFN's RMSNorm input);
+                     // x then accumulates the down projection's partial sums
+  int ffn_fused;     // 1: gate/up and down run as one stage with a split-K down projection
+  int jt;            // fused FFN: W_down columns per tile
+  int side_hloc;     // fused FFN: byte offset of the CTA's h slice [B][hloc] in the side region
+  int hloc;          //   floats per sequence of that slice (max gate/up pairs per CTA)
   int* route_exp;    // MoE: [L][S] expert of each slot (written by CTA 0)
   float* route_w;    // MoE: [L][S] weight of each slot
   float* part_ml;    // [B][nkv][G][group][2] per contributing CTA: (max in log2 units, sum)

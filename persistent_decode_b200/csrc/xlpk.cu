@@ -51,6 +51,21 @@ struct PackJob {
   long long sdst;       // FP8: byte offset of the row's scales in its first tile
 };
 
+// bf16 [R][C] row-major -> [C][R] row-major (32x32 tiles through shared memory).
+__global__ void transpose_bf16_kernel(const uint16_t* in, uint16_t* out, int R, int C) {
+  __shared__ uint16_t t[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < R && c < C) t[i][threadIdx.x] = in[static_cast<size_t>(r) * C + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < R && c < C) out[static_cast<size_t>(c) * R + r] = t[threadIdx.x][i];
+  }
+}
+
 // FP8: one thread per (row, chunk): the chunk's KC/128 block scales of the row.
 __global__ void pack_scales_kernel(const PackJob* jobs, int njobs, uint8_t* out, int nchunk, int kb_per_chunk) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -117,6 +132,8 @@ struct xlpk_engine {
   int smem = 0;
   int act_bytes = 0;
   int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, evb = 0;
+  int side_hloc = 0, hloc = 0;
+  bool ffn_fused = false;
   int esz = 2;
   int P = 0;
   uint8_t* packed = nullptr;
@@ -439,9 +456,18 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
   const int norm_stage = (B + 1) * H * 4;   // normed input vector + its RMSNorm gains
   e->act_bytes = static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
+  // Fused FFN stage (gate/up and a split-K down projection in one stage): bf16
+  // dense layers whose output rows fit two 8-row vectors per consumer thread
+  // and whose accumulators fit the register budget (XLPK_FFN_FUSED=0 turns it off).
+  {
+    const char* env = std::getenv("XLPK_FFN_FUSED");
+    const bool off = env && env[0] == '0';
+    e->ffn_fused = !off && c.n_experts == 0 && e->esz == 2 && H <= 2 * 8 * kConsumerThreads && H % 8 == 0 &&
+                   B <= 2;
+  }
   // epilogue side region: RoPE rows, then this CTA's rows of the residual (two
   // planes of float4) and of the embedding (bf16, 8-aligned) for the stages
-  // with H output rows
+  // with H output rows, then (fused FFN) the CTA's h slice
   {
     const int maxp = (H / 2 + e->G - 1) / e->G;
     const int rows_max = 2 * maxp;
@@ -450,7 +476,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     e->nvr = rows_max / 8 + 2;
     e->side_embed = e->side_resid + B * 2 * e->nvr * 16;
     e->evb = static_cast<int>(align_up(static_cast<size_t>(rows_max + 16) * 2, 16));
-    e->side_bytes = static_cast<int>(align_up(static_cast<size_t>(e->side_embed) + B * e->evb, 128));
+    e->side_hloc = static_cast<int>(align_up(static_cast<size_t>(e->side_embed) + B * e->evb, 16));
+    e->hloc = e->ffn_fused ? (F + e->G - 1) / e->G : 0;
+    e->side_bytes = static_cast<int>(align_up(static_cast<size_t>(e->side_hloc) + sizeof(float) * B * e->hloc, 128));
   }
   const int max_smem = static_cast<int>(prop.sharedMemPerBlockOptin);
   e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
@@ -471,7 +499,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
 
   // packed weights: per layer qkv, o, then gate/up + down (dense) or the
   // router + every expert's gate/up and down (MoE); then the LM head
-  enum Role { R_QKV, R_O, R_GU, R_DOWN, R_ROUTER, R_EGU, R_EDOWN, R_LM };
+  enum Role { R_QKV, R_O, R_GU, R_DOWN, R_DOWNT, R_ROUTER, R_EGU, R_EDOWN, R_LM };
   struct MatPlan {
     MatSrc src;
     int N, K;
@@ -498,7 +526,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     if (!moe) {
       add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr, L.w_gate.scale_dev, L.w_up.scale_dev},
           2 * F, H, l, R_GU, e->G);
-      add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev}, H, F, l, R_DOWN, e->G);
+      if (e->ffn_fused)
+        add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, F, H, l, R_DOWNT, 1);   // W_down^T [F][H]
+      else
+        add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev}, H, F, l, R_DOWN, e->G);
     } else {
       // router logits are bf16 whatever the weight dtype
       add({MatKind::PLAIN, u8(L.router_dev), nullptr, nullptr}, c.n_experts, H, l, R_ROUTER, 1);
@@ -557,9 +588,27 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   for (size_t i = 0; i < mats.size() && rc == XLPK_OK; ++i) {
     const MatPlan& mp = mats[i];
     Mat m{};
-    e->esz = mp.role == R_ROUTER ? 2 : esz_saved;
-    rc = pack_matrix(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, d_jobs, max_jobs, st, mp.split);
-    e->esz = esz_saved;
+    if (mp.role == R_DOWNT) {
+      // the fused FFN streams W_down columns: store W_down^T, plain bf16 [F][H]
+      const dim3 tb(32, 8), gr((mp.N + 31) / 32, (mp.K + 31) / 32);   // in: [H=K][F=N]
+      transpose_bf16_kernel<<<gr, tb, 0, st>>>(reinterpret_cast<const uint16_t*>(mp.src.a),
+                                               reinterpret_cast<uint16_t*>(e->packed + mp.off), mp.K, mp.N);
+      ce = cudaGetLastError();
+      if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+      if (ce != cudaSuccess) {
+        rc = cuda_fail(ce, "transpose_bf16_kernel");
+        break;
+      }
+      m.packed = e->packed + mp.off;
+      m.N = mp.N;
+      m.K = mp.K;
+      m.KC = mp.K;
+      m.fp8 = 0;
+    } else {
+      e->esz = mp.role == R_ROUTER ? 2 : esz_saved;
+      rc = pack_matrix(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, d_jobs, max_jobs, st, mp.split);
+      e->esz = esz_saved;
+    }
     if (rc != XLPK_OK) break;
     LayerParams* L = mp.layer >= 0 ? &lp[mp.layer] : nullptr;
     switch (mp.role) {
@@ -567,6 +616,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       case R_O: L->o = m; break;
       case R_GU: L->gu = m; break;
       case R_DOWN: L->down = m; break;
+      case R_DOWNT: L->downT = m; break;
       case R_ROUTER: L->router = m; break;
       case R_EGU:
         if (!L->egu.packed) L->egu = m;
@@ -621,6 +671,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const size_t o_q = take(sizeof(float) * B * qd);
   const size_t o_o = take(sizeof(float) * B * qd);
   const size_t o_h = take(sizeof(float) * B * std::max(F, S_moe * c.expert_ffn));
+  const size_t o_y = take(sizeof(float) * B * H);
   const size_t o_pml = take(sizeof(float) * prow * group * 2);
   const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * e->G * B);
@@ -687,6 +738,11 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.q = reinterpret_cast<float*>(e->ws + o_q);
   p.o = reinterpret_cast<float*>(e->ws + o_o);
   p.h = reinterpret_cast<float*>(e->ws + o_h);
+  p.y = reinterpret_cast<float*>(e->ws + o_y);
+  p.ffn_fused = e->ffn_fused ? 1 : 0;
+  p.jt = kTileBytes / (H * 2);
+  p.side_hloc = e->side_hloc;
+  p.hloc = e->hloc;
   p.route_exp = reinterpret_cast<int*>(e->ws + o_rte);
   p.route_w = reinterpret_cast<float*>(e->ws + o_rtw);
   p.E = c.n_experts;
@@ -838,7 +894,8 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   Params p = call_params(h, n_steps, tokens_out_dev, io);
   for (int s = 0; s < n_steps; ++s) {
     for (int l = 0; l < h->cfg.n_layers; ++l)
-      for (int k = 0; k < ST_LAYER; ++k) h->launch_stage(p, k, l, s, h->G, h->smem, st);
+      for (int k = 0; k < ST_LAYER; ++k)
+        if (!(k == ST_DOWN && h->ffn_fused)) h->launch_stage(p, k, l, s, h->G, h->smem, st);
     h->launch_stage(p, ST_LM, 0, s, h->G, h->smem, st);
   }
   XLPK_CUDA(cudaGetLastError());
@@ -874,6 +931,7 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   const size_t o_o = take(sizeof(float) * B * qd);
   const int S_moe = h->base.S;
   const size_t o_h = take(sizeof(float) * B * std::max(F, S_moe * c.expert_ffn));
+  const size_t o_y = take(sizeof(float) * B * H);
   const size_t o_pml = take(sizeof(float) * prow * group * 2);
   const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * h->G * B);
@@ -894,6 +952,7 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   p.q = reinterpret_cast<float*>(sc + o_q);
   p.o = reinterpret_cast<float*>(sc + o_o);
   p.h = reinterpret_cast<float*>(sc + o_h);
+  p.y = reinterpret_cast<float*>(sc + o_y);
   p.route_exp = reinterpret_cast<int*>(sc + o_rte);
   p.route_w = reinterpret_cast<float*>(sc + o_rtw);
   p.part_ml = reinterpret_cast<float*>(sc + o_pml);
@@ -950,7 +1009,7 @@ xlpk_status xlpk_get_info(xlpk_handle h, xlpk_info* out) {
   out->smem_bytes = h->smem;
   out->ring_slots = h->nslot;
   out->slot_bytes = kSlotBytes;
-  out->kernels_per_step_unfused = h->cfg.n_layers * ST_LAYER + 1;
+  out->kernels_per_step_unfused = h->cfg.n_layers * (h->ffn_fused ? ST_LAYER - 1 : ST_LAYER) + 1;
   out->packed_weight_bytes = static_cast<int64_t>(h->packed_bytes);
   out->workspace_bytes = static_cast<int64_t>(h->ws_bytes);
   out->weight_bytes_per_step = h->weight_bytes_per_step;

@@ -16,7 +16,7 @@ import torch
 import synth
 from persistent_decode_b200 import XlpkError, _abi, workload
 
-from tests.gpu_util import run_engine
+from tests.gpu_util import rel_l2, run_engine
 
 pytestmark = pytest.mark.gpu
 
@@ -30,9 +30,9 @@ def tiny_fast_fail(cuda_device):
 
 
 # stage index = layer * 5 + kind (0 QKV, 2 O-proj, 3 gate/up, 4 down); the tiny
-# model has 2 layers, so 9 is the last layer's down projection (its waiter is
-# the LM head)
-@pytest.mark.parametrize("stage", [0, 2, 3, 9])
+# bf16 model runs gate/up and down as one fused FFN stage (kind 3), so 8 is the
+# last layer's FFN (its waiter is the LM head)
+@pytest.mark.parametrize("stage", [0, 2, 3, 8])
 def test_withheld_release_times_out_and_handle_recovers(tiny_fast_fail, stage):
     m = tiny_fast_fail
     ref = run_engine(m, 8)
@@ -50,4 +50,4 @@ def test_withheld_release_times_out_and_handle_recovers(tiny_fast_fail, stage):
     # the status was reset with the counters: the handle works again
     again = run_engine(m, 8)
     assert torch.equal(again.tokens, ref.tokens)
-    assert torch.equal(again.logits, ref.logits)
+    assert rel_l2(again.logits, ref.logits) < 1e-5

@@ -41,12 +41,31 @@ def test_tiny_decode_matches_oracle(tiny, unfused):
     compare_with_oracle(tiny, run, o, tiny.cfg.steps)
 
 
-def test_tiny_persistent_equals_kernel_per_op_bitwise(tiny):
+def test_tiny_persistent_matches_kernel_per_op(tiny):
+    # the same tiles and arithmetic; the fused FFN stage adds the down
+    # projection's split-K partial sums with float atomics, so the two agree
+    # up to summation order
     a = run_engine(tiny, tiny.cfg.steps, unfused=False)
     b = run_engine(tiny, tiny.cfg.steps, unfused=True)
     assert torch.equal(a.tokens, b.tokens)
-    assert torch.equal(a.logits, b.logits)
-    assert torch.equal(a.hidden, b.hidden)
+    assert rel_l2(a.logits, b.logits) < 1e-5
+    assert rel_l2(a.hidden, b.hidden) < 1e-5
+
+
+def test_fused_ffn_matches_two_stage_ffn(cuda_device, monkeypatch):
+    # gate/up + split-K down in one stage (default for bf16 dense models) vs
+    # gate/up and down as two stages (XLPK_FFN_FUSED=0), same weights
+    cfg = synth.get_config("tiny", steps=10)
+    fused = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    monkeypatch.setenv("XLPK_FFN_FUSED", "0")
+    two = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=fused.weights)
+    assert two.engine.info().kernels_per_step_unfused == 5 * cfg.n_layers + 1
+    assert fused.engine.info().kernels_per_step_unfused == 4 * cfg.n_layers + 1
+    a = run_engine(fused, cfg.steps)
+    b = run_engine(two, cfg.steps)
+    assert torch.equal(a.tokens, b.tokens)
+    assert rel_l2(a.logits, b.logits) < 1e-5
+    compare_with_oracle(two, b, oracle_for(two), cfg.steps)
 
 
 def test_tiny_decode_is_deterministic_and_resumable(tiny):
