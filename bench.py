@@ -44,8 +44,8 @@ def parse():
 
 
 def dist_env():
-    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
-            int(os.environ.get("LOCAL_RANK", "0")))
+    from persistent_decode_b200.replicas import dist_env as _env
+    return _env()
 
 
 # ----------------------------------------------------------------- clocks
@@ -227,12 +227,11 @@ def main():
     import synth
     from persistent_decode_b200 import roofline, workload
 
+    from persistent_decode_b200 import replicas
     rank, world, local = dist_env()
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        replicas.init("nccl", device=torch.device("cuda", local))
     dev = torch.device("cuda", local if world > 1 else 0)
     cfg = synth.get_config(args.workload)
     if args.decode_steps:
@@ -274,14 +273,9 @@ def main():
     status = m.engine.status()
     if world > 1:
         dist.barrier()
-    total_ms = t_start.elapsed_time(t_end)
+    total_ms = replicas.max_over_ranks(t_start.elapsed_time(t_end), dev)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    tokens_total = args.steps * n * B * world
-    value = tokens_total / (total_ms / 1e3)
+    value = replicas.job_rate(args.steps * n * B, total_ms / 1e3, world)
     tpot_ms = total_ms / (args.steps * n)
 
     # roofline of the persistent kernel (one launch = one bench step)
@@ -307,12 +301,8 @@ def main():
         t0 = time.perf_counter()
         m.engine.generate(m.start_tokens.tolist(), [cfg.kv_len] * B, n, out_host)
         e2e_t.append(time.perf_counter() - t0)
-    e2e_s = statistics.mean(e2e_t)
-    if world > 1:
-        t = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e = {"value": n * B * world / e2e_s, "unit": UNIT, "h2d_bytes_per_step": 4 * B,
+    e2e_s = replicas.max_over_ranks(statistics.mean(e2e_t), dev)
+    e2e = {"value": replicas.job_rate(n * B, e2e_s, world), "unit": UNIT, "h2d_bytes_per_step": 4 * B,
            "d2h_bytes_per_step": 4 * B * n}
 
     extra = {}

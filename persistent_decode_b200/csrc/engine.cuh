@@ -1468,6 +1468,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     unsigned long long* e =
         p.trace + ((static_cast<size_t>(s) * n_st + stage_index(p, ST_ATTN, l)) * p.G + blockIdx.x) * kTraceSlots;
     for (int k = 0; k < 8; ++k) e[6 + k] = ta[k];
+    for (int k = 0; k < 8; ++k) ta[k] = 0;
   }
 }
 
@@ -1686,6 +1687,7 @@ __device__ __forceinline__ void init_ring(const Params& p, Ctx& cx) {
     cx.ctl->abort = 0;
     cx.ctl->flag = 0;
     cx.ctl->route_seq = 0;
+    for (int k = 0; k < 8; ++k) cx.ctl->tacc[k] = 0;
     fence_barrier_init();
   }
   __syncthreads();
