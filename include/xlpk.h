@@ -53,7 +53,9 @@ typedef enum xlpk_status {
 
 typedef enum xlpk_dtype {
   XLPK_DTYPE_BF16 = 0,         /* bf16 weights, row-major [N][K] */
-  XLPK_DTYPE_FP8_E4M3 = 1      /* e4m3 codes, row-major [N][K], + one fp32 scale per 128x128 block */
+  XLPK_DTYPE_FP8_E4M3 = 1      /* e4m3 codes, row-major [N][K], + one fp32 scale per 128x128 block;
+                                  dense models only, hidden / n_q_heads*head_dim / ffn multiples
+                                  of 256 and the other dims of 128 (else XLPK_ERR_UNSUPPORTED) */
 } xlpk_dtype;
 
 /* Model and launch shape.  All widths are element counts.

@@ -346,6 +346,9 @@ xlpk_status validate_config(const xlpk_config* c) {
     const int qd = c->n_q_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
     if (c->n_experts > 0) return XLPK_ERR_UNSUPPORTED;
     if (c->hidden % 128 || qd % 128 || kvd % 128 || c->ffn % 128 || c->vocab % 128) return XLPK_ERR_UNSUPPORTED;
+    // a packed FP8 row pair over K columns takes 2K + K/16 bytes; bulk copies
+    // of row-pair spans need 16-byte multiples, so every K is a multiple of 256
+    if (c->hidden % 256 || qd % 256 || c->ffn % 256) return XLPK_ERR_UNSUPPORTED;
   }
   if (c->n_experts > 0) {
     if (c->top_k < 1 || c->top_k > c->n_experts || c->expert_ffn <= 0) return XLPK_ERR_INVALID_ARG;
