@@ -319,10 +319,33 @@ def main():
         b.record(stream)
         torch.cuda.synchronize(dev)
         un_tpot = a.elapsed_time(b) / un_steps
+        # the same launches recorded once into a CUDA graph and replayed: the
+        # kernel-per-op baseline without host launch overhead
+        workload.reset_state(m)
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap):
+            m.engine.decode(un_steps, tok, unfused=True)
+        stream.wait_stream(cap)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        gt = []
+        for _ in range(3):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            gt.append(a.elapsed_time(b) / un_steps)
+        del g
+        m.engine.check()
+        un_graph = statistics.median(gt)
         info = m.engine.info()
         extra["unfused"] = {"tpot_ms": round(un_tpot, 4), "tok_s_per_user": round(1e3 / un_tpot, 2),
+                            "graph_tpot_ms": round(un_graph, 4),
                             "steps_timed": un_steps, "launches_per_token": info.kernels_per_step_unfused,
-                            "persistent_speedup": round(un_tpot / tpot_ms, 3)}
+                            "persistent_speedup": round(un_tpot / tpot_ms, 3),
+                            "persistent_speedup_vs_graph": round(un_graph / tpot_ms, 3)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_baselines:
         o, head, nl = build_cpu_sample(cfg, dev)

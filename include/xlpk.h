@@ -180,8 +180,14 @@ xlpk_status xlpk_set_state(xlpk_handle h, const int32_t* tokens_host,
 xlpk_status xlpk_decode(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                         const xlpk_decode_io* io, void* stream);
 
-/* The same decode as one kernel launch per operator stage (5 per layer + 1
- * per step), built from the same tiles: the kernel-per-op baseline. */
+/* The same decode as one kernel launch per operator stage, built from the same
+ * tiles: the kernel-per-op baseline.  Per layer: QKV, attention, O-projection
+ * and gate/up + down (one fused FFN launch where the persistent kernel fuses
+ * them); per step the LM head.  Each call first clears the handle's dependency
+ * counters on `stream` (an async memset) and calls nothing that synchronises,
+ * so its launches may be recorded by stream capture into a CUDA graph and
+ * replayed; a replay decodes the captured positions again, from the tokens the
+ * device holds. */
 xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                                 const xlpk_decode_io* io, void* stream);
 

@@ -895,6 +895,11 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   if (rc != XLPK_OK || n_steps == 0) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Params p = call_params(h, n_steps, tokens_out_dev, io);
+  // Fresh dependency counters for every call (the last-arriver decisions count
+  // from step 0), so the launches this call records can be captured into a CUDA
+  // graph and replayed; a later persistent call continues from step n_steps.
+  XLPK_CUDA(cudaMemsetAsync(h->base.cnt, 0, sizeof(unsigned) * h->base.cl.total, st));
+  p.step_base = 0;
   for (int s = 0; s < n_steps; ++s) {
     for (int l = 0; l < h->cfg.n_layers; ++l)
       for (int k = 0; k < ST_LAYER; ++k)
@@ -903,6 +908,7 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   }
   XLPK_CUDA(cudaGetLastError());
   advance(h, n_steps, st);
+  h->step_base = n_steps;
   return XLPK_OK;
 }
 

@@ -81,6 +81,41 @@ def test_tiny_decode_is_deterministic_and_resumable(tiny):
     assert torch.equal(torch.cat([t1, t2]).cpu(), a.tokens)
 
 
+def test_kernel_per_op_graph_replay_matches_eager(tiny):
+    # the kernel-per-op launches recorded by stream capture into a CUDA graph
+    # (each call clears its dependency counters on the stream) and replayed
+    cfg, dev = tiny.cfg, tiny.k.device
+    n = 6
+    a = run_engine(tiny, n, unfused=True)
+    workload.reset_state(tiny)
+    tok = torch.full((n, cfg.batch), -1, dtype=torch.int32, device=dev)
+    lg = torch.zeros(n, cfg.batch, cfg.vocab, dtype=torch.float32, device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        tiny.engine.decode(n, tok, logits=lg, unfused=True)
+    g.replay()
+    torch.cuda.synchronize()
+    tiny.engine.check()
+    assert torch.equal(tok.cpu(), a.tokens)
+    assert rel_l2(lg.cpu(), a.logits) < 1e-5
+    del g
+
+
+def test_decode_resumes_across_launch_modes(tiny):
+    # 8 kernel-per-op steps, then 8 persistent steps on the same handle, equal
+    # 16 persistent steps: the persistent call continues from the counters the
+    # kernel-per-op call left
+    a = run_engine(tiny, 16)
+    workload.reset_state(tiny)
+    dev = tiny.k.device
+    t1 = torch.empty(8, 1, dtype=torch.int32, device=dev)
+    t2 = torch.empty(8, 1, dtype=torch.int32, device=dev)
+    tiny.engine.decode(8, t1, unfused=True)
+    tiny.engine.decode(8, t2)
+    tiny.engine.check()
+    assert torch.equal(torch.cat([t1, t2]).cpu(), a.tokens)
+
+
 def test_tiny_kv_append_positions_exact(tiny):
     cfg = tiny.cfg
     T, n = cfg.kv_len, cfg.steps
