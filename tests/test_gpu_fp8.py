@@ -46,3 +46,15 @@ def test_llama8b_fp8_full_size_prefix(cuda_device):
     o = oracle_for(m)
     compare_with_oracle(m, run, o, 2, tol=REL_L2_FP8)
     assert int(run.tokens.min()) >= 0 and int(run.tokens.max()) < cfg.vocab
+
+
+def test_llama8b_fp8_batch2_full_size_prefix(cuda_device):
+    # the 8B FP8 shape at batch 2 (two sequences over the 1024-entry synthetic
+    # cache); its activation region holds 2 x 14336 floats, so the ring keeps
+    # 3 slots
+    cfg = synth.get_config("llama8b_fp8", batch=2)
+    m = workload.build(cfg, device=cuda_device)
+    assert m.engine.info().ring_slots >= 2
+    run = run_engine(m, 4)
+    compare_with_oracle(m, run, oracle_for(m), 2, tol=REL_L2_FP8)
+    assert int(run.tokens.min()) >= 0 and int(run.tokens.max()) < cfg.vocab

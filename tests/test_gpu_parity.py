@@ -234,3 +234,18 @@ def test_llama8b_full_size_prefix(cuda_device):
     # steps wrote exactly positions T .. T+15
     assert bool((m.k[:, :, :, T:T + 16].float().abs().sum(-1) > 0).all())
     assert int(m.k[:, :, :, T + 16:].float().abs().sum().item()) == 0
+
+
+def test_llama1b_batch4_prefix(cuda_device):
+    # the 1B shape at batch 4 (four independent prompts), with a 64-token
+    # prompt per sequence so that the oracle's prefill stays short; the
+    # activation region holds 4 x 8192 floats, so the ring keeps 2 slots
+    cfg = synth.get_config("llama1b", batch=4, kv_len=64, steps=8)
+    m = workload.build(cfg, device=cuda_device)
+    assert m.engine.info().ring_slots >= 2
+    run = run_engine(m, cfg.steps)
+    compare_with_oracle(m, run, oracle_for(m), 3)
+    T = cfg.kv_len
+    # every sequence wrote exactly positions T .. T+7 of its own cache rows
+    assert bool((m.k[:, :, :, T:T + 8].float().abs().sum(-1) > 0).all())
+    assert int(m.k[:, :, :, T + 8:].float().abs().sum().item()) == 0
