@@ -236,6 +236,25 @@ const char* xlpk_status_string(int32_t status);
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
 const char* xlpk_last_cuda_error(void);
 
+/* One batch-8 projection on the tcgen05 tensor cores:
+ *     y[n][b] = sum_k w[n][k] * bf16(x[b][k]),   n < N, b < 8,
+ * i.e. the decoder's linear layers (QKV, O, gate/up, down, LM head of the
+ * decode step above) for 8 sequences at once, where the GEMV becomes a dense
+ * [N x K] . [K x 8] contraction.  It is the tensor-core tile the batch-8
+ * decode is built from; xlpk_decode does not call it yet.
+ *  - w_dev: bf16 [N][K] row-major; x_dev: fp32 [8][K] row-major (rounded to
+ *    bf16, round-to-nearest-even, as it enters the MMA); y_dev: fp32 [N][8]
+ *    row-major, written.  All three 16-byte aligned, on the current device;
+ *    nothing is retained after the call.
+ *  - N >= 128 (one CTA per 128 rows; a ragged last block is fine),
+ *    64 <= K <= 4096 and K a multiple of 64; else XLPK_ERR_INVALID_ARG.
+ *  - Runs on `stream` and waits for it: returns XLPK_OK, XLPK_ERR_UNSUPPORTED
+ *    on a device that is not sm_100, XLPK_ERR_CUDA, or XLPK_ERR_TIMEOUT if a
+ *    device-side wait ran out (the kernel then leaves without writing y).
+ *    One call at a time per process (the device-side error word is shared). */
+xlpk_status xlpk_tc_gemm_tile(const void* w_dev, int32_t n, int32_t k, const float* x_dev, float* y_dev,
+                              void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -81,6 +81,7 @@ SIGNATURES = {
     "xlpk_get_info": (C.c_int32, [C.c_void_p, C.POINTER(xlpk_info)]),
     "xlpk_status_string": (C.c_char_p, [C.c_int32]),
     "xlpk_last_cuda_error": (C.c_char_p, []),
+    "xlpk_tc_gemm_tile": (C.c_int32, [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]),
 }
 
 

@@ -24,6 +24,7 @@
 
 #include "../../include/xlpk.h"
 #include "engine.cuh"
+#include "tc_tile.cuh"
 #include "params.h"
 
 using namespace xlpk;
@@ -811,6 +812,8 @@ void advance(xlpk_engine* h, int32_t n_steps, cudaStream_t st) {
 // loads the library.  Host code must not use the symbol's host address; the
 // device address comes from cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[XLPK_NOALLOC_SCRATCH_BYTES];
+// Error word of xlpk_tc_gemm_tile (one call at a time per process).
+static __device__ int g_tc_err;
 
 namespace {
 
@@ -1040,5 +1043,44 @@ const char* xlpk_status_string(int32_t s) {
 }
 
 const char* xlpk_last_cuda_error(void) { return g_cuda_err.c_str(); }
+
+xlpk_status xlpk_tc_gemm_tile(const void* w_dev, int32_t n, int32_t k, const float* x_dev, float* y_dev,
+                              void* stream) {
+  if (!w_dev || !x_dev || !y_dev) return XLPK_ERR_INVALID_ARG;
+  if (n < kTcRows || k < kTcKBox || k > kTcMaxK || k % kTcKBox) return XLPK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(w_dev) | reinterpret_cast<uintptr_t>(x_dev) |
+       reinterpret_cast<uintptr_t>(y_dev)) & 15u)
+    return XLPK_ERR_INVALID_ARG;
+  int dev = -1;
+  XLPK_CUDA(cudaGetDevice(&dev));
+  int major = 0;
+  XLPK_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  if (major != 10) {
+    g_cuda_err = "device is not sm_100";
+    return XLPK_ERR_UNSUPPORTED;
+  }
+  // the weight matrix as a 2-D [n][k] bf16 array read in [128 rows][64 columns]
+  // boxes with 128-byte swizzle: the layout of the MMA's A operand
+  CUtensorMap map;
+  xlpk_status rc = encode_kv_map(&map, const_cast<void*>(w_dev), static_cast<unsigned long long>(n), k, kTcRows);
+  if (rc != XLPK_OK) return rc;
+  const int smem = tc_smem_bytes(k);
+  XLPK_CUDA(cudaFuncSetAttribute(tc_gemm_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  int* err = nullptr;
+  XLPK_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tc_err));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  XLPK_CUDA(cudaMemsetAsync(err, 0, sizeof(int), st));
+  tc_gemm_tile_kernel<<<(n + kTcRows - 1) / kTcRows, kTcThreads, smem, st>>>(map, n, k, x_dev, y_dev, err,
+                                                                             200000000LL);
+  XLPK_CUDA(cudaGetLastError());
+  XLPK_CUDA(cudaStreamSynchronize(st));
+  int e = 0;
+  XLPK_CUDA(cudaMemcpy(&e, err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (e != 0) {
+    g_cuda_err = "xlpk_tc_gemm_tile: a device wait ran out";
+    return static_cast<xlpk_status>(e);
+  }
+  return XLPK_OK;
+}
 
 }  // extern "C"

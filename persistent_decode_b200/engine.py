@@ -46,6 +46,18 @@ def _ptr(t) -> int:
     return 0 if t is None else int(t.data_ptr())
 
 
+def tc_gemm_tile(w, x, stream=None):
+    """xlpk_tc_gemm_tile: Y[N][8] = W[N][K] . X[8][K]^T on the tcgen05 tensor cores.
+
+    `w` bf16 [N][K] and `x` fp32 [8][K] (contiguous, on the device); returns
+    fp32 [N][8].  The activations enter the MMA rounded to bf16."""
+    import torch
+    n, k = int(w.shape[0]), int(w.shape[1])
+    y = torch.empty(n, 8, dtype=torch.float32, device=w.device)
+    _check(lib.xlpk_tc_gemm_tile(_ptr(w), n, k, _ptr(x), _ptr(y), _stream_handle(stream)), "xlpk_tc_gemm_tile")
+    return y
+
+
 def _stream_handle(stream) -> Optional[int]:
     if stream is None:
         import torch

@@ -70,6 +70,12 @@ def test_host_side_argument_checks(lib):
     assert lib.xlpk_destroy(None) == _abi.XLPK_ERR_INVALID_ARG
     info = _abi.xlpk_info()
     assert lib.xlpk_get_info(None, C.byref(info)) == _abi.XLPK_ERR_INVALID_ARG
+    # the tensor-core tile: shapes and pointers are checked before any CUDA call
+    p = C.c_void_p(1 << 20)
+    for n, k in ((127, 64), (128, 0), (128, 96), (128, 8192)):
+        assert lib.xlpk_tc_gemm_tile(p, n, k, p, p, None) == _abi.XLPK_ERR_INVALID_ARG, (n, k)
+    assert lib.xlpk_tc_gemm_tile(None, 128, 64, p, p, None) == _abi.XLPK_ERR_INVALID_ARG
+    assert lib.xlpk_tc_gemm_tile(C.c_void_p((1 << 20) + 8), 128, 64, p, p, None) == _abi.XLPK_ERR_INVALID_ARG
 
 
 def test_struct_layout_matches_header(lib):
