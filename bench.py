@@ -112,10 +112,19 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+TILE_SECTION = b"\n// ---- tensor-core tile entry point"
+
+
 def kernel_source_hash() -> str:
+    """Hash of the sources the persistent decode kernel and its host planning
+    come from (the tensor-core tile entry point appended to xlpk.cu is not
+    among them)."""
     h = hashlib.sha256()
     for f in ("engine.cuh", "xlpk.cu", "params.h"):
-        h.update(open(os.path.join(ROOT, "persistent_decode_b200", "csrc", f), "rb").read())
+        data = open(os.path.join(ROOT, "persistent_decode_b200", "csrc", f), "rb").read()
+        if f == "xlpk.cu" and TILE_SECTION in data:
+            data = data[:data.index(TILE_SECTION)]
+        h.update(data)
     return h.hexdigest()[:16]
 
 

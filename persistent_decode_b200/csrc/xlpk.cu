@@ -24,7 +24,6 @@
 
 #include "../../include/xlpk.h"
 #include "engine.cuh"
-#include "tc_tile.cuh"
 #include "params.h"
 
 using namespace xlpk;
@@ -812,8 +811,6 @@ void advance(xlpk_engine* h, int32_t n_steps, cudaStream_t st) {
 // loads the library.  Host code must not use the symbol's host address; the
 // device address comes from cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[XLPK_NOALLOC_SCRATCH_BYTES];
-// Error word of xlpk_tc_gemm_tile (one call at a time per process).
-static __device__ int g_tc_err;
 
 namespace {
 
@@ -1044,8 +1041,18 @@ const char* xlpk_status_string(int32_t s) {
 
 const char* xlpk_last_cuda_error(void) { return g_cuda_err.c_str(); }
 
-xlpk_status xlpk_tc_gemm_tile(const void* w_dev, int32_t n, int32_t k, const float* x_dev, float* y_dev,
-                              void* stream) {
+}  // extern "C"
+
+// ---- tensor-core tile entry point: separate from the persistent decode (the
+// decode's kernels and planning above do not depend on anything below)
+
+#include "tc_tile.cuh"
+
+// Error word of xlpk_tc_gemm_tile (one call at a time per process).
+static __device__ int g_tc_err;
+
+extern "C" xlpk_status xlpk_tc_gemm_tile(const void* w_dev, int32_t n, int32_t k, const float* x_dev,
+                                         float* y_dev, void* stream) {
   if (!w_dev || !x_dev || !y_dev) return XLPK_ERR_INVALID_ARG;
   if (n < kTcRows || k < kTcKBox || k > kTcMaxK || k % kTcKBox) return XLPK_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(w_dev) | reinterpret_cast<uintptr_t>(x_dev) |
@@ -1082,5 +1089,3 @@ xlpk_status xlpk_tc_gemm_tile(const void* w_dev, int32_t n, int32_t k, const flo
   }
   return XLPK_OK;
 }
-
-}  // extern "C"
