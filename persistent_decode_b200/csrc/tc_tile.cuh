@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (!ok) {
       *ok_flag = 0;
-      atomicExch(err, -6);   // XLPK_ERR_TIMEOUT
+      atomicExch(err, static_cast<int>(kErrTimeout));
     }
   }
   __syncthreads();
