@@ -41,3 +41,16 @@ def test_call_bytes_sums_growing_steps():
     cfg = synth.get_config("tiny")
     assert roofline.call_bytes(cfg, 128, 3) == sum(roofline.step_bytes(cfg, 128 + s) for s in range(3))
     assert roofline.step_bytes(cfg, 129) - roofline.step_bytes(cfg, 128) == 2 * 2 * 64 * 2 * 2   # one more position
+
+
+def test_moe_counts_only_active_experts():
+    # 24 layers, hidden 2048, 16 q / 4 kv heads of 128, 64 experts (top-8) + 1 shared of width 1408, vocab 64000
+    #   attention per layer: (2048 + 2*512) * 2048 + 2048 * 2048 = 10,485,760
+    #   active experts per layer: (8 + 1) * 3 * 1408 * 2048 = 77,856,768
+    #   linear elements: 24 * 88,342,528 + 64000 * 2048 = 2,251,292,672 (bf16)
+    #   router (bf16, every layer): 64 * 2048 * 2 bytes = 262,144; norm gains 4 * 2048 * 49 = 401,408
+    #   one position's K and V: 24 * 4 * 128 * 4 = 49,152
+    cfg = synth.get_config("moe")
+    w = 2 * 2_251_292_672 + 24 * 262_144 + 401_408
+    assert roofline.weight_bytes(cfg) == w
+    assert roofline.step_bytes(cfg, 4096) == w + 4097 * 49_152 + 49_152 + 2048 * 2
