@@ -57,7 +57,9 @@ def test_host_side_argument_checks(lib):
                 dict(weight_dtype=7), dict(rope_theta=0.0)):
         c = _tiny_cfg(**bad)
         assert lib.xlpk_create(C.byref(c), C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_INVALID_ARG, bad
-    for unsup in (dict(head_dim=96), dict(batch=3), dict(n_q_heads=16, n_kv_heads=2)):
+    # FP8: K dims must be multiples of 256 (a row pair of 2K + K/16 bytes stays 16-byte aligned)
+    for unsup in (dict(head_dim=96), dict(batch=3), dict(n_q_heads=16, n_kv_heads=2),
+                  dict(weight_dtype=1, hidden=384)):
         c = _tiny_cfg(**unsup)
         assert lib.xlpk_create(C.byref(c), C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_UNSUPPORTED, unsup
     # a valid shape with missing weight pointers
