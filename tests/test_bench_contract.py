@@ -8,11 +8,12 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(extra_env=None):
+def _run(extra_env=None, steps=1, warmup=1):
     env = dict(os.environ)
     env.update(extra_env or {})
-    return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "1",
-                           "--warmup", "1"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--steps",
+                           str(steps), "--warmup", str(warmup)], cwd=ROOT, env=env, capture_output=True, text=True,
+                          timeout=600)
 
 
 def test_reference_arm_prints_one_contract_line():
@@ -39,3 +40,14 @@ def test_reference_arm_other_ranks_exit_without_work():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_survives_the_default_step_counts():
+    # warm-up 5 + 20 timed calls: every call must start from the sample's own
+    # start state (a sample whose position kept advancing would overrun its cache)
+    r = _run(steps=20, warmup=5)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, lines
+    d = json.loads(lines[0])
+    assert d["steps"] == 20 and d["warmup"] == 5 and d["value"] > 0
