@@ -331,3 +331,139 @@ def test_batch_sequences_are_independent():
         l0, _ = m0.step([a])
         l1, _ = m1.step([b])
         assert torch.equal(lb[0], l0[0]) and torch.equal(lb[1], l1[0])
+
+
+# ------------------------------------------------- FP8 weights inside the model
+
+def _bare_oracle(weights):
+    """An oracle over a hand-made weight dict (only W() is exercised)."""
+    cfg = DecoderConfig(name="w", n_layers=1, hidden=128, n_q_heads=2, n_kv_heads=1, head_dim=64,
+                        ffn=128, vocab=8, kv_len=0, steps=1)
+    return OracleDecoder(cfg, weights, 1, max_seq=1)
+
+
+def test_oracle_fp8_dequant_by_index_on_a_2x3_block_grid():
+    # 256 x 384 e4m3 codes: a 2 x 3 grid of 128x128 blocks, each with its own
+    # scale; every element must be table[code] * scale[row // 128][col // 128]
+    # (a transposed or mis-broadcast scale index fails on this non-square grid)
+    N, K = 256, 384
+    r = torch.arange(N)[:, None]
+    c = torch.arange(K)[None, :]
+    codes = ((r * 7 + c * 13) % 126).to(torch.uint8)          # finite codes only (0x7F is NaN)
+    codes[200, 300] = 0xFE                                     # -448
+    codes[5, 129] = 0x80                                       # -0
+    scales = torch.tensor([[0.5, 1.5, 3.0], [0.25, 2.0, 5.0]], dtype=torch.float32)
+    o = _bare_oracle({"m": codes, "m.scale": scales})
+    W = o.W("m")
+    assert W.shape == (N, K) and W.dtype == torch.float32
+    table = e4m3_decode_table()
+    for (i, j) in [(0, 0), (127, 127), (128, 0), (0, 128), (127, 255), (128, 256), (255, 383), (200, 300),
+                   (5, 129), (131, 17), (64, 200), (250, 130)]:
+        want = float(torch.tensor(float(table[int(codes[i, j])]) * float(scales[i // 128, j // 128]),
+                                  dtype=torch.float32))
+        assert float(W[i, j]) == want, (i, j)
+    # every block as a whole: block (bi, bj) / its scale is the decoded codes
+    for bi in range(2):
+        for bj in range(3):
+            blk = W[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128] / scales[bi, bj]
+            assert torch.equal(blk, table[codes[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128].long()])
+
+
+def test_oracle_fp8_weights_reproduce_the_bf16_originals():
+    # quantise seeded bf16 weights with the harness codec, widen them through the
+    # oracle's W(): each element is the original within e4m3's half-ulp of its block
+    w = synth.normal_bf16(0, "pin.fp8", (256, 384), 0.02)
+    codes, scales = synth.quantize_fp8_blocks(w)
+    W = _bare_oracle({"m": codes, "m.scale": scales}).W("m")
+    full_scale = scales.repeat_interleave(128, 0).repeat_interleave(128, 1)
+    q = w.float() / full_scale                                   # value in code units
+    err = (W - w.float()).abs() / full_scale                     # error in code units
+    normal = q.abs() >= 2.0 ** -6
+    # normal range: 3 mantissa bits -> |err| <= 2^-4 relative; subnormals: spacing 2^-9
+    assert bool((err[normal] <= q.abs()[normal] * 2.0 ** -4 * (1 + 1e-6)).all())
+    assert bool((err[~normal] <= 2.0 ** -10 * (1 + 1e-6)).all())
+    # and the block maximum is represented exactly (scale = amax / 448)
+    amax = w.float().view(2, 128, 3, 128).abs().amax(dim=(1, 3))
+    assert torch.allclose(W.view(2, 128, 3, 128).abs().amax(dim=(1, 3)), amax, rtol=1e-6)
+
+
+# ----------------------------------------------------- MoE composition, k > 1
+
+def _moe_structured():
+    """A one-layer MoE whose router and experts select entries by index.
+
+    H = 8, 4 routed experts (top-2) + 1 shared, expert width 4.  Router row e picks
+    xn[e] times c_e; expert e's gate row f picks xn[(f + e) % H] times a_e, its up
+    row f picks xn[(f + 2e + 1) % H] times b_e, and its down projection sends
+    h[(i + e) % 4] to output i.  The shared expert is built the same way with e = 4.
+    """
+    H, E, Fe = 8, 4, 4
+    cfg = DecoderConfig(name="m", n_layers=1, hidden=H, n_q_heads=2, n_kv_heads=1, head_dim=4, ffn=0,
+                        vocab=16, kv_len=0, steps=1, n_experts=E, top_k=2, n_shared_experts=1, expert_ffn=Fe)
+    w = synth.make_weights(cfg)
+    c = [1.0, 3.0, -2.0, 0.5]
+    a = [1.5, -0.75, 1.25, 2.0, 0.5]
+    bb = [-0.5, 1.0, 0.25, -1.5, 1.75]
+    router = torch.zeros(E, H)
+    for e in range(E):
+        router[e, e] = c[e]
+    w["layers.0.router"] = router.to(torch.bfloat16)
+
+    def expert(e):
+        g, u, d = torch.zeros(Fe, H), torch.zeros(Fe, H), torch.zeros(H, Fe)
+        for f in range(Fe):
+            g[f, (f + e) % H] = a[e]
+            u[f, (f + 2 * e + 1) % H] = bb[e]
+        for i in range(H):
+            d[i, (i + e) % Fe] = 1.0
+        return g, u, d
+
+    for e in range(E + 1):
+        g, u, d = expert(e)
+        q = f"layers.0.experts.{e}." if e < E else "layers.0.shared.0."
+        w[q + "w_gate"], w[q + "w_up"], w[q + "w_down"] = (t.to(torch.bfloat16) for t in (g, u, d))
+    return cfg, w, c, a, bb
+
+
+def test_moe_topk2_plus_shared_expert_closed_form():
+    cfg, w, c, a, bb = _moe_structured()
+    H, E, Fe = cfg.hidden, cfg.n_experts, cfg.expert_ffn
+    o = OracleDecoder(cfg, w, 1, max_seq=2)
+    for xn_vals in ([0.3, 0.9, -0.4, 1.1, -0.2, 0.7, 0.05, -1.3], [2.0, -0.1, 0.6, 0.2, 1.0, -0.8, 0.4, 0.9]):
+        xn = torch.tensor(xn_vals, dtype=torch.float32)
+        # hand routing: logits z_e = c_e xn[e], softmax, top-2 by probability (lower id on ties)
+        z = [c[e] * xn_vals[e] for e in range(E)]
+        mz = max(z)
+        ez = [math.exp(v - mz) for v in z]
+        p = [v / sum(ez) for v in ez]
+        top = sorted(range(E), key=lambda e: (-p[e], e))[:2]
+
+        def h(e):
+            out = []
+            for f in range(Fe):
+                g = a[e] * xn_vals[(f + e) % H]
+                out.append(g / (1 + math.exp(-g)) * bb[e] * xn_vals[(f + 2 * e + 1) % H])
+            return out
+
+        want = [sum(p[e] * h(e)[(i + e) % Fe] for e in top) + h(E)[(i + E) % Fe] for i in range(H)]
+        o._router_probs = []
+        got, ids = o._ffn(0, xn)
+        assert ids == top
+        assert torch.allclose(got, torch.tensor(want, dtype=torch.float32), rtol=1e-5, atol=1e-6), (got, want)
+        assert torch.allclose(o._router_probs[0], torch.tensor(p, dtype=torch.float32), rtol=1e-6)
+
+
+def test_moe_incremental_decode_equals_full_recompute():
+    cfg = DecoderConfig(name="m", n_layers=2, hidden=128, n_q_heads=2, n_kv_heads=1, head_dim=64, ffn=0,
+                        vocab=300, kv_len=9, steps=1, n_experts=4, top_k=2, n_shared_experts=1, expert_ffn=64)
+    w = synth.make_weights(cfg, norm_std=0.1)
+    toks = synth.make_prompt(cfg)                                   # [1][10]
+    full = OracleDecoder(cfg, w, 1, max_seq=12)
+    ref = full.forward_sequence(toks)[0]
+    inc = OracleDecoder(cfg, w, 1, max_seq=12)
+    for t in range(toks.shape[1]):
+        logits, _ = inc.step([int(toks[0, t])])
+        assert torch.allclose(logits[0], ref[t], rtol=1e-4, atol=1e-5), t
+    T = toks.shape[1]
+    assert torch.allclose(inc.K[:, :, :, :T].float(), full.K[:, :, :, :T].float(), atol=2e-2)
+    assert torch.allclose(inc.V[:, :, :, :T].float(), full.V[:, :, :, :T].float(), atol=2e-2)
