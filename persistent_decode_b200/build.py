@@ -12,7 +12,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "xlpk.cu")
-DEPS = [os.path.join(HERE, "csrc", f) for f in ("xlpk.cu", "engine.cuh", "tc_tile.cuh", "params.h")] + \
+DEPS = [os.path.join(HERE, "csrc", f) for f in ("xlpk.cu", "engine.cuh", "tcgen05.cuh", "tc_tile.cuh", "params.h")] + \
     [os.path.join(ROOT, "include", "xlpk.h")]
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libxlpk.so")

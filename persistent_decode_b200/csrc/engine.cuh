@@ -38,6 +38,7 @@
 #include <stdint.h>
 
 #include "params.h"
+#include "tcgen05.cuh"
 
 namespace xlpk {
 
@@ -246,6 +247,10 @@ struct alignas(16) SmemCtl {
   uint64_t full[kMaxSlots];
   uint64_t empty[kMaxSlots];
   uint64_t act_bar;      // completion of the activation bulk copy
+  uint64_t acc_bar;      // batch-8 tensor-core stages: the stage's MMAs have completed
+  uint64_t bop_bar;      //   the MMAs of a K window are done with its staged input
+  uint64_t fin_bar;      //   every MMA issued has completed (before the columns are freed)
+  uint32_t tmem_base;    //   this CTA's tensor-memory columns
   volatile int abort;
   int flag;
   int pad[2];
@@ -283,6 +288,8 @@ struct Ctx {
   int lane;
   int tid;
   uint32_t act_phase;   // parity of the next activation-copy phase (consumers)
+  uint32_t acc_phase;   // batch-8 tensor-core stages: parity of the next acc_bar / bop_bar phase
+  uint32_t bop_phase;
 };
 
 enum ErrCode : int { kErrNone = 0, kErrTimeout = -6, kErrAborted = -7 };
@@ -478,8 +485,17 @@ enum ActSrc : int { SRC_RESID = 0, SRC_EMBED = 1, SRC_PLAIN = 2 };
 //   SIDE_EMBED  this CTA's rows of the pending tokens' embeddings (layer-0 O-projection)
 enum SideKind : int { SIDE_NONE = 0, SIDE_ROPE = 1, SIDE_RESID = 2, SIDE_EMBED = 3 };
 
-// Row range [r0, r1) of this CTA in a stage whose matrix has H logical rows.
+// Row range [r0, r1) of this CTA in a stage whose matrix has H logical rows
+// (row pairs split evenly; with the batch-8 tensor-core tiles, 8-row units).
+template <int B>
 __device__ __forceinline__ void resid_rows(const Params& p, int c, int& r0, int& r1) {
+  if constexpr (B == kMaxBatch) {
+    if (p.tc) {
+      r0 = 8 * split_point(c, p.H >> 3, p.G);
+      r1 = 8 * split_point(c + 1, p.H >> 3, p.G);
+      return;
+    }
+  }
   r0 = 2 * split_point(c, p.H >> 1, p.G);
   r1 = 2 * split_point(c + 1, p.H >> 1, p.G);
 }
@@ -508,7 +524,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     asm volatile("fence.proxy.async;" ::: "memory");
     const uint32_t side_s = smem_addr(cx.side);
     int r0 = 0, r1 = 0;
-    if (side == SIDE_RESID || side == SIDE_EMBED) resid_rows(p, cx.c, r0, r1);
+    if (side == SIDE_RESID || side == SIDE_EMBED) resid_rows<B>(p, cx.c, r0, r1);
     int tok[B];
     if (side == SIDE_EMBED)
 #pragma unroll
@@ -706,6 +722,418 @@ __device__ __noinline__ void consume_gemv_t(const Params& p, Ctx& cx, const Mat&
       epi(g0 + cx.warp, a0, a1, cx.lane);
     }
   }
+}
+
+// K-windowed GEMV (the down projection when B x F fp32 inputs would crowd
+// out the ring): the CTA's tiles arrive window by window (all its groups'
+// chunks of one window, then the next), the activation region holds one window
+// of the input at a time (refilled by bulk copy after every consumer has left
+// the previous window), and each warp keeps its row pair's sums for every
+// group in registers until the last window.  The epilogue's side data (SIDE_RESID)
+// comes with the first window.
+template <int B, bool FP8, class Epi>
+__device__ __noinline__ void consume_gemv_win_t(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where,
+                                                const float* gsrc, int s, Epi& epi) {
+  const int NP = m.N >> 1;
+  const int p0 = split_point(cx.c, NP, p.G), p1 = split_point(cx.c + 1, NP, p.G);
+  const int np = p1 - p0;
+  const int ng = (np + kPairsPerTile - 1) / kPairsPerTile;   // <= kMaxWinGroups (checked at create)
+  const int KC = m.KC, nkc = m.K / KC, cw = p.down_win / KC;
+  const int nvKfull = m.K >> 3;
+  float a0[kMaxWinGroups][B], a1[kMaxWinGroups][B];
+#pragma unroll
+  for (int gi = 0; gi < kMaxWinGroups; ++gi)
+#pragma unroll
+    for (int b = 0; b < B; ++b) a0[gi][b] = a1[gi][b] = 0.f;
+  const uint32_t bar = smem_addr(&cx.ctl->act_bar);
+  for (int w = 0; w * cw < nkc; ++w) {
+    const int cww = min(cw, nkc - w * cw);
+    const int nvK = (cww * KC) >> 3;   // 8-column vectors of this window
+    // every consumer has left the previous window before it is overwritten
+    consumer_sync();
+    if (cx.tid == 0) {
+      asm volatile("fence.proxy.async;" ::: "memory");
+      uint32_t total = static_cast<uint32_t>(B) * 2u * nvK * 16u;
+      int r0 = 0, r1 = 0, v0 = 0, nv = 0;
+      if (w == 0) {
+        resid_rows<B>(p, cx.c, r0, r1);
+        v0 = r0 >> 3;
+        nv = r1 > r0 ? ((r1 - 1) >> 3) - v0 + 1 : 0;
+        total += static_cast<uint32_t>(B) * 2u * nv * 16u;
+      }
+      mbar_expect_tx(bar, total);
+      const int wv0 = (w * p.down_win) >> 3;   // first vector of the window in the full input
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        for (int pl = 0; pl < 2; ++pl)
+          bulk_g2s_nohint(smem_addr(cx.act) + ((pl * B + b) * nvK) * 16,
+                          gsrc + ((static_cast<size_t>(pl) * B + b) * nvKfull + wv0) * 4,
+                          static_cast<uint32_t>(nvK) * 16u, bar);
+      if (w == 0 && nv > 0) {
+        const uint32_t side_s = smem_addr(cx.side);
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          for (int pl = 0; pl < 2; ++pl)
+            bulk_g2s_nohint(side_s + p.side_resid + ((b * 2 + pl) * p.nvr) * 16,
+                            p.x + ((static_cast<size_t>(pl) * p.B + b) * (p.H >> 3) + v0) * 4,
+                            static_cast<uint32_t>(nv) * 16u, bar);
+      }
+    }
+    if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+    if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
+    cx.act_phase ^= 1u;
+    const uint32_t act_lo_s = smem_addr(cx.act);
+    const uint32_t act_hi_s = act_lo_s + B * nvK * 16;
+#pragma unroll
+    for (int gi = 0; gi < kMaxWinGroups; ++gi) {
+      if (gi >= ng) break;
+      const int gp = min(kPairsPerTile, np - gi * kPairsPerTile);
+      for (int kc = 0; kc < cww; ++kc) {
+        const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
+        const bool ok = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
+        if constexpr (FP8) {
+          if (ok && cx.warp < gp) {
+            const int nv8 = KC >> 4;
+            const uint32_t base = smem_addr(cx.ring) + rp.slot * kSlotBytes;
+            const uint32_t r0 = base + (2 * cx.warp) * KC;
+            const uint32_t r1 = r0 + KC;
+            const uint32_t s0 = base + 2 * gp * KC + (2 * cx.warp) * (KC >> 5);
+            const uint32_t s1 = s0 + (KC >> 5);
+            const uint32_t alo = act_lo_s + ((kc * KC) >> 3) * 16;
+            const uint32_t ahi = act_hi_s + ((kc * KC) >> 3) * 16;
+#pragma unroll 2
+            for (int v = cx.lane; v < nv8; v += 32) {
+              const uint4 w0 = lds_u4(r0 + v * 16);
+              const uint4 w1 = lds_u4(r1 + v * 16);
+              const float sc0 = __uint_as_float(lds_u1(s0 + (v >> 3) * 4));
+              const float sc1 = __uint_as_float(lds_u1(s1 + (v >> 3) * 4));
+#pragma unroll
+              for (int b = 0; b < B; ++b) {
+                const float4 x0 = lds_f4(alo + (b * nvK + 2 * v) * 16);
+                const float4 x1 = lds_f4(ahi + (b * nvK + 2 * v) * 16);
+                const float4 x2 = lds_f4(alo + (b * nvK + 2 * v + 1) * 16);
+                const float4 x3 = lds_f4(ahi + (b * nvK + 2 * v + 1) * 16);
+                a0[gi][b] = fmaf(sc0, dot16_e4m3(w0, x0, x1, x2, x3), a0[gi][b]);
+                a1[gi][b] = fmaf(sc1, dot16_e4m3(w1, x0, x1, x2, x3), a1[gi][b]);
+              }
+            }
+          }
+        } else if (ok && cx.warp < gp) {
+          const int nv = KC >> 3;
+          const uint32_t r0 = smem_addr(cx.ring) + rp.slot * kSlotBytes + (2 * cx.warp) * nv * 16;
+          const uint32_t r1 = r0 + nv * 16;
+          const uint32_t alo = act_lo_s + (kc * nv) * 16;
+          const uint32_t ahi = act_hi_s + (kc * nv) * 16;
+#pragma unroll 4
+          for (int v = cx.lane; v < nv; v += 32) {
+            const uint4 w0 = lds_u4(r0 + v * 16);
+            const uint4 w1 = lds_u4(r1 + v * 16);
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              const float4 lo = lds_f4(alo + (b * nvK + v) * 16);
+              const float4 hi = lds_f4(ahi + (b * nvK + v) * 16);
+              a0[gi][b] = dot8_bf16(w0, lo, hi, a0[gi][b]);
+              a1[gi][b] = dot8_bf16(w1, lo, hi, a1[gi][b]);
+            }
+          }
+        }
+        __syncwarp();
+        if (cx.lane == 0 && ok) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
+        rp.next(p.nslot);
+      }
+    }
+  }
+#pragma unroll
+  for (int gi = 0; gi < kMaxWinGroups; ++gi) {
+    if (gi >= ng) break;
+    const int gp = min(kPairsPerTile, np - gi * kPairsPerTile);
+    if (cx.warp < gp) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        a0[gi][b] = warp_sum(a0[gi][b]);
+        a1[gi][b] = warp_sum(a1[gi][b]);
+      }
+      epi(p0 + gi * kPairsPerTile + cx.warp, a0[gi], a1[gi], cx.lane);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ batch-8 tensor-core stages
+
+// The epilogue's side data alone (the batch-8 tensor-core stages stage their
+// input themselves): the same bulk copies as load_act's, on the act barrier.
+template <int B>
+__device__ __noinline__ void load_side(const Params& p, Ctx& cx, int side, int s, int where) {
+  if (side == SIDE_NONE) return;
+  const uint32_t bar = smem_addr(&cx.ctl->act_bar);
+  if (cx.tid == 0) {
+    asm volatile("fence.proxy.async;" ::: "memory");
+    const uint32_t side_s = smem_addr(cx.side);
+    int r0 = 0, r1 = 0;
+    resid_rows<B>(p, cx.c, r0, r1);
+    const uint32_t rope_bytes = static_cast<uint32_t>(p.d) * 4u;
+    const int v0 = r0 >> 3, nv = r1 > r0 ? ((r1 - 1) >> 3) - v0 + 1 : 0;
+    const int e0 = r0 & ~7, e1 = (r1 + 7) & ~7;
+    uint32_t total = 0;
+    if (side == SIDE_ROPE) total = B * rope_bytes;
+    if (side == SIDE_RESID) total = static_cast<uint32_t>(B) * 2u * nv * 16u;
+    if (side == SIDE_EMBED && r1 > r0) total = static_cast<uint32_t>(B) * (e1 - e0) * 2u;
+    mbar_expect_tx(bar, total);
+    if (side == SIDE_ROPE) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        bulk_g2s_nohint(side_s + p.side_rope + b * rope_bytes,
+                        p.rope + static_cast<size_t>(p.pos0[b] + s) * (p.d >> 1), rope_bytes, bar);
+    } else if (side == SIDE_RESID && nv > 0) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        for (int pl = 0; pl < 2; ++pl)
+          bulk_g2s_nohint(side_s + p.side_resid + ((b * 2 + pl) * p.nvr) * 16,
+                          p.x + ((static_cast<size_t>(pl) * p.B + b) * (p.H >> 3) + v0) * 4,
+                          static_cast<uint32_t>(nv) * 16u, bar);
+    } else if (side == SIDE_EMBED && r1 > r0) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        bulk_g2s_nohint(side_s + p.side_embed + b * p.evb,
+                        p.embed + static_cast<size_t>(__ldcg(p.cur_tok + b)) * p.H + e0,
+                        static_cast<uint32_t>(e1 - e0) * 2u, bar);
+    }
+  }
+  if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+  if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
+  cx.act_phase ^= 1u;
+}
+
+// Stage columns [k0, k0 + Kw) of the 8 sequences' input as the MMA's B
+// operand: bf16 boxes of [8 rows][64 columns] in the 128-byte-swizzle K-major
+// layout, box jb at act + jb * 1024.  The source is the two-plane fp32 layout
+// (or, SRC_EMBED, the pending tokens' bf16 embedding rows); with `gain` the
+// values are multiplied by it and the rows' RMSNorm factors returned in rn
+// (K = Kw = the whole input then).  `hidden_dbg` receives the raw input.
+__device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src, const float* gsrc, int K, int k0,
+                                            int Kw, const float* gain, float* hidden_dbg, float (&rn)[kMaxBatch]) {
+  constexpr int B = kMaxBatch;
+  const uint32_t act_s = smem_addr(cx.act);
+  float ss[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) ss[b] = 0.f;
+  const int nv = Kw >> 3;   // 8-column vectors of the window
+  int tok[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) tok[b] = src == SRC_EMBED ? __ldcg(p.cur_tok + b) : 0;
+  // one 8-column vector of all 8 sequences per thread and pass: its 16 (or 8)
+  // loads are independent and in flight together
+  for (int v = cx.tid; v < nv; v += kConsumerThreads) {
+    const int k = k0 + 8 * v;
+    float4 lo[B], hi[B];
+    if (src == SRC_EMBED) {
+      uint4 u[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        u[b] = __ldg(reinterpret_cast<const uint4*>(p.embed + static_cast<size_t>(tok[b]) * K + k));
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        lo[b] = make_float4(bf16_lo(u[b].x), bf16_hi(u[b].x), bf16_lo(u[b].y), bf16_hi(u[b].y));
+        hi[b] = make_float4(bf16_lo(u[b].z), bf16_hi(u[b].z), bf16_lo(u[b].w), bf16_hi(u[b].w));
+      }
+    } else {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        lo[b] = __ldcg(reinterpret_cast<const float4*>(gsrc + plane_index(b, k, B, K)));
+        hi[b] = __ldcg(reinterpret_cast<const float4*>(gsrc + plane_index(b, k + 4, B, K)));
+      }
+    }
+    float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
+    if (gain) {
+      g0 = __ldg(reinterpret_cast<const float4*>(gain + k));
+      g1 = __ldg(reinterpret_cast<const float4*>(gain + k + 4));
+    }
+    const int kk = k - k0, jb = kk >> 6, q = (kk & 63) >> 3;
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const float e[8] = {lo[b].x, lo[b].y, lo[b].z, lo[b].w, hi[b].x, hi[b].y, hi[b].z, hi[b].w};
+      if (hidden_dbg)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) hidden_dbg[static_cast<size_t>(b) * K + k + t] = e[t];
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc = fmaf(e[t], e[t], acc);
+      ss[b] += acc;
+      const uint32_t dst = act_s + jb * 1024 + b * 128 + ((q ^ b) << 4);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pack_bf16x2(e[0] * g0.x, e[1] * g0.y)),
+                   "r"(pack_bf16x2(e[2] * g0.z, e[3] * g0.w)), "r"(pack_bf16x2(e[4] * g1.x, e[5] * g1.y)),
+                   "r"(pack_bf16x2(e[6] * g1.z, e[7] * g1.w))
+                   : "memory");
+    }
+  }
+  // the MMAs read the operand through the async proxy
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+#pragma unroll
+  for (int b = 0; b < B; ++b) rn[b] = 1.f;
+  if (gain) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const float t = warp_sum(ss[b]);
+      if (cx.lane == 0) cx.ctl->red[cx.warp][b] = t;
+    }
+    consumer_sync();
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) t += cx.ctl->red[w][b];
+      rn[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
+    }
+  }
+  consumer_sync();
+}
+
+// Widen an FP8 tile in its ring slot to bf16 boxes in place: nb e4m3 boxes of
+// [rv][128 codes] (+ the rows' scales) become 2*nb bf16 boxes of [rv][64],
+// the codes times their block scale rounded to bf16, same swizzle.  Every
+// consumer thread reads its units before any is overwritten.
+__device__ __noinline__ void tc_widen_fp8(Ctx& cx, uint32_t slot_s, int rv, int nb) {
+  constexpr int kMaxUnits = 4;   // 16-byte code units per thread: nb * rv * 8 <= 1024
+  const int nu = nb * rv * 8;
+  uint4 code[kMaxUnits];
+  float sc[kMaxUnits];
+#pragma unroll
+  for (int t = 0; t < kMaxUnits; ++t) {
+    const int i = cx.tid + t * kConsumerThreads;
+    if (i < nu) {
+      const int j = i / (rv * 8), rem = i - j * rv * 8, r = rem >> 3;
+      code[t] = lds_u4(slot_s + i * 16);
+      sc[t] = __uint_as_float(lds_u1(slot_s + nb * rv * 128 + (j * rv + r) * 4));
+    }
+  }
+  consumer_sync();
+#pragma unroll
+  for (int t = 0; t < kMaxUnits; ++t) {
+    const int i = cx.tid + t * kConsumerThreads;
+    if (i < nu) {
+      const int j = i / (rv * 8), rem = i - j * rv * 8, r = rem >> 3, pq = rem & 7;
+      const int q = pq ^ (r & 7);                 // logical 16-code unit of the row
+      const uint32_t w[4] = {code[t].x, code[t].y, code[t].z, code[t].w};
+      uint32_t o[8];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 a = e4m3x2_to_float2(w[h] & 0xffffu);
+        const float2 c = e4m3x2_to_float2(w[h] >> 16);
+        o[2 * h] = pack_bf16x2(a.x * sc[t], a.y * sc[t]);
+        o[2 * h + 1] = pack_bf16x2(c.x * sc[t], c.y * sc[t]);
+      }
+      // columns 16q..16q+15 -> bf16 box 2j + q/4, its 8-column units 2(q%4), 2(q%4)+1
+      const uint32_t box = slot_s + (2 * j + (q >> 2)) * rv * 128 + r * 128;
+      const int u = 2 * (q & 3);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + ((u ^ (r & 7)) << 4)), "r"(o[0]),
+                   "r"(o[1]), "r"(o[2]), "r"(o[3])
+                   : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(box + (((u + 1) ^ (r & 7)) << 4)), "r"(o[4]),
+                   "r"(o[5]), "r"(o[6]), "r"(o[7])
+                   : "memory");
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  consumer_sync();
+}
+
+__device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(n) : "memory");
+}
+
+// One batch-8 projection on the tensor cores: the CTA's 8-row units of `m`
+// (M-tiles of <= 128 rows, each with kTcAccCols accumulator columns in tensor
+// memory, of which columns 0..7 are the 8 sequences),
+// the input staged as the B operand window by window (`win` columns; 0: the
+// whole K), one issuing thread (consumer warp 4, lane 0) driving the MMAs and
+// releasing each ring slot with tcgen05.commit, then warps 0..3 reading their
+// accumulator rows back and running `epi` on each row pair with rn applied.
+template <class Epi>
+__device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where, ActSrc src,
+                                        const float* gsrc, const float* gain, float* hidden_dbg, int win, Epi& epi) {
+  constexpr int B = kMaxBatch;
+  const int fp8 = m.fp8;
+  const int U = m.N >> 3;
+  const int u0 = split_point(cx.c, U, p.G), u1 = split_point(cx.c + 1, U, p.G);
+  const int R = 8 * (u1 - u0), nm = (R + 127) >> 7;
+  const int K = m.K, bc = tc_box_cols(fp8), kbox = tc_kbox(K, win, fp8);
+  const int nw = win > 0 ? (K + win - 1) / win : 1;
+  const bool issuer = cx.warp == 4 && cx.lane == 0;
+  const uint32_t idesc = tc_idesc_bf16(128, kTcAccCols);
+  const uint32_t tmem = cx.ctl->tmem_base;
+  float rn[B];
+  for (int w = 0; w < nw; ++w) {
+    const int k0 = w * win, Kw = win > 0 ? min(win, K - k0) : K;
+    if (w > 0) {
+      // the previous window's MMAs must be done with the staged input
+      if (!cx.ctl->abort) ring_wait(p, cx.ctl, smem_addr(&cx.ctl->bop_bar), cx.bop_phase, where);
+      cx.bop_phase ^= 1u;
+    }
+    float rw[B];
+    tc_stage_input(p, cx, src, gsrc, K, k0, Kw, w == 0 ? gain : nullptr, w == 0 ? hidden_dbg : nullptr, rw);
+    if (w == 0)
+#pragma unroll
+      for (int b = 0; b < B; ++b) rn[b] = rw[b];
+    if (issuer) tc_fence_after();
+    for (int mt = 0; mt < nm; ++mt) {
+      const int rv = min(128, R - 128 * mt);
+      const int nb = tc_nb(rv, kbox, fp8);
+      const int nt = (Kw / bc) / nb;
+      for (int t = 0; t < nt; ++t) {
+        const uint32_t slot_s = smem_addr(cx.ring) + rp.slot * kSlotBytes;
+        const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
+        const uint32_t eb = smem_addr(&cx.ctl->empty[rp.slot]);
+        bool ok;
+        if (fp8) {
+          const bool got = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
+          ok = !consumer_sync_any(!got);                 // uniform: the widening is CTA-collective
+          if (ok) tc_widen_fp8(cx, slot_s, rv, nb);
+        } else {
+          ok = issuer ? (cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where)) : true;
+        }
+        if (issuer && ok) {
+          tc_fence_after();
+          const int nbx = fp8 ? 2 * nb : nb;            // bf16 boxes of 64 columns in the slot
+          const int bx0 = t * nbx;                       // first B-operand box of the tile
+#pragma unroll 1
+          for (int j = 0; j < nbx; ++j)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              tc_mma(tmem + mt * kTcAccCols, tc_desc_sw128(slot_s + j * rv * 128 + ks * 32),
+                     tc_desc_sw128(smem_addr(cx.act) + (bx0 + j) * 1024 + ks * 32), idesc,
+                     (w | t | j | ks) != 0 ? 1u : 0u);
+          mbar_arrive_n(eb, kConsumerWarps - 1);
+          tc_commit(eb);                                 // the slot is free once these MMAs have read it
+        }
+        rp.next(p.nslot);
+      }
+    }
+    if (issuer && !cx.ctl->abort) tc_commit(smem_addr(w + 1 < nw ? &cx.ctl->bop_bar : &cx.ctl->acc_bar));
+  }
+  // accumulators -> epilogue, one row pair at a time
+  if (!cx.ctl->abort) ring_wait(p, cx.ctl, smem_addr(&cx.ctl->acc_bar), cx.acc_phase, where);
+  cx.acc_phase ^= 1u;
+  tc_fence_after();
+  const bool aborting = consumer_sync_any(cx.ctl->abort != 0);   // uniform: tcgen05.ld is warp-collective
+  if (cx.warp < 4 && !aborting) {
+    for (int mt = 0; mt < nm; ++mt) {
+      const int rv = min(128, R - 128 * mt);
+      if (cx.warp * 32 >= rv) continue;               // warp-uniform
+      uint32_t v[8];
+      tc_ld8(tmem + (static_cast<uint32_t>(cx.warp * 32) << 16) + mt * kTcAccCols, v);
+      for (int i = 0; i < 16; ++i) {
+        if (cx.warp * 32 + 2 * i >= rv) break;         // warp-uniform
+        float a0[B], a1[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          a0[b] = __uint_as_float(__shfl_sync(0xffffffffu, v[b], 2 * i)) * rn[b];
+          a1[b] = __uint_as_float(__shfl_sync(0xffffffffu, v[b], 2 * i + 1)) * rn[b];
+        }
+        epi(4 * u0 + 64 * mt + 16 * cx.warp + i, a0, a1, cx.lane);
+      }
+    }
+  }
+  tc_fence_before();
 }
 
 // e4m3 and bf16 tiles are separate instantiations, so neither inner loop
@@ -1496,13 +1924,23 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   if (kind == ST_LM) {
     if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ffn_done, G * S1, where, fused)) return false;
     float* hid = (p.hidden_out && cx.c == 0) ? p.hidden_out + static_cast<size_t>(s) * p.B * p.H : nullptr;
-    float rn[B];
-    load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, SIDE_NONE, s, rn, where);
-    if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     EpiLM<B> epi{p, s, &bv, &bi};
-    consume_gemv<B>(p, cx, p.lm, rp, where, rn, epi);
+    bool on_tc = false;
+    if constexpr (B == kMaxBatch && !MOE) {
+      if (p.tc) {
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+        consume_tc(p, cx, p.lm, rp, where, SRC_RESID, p.x, p.final_norm, hid, 0, epi);
+        on_tc = true;
+      }
+    }
+    if (!on_tc) {
+      float rn[B];
+      load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, SIDE_NONE, s, rn, where);
+      if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+      consume_gemv<B>(p, cx, p.lm, rp, where, rn, epi);
+    }
     if (cx.lane < B) {
       cx.ctl->redv[cx.warp][cx.lane] = bv;
       cx.ctl->redi[cx.warp][cx.lane] = bi;
@@ -1559,8 +1997,51 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   bool ok = true;
   float rn[B];
   int r0, r1;
-  resid_rows(p, cx.c, r0, r1);
-  switch (kind) {
+  resid_rows<B>(p, cx.c, r0, r1);
+  bool on_tc = false;
+  if constexpr (B == kMaxBatch && !MOE) {
+    if (p.tc) {
+      // batch-8 tensor-core stages: same waits, side data and epilogues
+      on_tc = true;
+      const unsigned* dep;
+      unsigned tgt;
+      if (kind == ST_QKV) {
+        dep = l == 0 ? p.cnt + p.cl.step_done : p.cnt + (l - 1) * ST_LAYER + ffn_done;
+        tgt = l == 0 ? S1 - 1u : G * S1;
+      } else if (kind == ST_OPROJ) {
+        dep = p.cnt + l * ST_LAYER + ST_ATTN;
+        tgt = static_cast<unsigned>(p.B * p.nkv) * S1;
+      } else if (kind == ST_GATEUP) {
+        dep = p.cnt + l * ST_LAYER + ST_OPROJ;
+        tgt = G * S1;
+      } else {
+        dep = p.cnt + l * ST_LAYER + ST_GATEUP;
+        tgt = G * S1;
+      }
+      if (!stage_wait(p, cx, dep, tgt, where, fused)) return false;
+      if (kind == ST_QKV) {
+        load_side<B>(p, cx, SIDE_ROPE, s, where);
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+        EpiQKV<B> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
+        consume_tc(p, cx, L.qkv, rp, where, l == 0 ? SRC_EMBED : SRC_RESID, p.x, L.attn_norm, nullptr, 0, epi);
+      } else if (kind == ST_OPROJ) {
+        load_side<B>(p, cx, l == 0 ? SIDE_EMBED : SIDE_RESID, s, where);
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+        EpiResid<B> epi{p, l == 0, cx.side, r0 >> 3, r0 & ~7};
+        consume_tc(p, cx, L.o, rp, where, SRC_PLAIN, p.o, nullptr, nullptr, 0, epi);
+      } else if (kind == ST_GATEUP) {
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+        EpiSwiGLU<B> epi{p};
+        consume_tc(p, cx, L.gu, rp, where, SRC_RESID, p.x, L.ffn_norm, nullptr, 0, epi);
+      } else {
+        load_side<B>(p, cx, SIDE_RESID, s, where);
+        if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+        EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
+        consume_tc(p, cx, L.down, rp, where, SRC_PLAIN, p.h, nullptr, nullptr, p.down_win, epi);
+      }
+    }
+  }
+  if (!on_tc) switch (kind) {
     case ST_QKV: {
       if (l == 0) {
         ok = stage_wait(p, cx, p.cnt + p.cl.step_done, S1 - 1u, where, fused);
@@ -1623,6 +2104,17 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
     }
     default: {  // ST_DOWN
       if (!stage_wait(p, cx, p.cnt + l * ST_LAYER + ST_GATEUP, G * S1, where, fused)) return false;
+      if constexpr (!MOE && B >= 2) {   // (batch 1 inputs always fit whole)
+        if (p.down_win > 0) {
+          if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
+          EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
+          if (L.down.fp8)
+            consume_gemv_win_t<B, true>(p, cx, L.down, rp, where, p.h, s, epi);
+          else
+            consume_gemv_win_t<B, false>(p, cx, L.down, rp, where, p.h, s, epi);
+          break;
+        }
+      }
       const int K = MOE ? p.S * p.Fe : p.F;
       load_act<B>(p, cx, K, SRC_PLAIN, p.h, nullptr, nullptr, SIDE_RESID, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
@@ -1664,6 +2156,8 @@ __device__ __forceinline__ Ctx make_ctx(uint8_t* smem, const Params& p) {
   cx.warp = threadIdx.x >> 5;
   cx.lane = threadIdx.x & 31;
   cx.act_phase = 0;
+  cx.acc_phase = 0;
+  cx.bop_phase = 0;
   return cx;
 }
 
@@ -1684,6 +2178,9 @@ __device__ __forceinline__ void init_ring(const Params& p, Ctx& cx) {
       mbar_init(smem_addr(&cx.ctl->empty[i]), kConsumerWarps);
     }
     mbar_init(smem_addr(&cx.ctl->act_bar), 1);
+    mbar_init(smem_addr(&cx.ctl->acc_bar), 1);
+    mbar_init(smem_addr(&cx.ctl->bop_bar), 1);
+    mbar_init(smem_addr(&cx.ctl->fin_bar), 1);
     cx.ctl->abort = 0;
     cx.ctl->flag = 0;
     cx.ctl->route_seq = 0;
@@ -1823,6 +2320,16 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         cu.KC = m.KC;
         cu.slot = 0;
         cu.grp = 0;
+      } else if (B == kMaxBatch && p.tc) {
+        // batch-8 tensor-core tiles: the CTA's 8-row units, runs per K window
+        const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
+        const int U = m.N >> 3;
+        const int u0 = split_point(c, U, p.G), u1 = split_point(c + 1, U, p.G);
+        cu.a = 4 * u0;
+        cu.a_end = 4 * u1;
+        cu.kc = 0;
+        cu.phase = 0;
+        cu.src = m.packed + static_cast<size_t>(8) * u0 * tc_row_bytes(m.K, m.fp8);
       } else {
         const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
         const int NP = m.N >> 1;
@@ -1890,6 +2397,50 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         }
         return CUR_TILE;
       }
+    } else if (!MOE && B == kMaxBatch && p.tc && cu.a < cu.a_end) {
+      // batch-8 tensor-core stage: per K window one run, the full 128-row
+      // M-tiles' tiles then the last M-tile's (params.h: tile geometry)
+      const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
+      const int win = cu.kind == ST_DOWN ? p.down_win : 0;
+      const int fp8 = m.fp8, bc = tc_box_cols(fp8), kbox = tc_kbox(m.K, win, fp8);
+      const int R = 2 * (cu.a_end - cu.a), w = cu.phase;
+      const int k0 = w * win, Kw = win > 0 ? min(win, m.K - k0) : m.K;
+      const int rl = R - 128 * ((R - 1) >> 7);    // rows of the last M-tile
+      const int nfull = (R - rl) >> 7;
+      const int nb1 = tc_nb(128, kbox, fp8), nbl = tc_nb(rl, kbox, fp8);
+      run->src = cu.src + static_cast<size_t>(w) * R * tc_row_bytes(win, fp8);
+      if (rl == 128) {
+        run->n1 = (nfull + 1) * ((Kw / bc) / nb1);
+        run->n2 = 0;
+      } else {
+        run->n1 = nfull * ((Kw / bc) / nb1);
+        run->n2 = (Kw / bc) / nbl;
+      }
+      run->b1 = static_cast<uint32_t>(tc_tile_bytes(128, nb1, fp8));
+      run->b2 = static_cast<uint32_t>(tc_tile_bytes(rl, nbl, fp8));
+      run->stage = t.stage;
+      run->layer = t.layer;
+      run->step = t.step;
+      ++cu.phase;
+      if (win == 0 || cu.phase * win >= m.K) cu.a = cu.a_end;
+      return CUR_RUN;
+    } else if (!MOE && B >= 2 && cu.kind == ST_DOWN && p.down_win > 0 && cu.a < cu.a_end) {
+      // K-windowed down projection: one run per window (its tiles: the full
+      // groups' chunks of the window, then the partial group's); cu.phase
+      // counts the windows
+      const int np = cu.a_end - cu.a;
+      const int cw = p.down_win / cu.KC, w = cu.phase;
+      const int cww = min(cw, cu.nkc - w * cw);
+      run->src = cu.src + static_cast<size_t>(2) * np * cw * w * cu.trow;
+      run->n1 = (np / kPairsPerTile) * cww;
+      run->b1 = 2u * kPairsPerTile * cu.trow;
+      run->n2 = (np % kPairsPerTile) ? cww : 0;
+      run->b2 = 2u * (np % kPairsPerTile) * cu.trow;
+      run->stage = t.stage;
+      run->layer = t.layer;
+      run->step = t.step;
+      if (++cu.phase * cw >= cu.nkc) cu.a = cu.a_end;
+      return CUR_RUN;
     } else if (cu.a < cu.a_end && !(moe && cu.kind == ST_GATEUP) && cu.kc == 0) {
       // a whole dense stage (the MoE router goes tile by tile)
       const int np = cu.a_end - cu.a;
@@ -2131,6 +2682,41 @@ __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
 }
 
 // The persistent engine: one launch decodes p.n_steps tokens.
+// Batch-8 tensor-core stages: consumer warp 0 allocates the CTA's accumulator
+// columns before the first stage and frees them after the last (every consumer
+// leaves consumer_main at the same point, abort included).
+template <int B>
+__device__ __forceinline__ void tc_open(const Params& p, Ctx& cx) {
+  if constexpr (B == kMaxBatch) {
+    if (!p.tc) return;
+    if (cx.warp == 0) tc_alloc(smem_addr(&cx.ctl->tmem_base), static_cast<uint32_t>(p.tc_cols));
+    tc_fence_before();
+    consumer_sync();
+    tc_fence_after();
+  }
+}
+template <int B>
+__device__ __forceinline__ void tc_close(const Params& p, Ctx& cx) {
+  if constexpr (B == kMaxBatch) {
+    if (!p.tc) return;
+    if (cx.warp == 4 && cx.lane == 0) {
+      // MMAs may still be in flight after an abort: free the columns only once
+      // every one this thread issued has completed (bounded)
+      tc_commit(smem_addr(&cx.ctl->fin_bar));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(smem_addr(&cx.ctl->fin_bar), 0) &&
+             static_cast<long long>(globaltimer() - t0) < 2 * p.spin_limit_ns) {
+      }
+    }
+    tc_fence_before();
+    consumer_sync();
+    if (cx.warp == 0) {
+      tc_fence_after();
+      tc_dealloc(cx.ctl->tmem_base, static_cast<uint32_t>(p.tc_cols));
+    }
+  }
+}
+
 template <int B, int D, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) engine_persistent(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -2140,7 +2726,9 @@ __global__ void __launch_bounds__(kThreads, 1) engine_persistent(const __grid_co
     if (cx.lane == 0) producer_main<B, MOE>(p, cx, 0, 0, 0, true);
     __syncwarp();
   } else {
+    tc_open<B>(p, cx);
     consumer_main<B, D, MOE>(p, cx, 0, 0, 0, true);
+    tc_close<B>(p, cx);
   }
 }
 
@@ -2164,7 +2752,9 @@ __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constan
     if (cx.lane == 0) producer_main<B, MOE>(p, cx, kind, layer, step, false);
     __syncwarp();
   } else {
+    tc_open<B>(p, cx);
     consumer_main<B, D, MOE>(p, cx, kind, layer, step, false);
+    tc_close<B>(p, cx);
   }
 }
 

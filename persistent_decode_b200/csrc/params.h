@@ -25,6 +25,7 @@ constexpr int kMaxExperts = 256;                      // routed experts per MoE 
 constexpr int kMaxMoeSlots = 16;                      // shared + selected experts per token
 constexpr int kMaxCtas = 160;                        // persistent grid limit (one CTA per SM; B200 has 148)
 constexpr int kTraceSlots = 16;                       // u64 stamps per (step, stage, CTA) in a trace
+constexpr int kMaxWinGroups = 4;                      // K-windowed down projection: row-pair groups per CTA
 
 // Stages of one layer, in dependency order, then the LM head.
 enum StageKind : int {
@@ -75,6 +76,46 @@ struct Mat {
 // Bytes of one packed row over `k` columns (codes or bf16 values, plus FP8 scales).
 __host__ __device__ __forceinline__ int packed_row_bytes(const Mat& m, int k) {
   return m.fp8 ? k + k / 32 : 2 * k;
+}
+
+// ------------------------------------------------------------------ batch-8 tensor-core tiles
+// With Params::tc (batch 8, dense layers) every projection runs on tcgen05
+// MMAs.  A CTA owns an even share of the matrix's 8-row units; its rows form
+// M-tiles of up to 128 rows.  Weights are packed per CTA span in (K window,
+// M-tile, tile) order; a tile is nb boxes of [rv rows][128 bytes] (64 bf16 or
+// 128 e4m3 columns), each box in the canonical K-major 128-byte-swizzle layout
+// (row r's 16-byte unit q at r*128 + ((q ^ (r % 8)) * 16)), followed for FP8 by
+// the rows' block scales [nb][rv] fp32.  A plain bulk copy of a tile into a
+// 1024-byte-aligned ring slot therefore lands as nb ready MMA operands.
+__host__ __device__ inline int tc_box_cols(int fp8) { return fp8 ? 128 : 64; }
+// Boxes per tile for M-tiles of rv rows: the largest power of two <= 16 whose
+// tile fits (bf16: 32 KB; FP8 codes: 16 KB, so that their in-place bf16
+// expansion fits the slot), whose last bf16 box still leaves the 128 rows an
+// M = 128 MMA reads inside the slot, and which divides `kbox`, the boxes per K
+// window.
+__host__ __device__ inline int tc_nb(int rv, int kbox, int fp8) {
+  const int cap = fp8 ? 16384 : 32768;
+  int nb = 16;
+  while (nb > 1 && (nb * rv * 128 > cap || ((fp8 ? 2 : 1) * nb - 1) * rv * 128 + 128 * 128 > kSlotBytes ||
+                    kbox % nb))
+    nb >>= 1;
+  return nb;
+}
+__host__ __device__ inline int tc_tile_bytes(int rv, int nb, int fp8) { return nb * rv * 128 + (fp8 ? nb * rv * 4 : 0); }
+// Packed bytes of one row over `cols` columns (codes or values + FP8 scales).
+__host__ __device__ inline long long tc_row_bytes(long long cols, int fp8) { return fp8 ? cols + cols / 32 : 2 * cols; }
+__host__ __device__ inline int tc_gcd(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+// Boxes per window common to every window of a K x (window) split.
+__host__ __device__ inline int tc_kbox(int K, int win, int fp8) {
+  const int bc = tc_box_cols(fp8);
+  return win > 0 ? tc_gcd(K / bc, win / bc) : K / bc;
 }
 
 struct LayerParams {
@@ -148,6 +189,10 @@ struct Params {
                      // x then accumulates the down projection's partial sums
   int ffn_fused;     // 1: gate/up and down run as one stage with a split-K down projection
   int jt;            // fused FFN: W_down columns per tile
+  int tc;            // 1: batch-8 projections on tcgen05 MMAs (tensor-core packing and stages)
+  int tc_cols;       //   tensor-memory columns each CTA allocates (8 per M-tile of its largest stage)
+  int down_win;      // K-windowed down projection: W_down columns per activation window (0: whole K);
+                     // the CTA's down tiles are packed window by window, groups inside a window
   int side_hloc;     // fused FFN: byte offset of the CTA's h slice [B][hloc] in the side region
   int hloc;          //   floats per sequence of that slice (max gate/up pairs per CTA)
   int* route_exp;    // MoE: [L][S] expert of each slot (written by CTA 0)

@@ -23,6 +23,7 @@
 // the tensor memory and leaves.
 #pragma once
 #include "engine.cuh"
+#include "tcgen05.cuh"
 
 namespace xlpk {
 
@@ -37,40 +38,9 @@ __host__ __device__ constexpr int tc_smem_bytes(int K) {
   return 1024 /* alignment slack */ + kTcRows * 128 /* A box */ + (K / kTcKBox) * kTcN * 128 /* B */ + 64;
 }
 
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (the leading-byte offset is not used by swizzled K-major
-// layouts and is set to one 16-byte unit), descriptor version 1.
-__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
-  uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(1u) << 16;
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
-  return d;
-}
-
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
 // K-major, N = kTcN, M = kTcRows.
-constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kTcN >> 3) << 17) | ((kTcRows >> 4) << 24);
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive on `bar` once every tcgen05.mma this thread issued so far has completed.
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
+constexpr uint32_t kTcIdesc = tc_idesc_bf16(kTcRows, kTcN);
 
 // Bounded wait on an mbarrier phase (plain polling; the tile is short).
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, long long limit_ns) {

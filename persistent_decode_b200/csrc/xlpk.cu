@@ -45,11 +45,24 @@ xlpk_status cuda_fail(cudaError_t e, const char* what) {
 
 struct PackJob {
   const uint8_t* src;   // source row
-  long long dst;        // byte offset of the row's first chunk in the packed buffer
-  long long stride;     // bytes between consecutive chunks of this row
   const float* scale;   // FP8: the row's block-scale row ([K/128] fp32), else null
-  long long sdst;       // FP8: byte offset of the row's scales in its first tile
+  long long base;       // byte offset of the CTA's span in the packed buffer
+  int row;              // row inside its tile (2 * pair-in-group + 0/1)
+  int j16;              // rows of the span before this row's group
+  int gp2;              // rows of this row's group
+  int np2;              // rows of the span
 };
+
+// Where chunk kc of a packed row starts.  The span's tiles are ordered
+// (window, group, chunk in window); with one window (cw = nkc) this is the
+// plain (group, chunk) order.  Returns the tile's offset; the row's codes sit
+// at + row * KC * esz, an FP8 tile's scales at + gp2 * KC + row * KC / 32.
+__host__ __device__ inline long long pack_tile_offset(const PackJob& j, int kc, int nkc, int cw, long long tile_row) {
+  const int w = kc / cw;
+  const int cww = (nkc - w * cw) < cw ? (nkc - w * cw) : cw;
+  return j.base + static_cast<long long>(j.np2) * cw * w * tile_row + static_cast<long long>(j.j16) * cww * tile_row +
+         static_cast<long long>(kc - w * cw) * j.gp2 * tile_row;
+}
 
 // bf16 [R][C] row-major -> [C][R] row-major (32x32 tiles through shared memory).
 __global__ void transpose_bf16_kernel(const uint16_t* in, uint16_t* out, int R, int C) {
@@ -67,18 +80,21 @@ __global__ void transpose_bf16_kernel(const uint16_t* in, uint16_t* out, int R, 
 }
 
 // FP8: one thread per (row, chunk): the chunk's KC/128 block scales of the row.
-__global__ void pack_scales_kernel(const PackJob* jobs, int njobs, uint8_t* out, int nchunk, int kb_per_chunk) {
+__global__ void pack_scales_kernel(const PackJob* jobs, int njobs, uint8_t* out, int nchunk, int kc_cols, int cw,
+                                   long long tile_row) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<long long>(njobs) * nchunk) return;
   const int jb = static_cast<int>(t / nchunk), c = static_cast<int>(t - static_cast<long long>(jb) * nchunk);
   const PackJob j = jobs[jb];
-  float* d = reinterpret_cast<float*>(out + j.sdst + c * j.stride);
+  const int kb_per_chunk = kc_cols / 128;
+  float* d = reinterpret_cast<float*>(out + pack_tile_offset(j, c, nchunk, cw, tile_row) +
+                                      static_cast<long long>(j.gp2) * kc_cols + j.row * (kc_cols / 32));
   for (int k = 0; k < kb_per_chunk; ++k) d[k] = j.scale[c * kb_per_chunk + k];
 }
 
-// One warp per packed row: chunk c of the row goes to dst + c*stride.
-__global__ void pack_rows_kernel(const PackJob* jobs, int njobs, uint8_t* out, int row_bytes,
-                                 int chunk_bytes) {
+// One warp per packed row: chunk c of the row goes to its tile (pack_tile_offset).
+__global__ void pack_rows_kernel(const PackJob* jobs, int njobs, uint8_t* out, int row_bytes, int chunk_bytes,
+                                 int nchunk, int cw, long long tile_row) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= njobs) return;
@@ -87,11 +103,80 @@ __global__ void pack_rows_kernel(const PackJob* jobs, int njobs, uint8_t* out, i
   const uint4* src = reinterpret_cast<const uint4*>(j.src);
   for (int v = lane; v < nvec; v += 32) {
     const int c = v / nvc, w = v - c * nvc;
-    *reinterpret_cast<uint4*>(out + j.dst + c * j.stride + static_cast<long long>(w) * 16) = src[v];
+    *reinterpret_cast<uint4*>(out + pack_tile_offset(j, c, nchunk, cw, tile_row) +
+                              static_cast<long long>(j.row) * chunk_bytes + static_cast<long long>(w) * 16) = src[v];
   }
 }
 
 long long split_host(long long c, long long n, long long G) { return (c * n) / G; }
+
+// ---- batch-8 tensor-core packing (params.h: "batch-8 tensor-core tiles")
+struct TcRowJob {
+  const uint8_t* src;   // source row (K codes or bf16 values)
+  const float* scale;   // FP8: the row's block-scale row ([K/128] fp32), else null
+  int n;                // logical row
+};
+
+static_assert(sizeof(TcRowJob) <= sizeof(PackJob), "the tensor-core packer reuses the job buffer");
+
+struct TcGeom {
+  int N, K, G, win, fp8;
+};
+
+// Byte offset of the tile holding column k of logical row n, and the row's
+// M-tile geometry (rows rv, boxes per tile nb, box j, row r, column in window kw).
+__device__ inline long long tc_tile_of(const TcGeom& g, int n, int k, int& rv, int& nb, int& j, int& r, int& kw) {
+  const int U = g.N / 8;
+  const int c = static_cast<int>(((static_cast<long long>(n / 8) + 1) * g.G - 1) / U);
+  const int u0 = static_cast<int>((static_cast<long long>(c) * U) / g.G);
+  const int u1 = static_cast<int>((static_cast<long long>(c + 1) * U) / g.G);
+  const int R = 8 * (u1 - u0);
+  const int lr = n - 8 * u0, m = lr / 128;
+  r = lr % 128;
+  rv = min(128, R - 128 * m);
+  const int bc = tc_box_cols(g.fp8);
+  nb = tc_nb(rv, tc_kbox(g.K, g.win, g.fp8), g.fp8);
+  const int w = g.win > 0 ? k / g.win : 0;
+  const int ws = w * g.win;
+  const int Kw = g.win > 0 ? min(g.win, g.K - ws) : g.K;
+  kw = k - ws;
+  const int bw = kw / bc;
+  j = bw % nb;
+  return 8LL * u0 * tc_row_bytes(g.K, g.fp8) + static_cast<long long>(w) * R * tc_row_bytes(g.win, g.fp8) +
+         128LL * m * tc_row_bytes(Kw, g.fp8) + static_cast<long long>(bw / nb) * tc_tile_bytes(rv, nb, g.fp8);
+}
+
+// One warp per row: its 16-byte units to their swizzled places.
+__global__ void pack_tc_rows_kernel(const TcRowJob* jobs, int njobs, uint8_t* out, TcGeom g) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= njobs) return;
+  const TcRowJob jb = jobs[warp];
+  const int esz = g.fp8 ? 1 : 2;
+  const int nvec = g.K * esz / 16, bc = tc_box_cols(g.fp8);
+  const uint4* src = reinterpret_cast<const uint4*>(jb.src);
+  for (int v = lane; v < nvec; v += 32) {
+    const int k = v * 16 / esz;
+    int rv, nb, j, r, kw;
+    const long long t = tc_tile_of(g, jb.n, k, rv, nb, j, r, kw);
+    const int q = ((kw % bc) * esz) / 16;
+    *reinterpret_cast<uint4*>(out + t + static_cast<long long>(j) * rv * 128 + r * 128 + ((q ^ (r & 7)) << 4)) =
+        src[v];
+  }
+}
+
+// FP8: one thread per (row, 128-column block): the block scale after the tile's boxes.
+__global__ void pack_tc_scales_kernel(const TcRowJob* jobs, int njobs, uint8_t* out, TcGeom g) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int nkb = g.K / 128;
+  if (t >= static_cast<long long>(njobs) * nkb) return;
+  const int i = static_cast<int>(t / nkb), kb = static_cast<int>(t - static_cast<long long>(i) * nkb);
+  const TcRowJob jb = jobs[i];
+  int rv, nb, j, r, kw;
+  const long long tile = tc_tile_of(g, jb.n, kb * 128, rv, nb, j, r, kw);
+  *reinterpret_cast<float*>(out + tile + static_cast<long long>(nb) * rv * 128 + (static_cast<long long>(j) * rv + r) * 4) =
+      jb.scale[kb];
+}
 
 // Largest k-chunk dividing K whose tile of 8 row pairs fits kTileBytes (FP8:
 // also a whole number of 128-column scale blocks).
@@ -134,6 +219,9 @@ struct xlpk_engine {
   int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, evb = 0;
   int side_hloc = 0, hloc = 0;
   bool ffn_fused = false;
+  bool tc = false;              // batch-8 projections on tcgen05 MMAs
+  int tc_cols = 0;
+  int down_win = 0;            // K-windowed down projection (columns per window; 0: off)
   int esz = 2;
   int P = 0;
   uint8_t* packed = nullptr;
@@ -235,13 +323,17 @@ SrcRow source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_conf
 // `split` CTAs share the rows (1: the whole matrix is one block streamed by
 // every CTA that needs it, e.g. the MoE router and expert gate/up blocks).
 xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t* dst, Mat* out,
-                        PackJob* d_jobs, size_t max_jobs, cudaStream_t st, int split) {
+                        PackJob* d_jobs, size_t max_jobs, cudaStream_t st, int split, int win_cols = 0) {
   const int esz = e->esz;
   const int KC = pick_kc(K, esz);
   if (KC == 0) return XLPK_ERR_UNSUPPORTED;
   const bool fp8 = esz == 1;
   if (fp8 && (!ms.sa || (ms.kind != MatKind::PLAIN && !ms.sb) || (ms.kind == MatKind::QKV && !ms.sc)))
     return XLPK_ERR_INVALID_ARG;
+  const int nkc = K / KC;
+  // chunks per window: the whole K unless the matrix is streamed window by window
+  const int cw = win_cols > 0 ? win_cols / KC : nkc;
+  if (cw < 1 || (win_cols > 0 && win_cols % KC)) return XLPK_ERR_UNSUPPORTED;
   // bytes per packed row over a chunk / over K (codes + FP8 block scales)
   const long long tile_row = static_cast<long long>(KC) * esz + (fp8 ? KC / 32 : 0);
   const long long full_row = static_cast<long long>(K) * esz + (fp8 ? K / 32 : 0);
@@ -254,15 +346,16 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
     for (long long lp = 0; lp < npc; ++lp) {
       const long long j = lp / kPairsPerTile, w = lp % kPairsPerTile;
       const long long gp = std::min<long long>(kPairsPerTile, npc - kPairsPerTile * j);
-      const long long group_off = (2 * p0 + 2LL * kPairsPerTile * j) * full_row;
       for (int r = 0; r < 2; ++r) {
         const SrcRow sr = source_row(ms, 2 * (p0 + lp) + r, K, esz, e->cfg);
         PackJob pj;
         pj.src = sr.w;
-        pj.dst = group_off + (2 * w + r) * static_cast<long long>(KC) * esz;
-        pj.stride = 2 * gp * tile_row;
         pj.scale = sr.s;
-        pj.sdst = group_off + 2 * gp * static_cast<long long>(KC) * esz + (2 * w + r) * (KC / 32);
+        pj.base = 2 * p0 * full_row;
+        pj.row = static_cast<int>(2 * w + r);
+        pj.j16 = static_cast<int>(2 * kPairsPerTile * j);
+        pj.gp2 = static_cast<int>(2 * gp);
+        pj.np2 = static_cast<int>(2 * npc);
         jobs.push_back(pj);
       }
     }
@@ -273,12 +366,13 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
     XLPK_CUDA(cudaMemcpyAsync(d_jobs, jobs.data() + off, n * sizeof(PackJob), cudaMemcpyHostToDevice, st));
     const int threads = 256;
     const int blocks = static_cast<int>((n * 32 + threads - 1) / threads);
-    pack_rows_kernel<<<blocks, threads, 0, st>>>(d_jobs, static_cast<int>(n), dst, row_bytes, chunk_bytes);
+    pack_rows_kernel<<<blocks, threads, 0, st>>>(d_jobs, static_cast<int>(n), dst, row_bytes, chunk_bytes, nkc, cw,
+                                                 tile_row);
     XLPK_CUDA(cudaGetLastError());
     if (fp8) {
-      const long long nt = static_cast<long long>(n) * (K / KC);
+      const long long nt = static_cast<long long>(n) * nkc;
       pack_scales_kernel<<<static_cast<int>((nt + threads - 1) / threads), threads, 0, st>>>(
-          d_jobs, static_cast<int>(n), dst, K / KC, KC / 128);
+          d_jobs, static_cast<int>(n), dst, nkc, KC, cw, tile_row);
       XLPK_CUDA(cudaGetLastError());
     }
     XLPK_CUDA(cudaStreamSynchronize(st));
@@ -288,6 +382,44 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
   out->N = N;
   out->K = K;
   out->KC = KC;
+  out->fp8 = fp8 ? 1 : 0;
+  return XLPK_OK;
+}
+
+xlpk_status pack_matrix_tc(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t* dst, Mat* out,
+                           TcRowJob* d_jobs, size_t max_jobs, cudaStream_t st, int win_cols) {
+  const int esz = e->esz;
+  const bool fp8 = esz == 1;
+  const int bc = tc_box_cols(fp8 ? 1 : 0);
+  if (N % 8 || K % bc || (win_cols > 0 && (win_cols % bc || win_cols >= K))) return XLPK_ERR_UNSUPPORTED;
+  if (fp8 && (!ms.sa || (ms.kind != MatKind::PLAIN && !ms.sb) || (ms.kind == MatKind::QKV && !ms.sc)))
+    return XLPK_ERR_INVALID_ARG;
+  std::vector<TcRowJob> jobs(static_cast<size_t>(N));
+  for (int n = 0; n < N; ++n) {
+    const SrcRow sr = source_row(ms, n, K, esz, e->cfg);
+    jobs[n] = TcRowJob{sr.w, sr.s, n};
+  }
+  const TcGeom g{N, K, e->G, win_cols, fp8 ? 1 : 0};
+  for (size_t off = 0; off < jobs.size(); off += max_jobs) {
+    const size_t n = std::min(max_jobs, jobs.size() - off);
+    XLPK_CUDA(cudaMemcpyAsync(d_jobs, jobs.data() + off, n * sizeof(TcRowJob), cudaMemcpyHostToDevice, st));
+    const int threads = 256;
+    pack_tc_rows_kernel<<<static_cast<int>((n * 32 + threads - 1) / threads), threads, 0, st>>>(
+        d_jobs, static_cast<int>(n), dst, g);
+    XLPK_CUDA(cudaGetLastError());
+    if (fp8) {
+      const long long nt = static_cast<long long>(n) * (K / 128);
+      pack_tc_scales_kernel<<<static_cast<int>((nt + threads - 1) / threads), threads, 0, st>>>(
+          d_jobs, static_cast<int>(n), dst, g);
+      XLPK_CUDA(cudaGetLastError());
+    }
+    XLPK_CUDA(cudaStreamSynchronize(st));
+  }
+  out->packed = dst;
+  out->scales = nullptr;
+  out->N = N;
+  out->K = K;
+  out->KC = bc;
   out->fp8 = fp8 ? 1 : 0;
   return XLPK_OK;
 }
@@ -453,12 +585,6 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const int group = c.n_q_heads / c.n_kv_heads;
   e->P = (kTileBytes / 2) / (d * 2);
 
-  // shared memory: ring + activation/scratch + control
-  const int S_moe = c.n_experts > 0 ? c.top_k + c.n_shared_experts : 0;
-  const int kmax = std::max(std::max(H, qd), std::max(F, S_moe * c.expert_ffn));
-  const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
-  const int norm_stage = (B + 1) * H * 4;   // normed input vector + its RMSNorm gains
-  e->act_bytes = static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
   // Fused FFN stage (gate/up and a split-K down projection in one stage): bf16
   // dense layers whose output rows fit two 8-row vectors per consumer thread
   // and whose accumulators fit the register budget (XLPK_FFN_FUSED=0 turns it off).
@@ -468,12 +594,33 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     e->ffn_fused = !off && c.n_experts == 0 && e->esz == 2 && H <= 2 * 8 * kConsumerThreads && H % 8 == 0 &&
                    B <= 2;
   }
+  // Batch 8, dense layers: every projection runs on tcgen05 MMAs (8-row units
+  // per CTA, M-tiles of <= 128 rows with kTcAccCols accumulator columns each in tensor
+  // memory; XLPK_TC=0 turns it off).
+  {
+    const char* env = std::getenv("XLPK_TC");
+    const int bc = e->esz == 1 ? 128 : 64;
+    const int nqkv = qd + 2 * kvd;
+    e->tc = !(env && env[0] == '0') && B == 8 && c.n_experts == 0 && H % bc == 0 && qd % bc == 0 &&
+            F % bc == 0 && nqkv % 8 == 0 && c.vocab % 8 == 0;
+    if (e->tc) {
+      int mt = 0;
+      for (const int n : {nqkv, H, 2 * F, c.vocab}) {
+        const int rows = 8 * ((n / 8 + e->G - 1) / e->G);
+        mt = std::max(mt, (rows + 127) / 128);
+      }
+      int cols = 32;
+      while (cols < kTcAccCols * mt) cols <<= 1;
+      if (cols > 512) e->tc = false;
+      e->tc_cols = cols;
+    }
+  }
   // epilogue side region: RoPE rows, then this CTA's rows of the residual (two
   // planes of float4) and of the embedding (bf16, 8-aligned) for the stages
   // with H output rows, then (fused FFN) the CTA's h slice
   {
     const int maxp = (H / 2 + e->G - 1) / e->G;
-    const int rows_max = 2 * maxp;
+    const int rows_max = std::max(2 * maxp, e->tc ? 8 * ((H / 8 + e->G - 1) / e->G) : 0);
     e->side_rope = 0;
     e->side_resid = static_cast<int>(align_up(static_cast<size_t>(B) * d * 4, 16));
     e->nvr = rows_max / 8 + 2;
@@ -483,7 +630,47 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     e->hloc = e->ffn_fused ? (F + e->G - 1) / e->G : 0;
     e->side_bytes = static_cast<int>(align_up(static_cast<size_t>(e->side_hloc) + sizeof(float) * B * e->hloc, 128));
   }
+  // shared memory: ring + activation/scratch + control
+  const int S_moe = c.n_experts > 0 ? c.top_k + c.n_shared_experts : 0;
+  const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
+  const int norm_stage = (B + 1) * H * 4;   // normed input vector + its RMSNorm gains
   const int max_smem = static_cast<int>(prop.sharedMemPerBlockOptin);
+  auto act_for = [&](int kmax) {
+    if (e->tc)   // the MMA's B operand: 8 sequences x kmax bf16, + one box of slack
+                 // that the N = 16 read of the last box's rows 8..15 may touch
+      return static_cast<int>(align_up(std::max(B * kmax * 2 + 1024, attn_scratch), 1024));
+    return static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
+  };
+  e->act_bytes = act_for(std::max(std::max(H, qd), std::max(F, S_moe * c.expert_ffn)));
+  // A two-stage dense FFN whose down-projection input (B x F fp32) would leave
+  // the ring fewer than 3 slots streams W_down window by window instead: the
+  // activation region then holds B x down_win floats of h at a time (windows of
+  // the largest whole number of k-chunks that fits the other stages' inputs).
+  // (XLPK_DOWN_WIN=<columns> asks for a given window where windows are possible;
+  // the tests compare windowed and whole-K down projections with it.)
+  e->down_win = 0;
+  {
+    const char* env = std::getenv("XLPK_DOWN_WIN");
+    const int forced = env ? std::atoi(env) : 0;
+    // window granule: whole k-chunks of the CUDA-core tiles, or 1024 columns
+    // (whole boxes of either weight type) for the tensor-core tiles
+    const int kc = e->tc ? 1024 : pick_kc(F, e->esz);
+    const int maxp = (H / 2 + e->G - 1) / e->G;
+    const bool possible = !e->ffn_fused && c.n_experts == 0 && B >= 2 && kc > 0 &&
+                          (e->tc || maxp <= kPairsPerTile * kMaxWinGroups);
+    int win = 0;
+    if (possible && forced > 0) {
+      if (forced % kc == 0 && forced < F) win = forced;
+    } else if (possible && F > std::max(H, qd) &&
+               (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes < 3) {
+      win = (std::max(H, qd) / kc) * kc;
+      if (win >= F) win = 0;
+    }
+    if (win > 0) {
+      e->down_win = win;
+      e->act_bytes = act_for(std::max(std::max(H, qd), win));
+    }
+  }
   e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
   e->smem = e->nslot * kSlotBytes + e->act_bytes + e->side_bytes + kMiscSmem;
@@ -609,7 +796,12 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       m.fp8 = 0;
     } else {
       e->esz = mp.role == R_ROUTER ? 2 : esz_saved;
-      rc = pack_matrix(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, d_jobs, max_jobs, st, mp.split);
+      if (e->tc && (mp.role == R_QKV || mp.role == R_O || mp.role == R_GU || mp.role == R_DOWN || mp.role == R_LM))
+        rc = pack_matrix_tc(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, reinterpret_cast<TcRowJob*>(d_jobs),
+                            max_jobs, st, mp.role == R_DOWN ? e->down_win : 0);
+      else
+        rc = pack_matrix(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, d_jobs, max_jobs, st, mp.split,
+                         mp.role == R_DOWN ? e->down_win : 0);
       e->esz = esz_saved;
     }
     if (rc != XLPK_OK) break;
@@ -744,6 +936,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.y = reinterpret_cast<float*>(e->ws + o_y);
   p.ffn_fused = e->ffn_fused ? 1 : 0;
   p.jt = kTileBytes / (H * 2);
+  p.down_win = e->down_win;
+  p.tc = e->tc ? 1 : 0;
+  p.tc_cols = e->tc_cols;
   p.side_hloc = e->side_hloc;
   p.hloc = e->hloc;
   p.route_exp = reinterpret_cast<int*>(e->ws + o_rte);

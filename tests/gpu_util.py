@@ -59,17 +59,55 @@ def check_experts(run: Run, o: OracleDecoder, s: int, b: int) -> None:
                 assert got == want, f"step {s} layer {l}: expert order {got} != oracle {want}"
 
 
-def oracle_for(m: workload.GpuModel, max_seq: Optional[int] = None) -> OracleDecoder:
+class HostWeights(dict):
+    """Host copies of the generator's weight tensors, fetched on first use.
+
+    A large model's oracle touches only what it reads (a MoE step reads the
+    router and the selected experts), so nothing else crosses to the host."""
+
+    def __init__(self, dev_weights):
+        super().__init__()
+        self._src = dev_weights
+
+    def __missing__(self, key):
+        t = self._src[key].cpu()
+        self[key] = t
+        return t
+
+    def __contains__(self, key):
+        return key in self._src
+
+
+class MemoOracle(OracleDecoder):
+    """The oracle with each matrix widened (or FP8-dequantised) by its own W()
+    once and kept in fp32, so that long replays do not redo the widening every
+    step.  The arithmetic is the oracle's: W() itself produces the cached values."""
+
+    def W(self, name: str) -> torch.Tensor:
+        memo = self.__dict__.setdefault("_memo", {})
+        t = memo.get(name)
+        if t is None:
+            t = super().W(name)
+            memo[name] = t
+            if isinstance(self.w, HostWeights):   # the fp32 copy replaces the stored bytes
+                self.w.pop(name, None)
+                self.w.pop(name + ".scale", None)
+        return t
+
+
+def oracle_for(m: workload.GpuModel, max_seq: Optional[int] = None, memo: bool = False) -> OracleDecoder:
     """An oracle at the same decode start state as the engine.
 
-    Weights are the generator's tensors copied to the host.  Prompt workloads
-    are prefilled by the oracle's own full causal recompute; synthetic-KV
-    workloads get the generator's cache contents (regenerated, not read back
-    from the engine's cache).
+    Weights are the generator's tensors, copied to the host as the oracle reads
+    them.  Prompt workloads are prefilled by the oracle's own full causal
+    recompute; synthetic-KV workloads get the generator's cache contents
+    (regenerated, not read back from the engine's cache).  `memo` keeps each
+    matrix's fp32 values after first use (long replays of large models).
     """
     cfg = m.cfg
-    w = {k: v.cpu() for k, v in m.weights.items()}
-    o = OracleDecoder(cfg, w, cfg.batch, max_seq=max_seq or m.k.shape[3])
+    w = HostWeights(m.weights)
+    cls = MemoOracle if memo else OracleDecoder
+    o = cls(cfg, w, cfg.batch, max_seq=max_seq or m.k.shape[3])
     if cfg.prefill:
         o.forward_sequence(m.prompt[:, : cfg.kv_len])
     else:

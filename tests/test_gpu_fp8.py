@@ -58,3 +58,22 @@ def test_llama8b_fp8_batch2_full_size_prefix(cuda_device):
     run = run_engine(m, 4)
     compare_with_oracle(m, run, oracle_for(m), 2, tol=REL_L2_FP8)
     assert int(run.tokens.min()) >= 0 and int(run.tokens.max()) < cfg.vocab
+
+
+@pytest.mark.parametrize("batch", [4, 8])
+def test_llama8b_fp8_large_batch_full_size_prefix(cuda_device, batch):
+    # the 8B FP8 shape at batch 4 and 8: B x 14336 fp32 down-projection inputs
+    # do not fit beside the ring, so W_down streams in K windows of 4096
+    cfg = synth.get_config("llama8b_fp8", batch=batch)
+    m = workload.build(cfg, device=cuda_device)
+    assert m.engine.info().ring_slots >= 2
+    run = run_engine(m, 3)
+    compare_with_oracle(m, run, oracle_for(m), 2, tol=REL_L2_FP8)
+
+
+def test_tiny_fp8_batch8_tensor_core(cuda_device):
+    # FP8 tiles widened to bf16 in their ring slot before the MMA
+    cfg = synth.get_config("tiny", weight_dtype="fp8_e4m3", batch=8, steps=6)
+    m = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    run = run_engine(m, cfg.steps)
+    compare_with_oracle(m, run, oracle_for(m), cfg.steps, tol=REL_L2_FP8)

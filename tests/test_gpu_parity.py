@@ -249,3 +249,52 @@ def test_llama1b_batch4_prefix(cuda_device):
     # every sequence wrote exactly positions T .. T+7 of its own cache rows
     assert bool((m.k[:, :, :, T:T + 8].float().abs().sum(-1) > 0).all())
     assert int(m.k[:, :, :, T + 8:].float().abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("batch", [2, 4])
+def test_windowed_down_projection_matches_whole_k(cuda_device, monkeypatch, batch):
+    # the down projection streamed in K windows of 1024 columns (4 windows of
+    # F = 4096) against the same model with the whole K staged at once: the
+    # per-lane sums run over the same chunks in the same order
+    monkeypatch.setenv("XLPK_FFN_FUSED", "0")
+    cfg = synth.get_config("tiny", ffn=4096, batch=batch, steps=6)
+    whole = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    monkeypatch.setenv("XLPK_DOWN_WIN", "1024")
+    win = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=whole.weights)
+    for unfused in (False, True):
+        a = run_engine(whole, cfg.steps, unfused=unfused)
+        b = run_engine(win, cfg.steps, unfused=unfused)
+        assert torch.equal(a.tokens, b.tokens)
+        assert torch.equal(a.logits, b.logits)
+    compare_with_oracle(win, b, oracle_for(win), cfg.steps)
+
+
+@pytest.mark.parametrize("unfused", [False, True], ids=["persistent", "kernel_per_op"])
+def test_batch8_tensor_core_path_matches_oracle(cuda_device, unfused):
+    # batch 8 runs every projection on tcgen05 MMAs (bf16 activations as the B
+    # operand, fp32 accumulators in tensor memory)
+    cfg = synth.get_config("tiny", batch=8, steps=6)
+    m = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    run = run_engine(m, cfg.steps, unfused=unfused)
+    compare_with_oracle(m, run, oracle_for(m), cfg.steps)
+
+
+def test_batch8_tensor_core_windowed_down_matches_whole_k(cuda_device, monkeypatch):
+    # the tensor-core down projection over K windows of 1024 columns keeps
+    # accumulating in the same tensor-memory columns: identical results
+    cfg = synth.get_config("tiny", ffn=4096, batch=8, steps=4)
+    whole = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    monkeypatch.setenv("XLPK_DOWN_WIN", "1024")
+    win = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=whole.weights)
+    a = run_engine(whole, cfg.steps)
+    b = run_engine(win, cfg.steps)
+    assert torch.equal(a.tokens, b.tokens)
+    assert torch.equal(a.logits, b.logits)
+    compare_with_oracle(win, b, oracle_for(win), cfg.steps)
+
+
+def test_llama1b_batch8_tensor_core_prefix(cuda_device):
+    cfg = synth.get_config("llama1b", batch=8, kv_len=32, steps=4)
+    m = workload.build(cfg, device=cuda_device)
+    run = run_engine(m, cfg.steps)
+    compare_with_oracle(m, run, oracle_for(m), 2)
