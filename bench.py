@@ -39,6 +39,7 @@ def parse():
     ap.add_argument("--impl", default="xlpk", choices=["xlpk", "reference"])
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--decode-steps", type=int, default=0, help="override tokens per call (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (sequences per call)")
     ap.add_argument("--no-baselines", action="store_true", help="skip the unfused and CPU legs")
     return ap.parse_args()
 
@@ -217,6 +218,18 @@ def run_reference(args):
     return 0
 
 
+def dtype_label(cfg) -> str:
+    """The arithmetic the decode runs in: weights as stored, fp32 accumulation."""
+    if cfg.weight_dtype == "fp8_e4m3":
+        w = "fp8_e4m3 weights (fp32 scale per 128x128 block)"
+    else:
+        w = "bf16 weights"
+    act = "fp32 activations"
+    if cfg.batch == 8 and not cfg.is_moe:
+        act = "activations as bf16 high + low parts into tcgen05 MMAs, fp32 accumulation"
+    return f"{w}, bf16 KV, {act}"
+
+
 def workload_config(cfg, n):
     return {"workload": f"{cfg.name}: {cfg.n_layers} layers, hidden {cfg.hidden}, {cfg.n_q_heads}q/"
                         f"{cfg.n_kv_heads}kv heads x {cfg.head_dim}, ffn {cfg.ffn}, vocab {cfg.vocab}, "
@@ -248,6 +261,8 @@ def main():
     cfg = synth.get_config(args.workload)
     if args.decode_steps:
         cfg = cfg.with_(steps=args.decode_steps)
+    if args.batch:
+        cfg = cfg.with_(batch=args.batch)
     n = cfg.steps
     B = cfg.batch
 
@@ -369,7 +384,7 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype_label(cfg), "data": "synthetic",
             "config": workload_config(cfg, world),
             "tpot_ms": round(tpot_ms, 4), "tok_s_per_user": round(1e3 / tpot_ms, 2),
             "roofline": roof,

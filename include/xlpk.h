@@ -14,7 +14,9 @@
  * the execution stays resident for the whole decode lifecycle).  The
  * kernel-per-op baseline the pages compare against (launch, load, compute,
  * store, synchronise per operator; "Persistent execution paradigm", section 1)
- * is xlpk_decode_unfused, built from the same tiles.
+ * is xlpk_decode_unfused, built from the same tiles.  The batch-8 decode runs
+ * its projections on the tcgen05 tensor cores (xlpk_tc_gemm_tile is the same
+ * contraction as a stand-alone call).
  *
  * Conventions for every entry point:
  *  - Pointers named *_dev are CUDA device pointers on the handle's device;
@@ -79,7 +81,21 @@ typedef struct xlpk_config {
   float rms_eps;               /* RMSNorm epsilon */
   int32_t n_ctas;              /* persistent grid size; 0 = one CTA per SM */
   int32_t spin_limit_us;       /* limit of every device-side wait; 0 = 200000 us */
+  int32_t flags;               /* XLPK_FLAG_* bits; 0 = the planner's defaults */
+  int32_t window;              /* K window (columns) of the windowed projections: the down projection at
+                                  batch >= 2 on CUDA cores (a multiple of its k-chunk) or every
+                                  tensor-core projection at batch 8 (a multiple of 1024); 0 = chosen by
+                                  the planner.  A value the planner cannot use is ignored on CUDA cores
+                                  and refused (XLPK_ERR_UNSUPPORTED) on tensor cores. */
 } xlpk_config;
+
+/* xlpk_config::flags.  The defaults are the fast paths; the flags select the
+ * alternatives they replace (both compute the same decode). */
+enum {
+  XLPK_FLAG_NO_FUSED_FFN = 1,      /* bf16 dense layers at batch <= 2: gate/up and down as two stages
+                                      instead of one fused stage with a split-K down projection */
+  XLPK_FLAG_NO_TENSOR_CORES = 2    /* batch 8: CUDA-core GEMV tiles instead of tcgen05 MMAs */
+};
 
 /* One linear weight: y = W x with W row-major [N][K] (PyTorch Linear layout).
  * `scale` is NULL for bf16; for FP8 it is fp32 [N/128][K/128], row-major. */
@@ -137,6 +153,10 @@ typedef struct xlpk_decode_io {
                                          combine), [8] q loads, [9] chunk math, [10] merge,
                                          [11] arrive, [12] combine, [13] chunks processed.
                                          n_stages = 5 * n_layers + 1 */
+  int32_t withhold_release;           /* failure-detection testing only: 1 + the index (layer * 5 +
+                                         stage kind, n_layers * 5 = LM head) of a stage whose
+                                         completion CTA 0 does not announce at the call's first
+                                         step, so the waits behind it run out; 0 = off */
 } xlpk_decode_io;
 
 /* Facts about a created handle (for measurement and tests). */
@@ -160,23 +180,44 @@ typedef struct xlpk_engine* xlpk_handle;
  * cache is written in place).  Weight buffers may be freed afterwards.
  * Runs on the current device and synchronises it first, so weights still
  * being written by work enqueued on any stream are complete before they are
- * packed. */
+ * packed.  Returns XLPK_ERR_INVALID_ARG for a bad shape or pointer (NULL,
+ * unaligned) and XLPK_ERR_UNSUPPORTED for a shape this build does not handle,
+ * before any device work; *out is NULL on every error.
+ * Source: the decode graph is compiled ahead of time into one resident engine
+ * whose tile shapes, placement and buffers are fixed before the first token
+ * ("Ultra-High Interactivity On NVIDIA GPUs? - TileRT InferenceX", digest,
+ * core views and the AoT static-compilation concept; the fixed temporary-
+ * tensor table of "Persistent execution paradigm", section 5.3). */
 xlpk_status xlpk_create(const xlpk_config* cfg, const xlpk_weights* weights,
                         const xlpk_kv* kv, xlpk_handle* out);
 
-/* Free everything the handle owns (not the caller's KV or weights). */
+/* Free everything the handle owns (not the caller's KV or weights).  Waits
+ * for the device first.  (The pages are silent; resource release of the
+ * handle above.) */
 xlpk_status xlpk_destroy(xlpk_handle h);
 
 /* Set the decode state: sequence b has seq_lens_host[b] positions already in
- * the KV cache and pending input token tokens_host[b].  Enqueued on `stream`. */
+ * the KV cache and pending input token tokens_host[b] (both host arrays of B
+ * entries, read during the call).  The tokens are copied to the device on
+ * `stream`.  XLPK_ERR_INVALID_ARG for a token outside [0, vocab) or a length
+ * outside [0, max_seq).  Host arrays let every value be checked before
+ * anything is enqueued.
+ * Source: the request's cache state at the start of decode ("XL-Persistent-
+ * Kernel", request lifecycle: the decode worker takes over the prefilled KV
+ * pages). */
 xlpk_status xlpk_set_state(xlpk_handle h, const int32_t* tokens_host,
                            const int32_t* seq_lens_host, void* stream);
 
 /* Greedy-decode n_steps tokens per sequence as ONE persistent kernel launch.
  * tokens_out_dev [n_steps][B] receives the argmax of every step.  Step s feeds
  * the pending token at position seq_len + s, appends K/V there, and makes
- * the argmax (or forced_tokens[s][b]) the next pending token.  Asynchronous
- * on `stream`; XLPK_ERR_KV_FULL if seq_len + n_steps > max_seq. */
+ * the argmax (or forced_tokens[s][b]) the next pending token.  `io` may be
+ * NULL.  Asynchronous on `stream`; XLPK_ERR_KV_FULL if seq_len + n_steps >
+ * max_seq; device-side failures are reported by xlpk_get_status.
+ * Source: the host launches the engine once and execution stays resident on
+ * the GPU for the whole decode ("Ultra-High Interactivity On NVIDIA GPUs? -
+ * TileRT InferenceX", digest, core views; "TileRT speed notes", Persistent
+ * Execution / Tile-Level Pipeline). */
 xlpk_status xlpk_decode(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                         const xlpk_decode_io* io, void* stream);
 
@@ -187,7 +228,11 @@ xlpk_status xlpk_decode(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
  * counters on `stream` (an async memset) and calls nothing that synchronises,
  * so its launches may be recorded by stream capture into a CUDA graph and
  * replayed; a replay decodes the captured positions again, from the tokens the
- * device holds. */
+ * device holds.  Errors as xlpk_decode.
+ * Source: the launch -> load -> compute -> store -> synchronise cycle per
+ * operator that persistent execution removes ("Persistent execution
+ * paradigm", section 1; "Ultra-High Interactivity On NVIDIA GPUs? - TileRT
+ * InferenceX", digest, section "GPU bottleneck is latency, not bandwidth"). */
 xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                                 const xlpk_decode_io* io, void* stream);
 
@@ -202,9 +247,10 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
  * compiled into the library: XLPK_NOALLOC_SCRATCH_BYTES bytes of file-scope
  * __device__ memory that every GPU which loads the library holds until the
  * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - The array's device address is looked up (cudaGetSymbolAddress) with the
+ *    device current at the first call on each device, and again if the
+ *    device's context has been replaced since (after cudaDeviceReset); make
+ *    the first call on a device before any stream capture.
  *  - Returns XLPK_ERR_UNSUPPORTED (with a message in xlpk_last_cuda_error) if
  *    the handle's scratch would exceed the array.
  *  - The counters in the array are cleared on `stream` at the start of each
@@ -216,21 +262,40 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
 xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                                 const xlpk_decode_io* io, void* stream);
 
+/* Parity mode: register device buffers logits_dev (fp32 [B][V]) and
+ * hidden_dev (fp32 [B][H], the residual after the last layer) into which every
+ * later decode call on the handle (xlpk_decode, xlpk_decode_unfused,
+ * xlpk_decode_noalloc) writes each step's values, one step over the other, so
+ * that after a call they hold its last step's.  A call whose `io` names its own
+ * logits or hidden buffer writes those instead.  Either pointer may be NULL;
+ * NULL, NULL turns parity mode off.  The buffers are borrowed until then; they
+ * must be 16-byte aligned (else XLPK_ERR_INVALID_ARG).
+ * Source: the oracle comparison of logits and hidden states that the decode is
+ * checked by (the pages are silent; a debug output of the boundary). */
+xlpk_status xlpk_debug_logits(xlpk_handle h, float* logits_dev, float* hidden_dev);
+
 /* End-to-end call with host buffers: uploads the state, decodes, downloads
  * tokens_out_host [n_steps][B], and synchronises `stream`.  Returns the
- * device status of the decode. */
+ * device status of the decode.
+ * Source: a request submitted with its prompt state and answered with its
+ * tokens ("XL-Persistent-Kernel", request lifecycle, steps 1 and 8). */
 xlpk_status xlpk_generate(xlpk_handle h, const int32_t* tokens_host, const int32_t* seq_lens_host,
                           int32_t n_steps, int32_t* tokens_out_host, void* stream);
 
 /* Synchronise the stream of the handle's last decode and return its device
  * status (XLPK_OK, XLPK_ERR_TIMEOUT or XLPK_ERR_ABORTED).  After an error the
  * handle's counters are reset; KV entries the failed call would have written
- * are unspecified. */
+ * are unspecified.
+ * Source: a persistent kernel has no per-operator failure boundary, so every
+ * device-side wait is bounded and reported ("Persistent execution paradigm",
+ * section 7.3, execution stability at the hardware's limits). */
 xlpk_status xlpk_get_status(xlpk_handle h);
 
+/* Facts about a created handle (grid, shared memory, ring, packed bytes).
+ * (The pages are silent; measurement support.) */
 xlpk_status xlpk_get_info(xlpk_handle h, xlpk_info* out);
 
-/* Human-readable name of a status. */
+/* Human-readable name of a status; "XLPK_ERR_UNKNOWN" for other values. */
 const char* xlpk_status_string(int32_t status);
 
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
@@ -238,10 +303,9 @@ const char* xlpk_last_cuda_error(void);
 
 /* One batch-8 projection on the tcgen05 tensor cores:
  *     y[n][b] = sum_k w[n][k] * bf16(x[b][k]),   n < N, b < 8,
- * i.e. the decoder's linear layers (QKV, O, gate/up, down, LM head of the
- * decode step above) for 8 sequences at once, where the GEMV becomes a dense
- * [N x K] . [K x 8] contraction.  It is the tensor-core tile the batch-8
- * decode is built from; xlpk_decode does not call it yet.
+ * the dense [N x K] . [K x 8] contraction that the decoder's linear layers
+ * become for 8 sequences at once, as a stand-alone call (the batch-8 decode
+ * runs the same MMAs inside the persistent kernel).
  *  - w_dev: bf16 [N][K] row-major; x_dev: fp32 [8][K] row-major (rounded to
  *    bf16, round-to-nearest-even, as it enters the MMA); y_dev: fp32 [N][8]
  *    row-major, written.  All three 16-byte aligned, on the current device;
@@ -251,7 +315,10 @@ const char* xlpk_last_cuda_error(void);
  *  - Runs on `stream` and waits for it: returns XLPK_OK, XLPK_ERR_UNSUPPORTED
  *    on a device that is not sm_100, XLPK_ERR_CUDA, or XLPK_ERR_TIMEOUT if a
  *    device-side wait ran out (the kernel then leaves without writing y).
- *    One call at a time per process (the device-side error word is shared). */
+ *    One call at a time per process (the device-side error word is shared).
+ * Source: tensor-core warp groups for the dense parts of the engine ("TileRT
+ * speed notes", Warp / Block Specialization; "Persistent execution paradigm",
+ * section 6.2, warp specialisation). */
 xlpk_status xlpk_tc_gemm_tile(const void* w_dev, int32_t n, int32_t k, const float* x_dev, float* y_dev,
                               void* stream);
 

@@ -21,13 +21,17 @@ XLPK_NOALLOC_SCRATCH_BYTES = 8 << 20
 XLPK_DTYPE_BF16 = 0
 XLPK_DTYPE_FP8_E4M3 = 1
 
+XLPK_FLAG_NO_FUSED_FFN = 1
+XLPK_FLAG_NO_TENSOR_CORES = 2
+
 
 class xlpk_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
         "n_experts", "top_k", "n_shared_experts", "expert_ffn", "weight_dtype", "batch",
         "max_seq")] + [("rope_theta", C.c_float), ("rms_eps", C.c_float),
-                       ("n_ctas", C.c_int32), ("spin_limit_us", C.c_int32)]
+                       ("n_ctas", C.c_int32), ("spin_limit_us", C.c_int32), ("flags", C.c_int32),
+                       ("window", C.c_int32)]
 
 
 class xlpk_linear(C.Structure):
@@ -54,7 +58,8 @@ class xlpk_kv(C.Structure):
 
 class xlpk_decode_io(C.Structure):
     _fields_ = [("forced_tokens_dev", C.c_void_p), ("logits_dev", C.c_void_p),
-                ("hidden_dev", C.c_void_p), ("experts_dev", C.c_void_p), ("trace_dev", C.c_void_p)]
+                ("hidden_dev", C.c_void_p), ("experts_dev", C.c_void_p), ("trace_dev", C.c_void_p),
+                ("withhold_release", C.c_int32)]
 
 
 class xlpk_info(C.Structure):
@@ -75,6 +80,7 @@ SIGNATURES = {
                                         C.POINTER(xlpk_decode_io), C.c_void_p]),
     "xlpk_decode_noalloc": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p,
                                         C.POINTER(xlpk_decode_io), C.c_void_p]),
+    "xlpk_debug_logits": (C.c_int32, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "xlpk_generate": (C.c_int32, [C.c_void_p, C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.c_int32,
                                   C.POINTER(C.c_int32), C.c_void_p]),
     "xlpk_get_status": (C.c_int32, [C.c_void_p]),

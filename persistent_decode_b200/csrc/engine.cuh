@@ -475,13 +475,27 @@ __host__ __device__ __forceinline__ size_t plane_index(int b, int k, int B, int 
   return ((static_cast<size_t>((k >> 2) & 1) * B + b) * (K >> 3) + (k >> 3)) * 4 + (k & 3);
 }
 
-enum ActSrc : int { SRC_RESID = 0, SRC_EMBED = 1, SRC_PLAIN = 2 };
+// Input vector sources: the residual (two-plane fp32), the pending tokens'
+// embedding rows, a plain two-plane vector without RMSNorm (o, h), or the
+// fused-FFN layers' residual accumulator (64-bit fixed point, below).
+enum ActSrc : int { SRC_RESID = 0, SRC_EMBED = 1, SRC_PLAIN = 2, SRC_FIXED = 3 };
+
+// The residual of the layers whose FFN runs as one fused stage lives in a
+// 64-bit fixed-point accumulator with 32 fractional bits: the split-K partial
+// sums of the down projection are added with integer atomics, and integer
+// addition does not depend on the order in which the CTAs arrive, so every run
+// gives the same bits (float atomics would not).  The range is +-2^31, the
+// resolution 2^-32; conversions round to nearest.
+__device__ __forceinline__ long long to_fixed(float v) { return __float2ll_rn(v * 4294967296.0f); }
+__device__ __forceinline__ float from_fixed(long long q) { return __ll2float_rn(q) * 2.3283064365386963e-10f; }
 
 // What the stage's epilogue reads besides its GEMV sums, staged in the CTA's
 // side region by the same bulk-copy phase as the input vector, so that no
 // epilogue waits on a global load of its own:
 //   SIDE_ROPE   cos/sin of this step's position per sequence (QKV)
-//   SIDE_RESID  this CTA's rows of the residual x (O-projection, down)
+//   SIDE_RESID  this CTA's rows of the residual x (O-projection, down): two
+//               planes of float4, or for the fused-FFN layers rows of the
+//               fixed-point accumulator [B][rows_side] int64
 //   SIDE_EMBED  this CTA's rows of the pending tokens' embeddings (layer-0 O-projection)
 enum SideKind : int { SIDE_NONE = 0, SIDE_ROPE = 1, SIDE_RESID = 2, SIDE_EMBED = 3 };
 
@@ -500,6 +514,12 @@ __device__ __forceinline__ void resid_rows(const Params& p, int c, int& r0, int&
   r1 = 2 * split_point(c + 1, p.H >> 1, p.G);
 }
 
+// The residual as the next layer's QKV stage and the LM head read it: the
+// fixed-point accumulator in the fused-FFN layers, else the two-plane x.
+__device__ __forceinline__ const void* resid_src(const Params& p) {
+  return p.ffn_fused ? static_cast<const void*>(p.xacc) : static_cast<const void*>(p.x);
+}
+
 // Stage the input vector and the epilogue's side data in shared memory.  A
 // residual / plain source (two-plane layout in global memory, written by other
 // CTAs in an earlier stage), the RMSNorm gains and the side data arrive by
@@ -509,10 +529,17 @@ __device__ __forceinline__ void resid_rows(const Params& p, int c, int& r0, int&
 // of squares; rn[b] = rsqrt(mean(v^2) + eps) is applied to the GEMV sums
 // (W (g v) r = W (r g v)), so the stage needs a single consumer barrier.
 // `hidden_dbg` (LM stage, CTA 0) receives the raw residual in natural [B][K] order.
+//
+// SRC_FIXED (the fused-FFN layers' residual accumulator) is read by all
+// consumer threads straight into registers (B*4096 values per pass, one round
+// trip), converted, scaled by the gains (read alongside) and written in the
+// two-plane layout; the side data still comes by bulk copy meanwhile.
 template <int B>
-__device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const float* gsrc,
+__device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const void* gsrc_v,
                                       const float* gain, float* hidden_dbg, int side, int s,
                                       float (&rn)[B], int where) {
+  const float* gsrc = static_cast<const float*>(gsrc_v);
+  const bool direct = src == SRC_FIXED;
   const int nvK = K >> 3;
   const int n4 = K >> 2;
   float4* act4 = reinterpret_cast<float4*>(cx.act);
@@ -531,22 +558,29 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
       for (int b = 0; b < B; ++b) tok[b] = __ldcg(p.cur_tok + b);
     // total bytes of this phase
     uint32_t total = 0;
-    if (src != SRC_EMBED) total += static_cast<uint32_t>(B) * K * 4u;
-    if (gain) total += static_cast<uint32_t>(K) * 4u;
+    if (src != SRC_EMBED && !direct) total += static_cast<uint32_t>(B) * K * 4u;
+    if (gain && !direct) total += static_cast<uint32_t>(K) * 4u;
     const uint32_t rope_bytes = static_cast<uint32_t>(p.d) * 4u;   // d/2 (cos, sin) pairs
     const int v0 = r0 >> 3, nv = r1 > r0 ? ((r1 - 1) >> 3) - v0 + 1 : 0;
     const int e0 = r0 & ~7, e1 = (r1 + 7) & ~7;
     if (side == SIDE_ROPE) total += B * rope_bytes;
-    if (side == SIDE_RESID) total += static_cast<uint32_t>(B) * 2u * nv * 16u;
+    if (side == SIDE_RESID)
+      total += p.ffn_fused ? static_cast<uint32_t>(B) * (r1 - r0) * 8u : static_cast<uint32_t>(B) * 2u * nv * 16u;
     if (side == SIDE_EMBED && r1 > r0) total += static_cast<uint32_t>(B) * (e1 - e0) * 2u;
     mbar_expect_tx(bar, total);
-    if (src != SRC_EMBED) bulk_g2s_nohint(smem_addr(cx.act), gsrc, static_cast<uint32_t>(B) * K * 4u, bar);
-    if (gain) bulk_g2s_nohint(gain_s, gain, static_cast<uint32_t>(K) * 4u, bar);
+    if (src != SRC_EMBED && !direct)
+      bulk_g2s_nohint(smem_addr(cx.act), gsrc, static_cast<uint32_t>(B) * K * 4u, bar);
+    if (gain && !direct) bulk_g2s_nohint(gain_s, gain, static_cast<uint32_t>(K) * 4u, bar);
     if (side == SIDE_ROPE) {
 #pragma unroll
       for (int b = 0; b < B; ++b)
         bulk_g2s_nohint(side_s + p.side_rope + b * rope_bytes,
                         p.rope + static_cast<size_t>(p.pos0[b] + s) * (p.d >> 1), rope_bytes, bar);
+    } else if (side == SIDE_RESID && p.ffn_fused && r1 > r0) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        bulk_g2s_nohint(side_s + p.side_resid + b * p.rows_side * 8, p.xacc + static_cast<size_t>(b) * p.H + r0,
+                        static_cast<uint32_t>(r1 - r0) * 8u, bar);
     } else if (side == SIDE_RESID && nv > 0) {
 #pragma unroll
       for (int b = 0; b < B; ++b)
@@ -561,6 +595,72 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
                         p.embed + static_cast<size_t>(tok[b]) * p.H + e0,
                         static_cast<uint32_t>(e1 - e0) * 2u, bar);
     }
+  }
+  if constexpr (B <= 2) {   // the fused FFN (and so SRC_FIXED) exists for batch <= 2 only
+  if (direct) {
+    constexpr int UF = 4 * B;   // groups of 4 per thread and pass: one pass for B*K <= 4096*B
+    const long long* xs = static_cast<const long long*>(gsrc_v);
+    const float4* g4p = reinterpret_cast<const float4*>(gain);
+    float ss[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) ss[b] = 0.f;
+    const int nit = B * n4;   // groups of 4 consecutive elements
+    for (int i0 = cx.tid; i0 < nit; i0 += UF * kConsumerThreads) {
+      longlong2 lo[UF], hi[UF];
+      float4 g[UF];
+#pragma unroll
+      for (int u = 0; u < UF; ++u) {
+        const int i = i0 + u * kConsumerThreads;
+        if (i < nit) {
+          const int b = i / n4, q = i - b * n4;
+          const longlong2* a = reinterpret_cast<const longlong2*>(xs + static_cast<size_t>(b) * K + 4 * q);
+          lo[u] = __ldcg(a);
+          hi[u] = __ldcg(a + 1);
+          g[u] = gain ? __ldg(g4p + q) : make_float4(1.f, 1.f, 1.f, 1.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UF; ++u) {
+        const int i = i0 + u * kConsumerThreads;
+        if (i < nit) {
+          const int b = i / n4, q = i - b * n4;
+          const float4 v = make_float4(from_fixed(lo[u].x), from_fixed(lo[u].y), from_fixed(hi[u].x),
+                                       from_fixed(hi[u].y));
+          if (hidden_dbg) *reinterpret_cast<float4*>(hidden_dbg + static_cast<size_t>(b) * K + 4 * q) = v;
+          const float sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
+#pragma unroll
+          for (int bb = 0; bb < B; ++bb)
+            if (bb == b) ss[bb] += sq;
+          act4[((q & 1) * B + b) * nvK + (q >> 1)] =
+              make_float4(v.x * g[u].x, v.y * g[u].y, v.z * g[u].z, v.w * g[u].w);
+        }
+      }
+    }
+    // the side data (RoPE rows)
+    if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
+    if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
+    cx.act_phase ^= 1u;
+#pragma unroll
+    for (int b = 0; b < B; ++b) rn[b] = 1.f;
+    if (gain) {
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float t = warp_sum(ss[b]);
+        if (cx.lane == 0) cx.ctl->red[cx.warp][b] = t;
+      }
+      consumer_sync();
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) t += cx.ctl->red[w][b];
+        rn[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
+      }
+    } else {
+      consumer_sync();
+    }
+    return;
+  }
   }
   if (src == SRC_EMBED) {
     int tok[B];
@@ -905,18 +1005,19 @@ __device__ __noinline__ void load_side(const Params& p, Ctx& cx, int side, int s
 }
 
 // Stage columns [k0, k0 + Kw) of the 8 sequences' input as the MMA's B
-// operand: bf16 boxes of [8 rows][64 columns] in the 128-byte-swizzle K-major
-// layout, box jb at act + jb * 1024.  The source is the two-plane fp32 layout
-// (or, SRC_EMBED, the pending tokens' bf16 embedding rows); with `gain` the
-// values are multiplied by it and the rows' RMSNorm factors returned in rn
-// (K = Kw = the whole input then).  `hidden_dbg` receives the raw input.
+// operand: boxes of [16 rows][64 columns] bf16 in the 128-byte-swizzle K-major
+// layout, box jb at act + jb * 2048.  Row b (< 8) holds bf16(v) of sequence b
+// and row 8 + b the rest, bf16(v - bf16(v)), so one M = 128, N = 16 MMA forms
+// both partial products and their sum (accumulator columns b and 8 + b) carries
+// about 16 significant bits of each input value instead of 8.  The source is
+// the two-plane fp32 layout (or, SRC_EMBED, the pending tokens' bf16 embedding
+// rows); with `gain` the values are multiplied by it and each thread's sums of
+// squares of the raw values are added to ss (the RMSNorm factor is formed once
+// every window has been staged).  `hidden_dbg` receives the raw input.
 __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src, const float* gsrc, int K, int k0,
-                                            int Kw, const float* gain, float* hidden_dbg, float (&rn)[kMaxBatch]) {
+                                            int Kw, const float* gain, float* hidden_dbg, float (&ss)[kMaxBatch]) {
   constexpr int B = kMaxBatch;
   const uint32_t act_s = smem_addr(cx.act);
-  float ss[B];
-#pragma unroll
-  for (int b = 0; b < B; ++b) ss[b] = 0.f;
   const int nv = Kw >> 3;   // 8-column vectors of the window
   int tok[B];
 #pragma unroll
@@ -959,32 +1060,21 @@ __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src
 #pragma unroll
       for (int t = 0; t < 8; ++t) acc = fmaf(e[t], e[t], acc);
       ss[b] += acc;
-      const uint32_t dst = act_s + jb * 1024 + b * 128 + ((q ^ b) << 4);
-      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pack_bf16x2(e[0] * g0.x, e[1] * g0.y)),
-                   "r"(pack_bf16x2(e[2] * g0.z, e[3] * g0.w)), "r"(pack_bf16x2(e[4] * g1.x, e[5] * g1.y)),
-                   "r"(pack_bf16x2(e[6] * g1.z, e[7] * g1.w))
+      const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      uint32_t h2[4], l2[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) split_bf16x2(e[2 * t] * gv[2 * t], e[2 * t + 1] * gv[2 * t + 1], h2[t], l2[t]);
+      const uint32_t dst = act_s + jb * 2048 + b * 128 + ((q ^ b) << 4);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(h2[0]), "r"(h2[1]), "r"(h2[2]),
+                   "r"(h2[3])
+                   : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 1024), "r"(l2[0]), "r"(l2[1]), "r"(l2[2]),
+                   "r"(l2[3])
                    : "memory");
     }
   }
   // the MMAs read the operand through the async proxy
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-#pragma unroll
-  for (int b = 0; b < B; ++b) rn[b] = 1.f;
-  if (gain) {
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      const float t = warp_sum(ss[b]);
-      if (cx.lane == 0) cx.ctl->red[cx.warp][b] = t;
-    }
-    consumer_sync();
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) t += cx.ctl->red[w][b];
-      rn[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
-    }
-  }
   consumer_sync();
 }
 
@@ -1043,25 +1133,29 @@ __device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t n) {
 
 // One batch-8 projection on the tensor cores: the CTA's 8-row units of `m`
 // (M-tiles of <= 128 rows, each with kTcAccCols accumulator columns in tensor
-// memory, of which columns 0..7 are the 8 sequences),
-// the input staged as the B operand window by window (`win` columns; 0: the
-// whole K), one issuing thread (consumer warp 4, lane 0) driving the MMAs and
-// releasing each ring slot with tcgen05.commit, then warps 0..3 reading their
-// accumulator rows back and running `epi` on each row pair with rn applied.
+// memory: columns b and 8 + b hold sequence b's high and low parts), the input
+// staged as the B operand window by window (tc_window: K windows of
+// Params::tc_win columns when K is larger, else the whole K), one issuing
+// thread (consumer warp 4, lane 0) driving the MMAs and releasing each ring
+// slot with tcgen05.commit, then warps 0..3 reading their accumulator rows back
+// and running `epi` on each row pair with the RMSNorm factor rn applied.
 template <class Epi>
 __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where, ActSrc src,
-                                        const float* gsrc, const float* gain, float* hidden_dbg, int win, Epi& epi) {
+                                        const float* gsrc, const float* gain, float* hidden_dbg, Epi& epi) {
   constexpr int B = kMaxBatch;
   const int fp8 = m.fp8;
   const int U = m.N >> 3;
   const int u0 = split_point(cx.c, U, p.G), u1 = split_point(cx.c + 1, U, p.G);
   const int R = 8 * (u1 - u0), nm = (R + 127) >> 7;
-  const int K = m.K, bc = tc_box_cols(fp8), kbox = tc_kbox(K, win, fp8);
+  const int K = m.K, win = tc_window(p.tc_win, K);
+  const int bc = tc_box_cols(fp8), kbox = tc_kbox(K, win, fp8);
   const int nw = win > 0 ? (K + win - 1) / win : 1;
   const bool issuer = cx.warp == 4 && cx.lane == 0;
   const uint32_t idesc = tc_idesc_bf16(128, kTcAccCols);
   const uint32_t tmem = cx.ctl->tmem_base;
-  float rn[B];
+  float ss[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) ss[b] = 0.f;
   for (int w = 0; w < nw; ++w) {
     const int k0 = w * win, Kw = win > 0 ? min(win, K - k0) : K;
     if (w > 0) {
@@ -1069,11 +1163,7 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
       if (!cx.ctl->abort) ring_wait(p, cx.ctl, smem_addr(&cx.ctl->bop_bar), cx.bop_phase, where);
       cx.bop_phase ^= 1u;
     }
-    float rw[B];
-    tc_stage_input(p, cx, src, gsrc, K, k0, Kw, w == 0 ? gain : nullptr, w == 0 ? hidden_dbg : nullptr, rw);
-    if (w == 0)
-#pragma unroll
-      for (int b = 0; b < B; ++b) rn[b] = rw[b];
+    tc_stage_input(p, cx, src, gsrc, K, k0, Kw, gain, hidden_dbg, ss);
     if (issuer) tc_fence_after();
     for (int mt = 0; mt < nm; ++mt) {
       const int rv = min(128, R - 128 * mt);
@@ -1100,7 +1190,7 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               tc_mma(tmem + mt * kTcAccCols, tc_desc_sw128(slot_s + j * rv * 128 + ks * 32),
-                     tc_desc_sw128(smem_addr(cx.act) + (bx0 + j) * 1024 + ks * 32), idesc,
+                     tc_desc_sw128(smem_addr(cx.act) + (bx0 + j) * 2048 + ks * 32), idesc,
                      (w | t | j | ks) != 0 ? 1u : 0u);
           mbar_arrive_n(eb, kConsumerWarps - 1);
           tc_commit(eb);                                 // the slot is free once these MMAs have read it
@@ -1109,6 +1199,25 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
       }
     }
     if (issuer && !cx.ctl->abort) tc_commit(smem_addr(w + 1 < nw ? &cx.ctl->bop_bar : &cx.ctl->acc_bar));
+  }
+  // the RMSNorm factor over the whole input, while the last MMAs run
+  float rn[B];
+#pragma unroll
+  for (int b = 0; b < B; ++b) rn[b] = 1.f;
+  if (gain) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const float t = warp_sum(ss[b]);
+      if (cx.lane == 0) cx.ctl->red[cx.warp][b] = t;
+    }
+    consumer_sync();
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) t += cx.ctl->red[w][b];
+      rn[b] = rsqrtf(t / static_cast<float>(K) + p.eps);
+    }
   }
   // accumulators -> epilogue, one row pair at a time
   if (!cx.ctl->abort) ring_wait(p, cx.ctl, smem_addr(&cx.ctl->acc_bar), cx.acc_phase, where);
@@ -1119,15 +1228,18 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
     for (int mt = 0; mt < nm; ++mt) {
       const int rv = min(128, R - 128 * mt);
       if (cx.warp * 32 >= rv) continue;               // warp-uniform
-      uint32_t v[8];
-      tc_ld8(tmem + (static_cast<uint32_t>(cx.warp * 32) << 16) + mt * kTcAccCols, v);
+      uint32_t v[16];
+      tc_ld16(tmem + (static_cast<uint32_t>(cx.warp * 32) << 16) + mt * kTcAccCols, v);
+      float row[B];   // this lane's accumulator row: high + low part of each sequence
+#pragma unroll
+      for (int b = 0; b < B; ++b) row[b] = __uint_as_float(v[b]) + __uint_as_float(v[8 + b]);
       for (int i = 0; i < 16; ++i) {
         if (cx.warp * 32 + 2 * i >= rv) break;         // warp-uniform
         float a0[B], a1[B];
 #pragma unroll
         for (int b = 0; b < B; ++b) {
-          a0[b] = __uint_as_float(__shfl_sync(0xffffffffu, v[b], 2 * i)) * rn[b];
-          a1[b] = __uint_as_float(__shfl_sync(0xffffffffu, v[b], 2 * i + 1)) * rn[b];
+          a0[b] = __shfl_sync(0xffffffffu, row[b], 2 * i) * rn[b];
+          a1[b] = __shfl_sync(0xffffffffu, row[b], 2 * i + 1) * rn[b];
         }
         epi(4 * u0 + 64 * mt + 16 * cx.warp + i, a0, a1, cx.lane);
       }
@@ -1200,25 +1312,32 @@ struct EpiResid {
   const Params& p;
   bool from_embed;
   const uint8_t* side;
-  int v0, e0;
+  int r0;                  // first row of this CTA's span (its side rows start there)
   float* also = nullptr;   // fused FFN (O-projection): the same sum also to y
   __device__ void operator()(int pg, const float (&a0)[B], const float (&a1)[B], int lane) const {
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       if (lane != b) continue;
       const int r = 2 * pg;
-      float2* xp = reinterpret_cast<float2*>(p.x + plane_index(b, r, p.B, p.H));
       float2 base;
       if (from_embed) {
         const uint32_t e =
-            *reinterpret_cast<const uint32_t*>(side + p.side_embed + b * p.evb + (r - e0) * 2);
+            *reinterpret_cast<const uint32_t*>(side + p.side_embed + b * p.evb + (r - (r0 & ~7)) * 2);
         base = make_float2(bf16_lo(e), bf16_hi(e));
+      } else if (p.ffn_fused) {
+        const longlong2 q =
+            *reinterpret_cast<const longlong2*>(side + p.side_resid + (b * p.rows_side + (r - r0)) * 8);
+        base = make_float2(from_fixed(q.x), from_fixed(q.y));
       } else {
         const float* rs = reinterpret_cast<const float*>(side + p.side_resid);
-        base = *reinterpret_cast<const float2*>(rs + ((b * 2 + ((r >> 2) & 1)) * p.nvr + (r >> 3) - v0) * 4 + (r & 3));
+        base = *reinterpret_cast<const float2*>(rs + ((b * 2 + ((r >> 2) & 1)) * p.nvr + (r >> 3) - (r0 >> 3)) * 4 +
+                                                (r & 3));
       }
       const float2 v = make_float2(base.x + a0[b], base.y + a1[b]);
-      *xp = v;
+      if (p.ffn_fused)
+        *reinterpret_cast<longlong2*>(p.xacc + static_cast<size_t>(b) * p.H + r) = make_longlong2(to_fixed(v.x), to_fixed(v.y));
+      else
+        *reinterpret_cast<float2*>(p.x + plane_index(b, r, p.B, p.H)) = v;
       if (also) *reinterpret_cast<float2*>(also + plane_index(b, r, p.B, p.H)) = v;
     }
   }
@@ -1255,8 +1374,9 @@ struct EpiSwiGLULocal {
 };
 
 // Fused FFN, second half: this CTA's columns [j0, j1) of W_down times its own
-// h slice, for all H output rows (split-K over the CTAs), added into x with
-// vector float atomics.  Tiles are jt rows of W_down^T (= W_down columns), H
+// h slice, for all H output rows (split-K over the CTAs), added into the
+// residual's fixed-point accumulator with 64-bit integer atomics (the sum does
+// not depend on the order of the adds).  Tiles are jt rows of W_down^T (= W_down columns), H
 // bf16 each; thread t owns the 8-row vectors t, t + 256, ... of the output.
 template <int B>
 __device__ __noinline__ void consume_downT(const Params& p, Ctx& cx, RingPos& rp, int where, int j0, int j1,
@@ -1301,19 +1421,25 @@ __device__ __noinline__ void consume_downT(const Params& p, Ctx& cx, RingPos& rp
     if (cx.lane == 0 && ok) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));   // this warp is done with it
     rp.next(p.nslot);
   }
+  // The partial sums go to the fixed-point accumulator: first through shared
+  // memory (the activation region, unused since the gate/up GEMV), so that
+  // each warp's integer adds then cover 32 consecutive rows.
+  float* part = cx.act;   // [B][H]
 #pragma unroll
   for (int q = 0; q < NV; ++q) {
     const int v = cx.tid + q * kConsumerThreads;
     if (v < V8) {
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        float4* x0 = reinterpret_cast<float4*>(p.x + plane_index(b, 8 * v, p.B, p.H));
-        float4* x1 = reinterpret_cast<float4*>(p.x + plane_index(b, 8 * v + 4, p.B, p.H));
-        atomicAdd(x0, make_float4(acc[q][0][b], acc[q][1][b], acc[q][2][b], acc[q][3][b]));
-        atomicAdd(x1, make_float4(acc[q][4][b], acc[q][5][b], acc[q][6][b], acc[q][7][b]));
+        float4* d = reinterpret_cast<float4*>(part + static_cast<size_t>(b) * p.H + 8 * v);
+        d[0] = make_float4(acc[q][0][b], acc[q][1][b], acc[q][2][b], acc[q][3][b]);
+        d[1] = make_float4(acc[q][4][b], acc[q][5][b], acc[q][6][b], acc[q][7][b]);
       }
     }
   }
+  consumer_sync();
+  for (int i = cx.tid; i < B * p.H; i += kConsumerThreads)
+    atomicAdd(reinterpret_cast<unsigned long long*>(p.xacc + i), static_cast<unsigned long long>(to_fixed(part[i])));
 }
 
 // LM-head epilogue: running (max, lowest index) per sequence in lane b.
@@ -1331,7 +1457,7 @@ struct EpiLM {
       argmax_merge(*best_v, *best_i, a0[b], row);
       argmax_merge(*best_v, *best_i, a1[b], row + 1);
       if (p.logits_out) {
-        float* lo = p.logits_out + (static_cast<size_t>(s) * p.B + b) * p.V + row;
+        float* lo = p.logits_out + (static_cast<size_t>(p.logits_overwrite ? 0 : s) * p.B + b) * p.V + row;
         lo[0] = a0[b];
         lo[1] = a1[b];
       }
@@ -1923,7 +2049,9 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
   if (kind == ST_DOWN && p.ffn_fused) return true;         // done inside the fused gate/up stage
   if (kind == ST_LM) {
     if (!stage_wait(p, cx, p.cnt + (p.L - 1) * ST_LAYER + ffn_done, G * S1, where, fused)) return false;
-    float* hid = (p.hidden_out && cx.c == 0) ? p.hidden_out + static_cast<size_t>(s) * p.B * p.H : nullptr;
+    float* hid = (p.hidden_out && cx.c == 0)
+                     ? p.hidden_out + static_cast<size_t>(p.hidden_overwrite ? 0 : s) * p.B * p.H
+                     : nullptr;
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     EpiLM<B> epi{p, s, &bv, &bi};
@@ -1931,13 +2059,13 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
     if constexpr (B == kMaxBatch && !MOE) {
       if (p.tc) {
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-        consume_tc(p, cx, p.lm, rp, where, SRC_RESID, p.x, p.final_norm, hid, 0, epi);
+        consume_tc(p, cx, p.lm, rp, where, SRC_RESID, p.x, p.final_norm, hid, epi);
         on_tc = true;
       }
     }
     if (!on_tc) {
       float rn[B];
-      load_act<B>(p, cx, p.H, SRC_RESID, p.x, p.final_norm, hid, SIDE_NONE, s, rn, where);
+      load_act<B>(p, cx, p.H, p.ffn_fused ? SRC_FIXED : SRC_RESID, resid_src(p), p.final_norm, hid, SIDE_NONE, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       consume_gemv<B>(p, cx, p.lm, rp, where, rn, epi);
     }
@@ -2023,21 +2151,21 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         load_side<B>(p, cx, SIDE_ROPE, s, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
         EpiQKV<B> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
-        consume_tc(p, cx, L.qkv, rp, where, l == 0 ? SRC_EMBED : SRC_RESID, p.x, L.attn_norm, nullptr, 0, epi);
+        consume_tc(p, cx, L.qkv, rp, where, l == 0 ? SRC_EMBED : SRC_RESID, p.x, L.attn_norm, nullptr, epi);
       } else if (kind == ST_OPROJ) {
         load_side<B>(p, cx, l == 0 ? SIDE_EMBED : SIDE_RESID, s, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-        EpiResid<B> epi{p, l == 0, cx.side, r0 >> 3, r0 & ~7};
-        consume_tc(p, cx, L.o, rp, where, SRC_PLAIN, p.o, nullptr, nullptr, 0, epi);
+        EpiResid<B> epi{p, l == 0, cx.side, r0};
+        consume_tc(p, cx, L.o, rp, where, SRC_PLAIN, p.o, nullptr, nullptr, epi);
       } else if (kind == ST_GATEUP) {
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
         EpiSwiGLU<B> epi{p};
-        consume_tc(p, cx, L.gu, rp, where, SRC_RESID, p.x, L.ffn_norm, nullptr, 0, epi);
+        consume_tc(p, cx, L.gu, rp, where, SRC_RESID, p.x, L.ffn_norm, nullptr, epi);
       } else {
         load_side<B>(p, cx, SIDE_RESID, s, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-        EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
-        consume_tc(p, cx, L.down, rp, where, SRC_PLAIN, p.h, nullptr, nullptr, p.down_win, epi);
+        EpiResid<B> epi{p, false, cx.side, r0};
+        consume_tc(p, cx, L.down, rp, where, SRC_PLAIN, p.h, nullptr, nullptr, epi);
       }
     }
   }
@@ -2051,7 +2179,8 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       } else {
         ok = stage_wait(p, cx, p.cnt + (l - 1) * ST_LAYER + ffn_done, G * S1, where, fused);
         if (!ok) return false;
-        load_act<B>(p, cx, p.H, SRC_RESID, p.x, L.attn_norm, nullptr, SIDE_ROPE, s, rn, where);
+        load_act<B>(p, cx, p.H, p.ffn_fused ? SRC_FIXED : SRC_RESID, resid_src(p), L.attn_norm, nullptr, SIDE_ROPE, s,
+                    rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       }
       EpiQKV<B> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
@@ -2064,7 +2193,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       load_act<B>(p, cx, p.nq * p.d, SRC_PLAIN, p.o, nullptr, nullptr, l == 0 ? SIDE_EMBED : SIDE_RESID, s,
                   rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      EpiResid<B> epi{p, l == 0, cx.side, r0 >> 3, r0 & ~7, p.ffn_fused ? p.y : nullptr};
+      EpiResid<B> epi{p, l == 0, cx.side, r0, p.ffn_fused ? p.y : nullptr};
       consume_gemv<B>(p, cx, L.o, rp, where, rn, epi);
       break;
     }
@@ -2107,7 +2236,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       if constexpr (!MOE && B >= 2) {   // (batch 1 inputs always fit whole)
         if (p.down_win > 0) {
           if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-          EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
+          EpiResid<B> epi{p, false, cx.side, r0};
           if (L.down.fp8)
             consume_gemv_win_t<B, true>(p, cx, L.down, rp, where, p.h, s, epi);
           else
@@ -2118,7 +2247,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       const int K = MOE ? p.S * p.Fe : p.F;
       load_act<B>(p, cx, K, SRC_PLAIN, p.h, nullptr, nullptr, SIDE_RESID, s, rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      EpiResid<B> epi{p, false, cx.side, r0 >> 3, r0 & ~7};
+      EpiResid<B> epi{p, false, cx.side, r0};
       if constexpr (MOE) {
         // K runs over [slot][expert column]: the producer streams each slot's expert
         Mat v = L.edown;
@@ -2401,7 +2530,7 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
       // batch-8 tensor-core stage: per K window one run, the full 128-row
       // M-tiles' tiles then the last M-tile's (params.h: tile geometry)
       const Mat& m = (cu.kind == ST_LM) ? p.lm : stage_mat(p.layers[cu.l], cu.kind);
-      const int win = cu.kind == ST_DOWN ? p.down_win : 0;
+      const int win = tc_window(p.tc_win, m.K);
       const int fp8 = m.fp8, bc = tc_box_cols(fp8), kbox = tc_kbox(m.K, win, fp8);
       const int R = 2 * (cu.a_end - cu.a), w = cu.phase;
       const int k0 = w * win, Kw = win > 0 ? min(win, m.K - k0) : m.K;

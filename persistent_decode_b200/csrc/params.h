@@ -112,6 +112,10 @@ __host__ __device__ inline int tc_gcd(int a, int b) {
   }
   return a;
 }
+// K window of a tensor-core projection: Params::tc_win columns when K is
+// larger (the activation region holds one window of the B operand), else 0
+// (the whole K at once).
+__host__ __device__ inline int tc_window(int tc_win, int K) { return tc_win > 0 && K > tc_win ? tc_win : 0; }
 // Boxes per window common to every window of a K x (window) split.
 __host__ __device__ inline int tc_kbox(int K, int win, int fp8) {
   const int bc = tc_box_cols(fp8);
@@ -158,6 +162,7 @@ struct Params {
   int side_resid;       //   byte offset of the residual slice [B][2 planes][nvr] float4
   int side_embed;       //   byte offset of the embedding slice [B][evb bytes]
   int nvr;              //   float4 vectors per (sequence, plane) of the residual slice
+  int rows_side;        //   fused-FFN layers: int64 rows per sequence of the accumulator slice
   int evb;              //   bytes per sequence of the embedding slice
   int attn_pos_per_tile;
   long long spin_limit_ns;
@@ -181,16 +186,19 @@ struct Params {
   const float2* rope;           // [max_seq][d/2] (cos, sin)
 
   // workspace
-  float* x;          // [B][H] residual stream
+  float* x;          // [B][H] residual stream (two-plane fp32; layers without the fused FFN)
+  long long* xacc;   // fused FFN: [B][H] residual stream, 64-bit fixed point with 32 fractional
+                     // bits, into which the down projection's split-K partials are added
   float* q;          // [B][nq*d] rotated queries
   float* o;          // [B][nq*d] attention output
   float* h;          // [B][F] SwiGLU output (MoE: [B][S*Fe], slot-major, gate-weighted)
   float* y;          // fused FFN: [B][H] residual after attention (the FFN's RMSNorm input);
-                     // x then accumulates the down projection's partial sums
+                     // xacc then accumulates the down projection's partial sums
   int ffn_fused;     // 1: gate/up and down run as one stage with a split-K down projection
   int jt;            // fused FFN: W_down columns per tile
   int tc;            // 1: batch-8 projections on tcgen05 MMAs (tensor-core packing and stages)
-  int tc_cols;       //   tensor-memory columns each CTA allocates (8 per M-tile of its largest stage)
+  int tc_cols;       //   tensor-memory columns each CTA allocates (16 per M-tile of its largest stage)
+  int tc_win;        //   K window of the tensor-core projections (tc_window), 0: whole K
   int down_win;      // K-windowed down projection: W_down columns per activation window (0: whole K);
                      // the CTA's down tiles are packed window by window, groups inside a window
   int side_hloc;     // fused FFN: byte offset of the CTA's h slice [B][hloc] in the side region
@@ -214,6 +222,8 @@ struct Params {
   const int32_t* forced;
   float* logits_out;
   float* hidden_out;
+  int logits_overwrite;        // 1: every step writes logits_out[0..B) (parity mode), else step s at [s]
+  int hidden_overwrite;        // the same for hidden_out
   int32_t* experts_out;        // MoE: [n_steps][L][B][topk] selected experts (may be null)
   unsigned long long* trace;   // optional stage timestamps
   int fault_drop_stage;        // failure-detection tests: CTA 0 withholds its release of this

@@ -7,11 +7,10 @@
 
 namespace xlpk {
 
-// N of the batch-8 MMAs.  kind::f16 with M = 128 takes N in multiples of 16,
-// so the 8 sequences' B operand is read as 16 rows: rows 8..15 are whatever
-// follows the staged operand in shared memory (the next box, or the slack kept
-// after the last one) and only reach accumulator columns 8..15, which are
-// never read.  Each M-tile therefore owns 16 tensor-memory columns.
+// N of the batch-8 MMAs (kind::f16 with M = 128 takes N in multiples of 16):
+// the B operand's rows 0..7 are the 8 sequences' inputs rounded to bf16 and
+// rows 8..15 the rounding remainders, so accumulator column b + 8 completes
+// column b.  Each M-tile owns 16 tensor-memory columns.
 constexpr int kTcAccCols = 16;
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -63,6 +62,17 @@ __device__ __forceinline__ void tc_alloc(uint32_t slot, uint32_t cols) {
 }
 __device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+// Warp-wide: 16 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15},"
+      " [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // Warp-wide: 8 consecutive fp32 columns of this warp's 32 tensor-memory lanes.

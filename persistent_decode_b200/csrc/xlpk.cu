@@ -216,12 +216,13 @@ struct xlpk_engine {
   int nslot = 0;
   int smem = 0;
   int act_bytes = 0;
-  int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, evb = 0;
+  int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, rows_side = 0, evb = 0;
   int side_hloc = 0, hloc = 0;
   bool ffn_fused = false;
   bool tc = false;              // batch-8 projections on tcgen05 MMAs
   int tc_cols = 0;
   int down_win = 0;            // K-windowed down projection (columns per window; 0: off)
+  int tc_win = 0;              // K window of the tensor-core projections (0: whole K)
   int esz = 2;
   int P = 0;
   uint8_t* packed = nullptr;
@@ -239,6 +240,8 @@ struct xlpk_engine {
   const void* kern_stage = nullptr;
   void (*launch_stage)(const Params&, int, int, int, int, int, cudaStream_t) = nullptr;
   int64_t weight_bytes_per_step = 0;
+  float* dbg_logits = nullptr;   // parity mode (xlpk_debug_logits): [B][V], [B][H], last step's
+  float* dbg_hidden = nullptr;
 };
 
 namespace {
@@ -589,20 +592,18 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   // dense layers whose output rows fit two 8-row vectors per consumer thread
   // and whose accumulators fit the register budget (XLPK_FFN_FUSED=0 turns it off).
   {
-    const char* env = std::getenv("XLPK_FFN_FUSED");
-    const bool off = env && env[0] == '0';
+    const bool off = (c.flags & XLPK_FLAG_NO_FUSED_FFN) != 0;
     e->ffn_fused = !off && c.n_experts == 0 && e->esz == 2 && H <= 2 * 8 * kConsumerThreads && H % 8 == 0 &&
                    B <= 2;
   }
   // Batch 8, dense layers: every projection runs on tcgen05 MMAs (8-row units
-  // per CTA, M-tiles of <= 128 rows with kTcAccCols accumulator columns each in tensor
-  // memory; XLPK_TC=0 turns it off).
+  // per CTA, M-tiles of <= 128 rows with kTcAccCols accumulator columns each in
+  // tensor memory; XLPK_FLAG_NO_TENSOR_CORES keeps the CUDA-core tiles).
   {
-    const char* env = std::getenv("XLPK_TC");
     const int bc = e->esz == 1 ? 128 : 64;
     const int nqkv = qd + 2 * kvd;
-    e->tc = !(env && env[0] == '0') && B == 8 && c.n_experts == 0 && H % bc == 0 && qd % bc == 0 &&
-            F % bc == 0 && nqkv % 8 == 0 && c.vocab % 8 == 0;
+    e->tc = !(c.flags & XLPK_FLAG_NO_TENSOR_CORES) && B == 8 && c.n_experts == 0 && H % bc == 0 &&
+            qd % bc == 0 && F % bc == 0 && nqkv % 8 == 0 && c.vocab % 8 == 0;
     if (e->tc) {
       int mt = 0;
       for (const int n : {nqkv, H, 2 * F, c.vocab}) {
@@ -624,7 +625,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     e->side_rope = 0;
     e->side_resid = static_cast<int>(align_up(static_cast<size_t>(B) * d * 4, 16));
     e->nvr = rows_max / 8 + 2;
-    e->side_embed = e->side_resid + B * 2 * e->nvr * 16;
+    e->rows_side = rows_max;
+    // the residual rows: two planes of float4, or (fused FFN) int64 rows of the accumulator
+    e->side_embed = e->side_resid + B * std::max(2 * e->nvr * 16, rows_max * 8);
     e->evb = static_cast<int>(align_up(static_cast<size_t>(rows_max + 16) * 2, 16));
     e->side_hloc = static_cast<int>(align_up(static_cast<size_t>(e->side_embed) + B * e->evb, 16));
     e->hloc = e->ffn_fused ? (F + e->G - 1) / e->G : 0;
@@ -635,34 +638,52 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const int attn_scratch = attn_scratch_floats(d, e->G) * 4;
   const int norm_stage = (B + 1) * H * 4;   // normed input vector + its RMSNorm gains
   const int max_smem = static_cast<int>(prop.sharedMemPerBlockOptin);
-  auto act_for = [&](int kmax) {
-    if (e->tc)   // the MMA's B operand: 8 sequences x kmax bf16, + one box of slack
-                 // that the N = 16 read of the last box's rows 8..15 may touch
-      return static_cast<int>(align_up(std::max(B * kmax * 2 + 1024, attn_scratch), 1024));
-    return static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
-  };
-  e->act_bytes = act_for(std::max(std::max(H, qd), std::max(F, S_moe * c.expert_ffn)));
-  // A two-stage dense FFN whose down-projection input (B x F fp32) would leave
-  // the ring fewer than 3 slots streams W_down window by window instead: the
-  // activation region then holds B x down_win floats of h at a time (windows of
-  // the largest whole number of k-chunks that fits the other stages' inputs).
-  // (XLPK_DOWN_WIN=<columns> asks for a given window where windows are possible;
-  // the tests compare windowed and whole-K down projections with it.)
+  auto slots_for = [&](int act) { return (max_smem - act - e->side_bytes - kMiscSmem) / kSlotBytes; };
   e->down_win = 0;
-  {
-    const char* env = std::getenv("XLPK_DOWN_WIN");
-    const int forced = env ? std::atoi(env) : 0;
-    // window granule: whole k-chunks of the CUDA-core tiles, or 1024 columns
-    // (whole boxes of either weight type) for the tensor-core tiles
-    const int kc = e->tc ? 1024 : pick_kc(F, e->esz);
+  e->tc_win = 0;
+  if (e->tc) {
+    // The MMA's B operand takes 32 bytes per input column (8 sequences, a bf16
+    // high and low part each).  Projections whose K is larger than a window
+    // stream it window by window (tc_window), the window chosen so that the
+    // ring keeps at least 4 slots: the whole K, else 4096, 2048 or 1024 columns
+    // (whole boxes of either weight type); xlpk_config::window asks for one.
+    const int kall = std::max(std::max(H, qd), F);
+    auto act_tc = [&](int kw) { return static_cast<int>(align_up(std::max(32 * kw, attn_scratch), 1024)); };
+    int win = -1;
+    if (c.window > 0) {
+      if (c.window % 1024) return XLPK_ERR_UNSUPPORTED;
+      win = c.window < kall ? c.window : 0;
+    } else {
+      for (const int cand : {0, 4096, 2048, 1024}) {
+        const int kw = cand > 0 ? std::min(cand, kall) : kall;
+        if (slots_for(act_tc(kw)) >= 4) {
+          win = cand > 0 && cand < kall ? cand : 0;
+          break;
+        }
+      }
+      if (win < 0) win = 1024;
+    }
+    e->tc_win = win;
+    e->act_bytes = act_tc(win > 0 ? win : kall);
+  } else {
+    auto act_for = [&](int kmax) {
+      return static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
+    };
+    e->act_bytes = act_for(std::max(std::max(H, qd), std::max(F, S_moe * c.expert_ffn)));
+    // A two-stage dense FFN whose down-projection input (B x F fp32) would leave
+    // the ring fewer than 3 slots streams W_down window by window instead: the
+    // activation region then holds B x down_win floats of h at a time (windows
+    // of the largest whole number of k-chunks that fits the other stages'
+    // inputs; xlpk_config::window asks for a given window where windows are
+    // possible).
+    const int kc = pick_kc(F, e->esz);
     const int maxp = (H / 2 + e->G - 1) / e->G;
-    const bool possible = !e->ffn_fused && c.n_experts == 0 && B >= 2 && kc > 0 &&
-                          (e->tc || maxp <= kPairsPerTile * kMaxWinGroups);
+    const bool possible =
+        !e->ffn_fused && c.n_experts == 0 && B >= 2 && kc > 0 && maxp <= kPairsPerTile * kMaxWinGroups;
     int win = 0;
-    if (possible && forced > 0) {
-      if (forced % kc == 0 && forced < F) win = forced;
-    } else if (possible && F > std::max(H, qd) &&
-               (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes < 3) {
+    if (possible && c.window > 0) {
+      if (c.window % kc == 0 && c.window < F) win = c.window;
+    } else if (possible && F > std::max(H, qd) && slots_for(e->act_bytes) < 3) {
       win = (std::max(H, qd) / kc) * kc;
       if (win >= F) win = 0;
     }
@@ -798,7 +819,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       e->esz = mp.role == R_ROUTER ? 2 : esz_saved;
       if (e->tc && (mp.role == R_QKV || mp.role == R_O || mp.role == R_GU || mp.role == R_DOWN || mp.role == R_LM))
         rc = pack_matrix_tc(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, reinterpret_cast<TcRowJob*>(d_jobs),
-                            max_jobs, st, mp.role == R_DOWN ? e->down_win : 0);
+                            max_jobs, st, tc_window(e->tc_win, mp.K));
       else
         rc = pack_matrix(e, mp.src, mp.N, mp.K, e->packed + mp.off, &m, d_jobs, max_jobs, st, mp.split,
                          mp.role == R_DOWN ? e->down_win : 0);
@@ -867,6 +888,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const size_t o_o = take(sizeof(float) * B * qd);
   const size_t o_h = take(sizeof(float) * B * std::max(F, S_moe * c.expert_ffn));
   const size_t o_y = take(sizeof(float) * B * H);
+  const size_t o_xacc = take(sizeof(long long) * B * H);
   const size_t o_pml = take(sizeof(float) * prow * group * 2);
   const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * e->G * B);
@@ -908,6 +930,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.side_resid = e->side_resid;
   p.side_embed = e->side_embed;
   p.nvr = e->nvr;
+  p.rows_side = e->rows_side;
   p.evb = e->evb;
   p.attn_pos_per_tile = e->P;
   p.spin_limit_ns = 1000LL * (c.spin_limit_us > 0 ? c.spin_limit_us : 200000);
@@ -934,11 +957,13 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.o = reinterpret_cast<float*>(e->ws + o_o);
   p.h = reinterpret_cast<float*>(e->ws + o_h);
   p.y = reinterpret_cast<float*>(e->ws + o_y);
+  p.xacc = reinterpret_cast<long long*>(e->ws + o_xacc);
   p.ffn_fused = e->ffn_fused ? 1 : 0;
   p.jt = kTileBytes / (H * 2);
   p.down_win = e->down_win;
   p.tc = e->tc ? 1 : 0;
   p.tc_cols = e->tc_cols;
+  p.tc_win = e->tc_win;
   p.side_hloc = e->side_hloc;
   p.hloc = e->hloc;
   p.route_exp = reinterpret_cast<int*>(e->ws + o_rte);
@@ -979,17 +1004,22 @@ Params call_params(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out, const x
   p.forced = io ? io->forced_tokens_dev : nullptr;
   p.logits_out = io ? io->logits_dev : nullptr;
   p.hidden_out = io ? io->hidden_dev : nullptr;
+  // parity mode: the registered buffers, each step over the last
+  p.logits_overwrite = 0;
+  p.hidden_overwrite = 0;
+  if (!p.logits_out && h->dbg_logits) {
+    p.logits_out = h->dbg_logits;
+    p.logits_overwrite = 1;
+  }
+  if (!p.hidden_out && h->dbg_hidden) {
+    p.hidden_out = h->dbg_hidden;
+    p.hidden_overwrite = 1;
+  }
   p.experts_out = io ? io->experts_dev : nullptr;
   p.trace = io ? reinterpret_cast<unsigned long long*>(io->trace_dev) : nullptr;
-  // L2 prefetch distance per CTA: a tuning knob read at each call (0 disables)
-  if (const char* env = std::getenv("XLPK_L2_PREFETCH_KB")) p.l2_prefetch_bytes = std::atoll(env) * 1024;
-  // suspend-time hint of the mbarrier waits (tuning knob; 0 polls)
-  if (const char* env = std::getenv("XLPK_WAIT_HINT_NS")) p.wait_hint_ns = static_cast<unsigned>(std::atoll(env));
-  // Failure-detection tests: make one dependency wait run out (a release that
-  // never happens) so the time limit, the abort path and the status report
-  // are exercised without faulting anything.
-  p.fault_drop_stage = -1;
-  if (const char* env = std::getenv("XLPK_FAULT_DROP_RELEASE")) p.fault_drop_stage = std::atoi(env);
+  // Failure-detection testing: CTA 0 withholds its release of one stage at the
+  // call's first step, so a dependency wait runs out (nothing faults).
+  p.fault_drop_stage = io && io->withhold_release > 0 ? io->withhold_release - 1 : -1;
   return p;
 }
 
@@ -1012,16 +1042,48 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 unsigned char* g_noalloc_addr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};   // context the address was taken in
 
-// Device address of the array on `dev` (which must be the current device).
+// Unique id of the current context (driver entry points reached through the
+// runtime, so the library does not link libcuda); 0 if unavailable.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    looked_up = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the array on `dev` (which must be the current device):
+// looked up once per device, and again if the device's context has been
+// replaced since (cudaDeviceReset reloads the module, which may move it).
 xlpk_status noalloc_scratch(int dev, unsigned char** out) {
   if (dev < 0 || dev >= kMaxDevices) return XLPK_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_noalloc_addr[dev] || ctx != g_noalloc_ctx[dev]) {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || !ptr) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
     g_noalloc_addr[dev] = static_cast<unsigned char*>(ptr);
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_addr[dev];
   return XLPK_OK;
@@ -1136,6 +1198,7 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   const int S_moe = h->base.S;
   const size_t o_h = take(sizeof(float) * B * std::max(F, S_moe * c.expert_ffn));
   const size_t o_y = take(sizeof(float) * B * H);
+  const size_t o_xacc = take(sizeof(long long) * B * H);
   const size_t o_pml = take(sizeof(float) * prow * group * 2);
   const size_t o_po = take(sizeof(float) * prow * group * d);
   const size_t o_lv = take(sizeof(float) * h->G * B);
@@ -1157,6 +1220,7 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
   p.o = reinterpret_cast<float*>(sc + o_o);
   p.h = reinterpret_cast<float*>(sc + o_h);
   p.y = reinterpret_cast<float*>(sc + o_y);
+  p.xacc = reinterpret_cast<long long*>(sc + o_xacc);
   p.route_exp = reinterpret_cast<int*>(sc + o_rte);
   p.route_w = reinterpret_cast<float*>(sc + o_rtw);
   p.part_ml = reinterpret_cast<float*>(sc + o_pml);
@@ -1169,6 +1233,14 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
                                         static_cast<size_t>(h->smem), st));
   for (int b = 0; b < B; ++b) h->pos[b] += n_steps;
   h->last_stream = st;
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_debug_logits(xlpk_handle h, float* logits_dev, float* hidden_dev) {
+  if (!h) return XLPK_ERR_INVALID_ARG;
+  if ((logits_dev && !aligned16(logits_dev)) || (hidden_dev && !aligned16(hidden_dev))) return XLPK_ERR_INVALID_ARG;
+  h->dbg_logits = logits_dev;
+  h->dbg_hidden = hidden_dev;
   return XLPK_OK;
 }
 

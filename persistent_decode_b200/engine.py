@@ -66,7 +66,7 @@ def _stream_handle(stream) -> Optional[int]:
 
 
 def make_config(cfg, n_ctas: int = 0, spin_limit_us: int = 0, batch: Optional[int] = None,
-                max_seq: Optional[int] = None) -> _abi.xlpk_config:
+                max_seq: Optional[int] = None, flags: int = 0, window: int = 0) -> _abi.xlpk_config:
     c = _abi.xlpk_config()
     for f in ("n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
               "n_experts", "top_k", "n_shared_experts", "expert_ffn"):
@@ -78,6 +78,8 @@ def make_config(cfg, n_ctas: int = 0, spin_limit_us: int = 0, batch: Optional[in
     c.rms_eps = float(cfg.rms_eps)
     c.n_ctas = int(n_ctas)
     c.spin_limit_us = int(spin_limit_us)
+    c.flags = int(flags)
+    c.window = int(window)
     return c
 
 
@@ -87,15 +89,17 @@ class Engine:
     `weights` maps names ("embed", "lm_head", "final_norm", "layers.{l}.wq", ...,
     with ".scale" companions for FP8) to CUDA tensors in row-major [out][in]
     layout; `k_cache`/`v_cache` are bf16 CUDA tensors [L][B][n_kv][max_seq][d]
-    that the engine writes in place.
+    that the engine writes in place.  `flags` (XLPK_FLAG_*) and `window` are the
+    config fields of the same names.
     """
 
     def __init__(self, cfg, weights: Dict[str, "object"], k_cache, v_cache, n_ctas: int = 0,
-                 spin_limit_us: int = 0):
+                 spin_limit_us: int = 0, flags: int = 0, window: int = 0):
         self.cfg = cfg
         self.B = int(k_cache.shape[1])
         self.max_seq = int(k_cache.shape[3])
-        self._c = make_config(cfg, n_ctas, spin_limit_us, batch=self.B, max_seq=self.max_seq)
+        self._c = make_config(cfg, n_ctas, spin_limit_us, batch=self.B, max_seq=self.max_seq, flags=flags,
+                              window=window)
         L = cfg.n_layers
         self._layers = (_abi.xlpk_layer_weights * max(L, 1))()
 
@@ -165,14 +169,17 @@ class Engine:
         _check(lib.xlpk_set_state(self.h, t, s, _stream_handle(stream)), "xlpk_set_state")
 
     @staticmethod
-    def _io(forced=None, logits=None, hidden=None, experts=None, trace=None):
-        if all(t is None for t in (forced, logits, hidden, experts, trace)):
+    def _io(forced=None, logits=None, hidden=None, experts=None, trace=None, withhold_release: int = 0):
+        if all(t is None for t in (forced, logits, hidden, experts, trace)) and not withhold_release:
             return None
-        return _abi.xlpk_decode_io(_ptr(forced), _ptr(logits), _ptr(hidden), _ptr(experts), _ptr(trace))
+        return _abi.xlpk_decode_io(_ptr(forced), _ptr(logits), _ptr(hidden), _ptr(experts), _ptr(trace),
+                                   int(withhold_release))
 
     def decode(self, n_steps: int, tokens_out, forced=None, logits=None, hidden=None, experts=None,
-               trace=None, stream=None, unfused: bool = False) -> None:
-        io = self._io(forced, logits, hidden, experts, trace)
+               trace=None, stream=None, unfused: bool = False, withhold_release: int = 0) -> None:
+        """xlpk_decode (or xlpk_decode_unfused); `withhold_release` is the io field
+        of that name (failure-detection tests only)."""
+        io = self._io(forced, logits, hidden, experts, trace, withhold_release)
         fn = lib.xlpk_decode_unfused if unfused else lib.xlpk_decode
         _check(fn(self.h, int(n_steps), _ptr(tokens_out), C.byref(io) if io is not None else None,
                   _stream_handle(stream)), "xlpk_decode_unfused" if unfused else "xlpk_decode")
@@ -184,6 +191,12 @@ class Engine:
         _check(lib.xlpk_decode_noalloc(self.h, int(n_steps), _ptr(tokens_out),
                                        C.byref(io) if io is not None else None, _stream_handle(stream)),
                "xlpk_decode_noalloc")
+
+    def debug_logits(self, logits=None, hidden=None) -> None:
+        """xlpk_debug_logits: parity-mode buffers ([B][V] and [B][H] fp32 CUDA tensors,
+        or None) that later decode calls overwrite with each step's values."""
+        self._dbg = (logits, hidden)   # borrowed by the library until replaced
+        _check(lib.xlpk_debug_logits(self.h, _ptr(logits), _ptr(hidden)), "xlpk_debug_logits")
 
     def status(self) -> int:
         return int(lib.xlpk_get_status(self.h))

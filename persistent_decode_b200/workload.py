@@ -33,7 +33,8 @@ def kv_shape(cfg, batch: int, max_seq: int):
 
 
 def build(cfg, device="cuda", norm_std: float = 0.0, n_ctas: int = 0, max_seq: Optional[int] = None,
-          spin_limit_us: int = 0, weights: Optional[Dict[str, torch.Tensor]] = None) -> GpuModel:
+          spin_limit_us: int = 0, weights: Optional[Dict[str, torch.Tensor]] = None, flags: int = 0,
+          window: int = 0) -> GpuModel:
     dev = torch.device(device)
     B = cfg.batch
     ms = max_seq if max_seq is not None else cfg.max_seq
@@ -50,7 +51,7 @@ def build(cfg, device="cuda", norm_std: float = 0.0, n_ctas: int = 0, max_seq: O
             k[l, :, :, : cfg.kv_len] = kl
             v[l, :, :, : cfg.kv_len] = vl
         start = synth.make_start_tokens(cfg, device="cpu")
-    eng = Engine(cfg, w, k, v, n_ctas=n_ctas, spin_limit_us=spin_limit_us)
+    eng = Engine(cfg, w, k, v, n_ctas=n_ctas, spin_limit_us=spin_limit_us, flags=flags, window=window)
     m = GpuModel(cfg, w, k, v, eng, prompt, start.to(torch.int32))
     if cfg.prefill:
         prefill(m)

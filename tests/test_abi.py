@@ -80,10 +80,34 @@ def test_host_side_argument_checks(lib):
     assert lib.xlpk_tc_gemm_tile(C.c_void_p((1 << 20) + 8), 128, 64, p, p, None) == _abi.XLPK_ERR_INVALID_ARG
 
 
-def test_struct_layout_matches_header(lib):
-    # 18 four-byte fields in xlpk_config; pointer-sized members elsewhere
-    assert C.sizeof(_abi.xlpk_config) == 18 * 4
-    assert C.sizeof(_abi.xlpk_linear) == 16
-    assert C.sizeof(_abi.xlpk_layer_weights) == 8 + 4 * 16 + 8 + 3 * 16 + 8 + 6 * 16
-    assert C.sizeof(_abi.xlpk_decode_io) == 40
-    assert C.sizeof(_abi.xlpk_info) == 6 * 4 + 3 * 8
+def test_struct_layout_matches_header(tmp_path):
+    # every field of every struct at the offset a C compiler gives it from
+    # include/xlpk.h (gcc on this host), against the ctypes mirror
+    import subprocess
+    structs = [_abi.xlpk_config, _abi.xlpk_linear, _abi.xlpk_layer_weights, _abi.xlpk_weights, _abi.xlpk_kv,
+               _abi.xlpk_decode_io, _abi.xlpk_info]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "xlpk.h"', 'int main(void) {']
+    for st in structs:
+        n = st.__name__
+        lines.append(f'  printf("{n} size %zu\\n", sizeof({n}));')
+        for f, _ in st._fields_:
+            lines.append(f'  printf("{n} {f} %zu\\n", offsetof({n}, {f}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {}
+    for line in out:
+        if line:
+            parts = line.split()
+            got[(parts[0], parts[1])] = int(parts[2])
+    for st in structs:
+        n = st.__name__
+        assert got[(n, "size")] == C.sizeof(st), n
+        for f, _ in st._fields_:
+            assert got[(n, f)] == getattr(st, f).offset, (n, f)
+
+def test_debug_logits_rejects_a_null_handle(lib):
+    assert lib.xlpk_debug_logits(None, None, None) == _abi.XLPK_ERR_INVALID_ARG

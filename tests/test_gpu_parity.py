@@ -42,23 +42,52 @@ def test_tiny_decode_matches_oracle(tiny, unfused):
 
 
 def test_tiny_persistent_matches_kernel_per_op(tiny):
-    # the same tiles and arithmetic; the fused FFN stage adds the down
-    # projection's split-K partial sums with float atomics, so the two agree
-    # up to summation order
+    # the same tiles and arithmetic in the same order (the fused FFN's split-K
+    # partial sums meet in a fixed-point accumulator, whose integer adds do not
+    # depend on arrival order): bit-identical results
     a = run_engine(tiny, tiny.cfg.steps, unfused=False)
     b = run_engine(tiny, tiny.cfg.steps, unfused=True)
     assert torch.equal(a.tokens, b.tokens)
-    assert rel_l2(a.logits, b.logits) < 1e-5
-    assert rel_l2(a.hidden, b.hidden) < 1e-5
+    assert torch.equal(a.logits, b.logits)
+    assert torch.equal(a.hidden, b.hidden)
 
 
-def test_fused_ffn_matches_two_stage_ffn(cuda_device, monkeypatch):
+def test_tiny_runs_are_bit_identical(tiny):
+    runs = [run_engine(tiny, tiny.cfg.steps) for _ in range(3)]
+    for r in runs[1:]:
+        assert torch.equal(r.logits, runs[0].logits)
+        assert torch.equal(r.hidden, runs[0].hidden)
+
+
+def test_debug_logits_hold_the_last_step(tiny):
+    # parity mode: buffers registered once, overwritten by every step
+    from persistent_decode_b200 import XlpkError
+    cfg, dev = tiny.cfg, tiny.k.device
+    ref = run_engine(tiny, 6)
+    lg = torch.full((cfg.batch, cfg.vocab), float("nan"), dtype=torch.float32, device=dev)
+    hd = torch.full((cfg.batch, cfg.hidden), float("nan"), dtype=torch.float32, device=dev)
+    tiny.engine.debug_logits(lg, hd)
+    try:
+        workload.reset_state(tiny)
+        tok = torch.empty(6, cfg.batch, dtype=torch.int32, device=dev)
+        tiny.engine.decode(6, tok)
+        tiny.engine.check()
+        assert torch.equal(lg.cpu(), ref.logits[5])
+        assert torch.equal(hd.cpu(), ref.hidden[5])
+    finally:
+        tiny.engine.debug_logits(None, None)
+    with pytest.raises(XlpkError):
+        tiny.engine.debug_logits(lg.view(-1)[1:], None)   # 4 bytes in: not 16-byte aligned
+
+
+def test_fused_ffn_matches_two_stage_ffn(cuda_device):
     # gate/up + split-K down in one stage (default for bf16 dense models) vs
-    # gate/up and down as two stages (XLPK_FFN_FUSED=0), same weights
+    # gate/up and down as two stages (XLPK_FLAG_NO_FUSED_FFN), same weights
+    from persistent_decode_b200 import _abi
     cfg = synth.get_config("tiny", steps=10)
     fused = workload.build(cfg, device=cuda_device, norm_std=0.1)
-    monkeypatch.setenv("XLPK_FFN_FUSED", "0")
-    two = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=fused.weights)
+    two = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=fused.weights,
+                         flags=_abi.XLPK_FLAG_NO_FUSED_FFN)
     assert two.engine.info().kernels_per_step_unfused == 5 * cfg.n_layers + 1
     assert fused.engine.info().kernels_per_step_unfused == 4 * cfg.n_layers + 1
     a = run_engine(fused, cfg.steps)
@@ -252,15 +281,15 @@ def test_llama1b_batch4_prefix(cuda_device):
 
 
 @pytest.mark.parametrize("batch", [2, 4])
-def test_windowed_down_projection_matches_whole_k(cuda_device, monkeypatch, batch):
+def test_windowed_down_projection_matches_whole_k(cuda_device, batch):
     # the down projection streamed in K windows of 1024 columns (4 windows of
     # F = 4096) against the same model with the whole K staged at once: the
     # per-lane sums run over the same chunks in the same order
-    monkeypatch.setenv("XLPK_FFN_FUSED", "0")
+    from persistent_decode_b200 import _abi
     cfg = synth.get_config("tiny", ffn=4096, batch=batch, steps=6)
-    whole = workload.build(cfg, device=cuda_device, norm_std=0.1)
-    monkeypatch.setenv("XLPK_DOWN_WIN", "1024")
-    win = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=whole.weights)
+    two = _abi.XLPK_FLAG_NO_FUSED_FFN
+    whole = workload.build(cfg, device=cuda_device, norm_std=0.1, flags=two)
+    win = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=whole.weights, flags=two, window=1024)
     for unfused in (False, True):
         a = run_engine(whole, cfg.steps, unfused=unfused)
         b = run_engine(win, cfg.steps, unfused=unfused)
@@ -279,18 +308,35 @@ def test_batch8_tensor_core_path_matches_oracle(cuda_device, unfused):
     compare_with_oracle(m, run, oracle_for(m), cfg.steps)
 
 
-def test_batch8_tensor_core_windowed_down_matches_whole_k(cuda_device, monkeypatch):
+def test_batch8_tensor_core_windowed_down_matches_whole_k(cuda_device):
     # the tensor-core down projection over K windows of 1024 columns keeps
-    # accumulating in the same tensor-memory columns: identical results
+    # accumulating in the same tensor-memory columns, in the same K order, as
+    # the whole K staged at once (window 4096 = F): identical results
     cfg = synth.get_config("tiny", ffn=4096, batch=8, steps=4)
-    whole = workload.build(cfg, device=cuda_device, norm_std=0.1)
-    monkeypatch.setenv("XLPK_DOWN_WIN", "1024")
-    win = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=whole.weights)
+    whole = workload.build(cfg, device=cuda_device, norm_std=0.1, window=4096)
+    win = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=whole.weights, window=1024)
     a = run_engine(whole, cfg.steps)
     b = run_engine(win, cfg.steps)
     assert torch.equal(a.tokens, b.tokens)
     assert torch.equal(a.logits, b.logits)
     compare_with_oracle(win, b, oracle_for(win), cfg.steps)
+
+
+def test_batch8_tensor_cores_match_cuda_cores(cuda_device):
+    # the MMA's B operand carries each input as a bf16 high part and a bf16
+    # remainder, so the tensor-core decode agrees with the fp32 CUDA-core
+    # tiles far inside the tolerance
+    from persistent_decode_b200 import _abi
+    cfg = synth.get_config("tiny", batch=8, steps=6)
+    tc = workload.build(cfg, device=cuda_device, norm_std=0.1)
+    cc = workload.build(cfg, device=cuda_device, norm_std=0.1, weights=tc.weights,
+                        flags=_abi.XLPK_FLAG_NO_TENSOR_CORES)
+    a = run_engine(tc, cfg.steps)
+    b = run_engine(cc, cfg.steps)
+    assert torch.equal(a.tokens, b.tokens)
+    assert rel_l2(a.logits, b.logits) < 1e-4
+    assert rel_l2(a.hidden, b.hidden) < 1e-4
+    compare_with_oracle(cc, b, oracle_for(cc), cfg.steps)
 
 
 def test_llama1b_batch8_tensor_core_prefix(cuda_device):
