@@ -130,11 +130,27 @@ typedef struct xlpk_weights {
   const xlpk_layer_weights* layers;   /* HOST array of n_layers entries */
 } xlpk_weights;
 
-/* Caller-owned KV cache, bf16 [L][B][n_kv][max_seq][d] for K and V each,
- * 16-byte aligned.  Entries are post-RoPE keys and values. */
+/* Caller-owned KV cache: post-RoPE keys and values, bf16, 16-byte aligned.
+ *  - Contiguous (page_table_dev NULL): K and V each [L][B][n_kv][max_seq][d].
+ *  - Paged: K and V each a pool [L][n_pages][n_kv][page_size][d] of pages of
+ *    page_size positions; page_table_dev int32 [B][ceil(max_seq / page_size)]
+ *    names the pool page that holds positions [j*page_size, (j+1)*page_size)
+ *    of sequence b.  page_size must be the attention chunk (64 positions for
+ *    head_dim 128, 128 for head_dim 64; else XLPK_ERR_UNSUPPORTED), so every
+ *    attention task reads exactly one page.  Sequences may share pages (a
+ *    common prefix).  The table is read by every decode; the caller may change
+ *    it between calls (stream order).  An entry outside [0, n_pages) that a
+ *    decode reaches is not followed: the decode stops with XLPK_ERR_INVALID_ARG
+ *    from xlpk_get_status.
+ * Source: the KV page planner that places each request's cache pages and the
+ * decode worker that follows them ("XL-Persistent-Kernel", request lifecycle
+ * steps 2-4 and the component table's KV row). */
 typedef struct xlpk_kv {
   void* k_dev;
   void* v_dev;
+  const int32_t* page_table_dev;   /* NULL: contiguous cache */
+  int32_t page_size;               /* paged: positions per page */
+  int32_t n_pages;                 /* paged: pages in each pool */
 } xlpk_kv;
 
 /* Optional per-step outputs and teacher forcing of one decode call.

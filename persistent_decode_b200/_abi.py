@@ -53,7 +53,8 @@ class xlpk_weights(C.Structure):
 
 
 class xlpk_kv(C.Structure):
-    _fields_ = [("k_dev", C.c_void_p), ("v_dev", C.c_void_p)]
+    _fields_ = [("k_dev", C.c_void_p), ("v_dev", C.c_void_p), ("page_table_dev", C.c_void_p),
+                ("page_size", C.c_int32), ("n_pages", C.c_int32)]
 
 
 class xlpk_decode_io(C.Structure):

@@ -292,7 +292,7 @@ struct Ctx {
   uint32_t bop_phase;
 };
 
-enum ErrCode : int { kErrNone = 0, kErrTimeout = -6, kErrAborted = -7 };
+enum ErrCode : int { kErrNone = 0, kErrBadPage = -1, kErrTimeout = -6, kErrAborted = -7 };
 
 __device__ __forceinline__ void raise_error(const Params& p, int code, int where) {
   if (atomicCAS(p.status, 0, code) == 0) {
@@ -1259,6 +1259,8 @@ __device__ __forceinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat
     consume_gemv_t<B, false>(p, cx, m, rp, where, rn, epi, q0, q1);
 }
 
+__device__ __forceinline__ size_t kv_row(const Params& p, int l, int b, int g, int t, bool& ok);
+
 // QKV epilogue: RoPE on q/k pairs, q -> workspace, bf16 k/v -> cache at pos.
 // The step's cos/sin rows were staged in shared memory (SIDE_ROPE).
 template <int B>
@@ -1286,18 +1288,27 @@ struct EpiQKV {
           qd[i] = y0;
           qd[i + half] = y1;
         } else {
-          uint16_t* kd =
-              p.kc + (((static_cast<size_t>(l) * p.B + b) * p.nkv + head) * p.max_seq + pos) * p.d;
-          kd[i] = f2bf(y0);
-          kd[i + half] = f2bf(y1);
+          bool ok;
+          const size_t row = kv_row(p, l, b, head, pos, ok);
+          if (ok) {
+            uint16_t* kd = p.kc + row;
+            kd[i] = f2bf(y0);
+            kd[i + half] = f2bf(y1);
+          } else {
+            raise_error(p, kErrBadPage, where_code(ST_QKV, l, s));
+          }
         }
       } else {
         const int pv = pg - hq - hk;
         const int head = pv / half, i2 = (pv - head * half) * 2;
-        uint16_t* vd =
-            p.vc + (((static_cast<size_t>(l) * p.B + b) * p.nkv + head) * p.max_seq + pos) * p.d;
-        const uint32_t packed = static_cast<uint32_t>(f2bf(r0)) | (static_cast<uint32_t>(f2bf(r1)) << 16);
-        *reinterpret_cast<uint32_t*>(vd + i2) = packed;
+        bool ok;
+        const size_t row = kv_row(p, l, b, head, pos, ok);
+        if (ok) {
+          const uint32_t packed = static_cast<uint32_t>(f2bf(r0)) | (static_cast<uint32_t>(f2bf(r1)) << 16);
+          *reinterpret_cast<uint32_t*>(p.vc + row + i2) = packed;
+        } else {
+          raise_error(p, kErrBadPage, where_code(ST_QKV, l, s));
+        }
       }
     }
   }
@@ -1640,8 +1651,24 @@ __device__ __forceinline__ void attn_item(const Params& p, const AttnPlan<B>& ap
   j = r - g * nch;
 }
 
-__device__ __forceinline__ size_t kv_row(const Params& p, int l, int b, int g, int t) {
-  return (((static_cast<size_t>(l) * p.B + b) * p.nkv + g) * p.max_seq + t) * p.d;
+// Element offset of cache row (layer l, sequence b, kv head g, position t).
+// Contiguous cache: [L][B][n_kv][max_seq][d].  Paged cache: a pool
+// [L][n_pages][n_kv][P][d] of pages of P positions (P = the attention chunk,
+// so a chunk is one page and one TMA box); positions [jP, (j+1)P) of
+// sequence b live in pool page page_table[b][j].  A page number outside the
+// pool gives offset 0 and ok = false: the caller skips the access and the
+// error is reported.
+__device__ __forceinline__ size_t kv_row(const Params& p, int l, int b, int g, int t, bool& ok) {
+  ok = true;
+  if (!p.page_table) return (((static_cast<size_t>(l) * p.B + b) * p.nkv + g) * p.max_seq + t) * p.d;
+  const int P = p.attn_pos_per_tile;
+  const int j = t / P;
+  const int pg = p.page_table[static_cast<size_t>(b) * p.pages_per_seq + j];
+  if (static_cast<unsigned>(pg) >= static_cast<unsigned>(p.n_pages)) {
+    ok = false;
+    return 0;
+  }
+  return ((((static_cast<size_t>(l) * p.n_pages + pg) * p.nkv + g) * P) + (t - j * P)) * p.d;
 }
 
 // Attention scratch in the activation region (the attention stage stages no
@@ -1756,10 +1783,13 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     if (have_tile && pg * 16 < npos) {   // warp-uniform
       if (npos > n_old && (n_old >> 4) == pg) {
         // this step's K/V entry of the head, from the cache (written by the QKV stage)
-        const size_t row = kv_row(p, l, b, g, T - 1);
+        bool row_ok;
+        const size_t row = kv_row(p, l, b, g, T - 1, row_ok);   // (a bad page was reported by the producer)
         const uint32_t ka = sw128_addr(kt, P, n_old, cx.lane * DV);
         const uint32_t va = sw128_addr(vt, P, n_old, cx.lane * DV);
-        if (DV == 4) {
+        if (!row_ok) {
+          // leave the chunk's row as loaded; the decode is abandoned
+        } else if (DV == 4) {
           const uint2 kk = __ldcg(reinterpret_cast<const uint2*>(p.kc + row + cx.lane * DV));
           const uint2 vv = __ldcg(reinterpret_cast<const uint2*>(p.vc + row + cx.lane * DV));
           asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(ka), "r"(kk.x), "r"(kk.y) : "memory");
@@ -2481,7 +2511,9 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         int b, g, j, nch, base;
         attn_item<B>(p, cu.ap, cu.a, b, g, j, nch, base);
         ++cu.a;
-        t.y = static_cast<int>(kv_row(p, cu.l, b, g, j * p.attn_pos_per_tile) / p.d);
+        bool ok;
+        t.y = static_cast<int>(kv_row(p, cu.l, b, g, j * p.attn_pos_per_tile, ok) / p.d);
+        if (!ok) raise_error(p, kErrBadPage, where_code(ST_ATTN, cu.l, cu.s));   // row 0 is read instead
         t.rows = min(p.attn_pos_per_tile, p.pos0[b] + cu.s + 1 - j * p.attn_pos_per_tile);
         t.src = nullptr;
         t.bytes = kTileBytes;

@@ -176,13 +176,17 @@ struct Params {
   Mat lm;
   const LayerParams* layers;    // device array [L]
 
-  // KV cache (caller-owned), bf16 [L][B][nkv][max_seq][d]; the tensor maps view
-  // each as a 2-D [L*B*nkv*max_seq rows][d] array read in 64-column boxes of
-  // attn_pos_per_tile rows with 128-byte swizzle
+  // KV cache (caller-owned), bf16 [L][B][nkv][max_seq][d], or paged: pools
+  // [L][n_pages][nkv][P][d] with P = attn_pos_per_tile; the tensor maps view
+  // each as a 2-D [rows][d] array read in 64-column boxes of P rows with
+  // 128-byte swizzle
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   uint16_t* kc;
   uint16_t* vc;
+  const int32_t* page_table;   // paged cache: [B][pages_per_seq] pool page of each chunk; null: contiguous
+  int pages_per_seq;
+  int n_pages;
   const float2* rope;           // [max_seq][d/2] (cos, sin)
 
   // workspace

@@ -505,6 +505,14 @@ xlpk_status validate_weights(const xlpk_config* c, const xlpk_weights* w, const 
     return XLPK_ERR_INVALID_ARG;
   if (!kv->k_dev || !kv->v_dev || !aligned16(kv->k_dev) || !aligned16(kv->v_dev))
     return XLPK_ERR_INVALID_ARG;
+  if (kv->page_table_dev) {
+    if ((reinterpret_cast<uintptr_t>(kv->page_table_dev) & 3u) || kv->page_size <= 0 || kv->n_pages <= 0)
+      return XLPK_ERR_INVALID_ARG;
+    // a page is one attention chunk (kTileBytes / 2 of K per chunk)
+    if (kv->page_size != (kTileBytes / 2) / (c->head_dim * 2)) return XLPK_ERR_UNSUPPORTED;
+  } else if (kv->page_size != 0 || kv->n_pages != 0) {
+    return XLPK_ERR_INVALID_ARG;
+  }
   if (!aligned16(w->embed_dev) || !aligned16(w->lm_head.w_dev)) return XLPK_ERR_INVALID_ARG;
   if (c->weight_dtype == XLPK_DTYPE_FP8_E4M3) {
     // every linear weight carries its block scales
@@ -943,9 +951,14 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.layers = e->d_layers;
   p.kc = static_cast<uint16_t*>(kv->k_dev);
   p.vc = static_cast<uint16_t*>(kv->v_dev);
+  p.page_table = kv->page_table_dev;
+  p.n_pages = kv->page_table_dev ? kv->n_pages : 0;
+  p.pages_per_seq = (c.max_seq + e->P - 1) / e->P;
   {
     const unsigned long long rows =
-        static_cast<unsigned long long>(c.n_layers) * B * c.n_kv_heads * static_cast<unsigned long long>(c.max_seq);
+        kv->page_table_dev
+            ? static_cast<unsigned long long>(c.n_layers) * kv->n_pages * c.n_kv_heads * static_cast<unsigned long long>(e->P)
+            : static_cast<unsigned long long>(c.n_layers) * B * c.n_kv_heads * static_cast<unsigned long long>(c.max_seq);
     xlpk_status st = encode_kv_map(&p.tmap_k, kv->k_dev, rows, d, e->P);
     if (st != XLPK_OK) return st;
     st = encode_kv_map(&p.tmap_v, kv->v_dev, rows, d, e->P);
@@ -1271,9 +1284,13 @@ xlpk_status xlpk_get_status(xlpk_handle h) {
   XLPK_CUDA(cudaMemset(h->base.abort_flag, 0, sizeof(int)));
   XLPK_CUDA(cudaDeviceSynchronize());
   h->step_base = 0;
-  char buf[128];
-  std::snprintf(buf, sizeof(buf), "device wait failed: stage %d layer %d step %d cta %d", st[1] & 0xff,
-                (st[1] >> 8) & 0xff, (st[1] >> 16) & 0x7fff, st[2]);
+  char buf[160];
+  if (st[0] == XLPK_ERR_INVALID_ARG)
+    std::snprintf(buf, sizeof(buf), "a KV page-table entry outside the pool: stage %d layer %d step %d cta %d",
+                  st[1] & 0xff, (st[1] >> 8) & 0xff, (st[1] >> 16) & 0x7fff, st[2]);
+  else
+    std::snprintf(buf, sizeof(buf), "device wait failed: stage %d layer %d step %d cta %d", st[1] & 0xff,
+                  (st[1] >> 8) & 0xff, (st[1] >> 16) & 0x7fff, st[2]);
   g_cuda_err = buf;
   return static_cast<xlpk_status>(st[0]);
 }

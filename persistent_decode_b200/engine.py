@@ -94,10 +94,16 @@ class Engine:
     """
 
     def __init__(self, cfg, weights: Dict[str, "object"], k_cache, v_cache, n_ctas: int = 0,
-                 spin_limit_us: int = 0, flags: int = 0, window: int = 0):
+                 spin_limit_us: int = 0, flags: int = 0, window: int = 0, page_table=None,
+                 max_seq: Optional[int] = None):
         self.cfg = cfg
-        self.B = int(k_cache.shape[1])
-        self.max_seq = int(k_cache.shape[3])
+        if page_table is None:
+            self.B = int(k_cache.shape[1])
+            self.max_seq = int(k_cache.shape[3])
+        else:
+            # paged: pools [L][n_pages][n_kv][page][d], page_table int32 [B][pages per sequence]
+            self.B = int(page_table.shape[0])
+            self.max_seq = int(max_seq if max_seq is not None else page_table.shape[1] * k_cache.shape[3])
         self._c = make_config(cfg, n_ctas, spin_limit_us, batch=self.B, max_seq=self.max_seq, flags=flags,
                               window=window)
         L = cfg.n_layers
@@ -139,8 +145,12 @@ class Engine:
                 lw.w_gate, lw.w_up, lw.w_down = lin(p + "w_gate"), lin(p + "w_up"), lin(p + "w_down")
         self._w = _abi.xlpk_weights(_ptr(weights["embed"]), _ptr(weights["final_norm"]),
                                     lin("lm_head"), self._layers)
-        self._kv = _abi.xlpk_kv(_ptr(k_cache), _ptr(v_cache))
-        self._refs = (weights, k_cache, v_cache)
+        if page_table is None:
+            self._kv = _abi.xlpk_kv(_ptr(k_cache), _ptr(v_cache), 0, 0, 0)
+        else:
+            self._kv = _abi.xlpk_kv(_ptr(k_cache), _ptr(v_cache), _ptr(page_table), int(k_cache.shape[3]),
+                                    int(k_cache.shape[1]))
+        self._refs = (weights, k_cache, v_cache, page_table)
         h = C.c_void_p()
         _check(lib.xlpk_create(C.byref(self._c), C.byref(self._w), C.byref(self._kv), C.byref(h)),
                "xlpk_create")

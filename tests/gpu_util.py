@@ -107,7 +107,7 @@ def oracle_for(m: workload.GpuModel, max_seq: Optional[int] = None, memo: bool =
     cfg = m.cfg
     w = HostWeights(m.weights)
     cls = MemoOracle if memo else OracleDecoder
-    o = cls(cfg, w, cfg.batch, max_seq=max_seq or m.k.shape[3])
+    o = cls(cfg, w, cfg.batch, max_seq=max_seq or m.engine.max_seq)
     if cfg.prefill:
         o.forward_sequence(m.prompt[:, : cfg.kv_len])
     else:
