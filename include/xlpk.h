@@ -290,6 +290,46 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
  * checked by (the pages are silent; a debug output of the boundary). */
 xlpk_status xlpk_debug_logits(xlpk_handle h, float* logits_dev, float* hidden_dev);
 
+/* Device-resident request loop ("serve mode").  xlpk_serve_start launches the
+ * persistent kernel once; it stays resident and decodes whatever steps the
+ * host posts, with no launch per request.  The host posts a request with
+ * xlpk_serve_post (a count of further greedy steps, written to a word in
+ * host-mapped memory); the kernel's first CTA polls that word, forwards it to
+ * the other CTAs through a device counter, decodes the steps, and publishes
+ * each step's tokens and a completed-step count to host-mapped memory, which
+ * xlpk_serve_wait reads.  While no request is pending the kernel waits at most
+ * idle_limit_us and then leaves on its own; a later post (or a wait that finds
+ * it gone) launches it again from the handle's state, transparently.  Every
+ * wait on the device is bounded.  During a session the handle's other decode
+ * calls and xlpk_set_state return XLPK_ERR_INVALID_ARG.
+ * Source: a GPU-resident scheduler drives the decode loop and the host only
+ * posts descriptors into a ring the kernel claims ("Persistent execution
+ * paradigm", section 5.6); device-resident request descriptors and work queue
+ * ("XL-Persistent-Kernel", features to be implemented). */
+
+/* Open a session on `stream` from the handle's current state (xlpk_set_state):
+ * allocates the mapped control words and token ring once per handle (pinned
+ * host memory) and launches the loop.  idle_limit_us > 0. */
+xlpk_status xlpk_serve_start(xlpk_handle h, int32_t idle_limit_us, void* stream);
+
+/* Post a request for n_steps more greedy steps (> 0) of every sequence;
+ * *first_step receives the session index of its first step (steps are
+ * numbered from 0 in posting order).  Returns without waiting;
+ * XLPK_ERR_KV_FULL if the session's steps would pass max_seq. */
+xlpk_status xlpk_serve_post(xlpk_handle h, int32_t n_steps, int64_t* first_step);
+
+/* Wait (host polling, at most timeout_us) until session steps
+ * [first_step, first_step + n_steps) are decoded and copy their tokens
+ * [n_steps][B] to tokens_out_host.  XLPK_ERR_TIMEOUT if they are not done in
+ * time; a device-side failure of the loop is returned as its status. */
+xlpk_status xlpk_serve_wait(xlpk_handle h, int64_t first_step, int32_t n_steps, int32_t* tokens_out_host,
+                            int32_t timeout_us);
+
+/* Ask the loop to leave once every posted step is decoded, wait for it, fold
+ * the session's steps into the handle's state (a later xlpk_decode continues
+ * after them) and close the session.  Returns the loop's device status. */
+xlpk_status xlpk_serve_stop(xlpk_handle h);
+
 /* End-to-end call with host buffers: uploads the state, decodes, downloads
  * tokens_out_host [n_steps][B], and synchronises `stream`.  Returns the
  * device status of the decode.

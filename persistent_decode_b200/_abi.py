@@ -82,6 +82,10 @@ SIGNATURES = {
     "xlpk_decode_noalloc": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p,
                                         C.POINTER(xlpk_decode_io), C.c_void_p]),
     "xlpk_debug_logits": (C.c_int32, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "xlpk_serve_start": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p]),
+    "xlpk_serve_post": (C.c_int32, [C.c_void_p, C.c_int32, C.POINTER(C.c_int64)]),
+    "xlpk_serve_wait": (C.c_int32, [C.c_void_p, C.c_int64, C.c_int32, C.POINTER(C.c_int32), C.c_int32]),
+    "xlpk_serve_stop": (C.c_int32, [C.c_void_p]),
     "xlpk_generate": (C.c_int32, [C.c_void_p, C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.c_int32,
                                   C.POINTER(C.c_int32), C.c_void_p]),
     "xlpk_get_status": (C.c_int32, [C.c_void_p]),

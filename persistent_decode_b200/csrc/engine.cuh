@@ -205,6 +205,16 @@ __device__ __forceinline__ int ld_volatile(const int* p) {
   asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned ld_acquire_sys(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_acquire_s32(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
@@ -401,6 +411,57 @@ __device__ __forceinline__ bool stage_wait(const Params& p, Ctx& cx, const unsig
     trace_stamp(p, s, stage_index(p, kind, l), 1);
   }
   return !consumer_sync_any(cx.ctl->abort != 0);
+}
+
+// ------------------------------------------------------------------ serve mode
+
+// Whether launch step s of a serve launch may run: 1 (requested), -1 (every
+// CTA stops at or before s), 0 (not decided yet).
+__device__ __forceinline__ int serve_state(const Params& p, int s) {
+  if (static_cast<int>(ld_acquire(p.serve_req_dev) - static_cast<unsigned>(p.serve_step0 + s + 1)) >= 0) return 1;
+  const int st = ld_acquire_s32(p.serve_stop_dev);
+  return st >= 0 && st <= s ? -1 : 0;
+}
+
+// Block (bounded) until launch step s is decided; true if it runs.  CTA 0's
+// first consumer thread is the poller: it reads the host-mapped request word,
+// forwards it, and decides the stop after serve_idle_ns without a request or
+// when the host asks to leave; every other waiter follows the device words,
+// with a limit above the poller's.
+__device__ __noinline__ bool serve_gate(const Params& p, SmemCtl* ctl, int s, bool poller) {
+  const unsigned want = static_cast<unsigned>(p.serve_step0 + s + 1);
+  const uint64_t t0 = globaltimer();
+  unsigned nap = 32;
+  for (;;) {
+    if (poller) {
+      const unsigned r = ld_acquire_sys(p.serve_req_host);
+      if (static_cast<int>(r - want) >= 0) {
+        __threadfence();
+        atomicMax(p.serve_req_dev, r);
+        return true;
+      }
+      const long long idle = static_cast<long long>(globaltimer() - t0);
+      if (*reinterpret_cast<const volatile int*>(p.serve_exit_host) || idle > p.serve_idle_ns) {
+        atomicExch(p.serve_stop_dev, s);
+        __threadfence();
+        return false;
+      }
+    } else {
+      const int st = serve_state(p, s);
+      if (st != 0) return st > 0;
+      if (static_cast<long long>(globaltimer() - t0) > p.serve_idle_ns + p.spin_limit_ns) {
+        raise_error(p, kErrTimeout, where_code(ST_QKV, 0, s) | (1 << 13));
+        ctl->abort = 1;
+        return false;
+      }
+    }
+    if (ctl->abort || ld_volatile(p.abort_flag)) {
+      ctl->abort = 1;
+      return false;
+    }
+    __nanosleep(nap);
+    if (nap < 1024) nap <<= 1;
+  }
 }
 
 // ------------------------------------------------------------------ math
@@ -2142,10 +2203,21 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
           }
           p.tokens_out[static_cast<size_t>(s) * p.B + b] = ix;
           p.cur_tok[b] = nxt;
+          if (p.serve)
+            p.serve_tokens_host[static_cast<size_t>((p.serve_step0 + s) % p.serve_cap) * p.B + b] = ix;
         }
       }
       consumer_sync();
-      if (cx.tid == 0) release_add(p.cnt + p.cl.step_done, 1u);
+      if (cx.tid == 0) {
+        release_add(p.cnt + p.cl.step_done, 1u);
+        if (p.serve) {
+          // the step's tokens (written above, ordered by the barrier) before its count, to the host
+          __threadfence_system();
+          asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p.serve_done_host),
+                       "r"(static_cast<unsigned>(p.serve_step0 + s + 1))
+                       : "memory");
+        }
+      }
     }
     const bool ab = consumer_sync_any(cx.ctl->abort != 0);
     if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
@@ -2435,7 +2507,7 @@ __device__ __forceinline__ void cursor_next_stage(const Params& p, Cursor<B>& cu
   }
 }
 
-enum CursorResult : int { CUR_DONE = 0, CUR_TILE = 1, CUR_BLOCKED = 2, CUR_RUN = 3 };
+enum CursorResult : int { CUR_DONE = 0, CUR_TILE = 1, CUR_BLOCKED = 2, CUR_RUN = 3, CUR_REQ = 4 };
 
 // A dense GEMV stage of one CTA is one contiguous byte range: n1 tiles of b1
 // bytes (full groups of 8 row pairs), then n2 tiles of b2 bytes (the last,
@@ -2450,6 +2522,15 @@ struct Run {
 template <int B, bool MOE>
 __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>& cu, Tile& t, Run* run) {
   while (!cu.done) {
+    if (p.serve && !cu.open && !cu.one_stage && cu.kind == ST_QKV && cu.l == 0) {
+      // serve mode: a step's tiles are streamed once the step is requested
+      const int st = serve_state(p, cu.s);
+      if (st < 0) {
+        cu.done = true;
+        break;
+      }
+      if (st == 0) return CUR_REQ;
+    }
     const bool moe = MOE && (cu.kind == ST_GATEUP || cu.kind == ST_DOWN);
     if (!cu.open) {
       cu.open = true;
@@ -2717,6 +2798,12 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
     int t_stage, t_layer, t_step, t_y = 0;
     if (r_n1 + r_n2 == 0) {
       int r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+      while (r == CUR_REQ) {
+        // serve mode: the next step is not requested yet (bounded wait)
+        if (!serve_gate(p, cx.ctl, cc.s, false) && serve_state(p, cc.s) >= 0) break;
+        r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+      }
+      if (r == CUR_REQ) break;
       if (r == CUR_BLOCKED) {
         // the next tile is an expert chosen by this CTA's own consumers: wait
         // (bounded) until they publish the layer's routing
@@ -2764,7 +2851,7 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
         continue;
       }
       const int pr = cursor_next<B, MOE>(p, cx.c, cx.ctl, pc, tp, &prun);
-      if (pr == CUR_BLOCKED) break;   // resume once the routing is known
+      if (pr == CUR_BLOCKED || pr == CUR_REQ) break;   // resume once the routing / the request is known
       if (pr == CUR_RUN) {
         pf_src = prun.src;
         pf_left = static_cast<long long>(prun.n1) * prun.b1 + static_cast<long long>(prun.n2) * prun.b2;
@@ -2832,6 +2919,11 @@ __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
   RingPos rp;
   if (fused) {
     for (int s = 0; s < p.n_steps; ++s) {
+      if (p.serve) {
+        // serve mode: run step s only once the host has asked for it
+        const bool go = cx.tid == 0 ? serve_gate(p, cx.ctl, s, cx.c == 0) : true;
+        if (consumer_sync_any(!go)) return;
+      }
       for (int l = 0; l < p.L; ++l)
         for (int k = 0; k < ST_LAYER; ++k)
           if (!consume_stage<B, D, MOE>(p, cx, k, l, s, rp, true)) return;

@@ -232,6 +232,23 @@ struct Params {
   unsigned long long* trace;   // optional stage timestamps
   int fault_drop_stage;        // failure-detection tests: CTA 0 withholds its release of this
                                // stage index at the call's first step (-1: never)
+
+  // Device-resident request loop (serve mode): launch step s runs once the
+  // host has asked for more than serve_step0 + s steps of the session.  CTA 0's
+  // first consumer thread polls the host-mapped request word and forwards it to
+  // serve_req_dev, which every other CTA polls; when no request comes for
+  // serve_idle_ns (or the host asks to leave while idle), CTA 0 names the step
+  // at which every CTA stops (serve_stop_dev) and the launch ends.
+  int serve;
+  int serve_step0;                  // session index of this launch's step 0
+  const unsigned* serve_req_host;   // host-mapped: steps requested in the session
+  const int* serve_exit_host;       // host-mapped: 1 = leave when idle
+  unsigned* serve_done_host;        // host-mapped: steps completed in the session
+  int32_t* serve_tokens_host;       // host-mapped ring [serve_cap][B]: token of session step t at t % cap
+  int serve_cap;
+  unsigned* serve_req_dev;          // workspace: the request count as CTA 0 forwarded it
+  int* serve_stop_dev;              // workspace: launch step at which every CTA leaves (-1: none yet)
+  long long serve_idle_ns;
 };
 
 }  // namespace xlpk

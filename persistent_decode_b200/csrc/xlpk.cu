@@ -14,6 +14,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -242,6 +244,19 @@ struct xlpk_engine {
   int64_t weight_bytes_per_step = 0;
   float* dbg_logits = nullptr;   // parity mode (xlpk_debug_logits): [B][V], [B][H], last step's
   float* dbg_hidden = nullptr;
+  // serve mode (xlpk_serve_*)
+  unsigned* serve_ctl = nullptr;     // host-mapped words: [0] requested, [1] leave, [2] done
+  int32_t* serve_tokens = nullptr;   // host-mapped token ring [serve_cap][B]
+  unsigned* serve_ctl_dev = nullptr; // the same memory as the device sees it
+  int32_t* serve_tokens_dev = nullptr;
+  int serve_cap = 0;
+  bool serve_active = false;         // a session is open
+  bool serve_launched = false;       // a serve launch may still be running
+  cudaStream_t serve_stream = nullptr;
+  long long serve_posted = 0;        // steps requested in the session
+  long long serve_step0 = 0;         // session steps done before the current launch
+  long long serve_idle_ns = 0;
+  unsigned* serve_dev_words = nullptr;   // workspace: [0] forwarded request count, [1] stop step
 };
 
 namespace {
@@ -562,6 +577,8 @@ void fill_rope(std::vector<float2>& t, int max_seq, int d, double theta) {
 
 void free_engine(xlpk_engine* e) {
   if (!e) return;
+  if (e->serve_ctl) cudaFreeHost(e->serve_ctl);
+  if (e->serve_tokens) cudaFreeHost(e->serve_tokens);
   cudaFree(e->packed);
   cudaFree(e->ws);
   cudaFree(e->d_layers);
@@ -908,6 +925,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const size_t o_st = take(sizeof(int) * 4);
   const size_t o_ab = take(sizeof(int));
   const size_t o_ts = take(sizeof(int) * static_cast<size_t>(c.max_seq) * B);
+  const size_t o_sv = take(sizeof(unsigned) * 2);
   e->ws_bytes = off;
   XLPK_CUDA(cudaMalloc(&e->ws, e->ws_bytes));
   XLPK_CUDA(cudaMemset(e->ws, 0, e->ws_bytes));
@@ -995,6 +1013,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.status = reinterpret_cast<int*>(e->ws + o_st);
   p.abort_flag = reinterpret_cast<int*>(e->ws + o_ab);
   e->tok_scratch = reinterpret_cast<int32_t*>(e->ws + o_ts);
+  e->serve_dev_words = reinterpret_cast<unsigned*>(e->ws + o_sv);
   e->pos.assign(B, 0);
   XLPK_CUDA(cudaDeviceSynchronize());
   return XLPK_OK;
@@ -1002,6 +1021,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
 
 xlpk_status check_decode_args(xlpk_engine* h, int32_t n_steps, int32_t* tokens_out) {
   if (!h || n_steps < 0) return XLPK_ERR_INVALID_ARG;
+  if (h->serve_active) return XLPK_ERR_INVALID_ARG;   // the serve loop owns the handle
   if (n_steps > 0 && !tokens_out) return XLPK_ERR_INVALID_ARG;
   for (int b = 0; b < h->cfg.batch; ++b)
     if (static_cast<long long>(h->pos[b]) + n_steps > h->cfg.max_seq) return XLPK_ERR_KV_FULL;
@@ -1102,9 +1122,147 @@ xlpk_status noalloc_scratch(int dev, unsigned char** out) {
   return XLPK_OK;
 }
 
+// ---- serve mode: one persistent launch that stays resident across requests
+
+// Steps of the current serve launch the host has seen completed.
+long long serve_done(const xlpk_engine* h) {
+  return static_cast<long long>(*reinterpret_cast<const volatile unsigned*>(h->serve_ctl + 2));
+}
+
+// Launch the serve loop from the handle's current state (session step serve_step0).
+xlpk_status serve_launch(xlpk_engine* h) {
+  const xlpk_config& c = h->cfg;
+  int room = c.max_seq;
+  for (int b = 0; b < c.batch; ++b) room = std::min(room, c.max_seq - h->pos[b]);
+  if (room <= 0) return XLPK_ERR_KV_FULL;
+  Params p = call_params(h, room, h->tok_scratch, nullptr);
+  p.serve = 1;
+  p.serve_step0 = static_cast<int>(h->serve_step0);
+  p.serve_req_host = h->serve_ctl_dev;
+  p.serve_exit_host = reinterpret_cast<const int*>(h->serve_ctl_dev + 1);
+  p.serve_done_host = h->serve_ctl_dev + 2;
+  p.serve_tokens_host = h->serve_tokens_dev;
+  p.serve_cap = h->serve_cap;
+  p.serve_req_dev = h->serve_dev_words;
+  p.serve_stop_dev = reinterpret_cast<int*>(h->serve_dev_words + 1);
+  p.serve_idle_ns = h->serve_idle_ns;
+  const unsigned init[2] = {static_cast<unsigned>(h->serve_step0), 0xffffffffu};   // forwarded = done; no stop
+  XLPK_CUDA(cudaMemcpyAsync(h->serve_dev_words, init, sizeof(init), cudaMemcpyHostToDevice, h->serve_stream));
+  void* args[] = {&p};
+  XLPK_CUDA(cudaLaunchCooperativeKernel(h->kern_persistent, dim3(h->G), dim3(kThreads), args,
+                                        static_cast<size_t>(h->smem), h->serve_stream));
+  h->serve_launched = true;
+  h->last_stream = h->serve_stream;
+  return XLPK_OK;
+}
+
+// The current launch has ended: fold the steps it decoded into the handle's
+// state.  Returns the launch's device status.
+xlpk_status serve_collect(xlpk_engine* h) {
+  XLPK_CUDA(cudaStreamSynchronize(h->serve_stream));
+  h->serve_launched = false;
+  const long long done = serve_done(h);
+  const int n = static_cast<int>(done - h->serve_step0);
+  for (int b = 0; b < h->cfg.batch; ++b) h->pos[b] += n;
+  h->step_base += n;
+  h->serve_step0 = done;
+  return xlpk_get_status(h);
+}
+
 }  // namespace
 
 extern "C" {
+
+xlpk_status xlpk_serve_start(xlpk_handle h, int32_t idle_limit_us, void* stream) {
+  if (!h || idle_limit_us <= 0 || h->serve_active) return XLPK_ERR_INVALID_ARG;
+  if (h->cfg.n_experts > 0 && h->cfg.batch != 1) return XLPK_ERR_UNSUPPORTED;
+  if (!h->serve_ctl) {
+    void* ctl = nullptr;
+    void* tok = nullptr;
+    XLPK_CUDA(cudaHostAlloc(&ctl, 64, cudaHostAllocMapped));
+    h->serve_ctl = static_cast<unsigned*>(ctl);
+    h->serve_cap = h->cfg.max_seq;
+    XLPK_CUDA(cudaHostAlloc(&tok, sizeof(int32_t) * static_cast<size_t>(h->serve_cap) * h->cfg.batch,
+                            cudaHostAllocMapped));
+    h->serve_tokens = static_cast<int32_t*>(tok);
+    XLPK_CUDA(cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->serve_ctl_dev), h->serve_ctl, 0));
+    XLPK_CUDA(cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->serve_tokens_dev), h->serve_tokens, 0));
+  }
+  volatile unsigned* w = h->serve_ctl;
+  w[0] = 0u;
+  w[1] = 0u;
+  w[2] = 0u;
+  h->serve_posted = 0;
+  h->serve_step0 = 0;
+  h->serve_idle_ns = 1000LL * idle_limit_us;
+  h->serve_stream = static_cast<cudaStream_t>(stream);
+  h->serve_active = true;
+  const xlpk_status rc = serve_launch(h);
+  if (rc != XLPK_OK) h->serve_active = false;
+  return rc;
+}
+
+xlpk_status xlpk_serve_post(xlpk_handle h, int32_t n_steps, int64_t* first_step) {
+  if (!h || !h->serve_active || n_steps <= 0 || !first_step) return XLPK_ERR_INVALID_ARG;
+  // every step of the session must fit the cache
+  const long long pos_start = h->pos[0] - h->serve_step0;   // pos at the session start (sequence 0)
+  for (int b = 0; b < h->cfg.batch; ++b)
+    if (h->pos[b] - h->serve_step0 + h->serve_posted + n_steps > h->cfg.max_seq) return XLPK_ERR_KV_FULL;
+  (void)pos_start;
+  if (h->serve_launched && cudaStreamQuery(h->serve_stream) == cudaSuccess) {
+    // the loop left while idle: fold in its steps and start it again
+    const xlpk_status rc = serve_collect(h);
+    if (rc != XLPK_OK) return rc;
+  }
+  if (!h->serve_launched) {
+    const xlpk_status rc = serve_launch(h);
+    if (rc != XLPK_OK) return rc;
+  }
+  *first_step = h->serve_posted;
+  h->serve_posted += n_steps;
+  std::atomic_thread_fence(std::memory_order_release);
+  *reinterpret_cast<volatile unsigned*>(h->serve_ctl) = static_cast<unsigned>(h->serve_posted);
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_serve_wait(xlpk_handle h, int64_t first_step, int32_t n_steps, int32_t* tokens_out_host,
+                            int32_t timeout_us) {
+  if (!h || !h->serve_active || n_steps <= 0 || first_step < 0 || !tokens_out_host || timeout_us <= 0)
+    return XLPK_ERR_INVALID_ARG;
+  const long long target = first_step + n_steps;
+  if (target > h->serve_posted) return XLPK_ERR_INVALID_ARG;
+  const auto t0 = std::chrono::steady_clock::now();
+  while (serve_done(h) < target) {
+    if (h->serve_launched && cudaStreamQuery(h->serve_stream) == cudaSuccess && serve_done(h) < target) {
+      // the launch ended (idle) before our steps: start it again
+      xlpk_status rc = serve_collect(h);
+      if (rc != XLPK_OK) return rc;
+      rc = serve_launch(h);
+      if (rc != XLPK_OK) return rc;
+    }
+    if (std::chrono::duration_cast<std::chrono::microseconds>(std::chrono::steady_clock::now() - t0).count() >
+        timeout_us)
+      return XLPK_ERR_TIMEOUT;
+  }
+  std::atomic_thread_fence(std::memory_order_acquire);
+  const volatile int32_t* ring = h->serve_tokens;
+  const int B = h->cfg.batch;
+  for (long long t = first_step; t < target; ++t)
+    for (int b = 0; b < B; ++b)
+      tokens_out_host[(t - first_step) * B + b] = ring[(t % h->serve_cap) * B + b];
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_serve_stop(xlpk_handle h) {
+  if (!h || !h->serve_active) return XLPK_ERR_INVALID_ARG;
+  std::atomic_thread_fence(std::memory_order_release);
+  *reinterpret_cast<volatile unsigned*>(h->serve_ctl + 1) = 1u;
+  xlpk_status rc = XLPK_OK;
+  if (h->serve_launched) rc = serve_collect(h);
+  h->serve_active = false;
+  return rc;
+}
+
 
 xlpk_status xlpk_create(const xlpk_config* cfg, const xlpk_weights* weights, const xlpk_kv* kv,
                         xlpk_handle* out) {
@@ -1134,6 +1292,7 @@ xlpk_status xlpk_destroy(xlpk_handle h) {
 xlpk_status xlpk_set_state(xlpk_handle h, const int32_t* tokens_host, const int32_t* seq_lens_host,
                            void* stream) {
   if (!h || !tokens_host || !seq_lens_host) return XLPK_ERR_INVALID_ARG;
+  if (h->serve_active) return XLPK_ERR_INVALID_ARG;   // the serve loop owns the handle
   for (int b = 0; b < h->cfg.batch; ++b) {
     if (tokens_host[b] < 0 || tokens_host[b] >= h->cfg.vocab) return XLPK_ERR_INVALID_ARG;
     if (seq_lens_host[b] < 0 || seq_lens_host[b] >= h->cfg.max_seq) return XLPK_ERR_INVALID_ARG;

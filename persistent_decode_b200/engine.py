@@ -208,6 +208,26 @@ class Engine:
         self._dbg = (logits, hidden)   # borrowed by the library until replaced
         _check(lib.xlpk_debug_logits(self.h, _ptr(logits), _ptr(hidden)), "xlpk_debug_logits")
 
+    # ---- device-resident request loop (xlpk_serve_*)
+
+    def serve_start(self, idle_limit_us: int = 1_000_000, stream=None) -> None:
+        _check(lib.xlpk_serve_start(self.h, int(idle_limit_us), _stream_handle(stream)), "xlpk_serve_start")
+
+    def serve_post(self, n_steps: int) -> int:
+        """Post n_steps more greedy steps; returns the session index of the first."""
+        first = C.c_int64()
+        _check(lib.xlpk_serve_post(self.h, int(n_steps), C.byref(first)), "xlpk_serve_post")
+        return int(first.value)
+
+    def serve_wait(self, first_step: int, n_steps: int, timeout_us: int = 10_000_000):
+        """Wait for the posted steps; returns their tokens as a list of [B] lists."""
+        out = (C.c_int32 * (int(n_steps) * self.B))()
+        _check(lib.xlpk_serve_wait(self.h, int(first_step), int(n_steps), out, int(timeout_us)), "xlpk_serve_wait")
+        return [[out[s * self.B + b] for b in range(self.B)] for s in range(int(n_steps))]
+
+    def serve_stop(self) -> None:
+        _check(lib.xlpk_serve_stop(self.h), "xlpk_serve_stop")
+
     def status(self) -> int:
         return int(lib.xlpk_get_status(self.h))
 
