@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=0, help="override tokens per call (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (sequences per call)")
     ap.add_argument("--no-baselines", action="store_true", help="skip the unfused and CPU legs")
+    ap.add_argument("--serve", action="store_true",
+                    help="also time one-step requests through the resident loop against one launch per request")
     return ap.parse_args()
 
 
@@ -240,6 +242,52 @@ def workload_config(cfg, n):
             "l2": "inputs larger than L2 (all weights streamed every token)"}
 
 
+def serve_latency(dev, requests: int = 200):
+    """Round trip of one-step requests on the tiny decoder (latency-bound): one
+    decode launch per request (launch, token copy to the host, synchronise)
+    against the device-resident loop (post a request word, wait for its
+    token in host-mapped memory).  Both decode consecutive steps."""
+    import torch
+
+    import synth
+    from persistent_decode_b200 import workload
+    cfg = synth.get_config("tiny")
+    m = workload.build(cfg, device=dev, max_seq=cfg.kv_len + 2 * requests + 16)
+    tok = torch.empty(1, cfg.batch, dtype=torch.int32, device=dev)
+    out = torch.empty(1, cfg.batch, dtype=torch.int32).pin_memory()
+
+    def per_launch(n):
+        workload.reset_state(m)
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for _ in range(n):
+            m.engine.decode(1, tok)
+            out.copy_(tok)            # synchronous copy: the token is on the host
+        return (time.perf_counter() - t0) / n
+
+    def resident(n):
+        workload.reset_state(m)
+        torch.cuda.synchronize(dev)
+        m.engine.serve_start(idle_limit_us=2_000_000)
+        try:
+            t0 = time.perf_counter()
+            for _ in range(n):
+                m.engine.serve_wait(m.engine.serve_post(1), 1)
+            dt = (time.perf_counter() - t0) / n
+        finally:
+            m.engine.serve_stop()
+        return dt
+
+    per_launch(16)
+    resident(16)
+    a = per_launch(requests)
+    b = resident(requests)
+    m.engine.check()
+    return {"workload": "tiny, batch 1, one greedy step per request", "requests": requests,
+            "launch_per_request_us": round(a * 1e6, 2), "resident_loop_us": round(b * 1e6, 2),
+            "speedup": round(a / b, 3)}
+
+
 # ----------------------------------------------------------------- main arm
 
 def main():
@@ -373,6 +421,8 @@ def main():
                             "steps_timed": un_steps, "launches_per_token": info.kernels_per_step_unfused,
                             "persistent_speedup": round(un_tpot / tpot_ms, 3),
                             "persistent_speedup_vs_graph": round(un_graph / tpot_ms, 3)}
+    if args.serve:
+        extra["serve_loop"] = serve_latency(dev)
     cpu = None
     if rank == 0 and world == 1 and not args.no_baselines:
         o, head, nl = build_cpu_sample(cfg, dev)
