@@ -156,6 +156,20 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   hi = *reinterpret_cast<const uint32_t*>(&h);
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
+// The same split into fp16 terms (11 significant bits each, for the fp16
+// tensor-core operands of FP8 models at batch 8).
+__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // Shared address of element (row r, dim d) of a K or V chunk of P rows as the
 // 128-byte-swizzled TMA boxes lay it out: box d/64 holds [P][64 dims]; the
 // 16-byte unit u of row r sits at unit u ^ (r % 8).
@@ -1076,7 +1090,8 @@ __device__ __noinline__ void load_side(const Params& p, Ctx& cx, int side, int s
 // squares of the raw values are added to ss (the RMSNorm factor is formed once
 // every window has been staged).  `hidden_dbg` receives the raw input.
 __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src, const float* gsrc, int K, int k0,
-                                            int Kw, const float* gain, float* hidden_dbg, float (&ss)[kMaxBatch]) {
+                                            int Kw, const float* gain, float* hidden_dbg, float (&ss)[kMaxBatch],
+                                            bool f16) {
   constexpr int B = kMaxBatch;
   const uint32_t act_s = smem_addr(cx.act);
   const int nv = Kw >> 3;   // 8-column vectors of the window
@@ -1124,7 +1139,12 @@ __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src
       const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       uint32_t h2[4], l2[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) split_bf16x2(e[2 * t] * gv[2 * t], e[2 * t + 1] * gv[2 * t + 1], h2[t], l2[t]);
+      for (int t = 0; t < 4; ++t) {
+        if (f16)
+          split_f16x2(e[2 * t] * gv[2 * t], e[2 * t + 1] * gv[2 * t + 1], h2[t], l2[t]);
+        else
+          split_bf16x2(e[2 * t] * gv[2 * t], e[2 * t + 1] * gv[2 * t + 1], h2[t], l2[t]);
+      }
       const uint32_t dst = act_s + jb * 2048 + b * 128 + ((q ^ b) << 4);
       asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(h2[0]), "r"(h2[1]), "r"(h2[2]),
                    "r"(h2[3])
@@ -1139,10 +1159,11 @@ __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src
   consumer_sync();
 }
 
-// Widen an FP8 tile in its ring slot to bf16 boxes in place: nb e4m3 boxes of
-// [rv][128 codes] (+ the rows' scales) become 2*nb bf16 boxes of [rv][64],
-// the codes times their block scale rounded to bf16, same swizzle.  Every
-// consumer thread reads its units before any is overwritten.
+// Widen an FP8 tile in its ring slot to fp16 boxes in place: nb e4m3 boxes of
+// [rv][128 codes] (+ the rows' scales) become 2*nb fp16 boxes of [rv][64],
+// the codes times their block scale rounded to fp16 (11 significant bits;
+// the MMAs of FP8 models take fp16 operands), same swizzle.  Every consumer
+// thread reads its units before any is overwritten.
 __device__ __noinline__ void tc_widen_fp8(Ctx& cx, uint32_t slot_s, int rv, int nb) {
   constexpr int kMaxUnits = 4;   // 16-byte code units per thread: nb * rv * 8 <= 1024
   const int nu = nb * rv * 8;
@@ -1170,8 +1191,8 @@ __device__ __noinline__ void tc_widen_fp8(Ctx& cx, uint32_t slot_s, int rv, int 
       for (int h = 0; h < 4; ++h) {
         const float2 a = e4m3x2_to_float2(w[h] & 0xffffu);
         const float2 c = e4m3x2_to_float2(w[h] >> 16);
-        o[2 * h] = pack_bf16x2(a.x * sc[t], a.y * sc[t]);
-        o[2 * h + 1] = pack_bf16x2(c.x * sc[t], c.y * sc[t]);
+        o[2 * h] = pack_f16x2(a.x * sc[t], a.y * sc[t]);
+        o[2 * h + 1] = pack_f16x2(c.x * sc[t], c.y * sc[t]);
       }
       // columns 16q..16q+15 -> bf16 box 2j + q/4, its 8-column units 2(q%4), 2(q%4)+1
       const uint32_t box = slot_s + (2 * j + (q >> 2)) * rv * 128 + r * 128;
@@ -1212,7 +1233,7 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
   const int bc = tc_box_cols(fp8), kbox = tc_kbox(K, win, fp8);
   const int nw = win > 0 ? (K + win - 1) / win : 1;
   const bool issuer = cx.warp == 4 && cx.lane == 0;
-  const uint32_t idesc = tc_idesc_bf16(128, kTcAccCols);
+  const uint32_t idesc = tc_idesc(128, kTcAccCols, fp8 != 0);   // FP8 weights: fp16 operands
   const uint32_t tmem = cx.ctl->tmem_base;
   float ss[B];
 #pragma unroll
@@ -1224,7 +1245,7 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
       if (!cx.ctl->abort) ring_wait(p, cx.ctl, smem_addr(&cx.ctl->bop_bar), cx.bop_phase, where);
       cx.bop_phase ^= 1u;
     }
-    tc_stage_input(p, cx, src, gsrc, K, k0, Kw, gain, hidden_dbg, ss);
+    tc_stage_input(p, cx, src, gsrc, K, k0, Kw, gain, hidden_dbg, ss, fp8 != 0);
     if (issuer) tc_fence_after();
     for (int mt = 0; mt < nm; ++mt) {
       const int rv = min(128, R - 128 * mt);

@@ -26,12 +26,13 @@ __device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, shape M x N.
-__host__ __device__ constexpr uint32_t tc_idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+// Instruction descriptor of kind::f16: fp32 accumulator, A and B both bf16
+// (or both fp16 with `f16`), both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool f16 = false) {
+  return (1u << 4) | (f16 ? 0u : (1u << 7) | (1u << 10)) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
+__host__ __device__ constexpr uint32_t tc_idesc_bf16(int M, int N) { return tc_idesc(M, N, false); }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
