@@ -94,7 +94,12 @@ typedef struct xlpk_config {
 enum {
   XLPK_FLAG_NO_FUSED_FFN = 1,      /* bf16 dense layers at batch <= 2: gate/up and down as two stages
                                       instead of one fused stage with a split-K down projection */
-  XLPK_FLAG_NO_TENSOR_CORES = 2    /* batch 8: CUDA-core GEMV tiles instead of tcgen05 MMAs */
+  XLPK_FLAG_NO_TENSOR_CORES = 2,   /* batch 8: CUDA-core GEMV tiles instead of tcgen05 MMAs */
+  XLPK_FLAG_FLOAT_FFN_REDUCE = 4   /* fused FFN: add the down projection's split-K partial sums into an
+                                      fp32 residual with float atomics instead of a 64-bit fixed-point
+                                      accumulator with integer atomics; fewer atomic operations, but
+                                      the rounding then depends on arrival order, so runs are not
+                                      bit-identical */
 };
 
 /* One linear weight: y = W x with W row-major [N][K] (PyTorch Linear layout).

@@ -23,6 +23,7 @@ XLPK_DTYPE_FP8_E4M3 = 1
 
 XLPK_FLAG_NO_FUSED_FFN = 1
 XLPK_FLAG_NO_TENSOR_CORES = 2
+XLPK_FLAG_FLOAT_FFN_REDUCE = 4
 
 
 class xlpk_config(C.Structure):

@@ -592,7 +592,7 @@ __device__ __forceinline__ void resid_rows(const Params& p, int c, int& r0, int&
 // The residual as the next layer's QKV stage and the LM head read it: the
 // fixed-point accumulator in the fused-FFN layers, else the two-plane x.
 __device__ __forceinline__ const void* resid_src(const Params& p) {
-  return p.ffn_fused ? static_cast<const void*>(p.xacc) : static_cast<const void*>(p.x);
+  return p.resid_fixed ? static_cast<const void*>(p.xacc) : static_cast<const void*>(p.x);
 }
 
 // Stage the input vector and the epilogue's side data in shared memory.  A
@@ -640,7 +640,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     const int e0 = r0 & ~7, e1 = (r1 + 7) & ~7;
     if (side == SIDE_ROPE) total += B * rope_bytes;
     if (side == SIDE_RESID)
-      total += p.ffn_fused ? static_cast<uint32_t>(B) * (r1 - r0) * 8u : static_cast<uint32_t>(B) * 2u * nv * 16u;
+      total += p.resid_fixed ? static_cast<uint32_t>(B) * (r1 - r0) * 8u : static_cast<uint32_t>(B) * 2u * nv * 16u;
     if (side == SIDE_EMBED && r1 > r0) total += static_cast<uint32_t>(B) * (e1 - e0) * 2u;
     mbar_expect_tx(bar, total);
     if (src != SRC_EMBED && !direct)
@@ -651,7 +651,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
       for (int b = 0; b < B; ++b)
         bulk_g2s_nohint(side_s + p.side_rope + b * rope_bytes,
                         p.rope + static_cast<size_t>(p.pos0[b] + s) * (p.d >> 1), rope_bytes, bar);
-    } else if (side == SIDE_RESID && p.ffn_fused && r1 > r0) {
+    } else if (side == SIDE_RESID && p.resid_fixed && r1 > r0) {
 #pragma unroll
       for (int b = 0; b < B; ++b)
         bulk_g2s_nohint(side_s + p.side_resid + b * p.rows_side * 8, p.xacc + static_cast<size_t>(b) * p.H + r0,
@@ -1417,7 +1417,7 @@ struct EpiResid {
         const uint32_t e =
             *reinterpret_cast<const uint32_t*>(side + p.side_embed + b * p.evb + (r - (r0 & ~7)) * 2);
         base = make_float2(bf16_lo(e), bf16_hi(e));
-      } else if (p.ffn_fused) {
+      } else if (p.resid_fixed) {
         const longlong2 q =
             *reinterpret_cast<const longlong2*>(side + p.side_resid + (b * p.rows_side + (r - r0)) * 8);
         base = make_float2(from_fixed(q.x), from_fixed(q.y));
@@ -1427,7 +1427,7 @@ struct EpiResid {
                                                 (r & 3));
       }
       const float2 v = make_float2(base.x + a0[b], base.y + a1[b]);
-      if (p.ffn_fused)
+      if (p.resid_fixed)
         *reinterpret_cast<longlong2*>(p.xacc + static_cast<size_t>(b) * p.H + r) = make_longlong2(to_fixed(v.x), to_fixed(v.y));
       else
         *reinterpret_cast<float2*>(p.x + plane_index(b, r, p.B, p.H)) = v;
@@ -1513,6 +1513,24 @@ __device__ __noinline__ void consume_downT(const Params& p, Ctx& cx, RingPos& rp
     __syncwarp();
     if (cx.lane == 0 && ok) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));   // this warp is done with it
     rp.next(p.nslot);
+  }
+  if (!p.resid_fixed) {
+    // fp32 residual: vector float atomics (the sum's rounding depends on the
+    // order in which the CTAs arrive)
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int v = cx.tid + q * kConsumerThreads;
+      if (v < V8) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          float4* x0 = reinterpret_cast<float4*>(p.x + plane_index(b, 8 * v, p.B, p.H));
+          float4* x1 = reinterpret_cast<float4*>(p.x + plane_index(b, 8 * v + 4, p.B, p.H));
+          atomicAdd(x0, make_float4(acc[q][0][b], acc[q][1][b], acc[q][2][b], acc[q][3][b]));
+          atomicAdd(x1, make_float4(acc[q][4][b], acc[q][5][b], acc[q][6][b], acc[q][7][b]));
+        }
+      }
+    }
+    return;
   }
   // The partial sums go to the fixed-point accumulator: first through shared
   // memory (the activation region, unused since the gate/up GEMV), so that
@@ -2177,7 +2195,8 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
     }
     if (!on_tc) {
       float rn[B];
-      load_act<B>(p, cx, p.H, p.ffn_fused ? SRC_FIXED : SRC_RESID, resid_src(p), p.final_norm, hid, SIDE_NONE, s, rn, where);
+      load_act<B>(p, cx, p.H, p.resid_fixed ? SRC_FIXED : SRC_RESID, resid_src(p), p.final_norm, hid, SIDE_NONE, s, rn,
+                  where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       consume_gemv<B>(p, cx, p.lm, rp, where, rn, epi);
     }
@@ -2302,7 +2321,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       } else {
         ok = stage_wait(p, cx, p.cnt + (l - 1) * ST_LAYER + ffn_done, G * S1, where, fused);
         if (!ok) return false;
-        load_act<B>(p, cx, p.H, p.ffn_fused ? SRC_FIXED : SRC_RESID, resid_src(p), L.attn_norm, nullptr, SIDE_ROPE, s,
+        load_act<B>(p, cx, p.H, p.resid_fixed ? SRC_FIXED : SRC_RESID, resid_src(p), L.attn_norm, nullptr, SIDE_ROPE, s,
                     rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       }

@@ -199,6 +199,8 @@ struct Params {
   float* y;          // fused FFN: [B][H] residual after attention (the FFN's RMSNorm input);
                      // xacc then accumulates the down projection's partial sums
   int ffn_fused;     // 1: gate/up and down run as one stage with a split-K down projection
+  int resid_fixed;   // fused FFN: 1 = residual in the fixed-point accumulator xacc (bit-reproducible
+                     // integer split-K adds), 0 = two-plane fp32 x with float atomics
   int jt;            // fused FFN: W_down columns per tile
   int tc;            // 1: batch-8 projections on tcgen05 MMAs (tensor-core packing and stages)
   int tc_cols;       //   tensor-memory columns each CTA allocates (16 per M-tile of its largest stage)

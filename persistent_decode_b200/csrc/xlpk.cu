@@ -990,6 +990,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.y = reinterpret_cast<float*>(e->ws + o_y);
   p.xacc = reinterpret_cast<long long*>(e->ws + o_xacc);
   p.ffn_fused = e->ffn_fused ? 1 : 0;
+  p.resid_fixed = e->ffn_fused && !(c.flags & XLPK_FLAG_FLOAT_FFN_REDUCE) ? 1 : 0;
   p.jt = kTileBytes / (H * 2);
   p.down_win = e->down_win;
   p.tc = e->tc ? 1 : 0;
