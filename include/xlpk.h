@@ -283,6 +283,26 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
 xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_out_dev,
                                 const xlpk_decode_io* io, void* stream);
 
+/* Speculative verification: check n_draft proposed tokens in ONE persistent
+ * launch and accept the longest correct prefix on the device.  The handle must
+ * have batch = n_draft + 1 and a paged cache whose sequences all name the same
+ * pages (one page-table row repeated): sequence b of the step feeds the pending
+ * token (b = 0) or draft b - 1 at position pos + b, writes its K/V row there and
+ * attends to every row up to it, including the rows the sequences before it write
+ * in the same step.  argmax_dev [n_draft + 1] receives the greedy token after
+ * each fed position; drafts are accepted while draft[a] == argmax[a], and the
+ * tokens emitted are draft[0..a-1] followed by argmax[a] (the bonus token):
+ * *emitted_host = a + 1.  The handle's state advances by a + 1 positions with
+ * argmax[a] pending (the K/V rows of rejected drafts are rewritten before they
+ * are read again).  Synchronises `stream`; returns the device status.  `io` may
+ * name per-position logits ([1][n_draft + 1][V]) and hidden states; NULL.
+ * Source: draft-token verification against the target model, accepted tokens
+ * committed and the rest discarded ("XL-Persistent-Kernel", request lifecycle
+ * steps 5-7; fused speculative verification among its features to implement;
+ * MTP in "Persistent execution paradigm", section 3). */
+xlpk_status xlpk_verify(xlpk_handle h, const int32_t* draft_dev, int32_t n_draft, int32_t* argmax_dev,
+                        int32_t* emitted_host, const xlpk_decode_io* io, void* stream);
+
 /* Parity mode: register device buffers logits_dev (fp32 [B][V]) and
  * hidden_dev (fp32 [B][H], the residual after the last layer) into which every
  * later decode call on the handle (xlpk_decode, xlpk_decode_unfused,

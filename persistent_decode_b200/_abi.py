@@ -83,6 +83,8 @@ SIGNATURES = {
     "xlpk_decode_noalloc": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p,
                                         C.POINTER(xlpk_decode_io), C.c_void_p]),
     "xlpk_debug_logits": (C.c_int32, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "xlpk_verify": (C.c_int32, [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.POINTER(C.c_int32),
+                                C.POINTER(xlpk_decode_io), C.c_void_p]),
     "xlpk_serve_start": (C.c_int32, [C.c_void_p, C.c_int32, C.c_void_p]),
     "xlpk_serve_post": (C.c_int32, [C.c_void_p, C.c_int32, C.POINTER(C.c_int64)]),
     "xlpk_serve_wait": (C.c_int32, [C.c_void_p, C.c_int64, C.c_int32, C.POINTER(C.c_int32), C.c_int32]),

@@ -2266,6 +2266,13 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         }
       }
       consumer_sync();
+      if (p.verify && cx.tid == 0) {
+        // accept drafts while the argmax after position pos0[a] is draft a
+        int a = 0;
+        while (a < p.B - 1 && p.tokens_out[a] == p.draft[a]) ++a;
+        p.accept_out[0] = a + 1;                 // the accepted drafts and the bonus token
+        p.cur_tok[0] = p.tokens_out[a];           // the next pending token
+      }
       if (cx.tid == 0) {
         release_add(p.cnt + p.cl.step_done, 1u);
         if (p.serve) {
@@ -2942,7 +2949,9 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
         // steps (or before the launch); make sure the previous step's write is
         // complete before reading it through the async proxy.
         if (fused) {
-          const unsigned target = static_cast<unsigned>(p.G) * static_cast<unsigned>(p.step_base + t_step);
+          // (verify: this step's rows of the sequences before this one, too)
+          const unsigned target =
+              static_cast<unsigned>(p.G) * static_cast<unsigned>(p.step_base + t_step + (p.verify ? 1 : 0));
           const int where = where_code(ST_ATTN, t_layer, t_step) | (1 << 15);
           if (!counter_wait(p, cx.ctl, p.cnt + t_layer * ST_LAYER + ST_QKV, target, where)) break;
         }

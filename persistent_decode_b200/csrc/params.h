@@ -236,6 +236,16 @@ struct Params {
   int fault_drop_stage;        // failure-detection tests: CTA 0 withholds its release of this
                                // stage index at the call's first step (-1: never)
 
+  // Speculative verify (one step): sequence b is the pending token (b = 0) or
+  // draft b - 1 fed at position pos0[b] = pos0[0] + b; every sequence reads the
+  // same pages, so attention needs this step's KV rows of the sequences before
+  // it (the producer waits for this step's QKV stage, not the previous one's).
+  // The LM head's last arriver accepts the longest prefix of drafts equal to the
+  // argmaxes and writes the number of tokens emitted (accepted + 1) to accept_out.
+  int verify;
+  const int32_t* draft;        // [B - 1] draft tokens
+  int32_t* accept_out;         // [1]
+
   // Device-resident request loop (serve mode): launch step s runs once the
   // host has asked for more than serve_step0 + s steps of the session.  CTA 0's
   // first consumer thread polls the host-mapped request word and forwards it to

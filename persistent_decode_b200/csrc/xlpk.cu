@@ -283,6 +283,7 @@ struct xlpk_engine {
   long long serve_step0 = 0;         // session steps done before the current launch
   long long serve_idle_ns = 0;
   unsigned* serve_dev_words = nullptr;   // workspace: [0] forwarded request count, [1] stop step
+  int32_t* verify_word = nullptr;        // workspace: tokens emitted by the last verify step
 };
 
 namespace {
@@ -961,6 +962,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   const size_t o_ab = take(sizeof(int));
   const size_t o_ts = take(sizeof(int) * static_cast<size_t>(c.max_seq) * B);
   const size_t o_sv = take(sizeof(unsigned) * 2);
+  const size_t o_acc = take(sizeof(int32_t));
   e->ws_bytes = off;
   XLPK_CUDA(cudaMalloc(&e->ws, e->ws_bytes));
   XLPK_CUDA(cudaMemset(e->ws, 0, e->ws_bytes));
@@ -1051,6 +1053,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.abort_flag = reinterpret_cast<int*>(e->ws + o_ab);
   e->tok_scratch = reinterpret_cast<int32_t*>(e->ws + o_ts);
   e->serve_dev_words = reinterpret_cast<unsigned*>(e->ws + o_sv);
+  e->verify_word = reinterpret_cast<int32_t*>(e->ws + o_acc);
   e->pos.assign(B, 0);
   XLPK_CUDA(cudaDeviceSynchronize());
   return XLPK_OK;
@@ -1442,6 +1445,35 @@ xlpk_status xlpk_decode_noalloc(xlpk_handle h, int32_t n_steps, int32_t* tokens_
                                         static_cast<size_t>(h->smem), st));
   for (int b = 0; b < B; ++b) h->pos[b] += n_steps;
   h->last_stream = st;
+  return XLPK_OK;
+}
+
+xlpk_status xlpk_verify(xlpk_handle h, const int32_t* draft_dev, int32_t n_draft, int32_t* argmax_dev,
+                        int32_t* emitted_host, const xlpk_decode_io* io, void* stream) {
+  if (!h || !draft_dev || !argmax_dev || !emitted_host || n_draft < 1) return XLPK_ERR_INVALID_ARG;
+  if (n_draft != h->cfg.batch - 1 || h->serve_active) return XLPK_ERR_INVALID_ARG;
+  if (h->cfg.n_experts > 0) return XLPK_ERR_UNSUPPORTED;
+  const int pos = h->pos[0];
+  if (pos + n_draft + 1 > h->cfg.max_seq) return XLPK_ERR_KV_FULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // sequence b > 0 feeds draft b - 1; sequence 0 keeps the pending token
+  XLPK_CUDA(cudaMemcpyAsync(h->base.cur_tok + 1, draft_dev, sizeof(int32_t) * n_draft, cudaMemcpyDeviceToDevice, st));
+  Params p = call_params(h, 1, argmax_dev, io);
+  for (int b = 0; b < h->cfg.batch; ++b) p.pos0[b] = pos + b;
+  p.forced = nullptr;
+  p.verify = 1;
+  p.draft = draft_dev;
+  p.accept_out = h->verify_word;
+  void* args[] = {&p};
+  XLPK_CUDA(cudaLaunchCooperativeKernel(h->kern_persistent, dim3(h->G), dim3(kThreads), args,
+                                        static_cast<size_t>(h->smem), st));
+  h->last_stream = st;
+  XLPK_CUDA(cudaMemcpyAsync(emitted_host, h->verify_word, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  const xlpk_status rc = xlpk_get_status(h);   // synchronises the stream
+  if (rc != XLPK_OK) return rc;
+  const int n = *emitted_host;
+  for (int b = 0; b < h->cfg.batch; ++b) h->pos[b] = pos + n;
+  h->step_base += 1;
   return XLPK_OK;
 }
 

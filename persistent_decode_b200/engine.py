@@ -208,6 +208,15 @@ class Engine:
         self._dbg = (logits, hidden)   # borrowed by the library until replaced
         _check(lib.xlpk_debug_logits(self.h, _ptr(logits), _ptr(hidden)), "xlpk_debug_logits")
 
+    def verify(self, drafts, argmax_out, logits=None, hidden=None, stream=None) -> int:
+        """xlpk_verify: `drafts` int32 CUDA tensor [B-1]; `argmax_out` int32 CUDA tensor [B];
+        returns the number of tokens emitted (accepted drafts + the bonus token)."""
+        n = C.c_int32()
+        io = self._io(None, logits, hidden, None, None)
+        _check(lib.xlpk_verify(self.h, _ptr(drafts), int(drafts.numel()), _ptr(argmax_out), C.byref(n),
+                               C.byref(io) if io is not None else None, _stream_handle(stream)), "xlpk_verify")
+        return int(n.value)
+
     # ---- device-resident request loop (xlpk_serve_*)
 
     def serve_start(self, idle_limit_us: int = 1_000_000, stream=None) -> None:
