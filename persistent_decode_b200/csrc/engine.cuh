@@ -1469,11 +1469,9 @@ struct EpiSwiGLULocal {
 // Fused FFN, second half: this CTA's columns [j0, j1) of W_down times its own
 // h slice, for all H output rows (split-K over the CTAs), added into the
 // residual's fixed-point accumulator with 64-bit integer atomics (the sum does
-// not depend on the order of the adds).  Tiles are jt rows of W_down^T (= W_down
-// columns) of p.downT_row bytes each: H bf16, or (FP8) H e4m3 codes followed by
-// the row's H/128 block scales; thread t owns the 8-row vectors t, t + 256, ...
-// of the output.
-template <int B, bool FP8>
+// not depend on the order of the adds).  Tiles are jt rows of W_down^T (= W_down columns), H
+// bf16 each; thread t owns the 8-row vectors t, t + 256, ... of the output.
+template <int B>
 __device__ __noinline__ void consume_downT(const Params& p, Ctx& cx, RingPos& rp, int where, int j0, int j1,
                                            const float* hl) {
   constexpr int NV = 2;                        // 8-row vectors per thread (H <= 4096)
@@ -1496,34 +1494,18 @@ __device__ __noinline__ void consume_downT(const Params& p, Ctx& cx, RingPos& rp
         float hv[B];
 #pragma unroll
         for (int b = 0; b < B; ++b) hv[b] = hl[b * p.hloc + t0 + jj];
-        const uint32_t col = base + jj * p.downT_row;
+        const uint32_t col = base + jj * p.H * 2;
 #pragma unroll
         for (int q = 0; q < NV; ++q) {
           const int v = cx.tid + q * kConsumerThreads;
           if (v < V8) {
-            float wf[8];
-            float hs[B];
-            if constexpr (FP8) {
-              // 8 codes of one 128-row scale block; the scale folds into h
-              const uint2 w = lds_u2(col + v * 8);
-              const float sc = __uint_as_float(lds_u1(col + p.H + (v >> 4) * 4));
-              const float2 f0 = e4m3x2_to_float2(w.x & 0xffffu), f1 = e4m3x2_to_float2(w.x >> 16);
-              const float2 f2 = e4m3x2_to_float2(w.y & 0xffffu), f3 = e4m3x2_to_float2(w.y >> 16);
-              wf[0] = f0.x; wf[1] = f0.y; wf[2] = f1.x; wf[3] = f1.y;
-              wf[4] = f2.x; wf[5] = f2.y; wf[6] = f3.x; wf[7] = f3.y;
-#pragma unroll
-              for (int b = 0; b < B; ++b) hs[b] = hv[b] * sc;
-            } else {
-              const uint4 w = lds_u4(col + v * 16);
-              wf[0] = bf16_lo(w.x); wf[1] = bf16_hi(w.x); wf[2] = bf16_lo(w.y); wf[3] = bf16_hi(w.y);
-              wf[4] = bf16_lo(w.z); wf[5] = bf16_hi(w.z); wf[6] = bf16_lo(w.w); wf[7] = bf16_hi(w.w);
-#pragma unroll
-              for (int b = 0; b < B; ++b) hs[b] = hv[b];
-            }
+            const uint4 w = lds_u4(col + v * 16);
+            const float wf[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                 bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
 #pragma unroll
             for (int e = 0; e < 8; ++e)
 #pragma unroll
-              for (int b = 0; b < B; ++b) acc[q][e][b] = fmaf(wf[e], hs[b], acc[q][e][b]);
+              for (int b = 0; b < B; ++b) acc[q][e][b] = fmaf(wf[e], hv[b], acc[q][e][b]);
           }
         }
       }
@@ -2391,10 +2373,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         EpiSwiGLULocal<B> epi{hl, p.hloc, q0};
         consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
         consumer_sync();
-        if (p.esz == 1)
-          consume_downT<B, true>(p, cx, rp, where, q0, q1, hl);
-        else
-          consume_downT<B, false>(p, cx, rp, where, q0, q1, hl);
+        consume_downT<B>(p, cx, rp, where, q0, q1, hl);
       } else {
         EpiSwiGLU<B> epi{p};
         consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
@@ -2780,7 +2759,7 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
       const int nj = j1 - j0;
       cu.phase = 1;
       if (nj > 0) {
-        const uint32_t colb = static_cast<uint32_t>(p.downT_row);
+        const uint32_t colb = static_cast<uint32_t>(p.H) * 2u;
         run->src = p.layers[cu.l].downT.packed + static_cast<size_t>(j0) * colb;
         run->n1 = nj / p.jt;
         run->b1 = static_cast<uint32_t>(p.jt) * colb;

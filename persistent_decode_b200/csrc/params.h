@@ -135,9 +135,9 @@ struct LayerParams {
   // CTAs); every expert's down projection is packed like a dense matrix
   // (rows split over the CTAs).  egu / edown describe expert 0; expert e's
   // block starts e * egu_stride (edown_stride) bytes further.
-  // Dense layers with the fused FFN stage: W_down transposed, [F][H] row-major
-  // (bf16, or e4m3 codes with each row's H/128 block scales after it); a CTA
-  // streams the rows (= W_down columns) matching its own gate/up pairs.
+  // Dense layers with the fused FFN stage: W_down transposed, bf16 [F][H]
+  // row-major; a CTA streams the rows (= W_down columns) matching its own
+  // gate/up pairs.
   Mat downT;
   Mat router;
   Mat egu;
@@ -202,7 +202,6 @@ struct Params {
   int resid_fixed;   // fused FFN: 1 = residual in the fixed-point accumulator xacc (bit-reproducible
                      // integer split-K adds), 0 = two-plane fp32 x with float atomics
   int jt;            // fused FFN: W_down columns per tile
-  int downT_row;     //   bytes of one W_down^T row: H bf16, or H e4m3 codes + H/128 fp32 block scales
   int tc;            // 1: batch-8 projections on tcgen05 MMAs (tensor-core packing and stages)
   int tc_cols;       //   tensor-memory columns each CTA allocates (16 per M-tile of its largest stage)
   int tc_win;        //   K window of the tensor-core projections (tc_window), 0: whole K

@@ -81,32 +81,6 @@ __global__ void transpose_bf16_kernel(const uint16_t* in, uint16_t* out, int R, 
   }
 }
 
-// bytes [R][C] row-major -> [C][R] row-major, rows of the output `ld` bytes apart
-// (32x32 tiles through shared memory).
-__global__ void transpose_u8_kernel(const uint8_t* in, uint8_t* out, int R, int C, int ld) {
-  __shared__ uint8_t t[32][33];
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < R && c < C) t[i][threadIdx.x] = in[static_cast<size_t>(r) * C + c];
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < R && c < C) out[static_cast<size_t>(c) * ld + r] = t[threadIdx.x][i];
-  }
-}
-
-// FP8 W_down^T rows: after row j's H codes, the scales of W_down's 128x128
-// blocks (hb, j / 128) for hb < H/128 (scale: [H/128][F/128] fp32).
-__global__ void downT_scales_kernel(const float* scale, uint8_t* out, int H, int F, int ld) {
-  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int nhb = H / 128;
-  if (t >= static_cast<long long>(F) * nhb) return;
-  const int j = static_cast<int>(t / nhb), hb = static_cast<int>(t - static_cast<long long>(j) * nhb);
-  reinterpret_cast<float*>(out + static_cast<size_t>(j) * ld + H)[hb] = scale[static_cast<size_t>(hb) * (F / 128) + j / 128];
-}
-
 // FP8: one thread per (row, chunk): the chunk's KC/128 block scales of the row.
 __global__ void pack_scales_kernel(const PackJob* jobs, int njobs, uint8_t* out, int nchunk, int kc_cols, int cw,
                                    long long tile_row) {
@@ -645,7 +619,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   // and whose accumulators fit the register budget (XLPK_FFN_FUSED=0 turns it off).
   {
     const bool off = (c.flags & XLPK_FLAG_NO_FUSED_FFN) != 0;
-    e->ffn_fused = !off && c.n_experts == 0 && H <= 2 * 8 * kConsumerThreads && H % 8 == 0 && B <= 2;
+    e->ffn_fused = !off && c.n_experts == 0 && e->esz == 2 && H <= 2 * 8 * kConsumerThreads && H % 8 == 0 &&
+                   B <= 2;
   }
   // Batch 8, dense layers: every projection runs on tcgen05 MMAs (8-row units
   // per CTA, M-tiles of <= 128 rows with kTcAccCols accumulator columns each in
@@ -789,8 +764,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr, L.w_gate.scale_dev, L.w_up.scale_dev},
           2 * F, H, l, R_GU, e->G);
       if (e->ffn_fused)
-        add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev}, F, H, l, R_DOWNT,
-            1);   // W_down^T [F][H]
+        add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, F, H, l, R_DOWNT, 1);   // W_down^T [F][H]
       else
         add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev}, H, F, l, R_DOWN, e->G);
     } else {
@@ -852,19 +826,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     const MatPlan& mp = mats[i];
     Mat m{};
     if (mp.role == R_DOWNT) {
-      // the fused FFN streams W_down columns: store W_down^T [F][H] (bf16, or
-      // e4m3 codes with each row's block scales after them)
+      // the fused FFN streams W_down columns: store W_down^T, plain bf16 [F][H]
       const dim3 tb(32, 8), gr((mp.N + 31) / 32, (mp.K + 31) / 32);   // in: [H=K][F=N]
-      if (e->esz == 2) {
-        transpose_bf16_kernel<<<gr, tb, 0, st>>>(reinterpret_cast<const uint16_t*>(mp.src.a),
-                                                 reinterpret_cast<uint16_t*>(e->packed + mp.off), mp.K, mp.N);
-      } else {
-        const int ld = mp.K + mp.K / 32;
-        transpose_u8_kernel<<<gr, tb, 0, st>>>(mp.src.a, e->packed + mp.off, mp.K, mp.N, ld);
-        const long long nt = static_cast<long long>(mp.N) * (mp.K / 128);
-        downT_scales_kernel<<<static_cast<int>((nt + 255) / 256), 256, 0, st>>>(mp.src.sa, e->packed + mp.off, mp.K,
-                                                                                mp.N, ld);
-      }
+      transpose_bf16_kernel<<<gr, tb, 0, st>>>(reinterpret_cast<const uint16_t*>(mp.src.a),
+                                               reinterpret_cast<uint16_t*>(e->packed + mp.off), mp.K, mp.N);
       ce = cudaGetLastError();
       if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
       if (ce != cudaSuccess) {
@@ -875,7 +840,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       m.N = mp.N;
       m.K = mp.K;
       m.KC = mp.K;
-      m.fp8 = e->esz == 1 ? 1 : 0;
+      m.fp8 = 0;
     } else {
       e->esz = mp.role == R_ROUTER ? 2 : esz_saved;
       if (e->tc && (mp.role == R_QKV || mp.role == R_O || mp.role == R_GU || mp.role == R_DOWN || mp.role == R_LM))
@@ -1028,8 +993,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.xacc = reinterpret_cast<long long*>(e->ws + o_xacc);
   p.ffn_fused = e->ffn_fused ? 1 : 0;
   p.resid_fixed = e->ffn_fused && !(c.flags & XLPK_FLAG_FLOAT_FFN_REDUCE) ? 1 : 0;
-  p.downT_row = e->esz == 1 ? H + H / 32 : 2 * H;
-  p.jt = kTileBytes / p.downT_row;
+  p.jt = kTileBytes / (H * 2);
   p.down_win = e->down_win;
   p.tc = e->tc ? 1 : 0;
   p.tc_cols = e->tc_cols;
