@@ -1920,25 +1920,24 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
       }
-      // ---- S = Q K^T for positions pg*16 .. pg*16+15
-      // (two accumulator chains: splitting them further measured slower)
+      // ---- S = Q K^T for positions pg*16 .. pg*16+15.  A rows 0..7 carry q's
+      // high bf16 terms and rows 8..15 its low terms, so one MMA forms both
+      // products: accumulator rows gid and gid + 8 add up to the score.
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       const int kr = pg * 16 + ((mi >> 1) << 3) + rr;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         uint32_t b00, b01, b10, b11;
         ldsm_x4(sw128_addr(kt, P, kr, ks * 16 + ((mi & 1) << 3)), b00, b01, b10, b11);
-        mma_16816(s0, qa0[ks], 0u, qa2[ks], 0u, b00, b01);
-        mma_16816(s1, qa0[ks], 0u, qa2[ks], 0u, b10, b11);
-        mma_16816(s0, qb0[ks], 0u, qb2[ks], 0u, b00, b01);
-        mma_16816(s1, qb0[ks], 0u, qb2[ks], 0u, b10, b11);
+        mma_16816(s0, qa0[ks], qb0[ks], qa2[ks], qb2[ks], b00, b01);
+        mma_16816(s1, qa0[ks], qb0[ks], qa2[ks], qb2[ks], b10, b11);
       }
       // ---- online softmax of head gid over the 16 positions (4 per lane)
       const int pa = pg * 16 + tig * 2;
-      const float v0 = pa < npos ? s0[0] : -INFINITY;
-      const float v1 = pa + 1 < npos ? s0[1] : -INFINITY;
-      const float v2 = pa + 8 < npos ? s1[0] : -INFINITY;
-      const float v3 = pa + 9 < npos ? s1[1] : -INFINITY;
+      const float v0 = pa < npos ? s0[0] + s0[2] : -INFINITY;
+      const float v1 = pa + 1 < npos ? s0[1] + s0[3] : -INFINITY;
+      const float v2 = pa + 8 < npos ? s1[0] + s1[2] : -INFINITY;
+      const float v3 = pa + 9 < npos ? s1[1] + s1[3] : -INFINITY;
       float mr = fmaxf(fmaxf(v0, v1), fmaxf(v2, v3));
       mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 1));
       mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 2));
@@ -1957,20 +1956,21 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       for (int nt = 0; nt < NT; ++nt) {
         o[nt][0] *= alpha;
         o[nt][1] *= alpha;
+        o[nt][2] *= alpha;
+        o[nt][3] *= alpha;
       }
       uint32_t pa0, pa2, pb0, pb2;
       split_bf16x2(p0, p1, pa0, pb0);
       split_bf16x2(p2, p3, pa2, pb2);
-      // ---- O += P V for this warp's dims
+      // ---- O += P V for this warp's dims (P's high terms in A rows 0..7, its
+      // low terms in rows 8..15: accumulator rows gid + 8 hold the low part)
       const int vr = pg * 16 + ((mi & 1) << 3) + rr;
 #pragma unroll
       for (int n2 = 0; n2 < NT / 2; ++n2) {
         uint32_t b00, b01, b10, b11;
         ldsm_x4_t(sw128_addr(vt, P, vr, ds * DW + n2 * 16 + ((mi >> 1) << 3)), b00, b01, b10, b11);
-        mma_16816(o[2 * n2], pa0, 0u, pa2, 0u, b00, b01);
-        mma_16816(o[2 * n2 + 1], pa0, 0u, pa2, 0u, b10, b11);
-        mma_16816(o[2 * n2], pb0, 0u, pb2, 0u, b00, b01);
-        mma_16816(o[2 * n2 + 1], pb0, 0u, pb2, 0u, b10, b11);
+        mma_16816(o[2 * n2], pa0, pb0, pa2, pb2, b00, b01);
+        mma_16816(o[2 * n2 + 1], pa0, pb0, pa2, pb2, b10, b11);
       }
     }
     __syncwarp();
@@ -2000,8 +2000,8 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     if (gid < kMaxGroup) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        sm_o[(cx.warp * kMaxGroup + gid) * DW + nt * 8 + tig * 2 + 0] = o[nt][0];
-        sm_o[(cx.warp * kMaxGroup + gid) * DW + nt * 8 + tig * 2 + 1] = o[nt][1];
+        sm_o[(cx.warp * kMaxGroup + gid) * DW + nt * 8 + tig * 2 + 0] = o[nt][0] + o[nt][2];
+        sm_o[(cx.warp * kMaxGroup + gid) * DW + nt * 8 + tig * 2 + 1] = o[nt][1] + o[nt][3];
       }
     }
     consumer_sync();
