@@ -605,10 +605,12 @@ __device__ __forceinline__ const void* resid_src(const Params& p) {
 // (W (g v) r = W (r g v)), so the stage needs a single consumer barrier.
 // `hidden_dbg` (LM stage, CTA 0) receives the raw residual in natural [B][K] order.
 //
-// SRC_FIXED (the fused-FFN layers' residual accumulator) is read by all
-// consumer threads straight into registers (B*4096 values per pass, one round
-// trip), converted, scaled by the gains (read alongside) and written in the
-// two-plane layout; the side data still comes by bulk copy meanwhile.
+// SRC_FIXED (the fused-FFN layers' residual accumulator) arrives by the same
+// bulk copy phase into a staging area behind the fp32 input (int64 [B][K] at
+// act + B*K*4 bytes); the threads convert it from shared memory, one group of 4
+// at a time, scaled by the gains they loaded before the wait.  (Reading it
+// straight into registers instead kept so many values live that the whole
+// kernel's register allocation spilled.)
 template <int B>
 __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc src, const void* gsrc_v,
                                       const float* gain, float* hidden_dbg, int side, int s,
@@ -634,6 +636,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     // total bytes of this phase
     uint32_t total = 0;
     if (src != SRC_EMBED && !direct) total += static_cast<uint32_t>(B) * K * 4u;
+    if (direct) total += static_cast<uint32_t>(B) * K * 8u;
     if (gain && !direct) total += static_cast<uint32_t>(K) * 4u;
     const uint32_t rope_bytes = static_cast<uint32_t>(p.d) * 4u;   // d/2 (cos, sin) pairs
     const int v0 = r0 >> 3, nv = r1 > r0 ? ((r1 - 1) >> 3) - v0 + 1 : 0;
@@ -645,6 +648,9 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     mbar_expect_tx(bar, total);
     if (src != SRC_EMBED && !direct)
       bulk_g2s_nohint(smem_addr(cx.act), gsrc, static_cast<uint32_t>(B) * K * 4u, bar);
+    if (direct)   // int64 [B][K] staged behind the fp32 area
+      bulk_g2s_nohint(smem_addr(cx.act) + static_cast<uint32_t>(B) * K * 4u, gsrc, static_cast<uint32_t>(B) * K * 8u,
+                      bar);
     if (gain && !direct) bulk_g2s_nohint(gain_s, gain, static_cast<uint32_t>(K) * 4u, bar);
     if (side == SIDE_ROPE) {
 #pragma unroll
@@ -673,48 +679,40 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
   }
   if constexpr (B <= 2) {   // the fused FFN (and so SRC_FIXED) exists for batch <= 2 only
   if (direct) {
-    constexpr int UF = 4 * B;   // groups of 4 per thread and pass: one pass for B*K <= 4096*B
-    const long long* xs = static_cast<const long long*>(gsrc_v);
-    const float4* g4p = reinterpret_cast<const float4*>(gain);
-    float ss[B];
+    // the gains of this thread's groups (K <= 4096 in the fused-FFN layers)
+    constexpr int GJ = 4;
+    float4 g[GJ];
 #pragma unroll
-    for (int b = 0; b < B; ++b) ss[b] = 0.f;
-    const int nit = B * n4;   // groups of 4 consecutive elements
-    for (int i0 = cx.tid; i0 < nit; i0 += UF * kConsumerThreads) {
-      longlong2 lo[UF], hi[UF];
-      float4 g[UF];
-#pragma unroll
-      for (int u = 0; u < UF; ++u) {
-        const int i = i0 + u * kConsumerThreads;
-        if (i < nit) {
-          const int b = i / n4, q = i - b * n4;
-          const longlong2* a = reinterpret_cast<const longlong2*>(xs + static_cast<size_t>(b) * K + 4 * q);
-          lo[u] = __ldcg(a);
-          hi[u] = __ldcg(a + 1);
-          g[u] = gain ? __ldg(g4p + q) : make_float4(1.f, 1.f, 1.f, 1.f);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < UF; ++u) {
-        const int i = i0 + u * kConsumerThreads;
-        if (i < nit) {
-          const int b = i / n4, q = i - b * n4;
-          const float4 v = make_float4(from_fixed(lo[u].x), from_fixed(lo[u].y), from_fixed(hi[u].x),
-                                       from_fixed(hi[u].y));
-          if (hidden_dbg) *reinterpret_cast<float4*>(hidden_dbg + static_cast<size_t>(b) * K + 4 * q) = v;
-          const float sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
-#pragma unroll
-          for (int bb = 0; bb < B; ++bb)
-            if (bb == b) ss[bb] += sq;
-          act4[((q & 1) * B + b) * nvK + (q >> 1)] =
-              make_float4(v.x * g[u].x, v.y * g[u].y, v.z * g[u].z, v.w * g[u].w);
-        }
-      }
+    for (int j = 0; j < GJ; ++j) {
+      const int q = cx.tid + j * kConsumerThreads;
+      g[j] = (gain && q < n4) ? __ldg(reinterpret_cast<const float4*>(gain) + q) : make_float4(1.f, 1.f, 1.f, 1.f);
     }
-    // the side data (RoPE rows)
     if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
     if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
     cx.act_phase ^= 1u;
+    const uint32_t stage = smem_addr(cx.act) + static_cast<uint32_t>(B) * K * 4u;
+    float ss[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      ss[b] = 0.f;
+#pragma unroll
+      for (int j = 0; j < GJ; ++j) {
+        const int q = cx.tid + j * kConsumerThreads;
+        if (q < n4) {
+          const uint32_t a = stage + static_cast<uint32_t>(b * K + 4 * q) * 8u;
+          const uint4 u0 = lds_u4(a), u1 = lds_u4(a + 16);
+          const float4 v = make_float4(
+              from_fixed(static_cast<long long>((static_cast<unsigned long long>(u0.y) << 32) | u0.x)),
+              from_fixed(static_cast<long long>((static_cast<unsigned long long>(u0.w) << 32) | u0.z)),
+              from_fixed(static_cast<long long>((static_cast<unsigned long long>(u1.y) << 32) | u1.x)),
+              from_fixed(static_cast<long long>((static_cast<unsigned long long>(u1.w) << 32) | u1.z)));
+          if (hidden_dbg) *reinterpret_cast<float4*>(hidden_dbg + static_cast<size_t>(b) * K + 4 * q) = v;
+          ss[b] = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss[b]))));
+          act4[((q & 1) * B + b) * nvK + (q >> 1)] =
+              make_float4(v.x * g[j].x, v.y * g[j].y, v.z * g[j].z, v.w * g[j].w);
+        }
+      }
+    }
 #pragma unroll
     for (int b = 0; b < B; ++b) rn[b] = 1.f;
     if (gain) {

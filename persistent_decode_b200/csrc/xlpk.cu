@@ -696,6 +696,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       return static_cast<int>(align_up(std::max(std::max(B * kmax * 4, norm_stage), attn_scratch), 1024));
     };
     e->act_bytes = act_for(std::max(std::max(H, qd), std::max(F, S_moe * c.expert_ffn)));
+    // the fused-FFN layers stage their int64 residual behind the fp32 input
+    if (e->ffn_fused) e->act_bytes = std::max(e->act_bytes, static_cast<int>(align_up(static_cast<size_t>(12) * B * H, 1024)));
     // A two-stage dense FFN whose down-projection input (B x F fp32) would leave
     // the ring fewer than 3 slots streams W_down window by window instead: the
     // activation region then holds B x down_win floats of h at a time (windows
