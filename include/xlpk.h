@@ -168,10 +168,11 @@ typedef struct xlpk_decode_io {
   uint64_t* trace_dev;                /* [n_steps][n_stages][n_ctas][16] globaltimer stamps (ns) per
                                          stage and CTA: [0] consumer entry, [1] dependency met,
                                          [2] inputs staged, [3] consumer done, [4] producer first
-                                         copy, [5] producer last copy.  Attention stages also record
-                                         totals of thread 0: [6] ns waiting for KV chunks, [7] ns
-                                         from the end of the chunks to leaving (merge, arrive,
-                                         combine), [8] q loads, [9] chunk math, [10] merge,
+                                         copy, [5] producer last copy.  A library built with
+                                         XLPK_TRACE_ATTN defined also records, for attention
+                                         stages, totals of thread 0: [6] ns waiting for KV chunks,
+                                         [7] ns from the end of the chunks to leaving (merge,
+                                         arrive, combine), [8] q loads, [9] chunk math, [10] merge,
                                          [11] arrive, [12] combine, [13] chunks processed.
                                          n_stages = 5 * n_layers + 1 */
   int32_t withhold_release;           /* failure-detection testing only: 1 + the index (layer * 5 +

@@ -1778,6 +1778,15 @@ __host__ __device__ constexpr int attn_scratch_floats(int D, int G) {
          + 3 * G * kMaxGroup + 2 * kMaxGroup;   // combine: (M, L, weight) per contributor, M*, L*
 }
 
+// Timers of the attention stage's internals (trace slots 6..13): a
+// diagnostic build's option (-DXLPK_TRACE_ATTN); the values they keep live cost
+// the release kernel about 2 % of a step on the 8B shape.
+#ifdef XLPK_TRACE_ATTN
+constexpr bool kTraceAttn = true;
+#else
+constexpr bool kTraceAttn = false;
+#endif
+
 // Flash-decoding over this CTA's chunks of the (sequence, kv head) space on
 // warp-level tensor cores.  A chunk is P = 64 (d=128) or 128 (d=64) positions
 // whose K and V rows arrive as 128-byte-swizzled TMA boxes.  Warp w takes the
@@ -1828,7 +1837,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
   // ring waits, from the end of the chunks to leaving, q loads, chunk math,
   // merge, arrive, combine; chunks processed
   unsigned long long* ta = cx.ctl->tacc;
-  if (p.trace && cx.tid == 0)
+  if (kTraceAttn && p.trace && cx.tid == 0)
     for (int k = 0; k < 8; ++k) ta[k] = 0;
 
   for (int i = i0; i < i1; ++i) {
@@ -1844,7 +1853,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       l_h = 0.f;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-      const unsigned long long tq0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+      const unsigned long long tq0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
       if (gid < GQ) {
         const float* qs = p.q + (static_cast<size_t>(b) * p.nq + g * GQ + gid) * D;
         const float sc = p.qk_scale_log2;
@@ -1859,7 +1868,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) qa0[ks] = qa2[ks] = qb0[ks] = qb2[ks] = 0u;
       }
-      if (p.trace && cx.tid == 0) ta[2] += globaltimer() - tq0;
+      if (kTraceAttn && p.trace && cx.tid == 0) ta[2] += globaltimer() - tq0;
     }
     ++seg_items;
     const int T = p.pos0[b] + s + 1;
@@ -1867,15 +1876,15 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     const int npos = min(t_lo + P, T) - t_lo;      // positions of this chunk (incl. the new token)
     const int n_old = min(t_lo + P, T - 1) - t_lo; // positions already in the cache before this step
     const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
-    const unsigned long long tw0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+    const unsigned long long tw0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
     // warp-uniform: the tile body below is warp-collective (ldmatrix, mma, shuffles)
     const bool have_tile =
         __all_sync(0xffffffffu, cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where));
-    if (p.trace && cx.tid == 0) {
+    if (kTraceAttn && p.trace && cx.tid == 0) {
       ta[0] += globaltimer() - tw0;
       ++ta[7];
     }
-    const unsigned long long tc0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+    const unsigned long long tc0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
     const uint32_t kt = ring_s + rp.slot * kSlotBytes;
     const uint32_t vt = kt + kTileBytes / 2;
     if (have_tile && pg * 16 < npos) {   // warp-uniform
@@ -1972,7 +1981,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       }
     }
     __syncwarp();
-    if (p.trace && cx.tid == 0) ta[3] += globaltimer() - tc0;
+    if (kTraceAttn && p.trace && cx.tid == 0) ta[3] += globaltimer() - tc0;
     if (cx.lane == 0 && have_tile) mbar_arrive(smem_addr(&cx.ctl->empty[rp.slot]));
     rp.next(p.nslot);
     // end of a (b, g) segment: merge the 8 warps into this CTA's partial, and
@@ -1980,7 +1989,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     const int ib = seg_base + seg_g * seg_nch;
     const int ie = ib + seg_nch;
     if (i + 1 < i1 && i + 1 < ie) continue;   // the segment goes on
-    const unsigned long long tm0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
+    const unsigned long long tm0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
 
     // contributors of this head: CTAs c_first .. c_first + ncov - 1 (partial rows 0 .. ncov-1)
     int c_first, ncov;
@@ -2030,8 +2039,8 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       fence_proxy_async_global();   // the combiner may read the partials by bulk copy
     }
     consumer_sync();
-    const unsigned long long ta0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
-    if (p.trace && cx.tid == 0) ta[4] += ta0 - tm0;
+    const unsigned long long ta0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
+    if (kTraceAttn && p.trace && cx.tid == 0) ta[4] += ta0 - tm0;
     unsigned* arrive = p.cnt + p.cl.attn_arrive + (l * p.B + seg_b) * p.nkv + seg_g;
     if (cx.tid == 0) {
       const unsigned old = release_add(arrive, static_cast<unsigned>(seg_items));
@@ -2039,10 +2048,10 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       cx.ctl->flag = (old + seg_items == static_cast<unsigned>(seg_nch)) ? 1 : 0;
     }
     consumer_sync();
-    const unsigned long long tb0 = (p.trace && cx.tid == 0) ? globaltimer() : 0;
-    if (p.trace && cx.tid == 0) ta[5] += tb0 - ta0;
+    const unsigned long long tb0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
+    if (kTraceAttn && p.trace && cx.tid == 0) ta[5] += tb0 - ta0;
     if (!cx.ctl->flag) {
-      if (p.trace && cx.tid == 0) ta[1] += globaltimer() - tm0;
+      if (kTraceAttn && p.trace && cx.tid == 0) ta[1] += globaltimer() - tm0;
       continue;
     }
     // ---- combine: contributors are CTAs c_first .. c_first + ncov - 1 (rows
@@ -2138,14 +2147,14 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       // release below, which the next step's contributors wait behind)
       *reinterpret_cast<volatile unsigned*>(arrive) = 0u;
       release_add(p.cnt + l * ST_LAYER + ST_ATTN, 1u);
-      if (p.trace) {
+      if (kTraceAttn && p.trace) {
         const unsigned long long te = globaltimer();
         ta[1] += te - tm0;
         ta[6] += te - tb0;
       }
     }
   }
-  if (p.trace && cx.tid == 0) {
+  if (kTraceAttn && p.trace && cx.tid == 0) {
     const size_t n_st = static_cast<size_t>(p.L) * ST_LAYER + 1;
     unsigned long long* e =
         p.trace + ((static_cast<size_t>(s) * n_st + stage_index(p, ST_ATTN, l)) * p.G + blockIdx.x) * kTraceSlots;

@@ -1238,7 +1238,12 @@ xlpk_status xlpk_serve_wait(xlpk_handle h, int64_t first_step, int32_t n_steps, 
   const long long target = first_step + n_steps;
   if (target > h->serve_posted) return XLPK_ERR_INVALID_ARG;
   const auto t0 = std::chrono::steady_clock::now();
+  auto last_check = t0;
   while (serve_done(h) < target) {
+    // whether the loop has left (idle) is asked of the driver only now and then
+    const auto now = std::chrono::steady_clock::now();
+    if (now - last_check < std::chrono::microseconds(200)) continue;
+    last_check = now;
     if (h->serve_launched && cudaStreamQuery(h->serve_stream) == cudaSuccess && serve_done(h) < target) {
       // the launch ended (idle) before our steps: start it again
       xlpk_status rc = serve_collect(h);
