@@ -24,7 +24,9 @@ The operations themselves follow the plain reading of a Llama-style decoder:
   logits = Wlm (x * rsqrt(mean(x^2) + eps) * g_final);  token = argmax (ties -> lowest id)
 
 Everything is fp32 on the CPU except the KV cache, which stores bf16 like the
-device cache (both sides round k and v to bf16 before attention reads them).
+device cache (both sides round k and v to bf16 before attention reads them), or
+for an e4m3 cache the e4m3 code of k / scale times a power-of-two scale per
+tensor (kv_round).
 The weights are widened from their stored bf16 / e4m3 bytes on use.
 """
 from __future__ import annotations
@@ -34,7 +36,7 @@ from typing import Dict, List, Optional, Tuple
 
 import torch
 
-from .fp8 import e4m3_to_fp32
+from .fp8 import e4m3_encode, e4m3_to_fp32
 
 
 # --------------------------------------------------------------------------- ops
@@ -113,6 +115,18 @@ def _bf16_round(x: torch.Tensor) -> torch.Tensor:
     return x.to(torch.bfloat16)
 
 
+def kv_round(x: torch.Tensor, kv_dtype: str, scale: float) -> torch.Tensor:
+    """The value a cache entry holds: bf16 (round to nearest even), or for an
+    e4m3 cache the code of x / scale (satfinite) times scale.  The scale is a
+    power of two, so x / scale and code * scale are exact and the result is
+    also exactly a bf16 value (4 significant bits)."""
+    if kv_dtype == "bf16":
+        return x.to(torch.bfloat16)
+    assert kv_dtype == "fp8_e4m3" and scale > 0 and math.frexp(scale)[0] == 0.5, scale
+    codes = e4m3_encode(x.float() / scale)
+    return (e4m3_to_fp32(codes) * scale).to(torch.bfloat16)
+
+
 # ------------------------------------------------------------------- the model
 
 class OracleDecoder:
@@ -145,7 +159,8 @@ class OracleDecoder:
         return t.float()
 
     def load_kv(self, layer: int, k: torch.Tensor, v: torch.Tensor) -> None:
-        """Install cache contents [B][n_kv][T][d] at positions [0, T) of `layer`."""
+        """Install cache contents [B][n_kv][T][d] at positions [0, T) of `layer`
+        (values a cache of the model's KV type can hold: they are stored as given)."""
         T = k.shape[2]
         self.K[layer, :, :, :T] = k.to(torch.bfloat16)
         self.V[layer, :, :, :T] = v.to(torch.bfloat16)
@@ -190,8 +205,8 @@ class OracleDecoder:
                 v = (self.W(p + "wv") @ xn).view(nkv, d)
                 q = rope_rotate(q, pos, cfg.rope_theta)
                 k = rope_rotate(k, pos, cfg.rope_theta)
-                self.K[l, b, :, pos] = _bf16_round(k)
-                self.V[l, b, :, pos] = _bf16_round(v)
+                self.K[l, b, :, pos] = kv_round(k, cfg.kv_dtype, cfg.k_scale)
+                self.V[l, b, :, pos] = kv_round(v, cfg.kv_dtype, cfg.v_scale)
                 o = attention_decode(q, self.K[l, b, :, : pos + 1], self.V[l, b, :, : pos + 1])
                 x = x + self.W(p + "wo") @ o.reshape(-1)
                 xn2 = rms_norm(x, self.w[p + "ffn_norm"], cfg.rms_eps)
@@ -236,7 +251,7 @@ class OracleDecoder:
                 for t in range(T):
                     qs[t] = rope_rotate(q[t], t, cfg.rope_theta)
                     ks[t] = rope_rotate(k[t], t, cfg.rope_theta)
-                kb, vb = _bf16_round(ks), _bf16_round(v)
+                kb, vb = kv_round(ks, cfg.kv_dtype, cfg.k_scale), kv_round(v, cfg.kv_dtype, cfg.v_scale)
                 if fill_cache:
                     self.K[l, b, :, :T] = kb.permute(1, 0, 2)
                     self.V[l, b, :, :T] = vb.permute(1, 0, 2)

@@ -5,7 +5,7 @@ contains none of the decoder's arithmetic (no norm, projection, attention,
 activation or routing).  Both sides of every parity test draw their inputs from
 here, on the host or on a CUDA device, bit-identically.
 """
-from .configs import DecoderConfig, CONFIGS, get_config  # noqa: F401
+from .configs import DecoderConfig, CONFIGS, fp8_kv, get_config  # noqa: F401
 from .gen import (  # noqa: F401
     splitmix64_stream,
     normal_bf16,

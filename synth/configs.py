@@ -35,6 +35,9 @@ class DecoderConfig:
     init_std: float = 0.02
     prefill: bool = True   # KV from a seeded prompt (True) or seeded synthetic KV (False)
     seed: int = 0
+    kv_dtype: str = "bf16"   # "bf16" or "fp8_e4m3" (one power-of-two scale per tensor)
+    k_scale: float = 0.0     # e4m3 cache: scales of K and V entries (powers of two)
+    v_scale: float = 0.0
 
     @property
     def max_seq(self) -> int:
@@ -79,6 +82,16 @@ MOE = DecoderConfig(
     n_shared_experts=1, expert_ffn=1408, prefill=False)
 
 CONFIGS = {c.name: c for c in (TINY, LLAMA_1B, LLAMA_8B, LLAMA_8B_FP8, MOE)}
+
+
+def fp8_kv(cfg: DecoderConfig) -> DecoderConfig:
+    """The same model with an e4m3 KV cache.  K and V entries are about
+    N(0, (init_std * sqrt(hidden))^2) (a projection of a unit-RMS activation); the
+    scale is the power of two that puts 6 sigma just under e4m3's largest value 448."""
+    import math
+    sigma = cfg.init_std * math.sqrt(cfg.hidden)
+    scale = 2.0 ** math.ceil(math.log2(6.0 * sigma / 448.0))
+    return cfg.with_(kv_dtype="fp8_e4m3", k_scale=scale, v_scale=scale)
 
 
 def get_config(name: str, **overrides) -> DecoderConfig:

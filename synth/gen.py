@@ -225,7 +225,23 @@ def make_synthetic_kv(cfg: DecoderConfig, layer: int, device: torch.device | str
     shape = (cfg.batch, cfg.n_kv_heads, cfg.kv_len, cfg.head_dim)
     k = normal_bf16(2, f"kv.k.{layer}", shape, std, device)
     v = normal_bf16(2, f"kv.v.{layer}", shape, std, device)
+    if cfg.kv_dtype == "fp8_e4m3":
+        # values an e4m3 cache holds (code x power-of-two scale), still as bf16
+        k = fp8_kv_values(k, cfg.k_scale)
+        v = fp8_kv_values(v, cfg.v_scale)
     return k, v
+
+
+def fp8_kv_values(x: torch.Tensor, scale: float) -> torch.Tensor:
+    """Synthetic entries of an e4m3 cache (input preparation): x / scale rounded to
+    e4m3 (satfinite, round to nearest even), times scale, as bf16 (exact)."""
+    q = (x.float() / scale).clamp(-FP8_E4M3_MAX, FP8_E4M3_MAX).to(torch.float8_e4m3fn)
+    return (q.float() * scale).to(torch.bfloat16)
+
+
+def fp8_kv_codes(x: torch.Tensor, scale: float) -> torch.Tensor:
+    """The uint8 e4m3 codes of cache values x that fp8_kv_values produced (exact)."""
+    return (x.float() / scale).clamp(-FP8_E4M3_MAX, FP8_E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
 
 
 def make_start_tokens(cfg: DecoderConfig, device: torch.device | str = "cpu") -> torch.Tensor:

@@ -467,3 +467,46 @@ def test_moe_incremental_decode_equals_full_recompute():
     T = toks.shape[1]
     assert torch.allclose(inc.K[:, :, :, :T].float(), full.K[:, :, :, :T].float(), atol=2e-2)
     assert torch.allclose(inc.V[:, :, :, :T].float(), full.V[:, :, :, :T].float(), atol=2e-2)
+
+
+# ----------------------------------------------------------- e4m3 encoding
+
+def test_e4m3_encoder_matches_library_rounding():
+    # the oracle's encoder (written from the format) against the library's
+    # conversion of the same values clamped to the finite range (satfinite)
+    from oracle import e4m3_encode
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.randn(200000, generator=g) * s for s in (1e-3, 0.05, 1.0, 30.0, 300.0)]
+                  + [torch.tensor([0.0, -0.0, 448.0, -448.0, 449.0, 1e6, -1e6, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11])])
+    lib = x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(e4m3_encode(x), lib)
+
+
+def test_e4m3_encoder_ties_go_to_the_even_code():
+    from oracle import e4m3_decode_table, e4m3_encode
+    t = e4m3_decode_table()
+    for c in (0x01, 0x08, 0x10, 0x30, 0x38, 0x3B, 0x50, 0x70, 0x7C):
+        mid = float((t[c] + t[c + 1]) / 2)                  # halfway between codes c and c + 1
+        want = c if c % 2 == 0 else c + 1
+        assert int(e4m3_encode(torch.tensor([mid]))) == want, hex(c)
+        assert int(e4m3_encode(torch.tensor([-mid]))) == want | 0x80, hex(c)
+
+
+def test_fp8_kv_round_is_code_times_a_power_of_two():
+    from oracle.decoder import kv_round
+    from oracle import e4m3_decode_table
+    table = e4m3_decode_table()
+    finite = table[~torch.isnan(table)]
+    x = torch.randn(4, 128) * 0.4
+    for scale in (2.0 ** -7, 2.0 ** -3):
+        r = kv_round(x, "fp8_e4m3", scale).float()
+        q = r / scale
+        assert bool(torch.isin(q, finite).all())          # every entry is an e4m3 value times the scale
+        assert torch.equal(kv_round(r, "fp8_e4m3", scale).float(), r)   # idempotent
+        # nearest: no e4m3 value is closer to x / scale than the chosen one
+        d = (x / scale).clamp(-448, 448)
+        err = (q - d).abs()
+        best = (finite[None, None, :] - d[..., None]).abs().min(dim=-1).values
+        assert bool((err <= best + 1e-7).all())
+    with pytest.raises(AssertionError):
+        kv_round(x, "fp8_e4m3", 0.3)                     # not a power of two
