@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--decode-steps", type=int, default=0, help="override tokens per call (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (sequences per call)")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="KV cache entries: bf16, or e4m3 codes with a power-of-two scale per tensor")
     ap.add_argument("--no-baselines", action="store_true", help="skip the unfused and CPU legs")
     ap.add_argument("--serve", action="store_true",
                     help="also time one-step requests through the resident loop against one launch per request")
@@ -123,7 +125,7 @@ def kernel_source_hash() -> str:
     come from (the tensor-core tile entry point appended to xlpk.cu is not
     among them)."""
     h = hashlib.sha256()
-    for f in ("engine.cuh", "xlpk.cu", "params.h"):
+    for f in ("engine.cuh", "xlpk.cu", "params.h", "kernels.cu", "kernels.h"):
         data = open(os.path.join(ROOT, "persistent_decode_b200", "csrc", f), "rb").read()
         if f == "xlpk.cu" and TILE_SECTION in data:
             data = data[:data.index(TILE_SECTION)]
@@ -188,6 +190,19 @@ def cpu_sample_desc(cfg, nl):
 
 # ----------------------------------------------------------------- reference arm
 
+def bench_config(args):
+    """The workload's config with the command line's overrides."""
+    import synth
+    cfg = synth.get_config(args.workload)
+    if getattr(args, "decode_steps", 0):
+        cfg = cfg.with_(steps=args.decode_steps)
+    if getattr(args, "batch", 0):
+        cfg = cfg.with_(batch=args.batch)
+    if getattr(args, "kv", "bf16") == "fp8":
+        cfg = synth.fp8_kv(cfg)
+    return cfg
+
+
 def run_reference(args):
     import torch
 
@@ -195,7 +210,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    cfg = synth.get_config(args.workload)
+    cfg = bench_config(args)
     dev = "cuda:0" if torch.cuda.is_available() else "cpu"
     o, head, nl = build_cpu_sample(cfg, dev)
     start = synth.make_start_tokens(cfg).tolist()
@@ -229,14 +244,16 @@ def dtype_label(cfg) -> str:
     act = "fp32 activations"
     if cfg.batch == 8 and not cfg.is_moe:
         act = "activations as bf16 high + low parts into tcgen05 MMAs, fp32 accumulation"
-    return f"{w}, bf16 KV, {act}"
+    kv = "e4m3 KV (power-of-two scale per tensor)" if cfg.kv_dtype == "fp8_e4m3" else "bf16 KV"
+    return f"{w}, {kv}, {act}"
 
 
 def workload_config(cfg, n):
     return {"workload": f"{cfg.name}: {cfg.n_layers} layers, hidden {cfg.hidden}, {cfg.n_q_heads}q/"
                         f"{cfg.n_kv_heads}kv heads x {cfg.head_dim}, ffn {cfg.ffn}, vocab {cfg.vocab}, "
-                        f"{cfg.weight_dtype} weights, KV {cfg.kv_len}, {cfg.steps} greedy steps, batch "
-                        f"{cfg.batch}",
+                        f"{cfg.weight_dtype} weights, KV {cfg.kv_len}"
+                        f"{' (e4m3 cache)' if cfg.kv_dtype == 'fp8_e4m3' else ''}, {cfg.steps} greedy steps, "
+                        f"batch {cfg.batch}",
             "global_batch": cfg.batch * n, "seq_len": cfg.kv_len, "decode_steps": cfg.steps,
             "parallelism": "replicas" if n > 1 else "single-gpu",
             "l2": "inputs larger than L2 (all weights streamed every token)"}
@@ -306,11 +323,7 @@ def main():
         torch.cuda.set_device(local)
         replicas.init("nccl", device=torch.device("cuda", local))
     dev = torch.device("cuda", local if world > 1 else 0)
-    cfg = synth.get_config(args.workload)
-    if args.decode_steps:
-        cfg = cfg.with_(steps=args.decode_steps)
-    if args.batch:
-        cfg = cfg.with_(batch=args.batch)
+    cfg = bench_config(args)
     n = cfg.steps
     B = cfg.batch
 

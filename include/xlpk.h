@@ -87,6 +87,11 @@ typedef struct xlpk_config {
                                   tensor-core projection at batch 8 (a multiple of 1024); 0 = chosen by
                                   the planner.  A value the planner cannot use is ignored on CUDA cores
                                   and refused (XLPK_ERR_UNSUPPORTED) on tensor cores. */
+  int32_t kv_dtype;            /* xlpk_dtype of the KV cache: XLPK_DTYPE_BF16 (entries are bf16) or
+                                  XLPK_DTYPE_FP8_E4M3 (entries are e4m3 codes; entry = code * scale) */
+  float k_scale;               /* e4m3 cache: the scale of every K entry, a power of two in
+                                  [2^-24, 2^24] (else XLPK_ERR_INVALID_ARG); ignored for bf16 */
+  float v_scale;               /* e4m3 cache: the scale of every V entry, the same rule */
 } xlpk_config;
 
 /* xlpk_config::flags.  The defaults are the fast paths; the flags select the
@@ -135,7 +140,11 @@ typedef struct xlpk_weights {
   const xlpk_layer_weights* layers;   /* HOST array of n_layers entries */
 } xlpk_weights;
 
-/* Caller-owned KV cache: post-RoPE keys and values, bf16, 16-byte aligned.
+/* Caller-owned KV cache: post-RoPE keys and values, 16-byte aligned, one
+ * element per entry of the config's kv_dtype: bf16, or an e4m3 code (one byte)
+ * whose value is code * k_scale (K) or code * v_scale (V).  A decode writes the
+ * new token's entries rounded to that type (e4m3: x / scale rounded to nearest
+ * even and saturated to +-448).
  *  - Contiguous (page_table_dev NULL): K and V each [L][B][n_kv][max_seq][d].
  *  - Paged: K and V each a pool [L][n_pages][n_kv][page_size][d] of pages of
  *    page_size positions; page_table_dev int32 [B][ceil(max_seq / page_size)]
@@ -149,7 +158,10 @@ typedef struct xlpk_weights {
  *    from xlpk_get_status.
  * Source: the KV page planner that places each request's cache pages and the
  * decode worker that follows them ("XL-Persistent-Kernel", request lifecycle
- * steps 2-4 and the component table's KV row). */
+ * steps 2-4 and the component table's KV row); a quantised (FP8) attention
+ * cache read inside the persistent kernel, which the survey of persistent
+ * execution names as an open combination ("持续执行范式：从 Kernel Boundary
+ * Elimination 到 Ultra-Low-Latency Engine", section 7.5). */
 typedef struct xlpk_kv {
   void* k_dev;
   void* v_dev;
@@ -171,8 +183,8 @@ typedef struct xlpk_decode_io {
                                          copy, [5] producer last copy.  A library built with
                                          XLPK_TRACE_ATTN defined also records, for attention
                                          stages, totals of thread 0: [6] ns waiting for KV chunks,
-                                         [7] ns from the end of the chunks to leaving (merge,
-                                         arrive, combine), [8] q loads, [9] chunk math, [10] merge,
+                                         [7] ns of the combining CTA's wait for the partials,
+                                         [8] q loads, [9] chunk math, [10] merge,
                                          [11] arrive, [12] combine, [13] chunks processed.
                                          n_stages = 5 * n_layers + 1 */
   int32_t withhold_release;           /* failure-detection testing only: 1 + the index (layer * 5 +

@@ -32,7 +32,8 @@ class xlpk_config(C.Structure):
         "n_experts", "top_k", "n_shared_experts", "expert_ffn", "weight_dtype", "batch",
         "max_seq")] + [("rope_theta", C.c_float), ("rms_eps", C.c_float),
                        ("n_ctas", C.c_int32), ("spin_limit_us", C.c_int32), ("flags", C.c_int32),
-                       ("window", C.c_int32)]
+                       ("window", C.c_int32), ("kv_dtype", C.c_int32), ("k_scale", C.c_float),
+                       ("v_scale", C.c_float)]
 
 
 class xlpk_linear(C.Structure):

@@ -12,7 +12,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "xlpk.cu")
-DEPS = [os.path.join(HERE, "csrc", f) for f in ("xlpk.cu", "engine.cuh", "tcgen05.cuh", "tc_tile.cuh", "params.h")] + \
+KERNELS = os.path.join(HERE, "csrc", "kernels.cu")
+KERNEL_UNITS = 9   # kKernelUnits in csrc/kernels.h
+DEPS = [os.path.join(HERE, "csrc", f) for f in ("xlpk.cu", "kernels.cu", "kernels.h", "engine.cuh", "tcgen05.cuh",
+                                                "tc_tile.cuh", "params.h")] + \
     [os.path.join(ROOT, "include", "xlpk.h")]
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libxlpk.so")
@@ -33,25 +36,60 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
+    """Compile the host code and the kernel units in parallel (one nvcc each),
+    then link libxlpk.so (or `out`).  `defines` are extra -D macros (build-time
+    options such as XLPK_TRACE_ATTN).  Every nvcc's output (with -Xptxas -v)
+    goes to lib/build.log (or beside `out`)."""
+    target = out or LIB
+    if not force and not defines and out is None and up_to_date():
         return LIB
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-Xptxas", "-v", "-I", os.path.join(ROOT, "include"), "-o", tmp, SRC]
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    log = os.path.join(LIB_DIR, "build.log")
+    import tempfile
+    obj_tmp = tempfile.TemporaryDirectory(dir=LIB_DIR, prefix="obj.")   # removed after the link
+    obj_dir = obj_tmp.name
+    nvcc = nvcc_path()
+    common = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v", "-Xfatbin", "-compress-all",
+              "-I", os.path.join(ROOT, "include"), *[f"-D{d}" for d in defines]]
+    jobs = [([nvcc, *common, "-c", SRC, "-o", os.path.join(obj_dir, "xlpk.o")], os.path.join(obj_dir, "xlpk.o"))]
+    for u in range(KERNEL_UNITS):
+        o = os.path.join(obj_dir, f"kernels{u}.o")
+        jobs.append(([nvcc, *common, f"-DXLPK_UNIT={u}", "-c", KERNELS, "-o", o], o))
+    width = max(1, min(len(jobs), os.cpu_count() or 1))
+    logs, failed, running, pending = [], False, [], list(jobs)
+    while pending or running:
+        while pending and len(running) < width:
+            cmd, _ = pending.pop(0)
+            running.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
+        cmd, proc = running.pop(0)
+        out, _ = proc.communicate()
+        logs.append(" ".join(cmd) + "\n" + out)
+        failed = failed or proc.returncode != 0
+    tmp = target + ".tmp"
+    if not failed:
+        link = [nvcc, *ARCH, "-shared", "-o", tmp, *[o for _, o in jobs]]
+        res = subprocess.run(link, capture_output=True, text=True)
+        logs.append(" ".join(link) + "\n" + res.stdout + res.stderr)
+        failed = res.returncode != 0
+    obj_tmp.cleanup()
+    log = os.path.join(LIB_DIR, "build.log") if out is None else target + ".build.log"
     with open(log, "w") as f:
-        f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
-    if res.returncode != 0:
-        sys.stderr.write(res.stderr[-8000:])
+        f.write("\n".join(logs))
+    if failed:
+        sys.stderr.write("\n".join(logs)[-8000:])
         raise RuntimeError(f"nvcc failed (see {log})")
-    os.replace(tmp, LIB)
+    os.replace(tmp, target)
     if verbose:
-        print(res.stderr)
-    return LIB
+        print("\n".join(logs))
+    return target
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser(description="build libxlpk.so")
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("-D", dest="defines", action="append", default=[], help="extra macro, e.g. -D XLPK_TRACE_ATTN")
+    ap.add_argument("-o", dest="out", default=None, help="output library (default: lib/libxlpk.so)")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.verbose, defines=a.defines, out=a.out))

@@ -142,6 +142,30 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// The same tile with fp16 operands.
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+      " {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+template <bool F16>
+__device__ __forceinline__ void mma_16816t(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  if constexpr (F16)
+    mma_16816_f16(d, a0, a1, a2, a3, b0, b1);
+  else
+    mma_16816(d, a0, a1, a2, a3, b0, b1);
+}
+// Two e4m3 codes (low byte first) -> their exact values as an f16x2 (low half
+// first); every e4m3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(r) : "r"(two_codes));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -175,6 +199,17 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // 16-byte unit u of row r sits at unit u ^ (r % 8).
 __device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int P, int r, int d) {
   return base + (d >> 6) * (P * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4) + ((d & 7) << 1);
+}
+// Byte (r, c) of an e4m3 K or V chunk: P rows of D bytes as the TMA writes
+// them with the 128-byte (D = 128) or 64-byte (D = 64) swizzle, i.e. the
+// 16-byte unit c/16 of row r is stored at unit (c/16) ^ (r & 7) or
+// (c/16) ^ ((r/2) & 3); the base is 1024-byte aligned.  Either way the eight
+// rows a warp quarter reads at one logical unit land in distinct banks.
+template <int D>
+__device__ __forceinline__ uint32_t kv8_addr(uint32_t base, int r, int c) {
+  static_assert(D == 64 || D == 128, "head_dim");
+  const int f = D == 128 ? (r & 7) : ((r >> 1) & 3);
+  return base + r * D + ((((c >> 4) ^ f) << 4) | (c & 15));
 }
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
@@ -347,7 +382,7 @@ __device__ __forceinline__ int stage_index(const Params& p, int kind, int l) {
 
 // Bounded wait on a ring barrier phase.  Returns false (and marks the CTA
 // aborted) if the global abort flag is raised or the time limit passes.
-__device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint32_t bar,
+static __device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint32_t bar,
                                             uint32_t parity, int where, int limit_mult = 1) {
   const uint64_t t0 = globaltimer();
   const long long limit = p.spin_limit_ns * limit_mult;
@@ -371,7 +406,7 @@ __device__ __noinline__ bool ring_wait_slow(const Params& p, SmemCtl* ctl, uint3
 // only read device memory and always complete; the bound (at least 2 s,
 // independent of the dependency-wait limit) only guards against a device that
 // stopped making progress.
-__device__ __noinline__ void copy_wait(const Params& p, uint32_t bar, uint32_t parity) {
+static __device__ __noinline__ void copy_wait(const Params& p, uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   const long long limit = p.spin_limit_ns > 2000000000LL ? p.spin_limit_ns : 2000000000LL;
   while (!(p.wait_hint_ns ? mbar_try_wait_suspend(bar, parity, p.wait_hint_ns) : mbar_try_wait(bar, parity))) {
@@ -386,7 +421,7 @@ __device__ __forceinline__ bool ring_wait(const Params& p, SmemCtl* ctl, uint32_
 }
 
 // Bounded wait (one thread) until *cnt >= target (wrap-safe).
-__device__ __noinline__ bool counter_wait_slow(const Params& p, SmemCtl* ctl, const unsigned* cnt,
+static __device__ __noinline__ bool counter_wait_slow(const Params& p, SmemCtl* ctl, const unsigned* cnt,
                                                unsigned target, int where) {
   const uint64_t t0 = globaltimer();
   unsigned nap = 16;
@@ -442,7 +477,7 @@ __device__ __forceinline__ int serve_state(const Params& p, int s) {
 // forwards it, and decides the stop after serve_idle_ns without a request or
 // when the host asks to leave; every other waiter follows the device words,
 // with a limit above the poller's.
-__device__ __noinline__ bool serve_gate(const Params& p, SmemCtl* ctl, int s, bool poller) {
+static __device__ __noinline__ bool serve_gate(const Params& p, SmemCtl* ctl, int s, bool poller) {
   const unsigned want = static_cast<unsigned>(p.serve_step0 + s + 1);
   const uint64_t t0 = globaltimer();
   unsigned nap = 32;
@@ -523,6 +558,10 @@ __device__ __forceinline__ float dot16_e4m3(const uint4 w, const float4 x0, cons
 __device__ __forceinline__ uint16_t f2bf(float v) {
   __nv_bfloat16 h = __float2bfloat16_rn(v);
   return *reinterpret_cast<uint16_t*>(&h);
+}
+// fp32 -> e4m3 code: round to nearest even, saturated to +-448 (NaN stays NaN).
+__device__ __forceinline__ uint8_t f2e4m3(float v) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -1087,7 +1126,7 @@ __device__ __noinline__ void load_side(const Params& p, Ctx& cx, int side, int s
 // rows); with `gain` the values are multiplied by it and each thread's sums of
 // squares of the raw values are added to ss (the RMSNorm factor is formed once
 // every window has been staged).  `hidden_dbg` receives the raw input.
-__device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src, const float* gsrc, int K, int k0,
+static __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src, const float* gsrc, int K, int k0,
                                             int Kw, const float* gain, float* hidden_dbg, float (&ss)[kMaxBatch],
                                             bool f16) {
   constexpr int B = kMaxBatch;
@@ -1162,7 +1201,7 @@ __device__ __noinline__ void tc_stage_input(const Params& p, Ctx& cx, ActSrc src
 // the codes times their block scale rounded to fp16 (11 significant bits;
 // the MMAs of FP8 models take fp16 operands), same swizzle.  Every consumer
 // thread reads its units before any is overwritten.
-__device__ __noinline__ void tc_widen_fp8(Ctx& cx, uint32_t slot_s, int rv, int nb) {
+static __device__ __noinline__ void tc_widen_fp8(Ctx& cx, uint32_t slot_s, int rv, int nb) {
   constexpr int kMaxUnits = 4;   // 16-byte code units per thread: nb * rv * 8 <= 1024
   const int nu = nb * rv * 8;
   uint4 code[kMaxUnits];
@@ -1343,7 +1382,7 @@ __device__ __forceinline__ size_t kv_row(const Params& p, int l, int b, int g, i
 
 // QKV epilogue: RoPE on q/k pairs, q -> workspace, bf16 k/v -> cache at pos.
 // The step's cos/sin rows were staged in shared memory (SIDE_ROPE).
-template <int B>
+template <int B, bool KV8>
 struct EpiQKV {
   const Params& p;
   int l, s;
@@ -1370,7 +1409,11 @@ struct EpiQKV {
         } else {
           bool ok;
           const size_t row = kv_row(p, l, b, head, pos, ok);
-          if (ok) {
+          if (KV8 && ok) {
+            uint8_t* kd = p.kc8 + row;
+            kd[i] = f2e4m3(y0 * p.k_inv);
+            kd[i + half] = f2e4m3(y1 * p.k_inv);
+          } else if (ok) {
             uint16_t* kd = p.kc + row;
             kd[i] = f2bf(y0);
             kd[i + half] = f2bf(y1);
@@ -1383,7 +1426,11 @@ struct EpiQKV {
         const int head = pv / half, i2 = (pv - head * half) * 2;
         bool ok;
         const size_t row = kv_row(p, l, b, head, pos, ok);
-        if (ok) {
+        if (KV8 && ok) {
+          const uint16_t packed = static_cast<uint16_t>(f2e4m3(r0 * p.v_inv)) |
+                                  static_cast<uint16_t>(static_cast<uint16_t>(f2e4m3(r1 * p.v_inv)) << 8);
+          *reinterpret_cast<uint16_t*>(p.vc8 + row + i2) = packed;
+        } else if (ok) {
           const uint32_t packed = static_cast<uint32_t>(f2bf(r0)) | (static_cast<uint32_t>(f2bf(r1)) << 16);
           *reinterpret_cast<uint32_t*>(p.vc + row + i2) = packed;
         } else {
@@ -1605,7 +1652,7 @@ struct EpiMoeGU {
 // probabilities as weights (not renormalised), shared experts first with
 // weight 1.  Writes this CTA's routing table; CTA 0 also records it globally
 // (for the kernel-per-op down launch and the caller's experts output).
-__device__ __noinline__ void moe_route(const Params& p, Ctx& cx, int l, int s) {
+static __device__ __noinline__ void moe_route(const Params& p, Ctx& cx, int l, int s) {
   constexpr int PER = kMaxExperts / 32;
   float v[PER];
   float mx = -INFINITY;
@@ -1799,7 +1846,19 @@ constexpr bool kTraceAttn = false;
 // operand of O += P V (the accumulator-to-A register reuse of FlashAttention-2).
 // The new token's K/V row (written by this step's QKV stage) is patched into
 // the chunk in shared memory.
-template <int B, int D>
+//
+// An e4m3 cache (KV8) arrives as two 8 KB boxes of codes (K at the slot's
+// start, V 8 KB further).  K codes feed the q.k MMAs straight from shared
+// memory: the dot product runs over a permutation of the head dims in which
+// k-step ks of lane quad tig covers dims 4*KS*tig + 4*ks + (0..3), so one
+// 32-bit word of a K row is the lane's whole B fragment (two f16x2 after an
+// exact e4m3 -> f16 conversion), and q is loaded in the same order.  Each warp
+// widens the V codes it multiplies (its 16 positions x DW dims) to f16 in the
+// bf16 path's swizzled V layout.  The MMAs take fp16 operands: q as two f16
+// terms (x 2^8), P as two f16 terms (x 2^12); the scales k_scale and v_scale
+// and those powers of two are applied to the scores and to the softmax sum, all
+// exact power-of-two multiplies.
+template <int B, int D, bool KV8>
 __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s, RingPos& rp,
                                          bool fused) {
   static_assert(kMaxGroup == 4, "query heads per kv head fill at most rows 0..3 of the A tile");
@@ -1811,6 +1870,10 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
   constexpr int KS = D / 16;                                  // q.k k-steps
   constexpr int DV = D / 32;                                  // new-row dims per lane
   static_assert(NPG * NDS == kConsumerWarps && NT % 2 == 0, "chunk shape");
+  static_assert(!KV8 || (DW == 64 && P * D == 8192), "e4m3 chunk: two 8 KB boxes, 64 dims per warp");
+  constexpr float kQMul = 256.f, kPMul = 4096.f;              // e4m3 path: operand pre-scales
+  const float smul = KV8 ? p.k_scale * (1.f / kQMul) : 1.f;   // score scale (a power of two)
+  const float lmul = KV8 ? kPMul * p.v_inv : 1.f;             // softmax-sum scale (a power of two)
   AttnPlan<B> ap;
   attn_plan<B>(p, s, ap);
   int i0, i1;
@@ -1854,7 +1917,17 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
       const unsigned long long tq0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
-      if (gid < GQ) {
+      if (KV8 && gid < GQ) {
+        // the permuted dim order of the e4m3 K fragments: dims 4*KS*tig + 4*ks + (0..3)
+        const float* qs = p.q + (static_cast<size_t>(b) * p.nq + g * GQ + gid) * D + tig * 4 * KS;
+        const float sc = p.qk_scale_log2 * kQMul;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const float4 u = __ldcg(reinterpret_cast<const float4*>(qs + ks * 4));
+          split_f16x2(u.x * sc, u.y * sc, qa0[ks], qb0[ks]);
+          split_f16x2(u.z * sc, u.w * sc, qa2[ks], qb2[ks]);
+        }
+      } else if (gid < GQ) {
         const float* qs = p.q + (static_cast<size_t>(b) * p.nq + g * GQ + gid) * D;
         const float sc = p.qk_scale_log2;
 #pragma unroll
@@ -1887,8 +1960,56 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     const unsigned long long tc0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
     const uint32_t kt = ring_s + rp.slot * kSlotBytes;
     const uint32_t vt = kt + kTileBytes / 2;
-    if (have_tile && pg * 16 < npos) {   // warp-uniform
+    const uint32_t vt8 = kt + 8192;                 // e4m3 V codes (K codes at kt)
+    if (KV8 && have_tile && pg * 16 < npos) {   // warp-uniform
       if (npos > n_old && (n_old >> 4) == pg) {
+        // this step's K/V codes of the head into the code chunks
+        bool row_ok;
+        const size_t row = kv_row(p, l, b, g, T - 1, row_ok);
+        constexpr int DB = D / 32;                  // bytes per lane
+        if (row_ok) {
+          const uint32_t ka = kv8_addr<D>(kt, n_old, cx.lane * DB);
+          const uint32_t va = kv8_addr<D>(vt8, n_old, cx.lane * DB);
+          if (DB == 4) {
+            const unsigned kk = __ldcg(reinterpret_cast<const unsigned*>(p.kc8 + row + cx.lane * DB));
+            const unsigned vv = __ldcg(reinterpret_cast<const unsigned*>(p.vc8 + row + cx.lane * DB));
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(ka), "r"(kk) : "memory");
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(va), "r"(vv) : "memory");
+          } else {
+            const unsigned short kk = __ldcg(reinterpret_cast<const unsigned short*>(p.kc8 + row + cx.lane * DB));
+            const unsigned short vv = __ldcg(reinterpret_cast<const unsigned short*>(p.vc8 + row + cx.lane * DB));
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(ka), "h"(kk) : "memory");
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(va), "h"(vv) : "memory");
+          }
+        }
+        __syncwarp();
+      }
+      // widen this warp's V codes (rows pg*16 + lane%16, 32 dims from ds*DW + 32*(lane/16))
+      {
+        const int r = pg * 16 + (cx.lane & 15);
+        const int c0 = ds * DW + (cx.lane >> 4) * 32;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w0, w1, w2, w3;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                       : "r"(kv8_addr<D>(vt8, r, c0 + 16 * h)));
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sw128_addr(vt, P, r, c0 + 16 * h)),
+                       "r"(e4m3x2_to_f16x2(w0 & 0xffffu)), "r"(e4m3x2_to_f16x2(w0 >> 16)),
+                       "r"(e4m3x2_to_f16x2(w1 & 0xffffu)), "r"(e4m3x2_to_f16x2(w1 >> 16))
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sw128_addr(vt, P, r, c0 + 16 * h + 8)),
+                       "r"(e4m3x2_to_f16x2(w2 & 0xffffu)), "r"(e4m3x2_to_f16x2(w2 >> 16)),
+                       "r"(e4m3x2_to_f16x2(w3 & 0xffffu)), "r"(e4m3x2_to_f16x2(w3 >> 16))
+                       : "memory");
+        }
+      }
+      // the slot is refilled by the async proxy later
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+    }
+    if (have_tile && pg * 16 < npos) {   // warp-uniform
+      if (!KV8 && npos > n_old && (n_old >> 4) == pg) {
         // this step's K/V entry of the head, from the cache (written by the QKV stage)
         bool row_ok;
         const size_t row = kv_row(p, l, b, g, T - 1, row_ok);   // (a bad page was reported by the producer)
@@ -1931,20 +2052,43 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       // high bf16 terms and rows 8..15 its low terms, so one MMA forms both
       // products: accumulator rows gid and gid + 8 add up to the score.
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-      const int kr = pg * 16 + ((mi >> 1) << 3) + rr;
+      if constexpr (KV8) {
+        // B fragments straight from the K codes: positions pg*16 + gid (n-tile 0)
+        // and pg*16 + 8 + gid (n-tile 1), this quad's 4*KS permuted dims
+        uint32_t k0[KS], k1[KS];
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        uint32_t b00, b01, b10, b11;
-        ldsm_x4(sw128_addr(kt, P, kr, ks * 16 + ((mi & 1) << 3)), b00, b01, b10, b11);
-        mma_16816(s0, qa0[ks], qb0[ks], qa2[ks], qb2[ks], b00, b01);
-        mma_16816(s1, qa0[ks], qb0[ks], qa2[ks], qb2[ks], b10, b11);
+        for (int h = 0; h < KS / 4; ++h) {
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(k0[4 * h]), "=r"(k0[4 * h + 1]), "=r"(k0[4 * h + 2]), "=r"(k0[4 * h + 3])
+                       : "r"(kv8_addr<D>(kt, pg * 16 + gid, tig * 4 * KS + 16 * h)));
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(k1[4 * h]), "=r"(k1[4 * h + 1]), "=r"(k1[4 * h + 2]), "=r"(k1[4 * h + 3])
+                       : "r"(kv8_addr<D>(kt, pg * 16 + 8 + gid, tig * 4 * KS + 16 * h)));
+        }
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          mma_16816_f16(s0, qa0[ks], qb0[ks], qa2[ks], qb2[ks], e4m3x2_to_f16x2(k0[ks] & 0xffffu),
+                        e4m3x2_to_f16x2(k0[ks] >> 16));
+          mma_16816_f16(s1, qa0[ks], qb0[ks], qa2[ks], qb2[ks], e4m3x2_to_f16x2(k1[ks] & 0xffffu),
+                        e4m3x2_to_f16x2(k1[ks] >> 16));
+        }
+      } else {
+        const int kr = pg * 16 + ((mi >> 1) << 3) + rr;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t b00, b01, b10, b11;
+          ldsm_x4(sw128_addr(kt, P, kr, ks * 16 + ((mi & 1) << 3)), b00, b01, b10, b11);
+          mma_16816(s0, qa0[ks], qb0[ks], qa2[ks], qb2[ks], b00, b01);
+          mma_16816(s1, qa0[ks], qb0[ks], qa2[ks], qb2[ks], b10, b11);
+        }
       }
       // ---- online softmax of head gid over the 16 positions (4 per lane)
       const int pa = pg * 16 + tig * 2;
-      const float v0 = pa < npos ? s0[0] + s0[2] : -INFINITY;
-      const float v1 = pa + 1 < npos ? s0[1] + s0[3] : -INFINITY;
-      const float v2 = pa + 8 < npos ? s1[0] + s1[2] : -INFINITY;
-      const float v3 = pa + 9 < npos ? s1[1] + s1[3] : -INFINITY;
+      auto score = [&](float hi, float lo) { return KV8 ? (hi + lo) * smul : hi + lo; };
+      const float v0 = pa < npos ? score(s0[0], s0[2]) : -INFINITY;
+      const float v1 = pa + 1 < npos ? score(s0[1], s0[3]) : -INFINITY;
+      const float v2 = pa + 8 < npos ? score(s1[0], s1[2]) : -INFINITY;
+      const float v3 = pa + 9 < npos ? score(s1[1], s1[3]) : -INFINITY;
       float mr = fmaxf(fmaxf(v0, v1), fmaxf(v2, v3));
       mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 1));
       mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 2));
@@ -1957,7 +2101,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       float rs = (p0 + p1) + (p2 + p3);
       rs += __shfl_xor_sync(0xffffffffu, rs, 1);
       rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-      l_h = l_h * alpha + rs;
+      l_h = l_h * alpha + (KV8 ? rs * lmul : rs);
       m_h = mn;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -1967,8 +2111,13 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
         o[nt][3] *= alpha;
       }
       uint32_t pa0, pa2, pb0, pb2;
-      split_bf16x2(p0, p1, pa0, pb0);
-      split_bf16x2(p2, p3, pa2, pb2);
+      if constexpr (KV8) {
+        split_f16x2(p0 * kPMul, p1 * kPMul, pa0, pb0);
+        split_f16x2(p2 * kPMul, p3 * kPMul, pa2, pb2);
+      } else {
+        split_bf16x2(p0, p1, pa0, pb0);
+        split_bf16x2(p2, p3, pa2, pb2);
+      }
       // ---- O += P V for this warp's dims (P's high terms in A rows 0..7, its
       // low terms in rows 8..15: accumulator rows gid + 8 hold the low part)
       const int vr = pg * 16 + ((mi & 1) << 3) + rr;
@@ -1976,8 +2125,8 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       for (int n2 = 0; n2 < NT / 2; ++n2) {
         uint32_t b00, b01, b10, b11;
         ldsm_x4_t(sw128_addr(vt, P, vr, ds * DW + n2 * 16 + ((mi >> 1) << 3)), b00, b01, b10, b11);
-        mma_16816(o[2 * n2], pa0, pb0, pa2, pb2, b00, b01);
-        mma_16816(o[2 * n2 + 1], pa0, pb0, pa2, pb2, b10, b11);
+        mma_16816t<KV8>(o[2 * n2], pa0, pb0, pa2, pb2, b00, b01);
+        mma_16816t<KV8>(o[2 * n2 + 1], pa0, pb0, pa2, pb2, b10, b11);
       }
     }
     __syncwarp();
@@ -2050,10 +2199,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
     consumer_sync();
     const unsigned long long tb0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
     if (kTraceAttn && p.trace && cx.tid == 0) ta[5] += tb0 - ta0;
-    if (!cx.ctl->flag) {
-      if (kTraceAttn && p.trace && cx.tid == 0) ta[1] += globaltimer() - tm0;
-      continue;
-    }
+    if (!cx.ctl->flag) continue;
     // ---- combine: contributors are CTAs c_first .. c_first + ncov - 1 (rows
     // 0..ncov-1); a CTA in that range with no chunk of this head contributes
     // nothing.  Each thread owns 4 consecutive output dims of one query head
@@ -2105,6 +2251,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       mlsrc = cp_ml;
       osrc = cp_o;
     }
+    if (kTraceAttn && p.trace && cx.tid == 0) ta[1] += globaltimer() - tb0;
     for (int o4 = cx.tid; o4 < GQ * D / 4; o4 += kConsumerThreads) {
       const int h = (o4 * 4) / D, dd = o4 * 4 - h * D;
       const float* mlh = mlsrc + h * 2;
@@ -2149,7 +2296,6 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       release_add(p.cnt + l * ST_LAYER + ST_ATTN, 1u);
       if (kTraceAttn && p.trace) {
         const unsigned long long te = globaltimer();
-        ta[1] += te - tm0;
         ta[6] += te - tb0;
       }
     }
@@ -2170,14 +2316,14 @@ __device__ __forceinline__ const Mat& stage_mat(const LayerParams& L, int kind) 
 }
 
 // Consumers: one stage.  Returns false once the CTA is aborting.
-template <int B, int D, bool MOE>
+template <int B, int D, bool MOE, bool KV8>
 __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s,
                                            RingPos& rp, bool fused) {
   const unsigned G = static_cast<unsigned>(p.G);
   const unsigned S1 = static_cast<unsigned>(p.step_base + s + 1);
   const int where = where_code(kind, l, s);
   if (kind == ST_ATTN) {
-    consume_attn<B, D>(p, cx, l, s, rp, fused);
+    consume_attn<B, D, KV8>(p, cx, l, s, rp, fused);
     const bool ab = consumer_sync_any(cx.ctl->abort != 0);
     if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 3);
     return !ab;
@@ -2306,7 +2452,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       if (kind == ST_QKV) {
         load_side<B>(p, cx, SIDE_ROPE, s, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-        EpiQKV<B> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
+        EpiQKV<B, KV8> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
         consume_tc(p, cx, L.qkv, rp, where, l == 0 ? SRC_EMBED : SRC_RESID, p.x, L.attn_norm, nullptr, epi);
       } else if (kind == ST_OPROJ) {
         load_side<B>(p, cx, l == 0 ? SIDE_EMBED : SIDE_RESID, s, where);
@@ -2339,7 +2485,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
                     rn, where);
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       }
-      EpiQKV<B> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
+      EpiQKV<B, KV8> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
       consume_gemv<B>(p, cx, L.qkv, rp, where, rn, epi);
       break;
     }
@@ -2477,7 +2623,7 @@ __device__ __forceinline__ void init_ring(const Params& p, Ctx& cx) {
 
 // Producer epilogue: wait until every issued copy has landed so the CTA's
 // shared memory is not released under an in-flight bulk copy.
-__device__ void drain_ring(const Params& p, Ctx& cx, const RingPos& rp, int issued) {
+static __device__ void drain_ring(const Params& p, Ctx& cx, const RingPos& rp, int issued) {
   if (issued <= 0) return;
   const int n = min(issued, p.nslot);
   RingPos q = rp;
@@ -2573,7 +2719,7 @@ struct Run {
   int stage, layer, step;
 };
 
-template <int B, bool MOE>
+template <int B, bool MOE, bool KV8>
 __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>& cu, Tile& t, Run* run) {
   while (!cu.done) {
     if (p.serve && !cu.open && !cu.one_stage && cu.kind == ST_QKV && cu.l == 0) {
@@ -2651,7 +2797,7 @@ __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>
         if (!ok) raise_error(p, kErrBadPage, where_code(ST_ATTN, cu.l, cu.s));   // row 0 is read instead
         t.rows = min(p.attn_pos_per_tile, p.pos0[b] + cu.s + 1 - j * p.attn_pos_per_tile);
         t.src = nullptr;
-        t.bytes = kTileBytes;
+        t.bytes = KV8 ? kTileBytes / 2 : kTileBytes;   // two boxes of P x d entries
         t.attn = true;
         return CUR_TILE;
       }
@@ -2801,7 +2947,7 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 }
 
 // Bounded wait of the producer for its CTA's routing of (step, layer).
-__device__ __noinline__ bool route_wait(const Params& p, SmemCtl* ctl, int want, int where) {
+static __device__ __noinline__ bool route_wait(const Params& p, SmemCtl* ctl, int want, int where) {
   const uint64_t t0 = globaltimer();
   while (ctl->route_seq != want) {
     if (ctl->abort) return false;
@@ -2824,7 +2970,7 @@ __device__ __noinline__ bool route_wait(const Params& p, SmemCtl* ctl, int want,
 // `p.l2_prefetch_bytes` ahead.  Weights do not depend on activations, so both
 // run ahead of the consumers across stage boundaries; only attention chunks
 // wait for the previous step's KV write of their layer.
-template <int B, bool MOE>
+template <int B, bool MOE, bool KV8>
 __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
   RingPos rp;
   const uint64_t pol = evict_first_policy();
@@ -2851,18 +2997,18 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
     bool t_attn = false;
     int t_stage, t_layer, t_step, t_y = 0;
     if (r_n1 + r_n2 == 0) {
-      int r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+      int r = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, cc, t, &nr);
       while (r == CUR_REQ) {
         // serve mode: the next step is not requested yet (bounded wait)
         if (!serve_gate(p, cx.ctl, cc.s, false) && serve_state(p, cc.s) >= 0) break;
-        r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+        r = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, cc, t, &nr);
       }
       if (r == CUR_REQ) break;
       if (r == CUR_BLOCKED) {
         // the next tile is an expert chosen by this CTA's own consumers: wait
         // (bounded) until they publish the layer's routing
         if (!route_wait(p, cx.ctl, route_want(p, cc.s, cc.l), where_code(cc.kind, cc.l, cc.s) | (1 << 15))) break;
-        r = cursor_next<B, MOE>(p, cx.c, cx.ctl, cc, t, &nr);
+        r = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, cc, t, &nr);
       }
       if (r == CUR_RUN) {
         r_src = nr.src;
@@ -2904,7 +3050,7 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
         ahead += nb;
         continue;
       }
-      const int pr = cursor_next<B, MOE>(p, cx.c, cx.ctl, pc, tp, &prun);
+      const int pr = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, pc, tp, &prun);
       if (pr == CUR_BLOCKED || pr == CUR_REQ) break;   // resume once the routing / the request is known
       if (pr == CUR_RUN) {
         pf_src = prun.src;
@@ -2918,10 +3064,11 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
       } else {
         // the chunk's existing K and V rows (contiguous, 16-byte multiples);
         // L2 is the coherence point, so a row rewritten later is still read fresh
-        const size_t off = static_cast<size_t>(tp.y) * p.d;
-        const uint32_t nb = static_cast<uint32_t>(tp.rows) * p.d * 2u;
-        prefetch_l2(p.kc + off, nb);
-        prefetch_l2(p.vc + off, nb);
+        constexpr int esz = KV8 ? 1 : 2;
+        const size_t off = static_cast<size_t>(tp.y) * p.d * esz;
+        const uint32_t nb = static_cast<uint32_t>(tp.rows) * p.d * esz;
+        prefetch_l2((KV8 ? p.kc8 : reinterpret_cast<const uint8_t*>(p.kc)) + off, nb);
+        prefetch_l2((KV8 ? p.vc8 : reinterpret_cast<const uint8_t*>(p.vc)) + off, nb);
       }
       ahead += tp.bytes;
     }
@@ -2954,7 +3101,11 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
     const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
     mbar_expect_tx(fb, tb);
     const uint32_t dst = smem_addr(cx.ring + static_cast<size_t>(rp.slot) * kSlotBytes);
-    if (t_attn) {
+    if (KV8 && t_attn) {
+      // e4m3 chunk: one box of P rows x d bytes each for K and V
+      tma_load_2d(dst, &p.tmap_k, 0, t_y, fb, pol);
+      tma_load_2d(dst + 8192, &p.tmap_v, 0, t_y, fb, pol);
+    } else if (t_attn) {
       const int box = p.attn_pos_per_tile * 128;
       for (int x = 0; x < p.d; x += 64) {
         tma_load_2d(dst + (x >> 6) * box, &p.tmap_k, x, t_y, fb, pol);
@@ -2970,7 +3121,7 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
   drain_ring(p, cx, rp, p.nslot);
 }
 
-template <int B, int D, bool MOE>
+template <int B, int D, bool MOE, bool KV8>
 __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
   RingPos rp;
   if (fused) {
@@ -2982,11 +3133,11 @@ __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
       }
       for (int l = 0; l < p.L; ++l)
         for (int k = 0; k < ST_LAYER; ++k)
-          if (!consume_stage<B, D, MOE>(p, cx, k, l, s, rp, true)) return;
-      if (!consume_stage<B, D, MOE>(p, cx, ST_LM, 0, s, rp, true)) return;
+          if (!consume_stage<B, D, MOE, KV8>(p, cx, k, l, s, rp, true)) return;
+      if (!consume_stage<B, D, MOE, KV8>(p, cx, ST_LM, 0, s, rp, true)) return;
     }
   } else {
-    consume_stage<B, D, MOE>(p, cx, kind0, l0, s0, rp, false);
+    consume_stage<B, D, MOE, KV8>(p, cx, kind0, l0, s0, rp, false);
   }
 }
 
@@ -3026,23 +3177,23 @@ __device__ __forceinline__ void tc_close(const Params& p, Ctx& cx) {
   }
 }
 
-template <int B, int D, bool MOE>
+template <int B, int D, bool MOE, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1) engine_persistent(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctx cx = make_ctx(smem, p);
   init_ring(p, cx);
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<B, MOE>(p, cx, 0, 0, 0, true);
+    if (cx.lane == 0) producer_main<B, MOE, KV8>(p, cx, 0, 0, 0, true);
     __syncwarp();
   } else {
     tc_open<B>(p, cx);
-    consumer_main<B, D, MOE>(p, cx, 0, 0, 0, true);
+    consumer_main<B, D, MOE, KV8>(p, cx, 0, 0, 0, true);
     tc_close<B>(p, cx);
   }
 }
 
 // Kernel-per-op baseline: one launch runs one stage (same tiles, no waits).
-template <int B, int D, bool MOE>
+template <int B, int D, bool MOE, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constant__ Params p, int kind,
                                                             int layer, int step) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -3058,11 +3209,11 @@ __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constan
     __syncthreads();
   }
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<B, MOE>(p, cx, kind, layer, step, false);
+    if (cx.lane == 0) producer_main<B, MOE, KV8>(p, cx, kind, layer, step, false);
     __syncwarp();
   } else {
     tc_open<B>(p, cx);
-    consumer_main<B, D, MOE>(p, cx, kind, layer, step, false);
+    consumer_main<B, D, MOE, KV8>(p, cx, kind, layer, step, false);
     tc_close<B>(p, cx);
   }
 }

@@ -182,8 +182,13 @@ struct Params {
   // 128-byte swizzle
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
-  uint16_t* kc;
+  uint16_t* kc;          // bf16 cache (null for an e4m3 cache)
   uint16_t* vc;
+  uint8_t* kc8;          // e4m3 cache: codes (null for a bf16 cache)
+  uint8_t* vc8;
+  int kv_fp8;            // 1: the cache holds e4m3 codes; entry = code * k_scale / v_scale
+  float k_inv, v_inv;    // 1 / k_scale, 1 / v_scale (powers of two)
+  float k_scale, v_scale;
   const int32_t* page_table;   // paged cache: [B][pages_per_seq] pool page of each chunk; null: contiguous
   int pages_per_seq;
   int n_pages;

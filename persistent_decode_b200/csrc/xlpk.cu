@@ -26,6 +26,7 @@
 
 #include "../../include/xlpk.h"
 #include "engine.cuh"
+#include "kernels.h"
 #include "params.h"
 
 using namespace xlpk;
@@ -262,31 +263,31 @@ struct xlpk_engine {
 
 namespace {
 
-template <int B, int D, bool MOE>
-void launch_stage_impl(const Params& p, int kind, int layer, int step, int G, int smem,
-                       cudaStream_t st) {
-  engine_stage<B, D, MOE><<<G, kThreads, smem, st>>>(p, kind, layer, step);
-}
-
 // Dense and MoE models use separate kernel instantiations, so the dense
-// kernels carry none of the routing code.
-template <int B, int D, bool MOE = false>
+// kernels carry none of the routing code; likewise bf16 and e4m3 caches, so
+// the bf16 kernels carry none of the e4m3 code (nor its register pressure).
+template <int B, int D, bool MOE = false, bool KV8 = false>
 void bind_kernels(xlpk_engine* e) {
-  e->kern_persistent = reinterpret_cast<const void*>(&engine_persistent<B, D, MOE>);
-  e->kern_stage = reinterpret_cast<const void*>(&engine_stage<B, D, MOE>);
-  e->launch_stage = &launch_stage_impl<B, D, MOE>;
+  const KernelSet k = kernel_set<B, D, MOE, KV8>();
+  e->kern_persistent = k.persistent;
+  e->kern_stage = k.stage;
+  e->launch_stage = k.launch_stage;
 }
 
-bool bind_by_shape(xlpk_engine* e, int B, int D, bool moe) {
-  if (moe) {   // MoE is built for batch 1
+bool bind_by_shape(xlpk_engine* e, int B, int D, bool moe, bool kv8) {
+  if (moe) {   // MoE is built for batch 1 with a bf16 cache
+    if (kv8) return false;
     if (B == 1 && D == 64) return bind_kernels<1, 64, true>(e), true;
     if (B == 1 && D == 128) return bind_kernels<1, 128, true>(e), true;
     return false;
   }
-#define XLPK_BIND(b, d)          \
-  if (B == b && D == d) {        \
-    bind_kernels<b, d>(e);       \
-    return true;                 \
+#define XLPK_BIND(b, d)                     \
+  if (B == b && D == d) {                   \
+    if (kv8)                                \
+      bind_kernels<b, d, false, true>(e);   \
+    else                                    \
+      bind_kernels<b, d>(e);                \
+    return true;                            \
   }
   XLPK_BIND(1, 64)
   XLPK_BIND(1, 128)
@@ -450,7 +451,10 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // tile's ldmatrix addressing expects).  The encoder is the driver's
 // cuTensorMapEncodeTiled, reached through the runtime's entry-point query so
 // the library does not link libcuda.
-xlpk_status encode_kv_map(CUtensorMap* map, void* base, unsigned long long rows, int d, int P) {
+// bf16 cache: boxes of 64 elements x P rows with the 128-byte swizzle (d/64
+// boxes per chunk).  e4m3 cache: one box of d bytes x P rows per chunk with the
+// 128-byte (d = 128) or 64-byte (d = 64) swizzle.
+xlpk_status encode_kv_map(CUtensorMap* map, void* base, unsigned long long rows, int d, int P, bool fp8 = false) {
   static PFN_cuTensorMapEncodeTiled encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -463,11 +467,12 @@ xlpk_status encode_kv_map(CUtensorMap* map, void* base, unsigned long long rows,
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
   }
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(P)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * (fp8 ? 1 : 2)};
+  const cuuint32_t box[2] = {fp8 ? static_cast<cuuint32_t>(d) : 64u, static_cast<cuuint32_t>(P)};
   const cuuint32_t estr[2] = {1u, 1u};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const CUtensorMapSwizzle sw = (fp8 && d == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUresult r = encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     g_cuda_err = "cuTensorMapEncodeTiled failed (" + std::to_string(static_cast<int>(r)) + ")";
@@ -486,6 +491,15 @@ xlpk_status validate_config(const xlpk_config* c) {
     return XLPK_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return XLPK_ERR_INVALID_ARG;
   if (c->n_ctas < 0 || c->spin_limit_us < 0) return XLPK_ERR_INVALID_ARG;
+  if (c->kv_dtype != XLPK_DTYPE_BF16 && c->kv_dtype != XLPK_DTYPE_FP8_E4M3) return XLPK_ERR_INVALID_ARG;
+  if (c->kv_dtype == XLPK_DTYPE_FP8_E4M3) {
+    // the scales are powers of two in [2^-24, 2^24]: every rescale is exact
+    for (const float sc : {c->k_scale, c->v_scale}) {
+      int ex = 0;
+      if (!(sc > 0.f) || !std::isfinite(sc) || std::frexp(sc, &ex) != 0.5f || ex - 1 < -24 || ex - 1 > 24)
+        return XLPK_ERR_INVALID_ARG;
+    }
+  }
   if (c->n_experts < 0 || c->top_k < 0 || c->n_shared_experts < 0 || c->expert_ffn < 0)
     return XLPK_ERR_INVALID_ARG;
   // shapes this build handles
@@ -525,6 +539,7 @@ xlpk_status validate_weights(const xlpk_config* c, const xlpk_weights* w, const 
     if ((reinterpret_cast<uintptr_t>(kv->page_table_dev) & 3u) || kv->page_size <= 0 || kv->n_pages <= 0)
       return XLPK_ERR_INVALID_ARG;
     // a page is one attention chunk (kTileBytes / 2 of K per chunk)
+    // (the same positions for an e4m3 cache: its page is half the bytes)
     if (kv->page_size != (kTileBytes / 2) / (c->head_dim * 2)) return XLPK_ERR_UNSUPPORTED;
   } else if (kv->page_size != 0 || kv->n_pages != 0) {
     return XLPK_ERR_INVALID_ARG;
@@ -723,7 +738,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
   e->smem = e->nslot * kSlotBytes + e->act_bytes + e->side_bytes + kMiscSmem;
-  if (!bind_by_shape(e, B, d, c.n_experts > 0)) return XLPK_ERR_UNSUPPORTED;
+  if (!bind_by_shape(e, B, d, c.n_experts > 0, c.kv_dtype == XLPK_DTYPE_FP8_E4M3)) return XLPK_ERR_UNSUPPORTED;
 
   // The attribute is per kernel function, shared by every handle that uses the
   // same instantiation: allow the device maximum rather than this handle's size.
@@ -971,8 +986,16 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.final_norm = final_norm_copy;
   p.lm = lm;
   p.layers = e->d_layers;
-  p.kc = static_cast<uint16_t*>(kv->k_dev);
-  p.vc = static_cast<uint16_t*>(kv->v_dev);
+  const bool kv8 = c.kv_dtype == XLPK_DTYPE_FP8_E4M3;
+  p.kv_fp8 = kv8 ? 1 : 0;
+  p.kc = kv8 ? nullptr : static_cast<uint16_t*>(kv->k_dev);
+  p.vc = kv8 ? nullptr : static_cast<uint16_t*>(kv->v_dev);
+  p.kc8 = kv8 ? static_cast<uint8_t*>(kv->k_dev) : nullptr;
+  p.vc8 = kv8 ? static_cast<uint8_t*>(kv->v_dev) : nullptr;
+  p.k_scale = kv8 ? c.k_scale : 1.f;
+  p.v_scale = kv8 ? c.v_scale : 1.f;
+  p.k_inv = 1.f / p.k_scale;   // exact: powers of two
+  p.v_inv = 1.f / p.v_scale;
   p.page_table = kv->page_table_dev;
   p.n_pages = kv->page_table_dev ? kv->n_pages : 0;
   p.pages_per_seq = (c.max_seq + e->P - 1) / e->P;
@@ -981,9 +1004,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
         kv->page_table_dev
             ? static_cast<unsigned long long>(c.n_layers) * kv->n_pages * c.n_kv_heads * static_cast<unsigned long long>(e->P)
             : static_cast<unsigned long long>(c.n_layers) * B * c.n_kv_heads * static_cast<unsigned long long>(c.max_seq);
-    xlpk_status st = encode_kv_map(&p.tmap_k, kv->k_dev, rows, d, e->P);
+    xlpk_status st = encode_kv_map(&p.tmap_k, kv->k_dev, rows, d, e->P, kv8);
     if (st != XLPK_OK) return st;
-    st = encode_kv_map(&p.tmap_v, kv->v_dev, rows, d, e->P);
+    st = encode_kv_map(&p.tmap_v, kv->v_dev, rows, d, e->P, kv8);
     if (st != XLPK_OK) return st;
   }
   p.rope = e->rope;

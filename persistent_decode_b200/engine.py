@@ -80,6 +80,12 @@ def make_config(cfg, n_ctas: int = 0, spin_limit_us: int = 0, batch: Optional[in
     c.spin_limit_us = int(spin_limit_us)
     c.flags = int(flags)
     c.window = int(window)
+    if getattr(cfg, "kv_dtype", "bf16") == "fp8_e4m3":
+        c.kv_dtype = _abi.XLPK_DTYPE_FP8_E4M3
+        c.k_scale = float(cfg.k_scale)
+        c.v_scale = float(cfg.v_scale)
+    else:
+        c.kv_dtype = _abi.XLPK_DTYPE_BF16
     return c
 
 
@@ -88,8 +94,9 @@ class Engine:
 
     `weights` maps names ("embed", "lm_head", "final_norm", "layers.{l}.wq", ...,
     with ".scale" companions for FP8) to CUDA tensors in row-major [out][in]
-    layout; `k_cache`/`v_cache` are bf16 CUDA tensors [L][B][n_kv][max_seq][d]
-    that the engine writes in place.  `flags` (XLPK_FLAG_*) and `window` are the
+    layout; `k_cache`/`v_cache` are CUDA tensors [L][B][n_kv][max_seq][d] (bf16,
+    or uint8 e4m3 codes when cfg.kv_dtype is "fp8_e4m3") that the engine writes
+    in place.  `flags` (XLPK_FLAG_*) and `window` are the
     config fields of the same names.
     """
 
@@ -97,6 +104,10 @@ class Engine:
                  spin_limit_us: int = 0, flags: int = 0, window: int = 0, page_table=None,
                  max_seq: Optional[int] = None):
         self.cfg = cfg
+        import torch
+        want = torch.uint8 if getattr(cfg, "kv_dtype", "bf16") == "fp8_e4m3" else torch.bfloat16
+        if k_cache.dtype != want or v_cache.dtype != want:
+            raise ValueError(f"KV cache must be {want} for kv_dtype {getattr(cfg, 'kv_dtype', 'bf16')}")
         if page_table is None:
             self.B = int(k_cache.shape[1])
             self.max_seq = int(k_cache.shape[3])

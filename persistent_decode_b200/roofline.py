@@ -36,7 +36,8 @@ def step_bytes(cfg, kv_positions: int, batch: int = None) -> int:
     """Bytes of one decode step whose new token lands at position `kv_positions`
     (so kv_positions + 1 entries are attended per sequence)."""
     B = cfg.batch if batch is None else batch
-    kv_entry = cfg.n_layers * cfg.n_kv_heads * cfg.head_dim * 2 * 2      # K and V, bf16
+    kv_esz = 1 if getattr(cfg, "kv_dtype", "bf16") == "fp8_e4m3" else 2
+    kv_entry = cfg.n_layers * cfg.n_kv_heads * cfg.head_dim * 2 * kv_esz   # K and V entries
     per_seq = kv_entry * (kv_positions + 1) + kv_entry + cfg.hidden * 2  # read, write, embed row
     return weight_bytes(cfg) + B * per_seq
 

@@ -62,6 +62,21 @@ def contiguous_view(m: "GpuModel", which: str = "k") -> torch.Tensor:
     return g.permute(0, 1, 3, 2, 4, 5).reshape(L, B, nkv, npg * P, d)[:, :, :, : m.engine.max_seq]
 
 
+def kv_dtype(cfg) -> torch.dtype:
+    """Element type of the cache tensors: bf16, or uint8 e4m3 codes."""
+    return torch.uint8 if getattr(cfg, "kv_dtype", "bf16") == "fp8_e4m3" else torch.bfloat16
+
+
+def kv_values(m: "GpuModel", which: str = "k") -> torch.Tensor:
+    """The cache entries' values as bf16 [L][B][n_kv][max_seq][d] (an e4m3 cache:
+    code * scale, exact in bf16)."""
+    c = contiguous_view(m, which)
+    if c.dtype != torch.uint8:
+        return c
+    scale = m.cfg.k_scale if which == "k" else m.cfg.v_scale
+    return (c.view(torch.float8_e4m3fn).float() * scale).to(torch.bfloat16)
+
+
 def build(cfg, device="cuda", norm_std: float = 0.0, n_ctas: int = 0, max_seq: Optional[int] = None,
           spin_limit_us: int = 0, weights: Optional[Dict[str, torch.Tensor]] = None, flags: int = 0,
           window: int = 0, paged: bool = False, spare_pages: int = 3, shared_prefix_pages: int = 0,
@@ -79,10 +94,10 @@ def build(cfg, device="cuda", norm_std: float = 0.0, n_ctas: int = 0, max_seq: O
         nps = (ms + P - 1) // P
         n_pages = B * nps + spare_pages
         pt = make_page_table(B, nps, n_pages, page_seed, shared_prefix_pages)
-        k = torch.zeros((cfg.n_layers, n_pages, cfg.n_kv_heads, P, cfg.head_dim), dtype=torch.bfloat16,
+        k = torch.zeros((cfg.n_layers, n_pages, cfg.n_kv_heads, P, cfg.head_dim), dtype=kv_dtype(cfg),
                         device=dev)
     else:
-        k = torch.zeros(kv_shape(cfg, B, ms), dtype=torch.bfloat16, device=dev)
+        k = torch.zeros(kv_shape(cfg, B, ms), dtype=kv_dtype(cfg), device=dev)
     v = torch.zeros_like(k)
     prompt = None
     if cfg.prefill:
@@ -93,6 +108,8 @@ def build(cfg, device="cuda", norm_std: float = 0.0, n_ctas: int = 0, max_seq: O
     else:
         for l in range(cfg.n_layers):
             kl, vl = synth.make_synthetic_kv(cfg, l, device=dev)
+            if k.dtype == torch.uint8:   # the e4m3 codes of those values (exact)
+                kl, vl = synth.fp8_kv_codes(kl, cfg.k_scale), synth.fp8_kv_codes(vl, cfg.v_scale)
             if pt is None:
                 k[l, :, :, : cfg.kv_len] = kl
                 v[l, :, :, : cfg.kv_len] = vl

@@ -15,6 +15,8 @@ from .gen import (  # noqa: F401
     make_weights,
     make_prompt,
     make_synthetic_kv,
+    fp8_kv_values,
+    fp8_kv_codes,
     make_start_tokens,
     stream_key,
 )

@@ -54,7 +54,11 @@ def test_host_side_argument_checks(lib):
     assert lib.xlpk_create(None, C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_INVALID_ARG
     # bad shapes are rejected before any CUDA call
     for bad in (dict(n_layers=0), dict(n_q_heads=3), dict(batch=0), dict(max_seq=0), dict(vocab=1),
-                dict(weight_dtype=7), dict(rope_theta=0.0)):
+                dict(weight_dtype=7), dict(rope_theta=0.0), dict(kv_dtype=2),
+                # e4m3 cache: scales must be powers of two in [2^-24, 2^24]
+                dict(kv_dtype=1, k_scale=0.3, v_scale=0.25), dict(kv_dtype=1, k_scale=0.0, v_scale=1.0),
+                dict(kv_dtype=1, k_scale=1.0, v_scale=2.0 ** -30), dict(kv_dtype=1, k_scale=-0.5, v_scale=0.5),
+                dict(kv_dtype=1, k_scale=float("inf"), v_scale=0.5)):
         c = _tiny_cfg(**bad)
         assert lib.xlpk_create(C.byref(c), C.byref(w), C.byref(kv), C.byref(h)) == _abi.XLPK_ERR_INVALID_ARG, bad
     # FP8: K dims must be multiples of 256 (a row pair of 2K + K/16 bytes stays 16-byte aligned)
