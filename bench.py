@@ -239,6 +239,8 @@ def dtype_label(cfg) -> str:
     """The arithmetic the decode runs in: weights as stored, fp32 accumulation."""
     if cfg.weight_dtype == "fp8_e4m3":
         w = "fp8_e4m3 weights (fp32 scale per 128x128 block)"
+    elif cfg.weight_dtype == "nvfp4":
+        w = "nvfp4 weights (e2m1, e4m3 scale per 16 elements, fp32 scale per matrix)"
     else:
         w = "bf16 weights"
     act = "fp32 activations"

@@ -55,9 +55,13 @@ typedef enum xlpk_status {
 
 typedef enum xlpk_dtype {
   XLPK_DTYPE_BF16 = 0,         /* bf16 weights, row-major [N][K] */
-  XLPK_DTYPE_FP8_E4M3 = 1      /* e4m3 codes, row-major [N][K], + one fp32 scale per 128x128 block;
+  XLPK_DTYPE_FP8_E4M3 = 1,     /* e4m3 codes, row-major [N][K], + one fp32 scale per 128x128 block;
                                   dense models only, hidden / n_q_heads*head_dim / ffn multiples
                                   of 256 and the other dims of 128 (else XLPK_ERR_UNSUPPORTED) */
+  XLPK_DTYPE_NVFP4 = 2         /* weights only: e2m1 codes [N][K/2] (element 2j in the low nibble of
+                                  byte j), one e4m3 scale per 16 consecutive elements of a row and one
+                                  fp32 scale per matrix (xlpk_linear); dense models at batch 1, hidden /
+                                  n_q_heads*head_dim / ffn multiples of 128 (else XLPK_ERR_UNSUPPORTED) */
 } xlpk_dtype;
 
 /* Model and launch shape.  All widths are element counts.
@@ -108,10 +112,16 @@ enum {
 };
 
 /* One linear weight: y = W x with W row-major [N][K] (PyTorch Linear layout).
- * `scale` is NULL for bf16; for FP8 it is fp32 [N/128][K/128], row-major. */
+ * `scale_dev` is NULL for bf16; for FP8 it is fp32 [N/128][K/128], row-major;
+ * for NVFP4 the e4m3 block scales, uint8 [N][K/16], and `global_scale` the
+ * matrix's fp32 scale (finite, > 0): element = e2m1 code * block scale *
+ * global_scale.  `global_scale` is ignored for the other types.
+ * Source: the NVFP4 bytes-per-token roofline ("Ultra-High Interactivity On
+ * NVIDIA GPUs? - TileRT InferenceX", digest, core views). */
 typedef struct xlpk_linear {
   const void* w_dev;
-  const float* scale_dev;
+  const void* scale_dev;
+  float global_scale;
 } xlpk_linear;
 
 typedef struct xlpk_layer_weights {
@@ -185,7 +195,9 @@ typedef struct xlpk_decode_io {
                                          stages, totals of thread 0: [6] ns waiting for KV chunks,
                                          [7] ns of the combining CTA's wait for the partials,
                                          [8] q loads, [9] chunk math, [10] merge,
-                                         [11] arrive, [12] combine, [13] chunks processed.
+                                         [11] arrive, [12] combine, [13] chunks processed; for the
+                                         other stages, thread 0's input staging: [6] copies issued,
+                                         [7] landed, [8] converted, [9] RMSNorm factor ready.
                                          n_stages = 5 * n_layers + 1 */
   int32_t withhold_release;           /* failure-detection testing only: 1 + the index (layer * 5 +
                                          stage kind, n_layers * 5 = LM head) of a stage whose

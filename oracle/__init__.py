@@ -16,6 +16,7 @@ synthetic models has no printed worked example on the pages: beyond those pins
 it is "parity unpinned" (no page prints a decoded sequence or logit for them).
 """
 from .fp8 import e4m3_decode_table, e4m3_encode, e4m3_to_fp32  # noqa: F401
+from .fp4 import e2m1_decode_table, nvfp4_dequant  # noqa: F401
 from .decoder import (  # noqa: F401
     rms_norm,
     rope_rotate,

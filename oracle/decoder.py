@@ -36,6 +36,7 @@ from typing import Dict, List, Optional, Tuple
 
 import torch
 
+from .fp4 import nvfp4_dequant
 from .fp8 import e4m3_encode, e4m3_to_fp32
 
 
@@ -151,6 +152,9 @@ class OracleDecoder:
     # weights widened to fp32 on use
     def W(self, name: str) -> torch.Tensor:
         t = self.w[name]
+        if t.dtype == torch.uint8 and (name + ".gscale") in self.w:
+            # NVFP4: e2m1 codes, an e4m3 scale per 16 elements of a row, an fp32 tensor scale
+            return nvfp4_dequant(t, self.w[name + ".scale"], float(self.w[name + ".gscale"].reshape(-1)[0]))
         if t.dtype == torch.uint8:
             sc = self.w[name + ".scale"]
             N, K = t.shape

@@ -20,6 +20,7 @@ XLPK_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 XLPK_DTYPE_BF16 = 0
 XLPK_DTYPE_FP8_E4M3 = 1
+XLPK_DTYPE_NVFP4 = 2
 
 XLPK_FLAG_NO_FUSED_FFN = 1
 XLPK_FLAG_NO_TENSOR_CORES = 2
@@ -37,7 +38,7 @@ class xlpk_config(C.Structure):
 
 
 class xlpk_linear(C.Structure):
-    _fields_ = [("w_dev", C.c_void_p), ("scale_dev", C.c_void_p)]
+    _fields_ = [("w_dev", C.c_void_p), ("scale_dev", C.c_void_p), ("global_scale", C.c_float)]
 
 
 class xlpk_layer_weights(C.Structure):

@@ -62,8 +62,8 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str = Non
             cmd, _ = pending.pop(0)
             running.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
         cmd, proc = running.pop(0)
-        out, _ = proc.communicate()
-        logs.append(" ".join(cmd) + "\n" + out)
+        text, _ = proc.communicate()
+        logs.append(" ".join(cmd) + "\n" + text)
         failed = failed or proc.returncode != 0
     tmp = target + ".tmp"
     if not failed:

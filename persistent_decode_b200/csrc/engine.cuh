@@ -34,6 +34,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -98,6 +99,11 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t a) {
 __device__ __forceinline__ uint2 lds_u2(uint32_t a) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds_u1(uint32_t a) {
@@ -365,6 +371,16 @@ __device__ __forceinline__ void raise_error(const Params& p, int code, int where
 // layer l) is in its table.
 __device__ __forceinline__ int route_want(const Params& p, int s, int l) { return s * p.L + l + 1; }
 
+// Timers of stage internals (trace slots 6..13: the attention stage's phases,
+// the other stages' input staging): a diagnostic build's option
+// (-DXLPK_TRACE_ATTN); the values they keep live cost the release kernel about
+// 2 % of a step on the 8B shape.
+#ifdef XLPK_TRACE_ATTN
+constexpr bool kTraceAttn = true;
+#else
+constexpr bool kTraceAttn = false;
+#endif
+
 __device__ __forceinline__ int where_code(int kind, int layer, int step) {
   return (step << 16) | ((layer & 0xff) << 8) | (kind & 0xff);
 }
@@ -555,6 +571,30 @@ __device__ __forceinline__ float dot16_e4m3(const uint4 w, const float4 x0, cons
   return acc;
 }
 
+// Two e2m1 codes (one byte, the low nibble first) -> two floats, through the
+// CUDA fp4 conversion to half precision (every e2m1 value is exact).
+__device__ __forceinline__ float2 e2m1x2_to_float2(uint32_t byte) {
+  const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Sum over 16 e2m1 codes (two 32-bit words, element 2j in the low nibble of
+// byte j) times 16 fp32 activations x0 = elements 0..3, .., x3 = 12..15.
+__device__ __forceinline__ float dot16_e2m1(uint32_t a, uint32_t b, const float4 x0, const float4 x1,
+                                           const float4 x2, const float4 x3) {
+  float acc = 0.f;
+  float2 f;
+  f = e2m1x2_to_float2(a & 0xffu);          acc = fmaf(f.x, x0.x, fmaf(f.y, x0.y, acc));
+  f = e2m1x2_to_float2((a >> 8) & 0xffu);   acc = fmaf(f.x, x0.z, fmaf(f.y, x0.w, acc));
+  f = e2m1x2_to_float2((a >> 16) & 0xffu);  acc = fmaf(f.x, x1.x, fmaf(f.y, x1.y, acc));
+  f = e2m1x2_to_float2(a >> 24);            acc = fmaf(f.x, x1.z, fmaf(f.y, x1.w, acc));
+  f = e2m1x2_to_float2(b & 0xffu);          acc = fmaf(f.x, x2.x, fmaf(f.y, x2.y, acc));
+  f = e2m1x2_to_float2((b >> 8) & 0xffu);   acc = fmaf(f.x, x2.z, fmaf(f.y, x2.w, acc));
+  f = e2m1x2_to_float2((b >> 16) & 0xffu);  acc = fmaf(f.x, x3.x, fmaf(f.y, x3.y, acc));
+  f = e2m1x2_to_float2(b >> 24);            acc = fmaf(f.x, x3.z, fmaf(f.y, x3.w, acc));
+  return acc;
+}
+
 __device__ __forceinline__ uint16_t f2bf(float v) {
   __nv_bfloat16 h = __float2bfloat16_rn(v);
   return *reinterpret_cast<uint16_t*>(&h);
@@ -656,6 +696,12 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
                                       float (&rn)[B], int where) {
   const float* gsrc = static_cast<const float*>(gsrc_v);
   const bool direct = src == SRC_FIXED;
+  // diagnostic build (XLPK_TRACE_ATTN): thread 0's progress through the input
+  // staging in trace slots 6..9 (copies issued, landed, converted, reduced)
+  auto tstamp = [&](int k) {
+    if (kTraceAttn && p.trace && cx.tid == 0)
+      trace_stamp(p, where >> 16, stage_index(p, where & 0xff, (where >> 8) & 0xff), k);
+  };
   const int nvK = K >> 3;
   const int n4 = K >> 2;
   float4* act4 = reinterpret_cast<float4*>(cx.act);
@@ -684,6 +730,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     if (side == SIDE_RESID)
       total += p.resid_fixed ? static_cast<uint32_t>(B) * (r1 - r0) * 8u : static_cast<uint32_t>(B) * 2u * nv * 16u;
     if (side == SIDE_EMBED && r1 > r0) total += static_cast<uint32_t>(B) * (e1 - e0) * 2u;
+    tstamp(6);
     mbar_expect_tx(bar, total);
     if (src != SRC_EMBED && !direct)
       bulk_g2s_nohint(smem_addr(cx.act), gsrc, static_cast<uint32_t>(B) * K * 4u, bar);
@@ -729,6 +776,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     if (!cx.ctl->abort) ring_wait(p, cx.ctl, bar, cx.act_phase, where);
     if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
     cx.act_phase ^= 1u;
+    tstamp(7);
     const uint32_t stage = smem_addr(cx.act) + static_cast<uint32_t>(B) * K * 4u;
     float ss[B];
 #pragma unroll
@@ -754,6 +802,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     }
 #pragma unroll
     for (int b = 0; b < B; ++b) rn[b] = 1.f;
+    tstamp(8);
     if (gain) {
 #pragma unroll
       for (int b = 0; b < B; ++b) {
@@ -771,6 +820,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
     } else {
       consumer_sync();
     }
+    tstamp(9);
     return;
   }
   }
@@ -802,6 +852,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
   // even when aborting, the copies must land before the CTA may exit
   if (cx.ctl->abort) copy_wait(p, bar, cx.act_phase);
   cx.act_phase ^= 1u;
+  tstamp(7);
   if (hidden_dbg) {
     if (src == SRC_EMBED) consumer_sync();
     for (int k = cx.tid; k < K; k += kConsumerThreads)
@@ -827,6 +878,7 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
         a = make_float4(x.x * g4.x, x.y * g4.y, x.z * g4.z, x.w * g4.w);
       }
     }
+    tstamp(8);
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       const float t = warp_sum(ss[b]);
@@ -843,15 +895,17 @@ __device__ __noinline__ void load_act(const Params& p, Ctx& cx, int K, ActSrc sr
   } else if (src == SRC_EMBED) {
     consumer_sync();
   }
+  tstamp(9);
 }
 
 // ------------------------------------------------------------------ GEMV stages
 
 // Consumer side: each warp owns one row pair of every tile of a group and
 // accumulates it over the group's k-chunks; `epi(pair, acc0, acc1)` runs on
-// the reduced sums (identical in every lane).
+// the reduced sums (identical in every lane).  WF: 0 bf16, 1 e4m3 (fp32 scale
+// per 128x128 block), 2 NVFP4 (e4m3 scale per 16 columns, matrix scale per row).
 // [q0, q1) overrides the CTA's pair range (default: the even split of m's pairs).
-template <int B, bool FP8, class Epi>
+template <int B, int WF, class Epi>
 __device__ __noinline__ void consume_gemv_t(const Params& p, Ctx& cx, const Mat& m, RingPos& rp,
                                             int where, const float (&rn)[B], Epi& epi, int q0, int q1) {
   const int NP = m.N >> 1;
@@ -871,7 +925,40 @@ __device__ __noinline__ void consume_gemv_t(const Params& p, Ctx& cx, const Mat&
     for (int kc = 0; kc < nkc; ++kc) {
       const uint32_t fb = smem_addr(&cx.ctl->full[rp.slot]);
       const bool ok = cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where);
-      if constexpr (FP8) {
+      if constexpr (WF == 2) {
+        if (ok && cx.warp < gp) {
+          // NVFP4 tile: [2gp rows][KC/2 code bytes] then [2gp rows][KC/16 e4m3
+          // scales]; lane vectors of 32 codes (16 bytes) = two 16-column scale
+          // blocks, each block's sum scaled once
+          const int nv32 = KC >> 5;
+          const uint32_t base = smem_addr(cx.ring) + rp.slot * kSlotBytes;
+          const uint32_t r0 = base + (2 * cx.warp) * (KC >> 1);
+          const uint32_t r1 = r0 + (KC >> 1);
+          const uint32_t s0 = base + gp * KC + (2 * cx.warp) * (KC >> 4);
+          const uint32_t s1 = s0 + (KC >> 4);
+          const uint32_t alo = act_lo_s + ((kc * KC) >> 3) * 16;
+          const uint32_t ahi = act_hi_s + ((kc * KC) >> 3) * 16;
+#pragma unroll 2
+          for (int v = cx.lane; v < nv32; v += 32) {
+            const uint4 w0 = lds_u4(r0 + v * 16);
+            const uint4 w1 = lds_u4(r1 + v * 16);
+            const float2 sc0 = e4m3x2_to_float2(lds_u16(s0 + v * 2));
+            const float2 sc1 = e4m3x2_to_float2(lds_u16(s1 + v * 2));
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              const uint32_t xv = (b * nvK + 4 * v) * 16;
+              const float4 x0 = lds_f4(alo + xv), x1 = lds_f4(ahi + xv);
+              const float4 x2 = lds_f4(alo + xv + 16), x3 = lds_f4(ahi + xv + 16);
+              const float4 x4 = lds_f4(alo + xv + 32), x5 = lds_f4(ahi + xv + 32);
+              const float4 x6 = lds_f4(alo + xv + 48), x7 = lds_f4(ahi + xv + 48);
+              a0[b] = fmaf(sc0.x, dot16_e2m1(w0.x, w0.y, x0, x1, x2, x3), a0[b]);
+              a0[b] = fmaf(sc0.y, dot16_e2m1(w0.z, w0.w, x4, x5, x6, x7), a0[b]);
+              a1[b] = fmaf(sc1.x, dot16_e2m1(w1.x, w1.y, x0, x1, x2, x3), a1[b]);
+              a1[b] = fmaf(sc1.y, dot16_e2m1(w1.z, w1.w, x4, x5, x6, x7), a1[b]);
+            }
+          }
+        }
+      } else if constexpr (WF == 1) {
         if (ok && cx.warp < gp) {
         // e4m3 tile: lane vectors of 16 codes, each inside one 128-column
         // scale block; the block's sum is scaled once
@@ -926,10 +1013,12 @@ __device__ __noinline__ void consume_gemv_t(const Params& p, Ctx& cx, const Mat&
       rp.next(p.nslot);
     }
     if (cx.warp < gp) {
+      // NVFP4: the rows' matrix scales
+      const float2 gs = WF == 2 ? __ldg(m.gsc + g0 + cx.warp) : make_float2(1.f, 1.f);
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        a0[b] = warp_sum(a0[b]) * rn[b];
-        a1[b] = warp_sum(a1[b]) * rn[b];
+        a0[b] = warp_sum(a0[b]) * (WF == 2 ? rn[b] * gs.x : rn[b]);
+        a1[b] = warp_sum(a1[b]) * (WF == 2 ? rn[b] * gs.y : rn[b]);
       }
       epi(g0 + cx.warp, a0, a1, cx.lane);
     }
@@ -1372,10 +1461,16 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
 template <int B, class Epi>
 __device__ __forceinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where,
                                              const float (&rn)[B], Epi& epi, int q0 = -1, int q1 = -1) {
+  if constexpr (B == 1) {   // NVFP4 weights are built for batch 1
+    if (m.fp4) {
+      consume_gemv_t<B, 2>(p, cx, m, rp, where, rn, epi, q0, q1);
+      return;
+    }
+  }
   if (m.fp8)
-    consume_gemv_t<B, true>(p, cx, m, rp, where, rn, epi, q0, q1);
+    consume_gemv_t<B, 1>(p, cx, m, rp, where, rn, epi, q0, q1);
   else
-    consume_gemv_t<B, false>(p, cx, m, rp, where, rn, epi, q0, q1);
+    consume_gemv_t<B, 0>(p, cx, m, rp, where, rn, epi, q0, q1);
 }
 
 __device__ __forceinline__ size_t kv_row(const Params& p, int l, int b, int g, int t, bool& ok);
@@ -1825,14 +1920,6 @@ __host__ __device__ constexpr int attn_scratch_floats(int D, int G) {
          + 3 * G * kMaxGroup + 2 * kMaxGroup;   // combine: (M, L, weight) per contributor, M*, L*
 }
 
-// Timers of the attention stage's internals (trace slots 6..13): a
-// diagnostic build's option (-DXLPK_TRACE_ATTN); the values they keep live cost
-// the release kernel about 2 % of a step on the 8B shape.
-#ifdef XLPK_TRACE_ATTN
-constexpr bool kTraceAttn = true;
-#else
-constexpr bool kTraceAttn = false;
-#endif
 
 // Flash-decoding over this CTA's chunks of the (sequence, kv head) space on
 // warp-level tensor cores.  A chunk is P = 64 (d=128) or 128 (d=64) positions

@@ -66,16 +66,18 @@ struct CounterLayout {
 // bulk copy; a packed row then takes K + K/32 bytes.
 struct Mat {
   const uint8_t* packed;
-  const float* scales;   // unused (FP8 scales travel inside the tiles)
+  const float2* gsc;     // NVFP4: per row pair, the two rows' matrix scales; else null
   int N;                 // logical rows (even)
   int K;                 // columns
   int KC;                // k-chunk (divides K)
-  int fp8;               // 1: e4m3 codes + in-tile block scales; 0: bf16
+  int fp8;               // 1: e4m3 codes + in-tile fp32 scales per 128x128 block
+  int fp4;               // 1: NVFP4 e2m1 codes + in-tile e4m3 scales per 16 columns (and gsc)
 };
 
-// Bytes of one packed row over `k` columns (codes or bf16 values, plus FP8 scales).
+// Bytes of one packed row over `k` columns (codes or bf16 values, plus the
+// in-tile block scales: FP8 one fp32 per 128 columns, NVFP4 one byte per 16).
 __host__ __device__ __forceinline__ int packed_row_bytes(const Mat& m, int k) {
-  return m.fp8 ? k + k / 32 : 2 * k;
+  return m.fp4 ? k / 2 + k / 16 : m.fp8 ? k + k / 32 : 2 * k;
 }
 
 // ------------------------------------------------------------------ batch-8 tensor-core tiles

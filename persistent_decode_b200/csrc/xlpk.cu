@@ -48,7 +48,7 @@ xlpk_status cuda_fail(cudaError_t e, const char* what) {
 
 struct PackJob {
   const uint8_t* src;   // source row
-  const float* scale;   // FP8: the row's block-scale row ([K/128] fp32), else null
+  const void* scale;    // FP8: the row's block-scale row ([K/128] fp32); NVFP4: [K/16] e4m3; else null
   long long base;       // byte offset of the CTA's span in the packed buffer
   int row;              // row inside its tile (2 * pair-in-group + 0/1)
   int j16;              // rows of the span before this row's group
@@ -92,7 +92,23 @@ __global__ void pack_scales_kernel(const PackJob* jobs, int njobs, uint8_t* out,
   const int kb_per_chunk = kc_cols / 128;
   float* d = reinterpret_cast<float*>(out + pack_tile_offset(j, c, nchunk, cw, tile_row) +
                                       static_cast<long long>(j.gp2) * kc_cols + j.row * (kc_cols / 32));
-  for (int k = 0; k < kb_per_chunk; ++k) d[k] = j.scale[c * kb_per_chunk + k];
+  const float* sr = static_cast<const float*>(j.scale);
+  for (int k = 0; k < kb_per_chunk; ++k) d[k] = sr[c * kb_per_chunk + k];
+}
+
+// NVFP4: one thread per (row, chunk): the chunk's KC/16 e4m3 block scales of
+// the row, after the tile's code rows ([gp2 rows][KC/2 bytes]).
+__global__ void pack_scales4_kernel(const PackJob* jobs, int njobs, uint8_t* out, int nchunk, int kc_cols, int cw,
+                                    long long tile_row) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= static_cast<long long>(njobs) * nchunk) return;
+  const int jb = static_cast<int>(t / nchunk), c = static_cast<int>(t - static_cast<long long>(jb) * nchunk);
+  const PackJob j = jobs[jb];
+  const int nb = kc_cols / 16;
+  uint8_t* d = out + pack_tile_offset(j, c, nchunk, cw, tile_row) + static_cast<long long>(j.gp2) * (kc_cols / 2) +
+               static_cast<long long>(j.row) * nb;
+  const uint8_t* sr = static_cast<const uint8_t*>(j.scale) + static_cast<long long>(c) * nb;
+  for (int k = 0; k < nb; ++k) d[k] = sr[k];
 }
 
 // One warp per packed row: chunk c of the row goes to its tile (pack_tile_offset).
@@ -182,8 +198,14 @@ __global__ void pack_tc_scales_kernel(const TcRowJob* jobs, int njobs, uint8_t* 
 }
 
 // Largest k-chunk dividing K whose tile of 8 row pairs fits kTileBytes (FP8:
-// also a whole number of 128-column scale blocks).
-int pick_kc(int K, int esz) {
+// also a whole number of 128-column scale blocks; NVFP4: rows of KC/2 code
+// bytes + KC/16 scale bytes, KC a multiple of 128 so tiles stay 16-byte sized).
+int pick_kc(int K, int esz, bool fp4 = false) {
+  if (fp4) {
+    for (int kc = std::min(K, kTileBytes * 16 / (2 * kPairsPerTile * 9)); kc >= 128; --kc)
+      if (K % kc == 0 && kc % 128 == 0) return kc;
+    return 0;
+  }
   const int vec = esz == 1 ? 128 : 16 / esz;
   const int cap = kTileBytes / (2 * kPairsPerTile * esz);
   for (int kc = std::min(K, cap); kc >= vec; --kc)
@@ -192,6 +214,7 @@ int pick_kc(int K, int esz) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 enum class MatKind { QKV, PLAIN, GATEUP };
 
@@ -200,14 +223,16 @@ struct MatSrc {
   const uint8_t* a;   // QKV: wq; GATEUP: gate; PLAIN: w
   const uint8_t* b;   // QKV: wk; GATEUP: up
   const uint8_t* c;   // QKV: wv
-  const float* sa = nullptr;   // FP8 block scales [rows/128][K/128] of a, b, c
-  const float* sb = nullptr;
-  const float* sc = nullptr;
+  const void* sa = nullptr;   // block scales of a, b, c: FP8 fp32 [rows/128][K/128], NVFP4 e4m3 [rows][K/16]
+  const void* sb = nullptr;
+  const void* sc = nullptr;
+  float ga = 1.f, gb = 1.f, gc = 1.f;   // NVFP4: the matrix scales of a, b, c
 };
 
 struct SrcRow {
   const uint8_t* w;
-  const float* s;   // FP8: the row's block-scale row
+  const void* s;   // the row's block-scale row (FP8: fp32, NVFP4: e4m3), else null
+  float g;         // NVFP4: the source matrix's scale
 };
 
 }  // namespace
@@ -226,7 +251,8 @@ struct xlpk_engine {
   int tc_cols = 0;
   int down_win = 0;            // K-windowed down projection (columns per window; 0: off)
   int tc_win = 0;              // K window of the tensor-core projections (0: whole K)
-  int esz = 2;
+  int esz = 2;                 // bytes per weight element (1: e4m3 codes, or NVFP4 with fp4 set)
+  bool fp4 = false;            // NVFP4 weights
   int P = 0;
   uint8_t* packed = nullptr;
   size_t packed_bytes = 0;
@@ -301,20 +327,21 @@ bool bind_by_shape(xlpk_engine* e, int B, int D, bool moe, bool kv8) {
   return false;
 }
 
-// Logical row n of a packed matrix -> source row (and its FP8 block-scale row).
-SrcRow source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_config& c) {
-  const long long row_bytes = static_cast<long long>(K) * esz;
+// Logical row n of a packed matrix -> source row (and its block-scale row).
+SrcRow source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_config& c, bool fp4 = false) {
+  const long long row_bytes = fp4 ? K / 2 : static_cast<long long>(K) * esz;
   const long long pr = n >> 1;
   const int r = static_cast<int>(n & 1);
   const uint8_t* base = nullptr;
-  const float* sbase = nullptr;
+  const void* sbase = nullptr;
+  float g = 1.f;
   long long row = 0;
   switch (ms.kind) {
     case MatKind::PLAIN:
-      base = ms.a, sbase = ms.sa, row = n;
+      base = ms.a, sbase = ms.sa, g = ms.ga, row = n;
       break;
     case MatKind::GATEUP:
-      base = r == 0 ? ms.a : ms.b, sbase = r == 0 ? ms.sa : ms.sb, row = pr;
+      base = r == 0 ? ms.a : ms.b, sbase = r == 0 ? ms.sa : ms.sb, g = r == 0 ? ms.ga : ms.gb, row = pr;
       break;
     case MatKind::QKV: {
       const long long half = c.head_dim / 2;
@@ -325,17 +352,23 @@ SrcRow source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_conf
         const long long pp = isq ? pr : pr - hq;
         const long long head = pp / half, i = pp % half;
         row = head * c.head_dim + i + r * half;
-        base = isq ? ms.a : ms.b, sbase = isq ? ms.sa : ms.sb;
+        base = isq ? ms.a : ms.b, sbase = isq ? ms.sa : ms.sb, g = isq ? ms.ga : ms.gb;
       } else {
         row = 2 * (pr - hq - hk) + r;
-        base = ms.c, sbase = ms.sc;
+        base = ms.c, sbase = ms.sc, g = ms.gc;
       }
       break;
     }
   }
   SrcRow out;
   out.w = base + row * row_bytes;
-  out.s = sbase ? sbase + (row / 128) * (K / 128) : nullptr;
+  if (!sbase)
+    out.s = nullptr;
+  else if (fp4)
+    out.s = static_cast<const uint8_t*>(sbase) + row * (K / 16);
+  else
+    out.s = static_cast<const float*>(sbase) + (row / 128) * (K / 128);
+  out.g = g;
   return out;
 }
 
@@ -345,18 +378,20 @@ SrcRow source_row(const MatSrc& ms, long long n, int K, int esz, const xlpk_conf
 xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t* dst, Mat* out,
                         PackJob* d_jobs, size_t max_jobs, cudaStream_t st, int split, int win_cols = 0) {
   const int esz = e->esz;
-  const int KC = pick_kc(K, esz);
+  const bool fp4 = e->fp4 && esz == 1;   // (the MoE router stays bf16)
+  const int KC = pick_kc(K, esz, fp4);
   if (KC == 0) return XLPK_ERR_UNSUPPORTED;
-  const bool fp8 = esz == 1;
-  if (fp8 && (!ms.sa || (ms.kind != MatKind::PLAIN && !ms.sb) || (ms.kind == MatKind::QKV && !ms.sc)))
+  const bool fp8 = esz == 1 && !fp4;
+  if ((fp8 || fp4) && (!ms.sa || (ms.kind != MatKind::PLAIN && !ms.sb) || (ms.kind == MatKind::QKV && !ms.sc)))
     return XLPK_ERR_INVALID_ARG;
   const int nkc = K / KC;
   // chunks per window: the whole K unless the matrix is streamed window by window
   const int cw = win_cols > 0 ? win_cols / KC : nkc;
   if (cw < 1 || (win_cols > 0 && win_cols % KC)) return XLPK_ERR_UNSUPPORTED;
-  // bytes per packed row over a chunk / over K (codes + FP8 block scales)
-  const long long tile_row = static_cast<long long>(KC) * esz + (fp8 ? KC / 32 : 0);
-  const long long full_row = static_cast<long long>(K) * esz + (fp8 ? K / 32 : 0);
+  // bytes per packed row over a chunk / over K (codes + block scales)
+  const long long tile_row =
+      fp4 ? KC / 2 + KC / 16 : static_cast<long long>(KC) * esz + (fp8 ? KC / 32 : 0);
+  const long long full_row = fp4 ? K / 2 + K / 16 : static_cast<long long>(K) * esz + (fp8 ? K / 32 : 0);
   const long long NP = N / 2, G = split;
   std::vector<PackJob> jobs;
   jobs.reserve(static_cast<size_t>(N));
@@ -367,7 +402,7 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
       const long long j = lp / kPairsPerTile, w = lp % kPairsPerTile;
       const long long gp = std::min<long long>(kPairsPerTile, npc - kPairsPerTile * j);
       for (int r = 0; r < 2; ++r) {
-        const SrcRow sr = source_row(ms, 2 * (p0 + lp) + r, K, esz, e->cfg);
+        const SrcRow sr = source_row(ms, 2 * (p0 + lp) + r, K, esz, e->cfg, fp4);
         PackJob pj;
         pj.src = sr.w;
         pj.scale = sr.s;
@@ -380,7 +415,7 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
       }
     }
   }
-  const int row_bytes = K * esz, chunk_bytes = KC * esz;
+  const int row_bytes = fp4 ? K / 2 : K * esz, chunk_bytes = fp4 ? KC / 2 : KC * esz;
   for (size_t off = 0; off < jobs.size(); off += max_jobs) {
     const size_t n = std::min(max_jobs, jobs.size() - off);
     XLPK_CUDA(cudaMemcpyAsync(d_jobs, jobs.data() + off, n * sizeof(PackJob), cudaMemcpyHostToDevice, st));
@@ -394,15 +429,30 @@ xlpk_status pack_matrix(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8_t*
       pack_scales_kernel<<<static_cast<int>((nt + threads - 1) / threads), threads, 0, st>>>(
           d_jobs, static_cast<int>(n), dst, nkc, KC, cw, tile_row);
       XLPK_CUDA(cudaGetLastError());
+    } else if (fp4) {
+      const long long nt = static_cast<long long>(n) * nkc;
+      pack_scales4_kernel<<<static_cast<int>((nt + threads - 1) / threads), threads, 0, st>>>(
+          d_jobs, static_cast<int>(n), dst, nkc, KC, cw, tile_row);
+      XLPK_CUDA(cudaGetLastError());
     }
     XLPK_CUDA(cudaStreamSynchronize(st));
   }
   out->packed = dst;
-  out->scales = nullptr;
+  out->gsc = nullptr;
   out->N = N;
   out->K = K;
   out->KC = KC;
   out->fp8 = fp8 ? 1 : 0;
+  out->fp4 = fp4 ? 1 : 0;
+  if (fp4) {
+    // the rows' matrix scales per row pair, behind the packed rows (16-byte aligned)
+    std::vector<float> gs(static_cast<size_t>(N));
+    for (long long n = 0; n < N; ++n) gs[n] = source_row(ms, n, K, esz, e->cfg, true).g;
+    float* d = reinterpret_cast<float*>(dst + align_up(static_cast<size_t>(N) * full_row, 16));
+    XLPK_CUDA(cudaMemcpyAsync(d, gs.data(), gs.size() * sizeof(float), cudaMemcpyHostToDevice, st));
+    XLPK_CUDA(cudaStreamSynchronize(st));
+    out->gsc = reinterpret_cast<const float2*>(d);
+  }
   return XLPK_OK;
 }
 
@@ -417,7 +467,7 @@ xlpk_status pack_matrix_tc(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8
   std::vector<TcRowJob> jobs(static_cast<size_t>(N));
   for (int n = 0; n < N; ++n) {
     const SrcRow sr = source_row(ms, n, K, esz, e->cfg);
-    jobs[n] = TcRowJob{sr.w, sr.s, n};
+    jobs[n] = TcRowJob{sr.w, static_cast<const float*>(sr.s), n};
   }
   const TcGeom g{N, K, e->G, win_cols, fp8 ? 1 : 0};
   for (size_t off = 0; off < jobs.size(); off += max_jobs) {
@@ -436,7 +486,7 @@ xlpk_status pack_matrix_tc(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8
     XLPK_CUDA(cudaStreamSynchronize(st));
   }
   out->packed = dst;
-  out->scales = nullptr;
+  out->gsc = nullptr;
   out->N = N;
   out->K = K;
   out->KC = bc;
@@ -444,7 +494,6 @@ xlpk_status pack_matrix_tc(xlpk_engine* e, const MatSrc& ms, int N, int K, uint8
   return XLPK_OK;
 }
 
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Tensor map of one KV cache viewed as a 2-D [rows][d] bf16 array, read in
 // boxes of 64 columns x P rows with 128-byte swizzle (the layout the attention
@@ -487,7 +536,8 @@ xlpk_status validate_config(const xlpk_config* c) {
       c->n_kv_heads <= 0 || c->head_dim <= 0 || c->vocab <= 1 || c->batch < 1 || c->max_seq < 1)
     return XLPK_ERR_INVALID_ARG;
   if (c->n_q_heads % c->n_kv_heads != 0) return XLPK_ERR_INVALID_ARG;
-  if (c->weight_dtype != XLPK_DTYPE_BF16 && c->weight_dtype != XLPK_DTYPE_FP8_E4M3)
+  if (c->weight_dtype != XLPK_DTYPE_BF16 && c->weight_dtype != XLPK_DTYPE_FP8_E4M3 &&
+      c->weight_dtype != XLPK_DTYPE_NVFP4)
     return XLPK_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return XLPK_ERR_INVALID_ARG;
   if (c->n_ctas < 0 || c->spin_limit_us < 0) return XLPK_ERR_INVALID_ARG;
@@ -514,6 +564,12 @@ xlpk_status validate_config(const xlpk_config* c) {
     // a packed FP8 row pair over K columns takes 2K + K/16 bytes; bulk copies
     // of row-pair spans need 16-byte multiples, so every K is a multiple of 256
     if (c->hidden % 256 || qd % 256 || c->ffn % 256) return XLPK_ERR_UNSUPPORTED;
+  }
+  if (c->weight_dtype == XLPK_DTYPE_NVFP4) {
+    // dense models at batch 1; K dims in whole 128-column chunks
+    const int qd = c->n_q_heads * c->head_dim;
+    if (c->n_experts > 0 || c->batch != 1) return XLPK_ERR_UNSUPPORTED;
+    if (c->hidden % 128 || qd % 128 || c->ffn % 128) return XLPK_ERR_UNSUPPORTED;
   }
   if (c->n_experts > 0) {
     if (c->top_k < 1 || c->top_k > c->n_experts || c->expert_ffn <= 0) return XLPK_ERR_INVALID_ARG;
@@ -553,6 +609,18 @@ xlpk_status validate_weights(const xlpk_config* c, const xlpk_weights* w, const 
       const xlpk_linear* lin[] = {&L.wq, &L.wk, &L.wv, &L.wo, &L.w_gate, &L.w_up, &L.w_down};
       for (const xlpk_linear* x : lin)
         if (!x->scale_dev || (reinterpret_cast<uintptr_t>(x->scale_dev) & 3u)) return XLPK_ERR_INVALID_ARG;
+    }
+  }
+  if (c->weight_dtype == XLPK_DTYPE_NVFP4) {
+    // every linear weight carries its block scales and a finite positive matrix scale
+    auto bad = [](const xlpk_linear& x) {
+      return !x.scale_dev || !(x.global_scale > 0.f) || !std::isfinite(x.global_scale);
+    };
+    if (bad(w->lm_head)) return XLPK_ERR_INVALID_ARG;
+    for (int l = 0; l < c->n_layers; ++l) {
+      const xlpk_layer_weights& L = w->layers[l];
+      for (const xlpk_linear* x : {&L.wq, &L.wk, &L.wv, &L.wo, &L.w_gate, &L.w_up, &L.w_down})
+        if (bad(*x)) return XLPK_ERR_INVALID_ARG;
     }
   }
   for (int l = 0; l < c->n_layers; ++l) {
@@ -623,7 +691,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
     g_cuda_err = "persistent grid larger than " + std::to_string(kMaxCtas) + " CTAs";
     return XLPK_ERR_UNSUPPORTED;
   }
-  e->esz = c.weight_dtype == XLPK_DTYPE_FP8_E4M3 ? 1 : 2;
+  e->esz = c.weight_dtype == XLPK_DTYPE_BF16 ? 2 : 1;
+  e->fp4 = c.weight_dtype == XLPK_DTYPE_NVFP4;
   const int B = c.batch, H = c.hidden, d = c.head_dim, F = c.ffn;
   const int qd = c.n_q_heads * d, kvd = c.n_kv_heads * d;
   const int group = c.n_q_heads / c.n_kv_heads;
@@ -767,23 +836,31 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   auto add = [&](MatSrc s, int N, int K, int layer, int role, int split) {
     mats.push_back({s, N, K, total, layer, role, split});
     const size_t esz_m = role == R_ROUTER ? 2 : e->esz;
-    total += align_up(static_cast<size_t>(N) * K * esz_m + (esz_m == 1 ? static_cast<size_t>(N) * K / 32 : 0), 256);
+    const size_t nk = static_cast<size_t>(N) * K;
+    if (e->fp4 && role != R_ROUTER)   // codes + e4m3 block scales, then the per-row matrix scales
+      total += align_up(align_up(nk / 2 + nk / 16, 16) + static_cast<size_t>(N) * 4, 256);
+    else
+      total += align_up(nk * esz_m + (esz_m == 1 ? nk / 32 : 0), 256);
   };
   auto u8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
   const size_t eg_bytes = static_cast<size_t>(Fe) * H * e->esz;   // one expert's gate (or up, or down)
   for (int l = 0; l < c.n_layers; ++l) {
     const xlpk_layer_weights& L = w->layers[l];
     add({MatKind::QKV, u8(L.wq.w_dev), u8(L.wk.w_dev), u8(L.wv.w_dev), L.wq.scale_dev, L.wk.scale_dev,
-         L.wv.scale_dev},
+         L.wv.scale_dev, L.wq.global_scale, L.wk.global_scale, L.wv.global_scale},
         qd + 2 * kvd, H, l, R_QKV, e->G);
-    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr, L.wo.scale_dev}, H, qd, l, R_O, e->G);
+    add({MatKind::PLAIN, u8(L.wo.w_dev), nullptr, nullptr, L.wo.scale_dev, nullptr, nullptr, L.wo.global_scale}, H,
+        qd, l, R_O, e->G);
     if (!moe) {
-      add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr, L.w_gate.scale_dev, L.w_up.scale_dev},
+      add({MatKind::GATEUP, u8(L.w_gate.w_dev), u8(L.w_up.w_dev), nullptr, L.w_gate.scale_dev, L.w_up.scale_dev,
+           nullptr, L.w_gate.global_scale, L.w_up.global_scale},
           2 * F, H, l, R_GU, e->G);
       if (e->ffn_fused)
         add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr}, F, H, l, R_DOWNT, 1);   // W_down^T [F][H]
       else
-        add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev}, H, F, l, R_DOWN, e->G);
+        add({MatKind::PLAIN, u8(L.w_down.w_dev), nullptr, nullptr, L.w_down.scale_dev, nullptr, nullptr,
+             L.w_down.global_scale},
+            H, F, l, R_DOWN, e->G);
     } else {
       // router logits are bf16 whatever the weight dtype
       add({MatKind::PLAIN, u8(L.router_dev), nullptr, nullptr}, c.n_experts, H, l, R_ROUTER, 1);
@@ -802,7 +879,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       }
     }
   }
-  add({MatKind::PLAIN, u8(w->lm_head.w_dev), nullptr, nullptr, w->lm_head.scale_dev}, c.vocab, H, -1, R_LM, e->G);
+  add({MatKind::PLAIN, u8(w->lm_head.w_dev), nullptr, nullptr, w->lm_head.scale_dev, nullptr, nullptr,
+       w->lm_head.global_scale},
+      c.vocab, H, -1, R_LM, e->G);
   // library-owned copies of the embedding table and the norm gains, so the
   // caller may free every weight buffer after create
   const size_t off_embed = total;
@@ -820,7 +899,10 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   for (const MatPlan& m : mats) {
     if (m.role == R_EGU || m.role == R_EDOWN) continue;
     const int64_t nk = static_cast<int64_t>(m.N) * m.K;
-    e->weight_bytes_per_step += m.role == R_ROUTER ? 2 * nk : e->esz == 1 ? nk + nk / 32 : 2 * nk;
+    e->weight_bytes_per_step += m.role == R_ROUTER ? 2 * nk
+                                : e->fp4       ? nk / 2 + nk / 16 + 4
+                                : e->esz == 1  ? nk + nk / 32
+                                               : 2 * nk;
   }
   if (moe)
     e->weight_bytes_per_step += static_cast<int64_t>(c.n_layers) * (c.top_k + c.n_shared_experts) * 3 *

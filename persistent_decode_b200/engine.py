@@ -71,7 +71,8 @@ def make_config(cfg, n_ctas: int = 0, spin_limit_us: int = 0, batch: Optional[in
     for f in ("n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
               "n_experts", "top_k", "n_shared_experts", "expert_ffn"):
         setattr(c, f, int(getattr(cfg, f)))
-    c.weight_dtype = _abi.XLPK_DTYPE_FP8_E4M3 if cfg.weight_dtype == "fp8_e4m3" else _abi.XLPK_DTYPE_BF16
+    c.weight_dtype = {"fp8_e4m3": _abi.XLPK_DTYPE_FP8_E4M3, "nvfp4": _abi.XLPK_DTYPE_NVFP4}.get(
+        cfg.weight_dtype, _abi.XLPK_DTYPE_BF16)
     c.batch = int(batch if batch is not None else cfg.batch)
     c.max_seq = int(max_seq if max_seq is not None else cfg.max_seq)
     c.rope_theta = float(cfg.rope_theta)
@@ -121,7 +122,9 @@ class Engine:
         self._layers = (_abi.xlpk_layer_weights * max(L, 1))()
 
         def lin(name):
-            return _abi.xlpk_linear(_ptr(weights[name]), _ptr(weights.get(name + ".scale")))
+            gs = weights.get(name + ".gscale")   # NVFP4: the matrix scale (a one-element tensor)
+            return _abi.xlpk_linear(_ptr(weights[name]), _ptr(weights.get(name + ".scale")),
+                                    float(gs.reshape(-1)[0]) if gs is not None else 0.0)
 
         import torch
 

@@ -14,6 +14,8 @@ from __future__ import annotations
 
 
 def weight_bytes(cfg) -> int:
+    if cfg.weight_dtype == "nvfp4":
+        return _nvfp4_weight_bytes(cfg)
     esz = 1 if cfg.weight_dtype == "fp8_e4m3" else 2
     H, qd, kvd = cfg.hidden, cfg.q_dim, cfg.kv_dim
     per_layer = (qd + 2 * kvd) * H + H * qd
@@ -30,6 +32,17 @@ def weight_bytes(cfg) -> int:
         scales = 4 * (cfg.n_layers * per_layer + cfg.vocab * H) // (128 * 128)
     norms = 4 * H * (2 * cfg.n_layers + 1)
     return lin + scales + norms + cfg.n_layers * router
+
+
+def _nvfp4_weight_bytes(cfg) -> int:
+    """NVFP4 (dense): half a byte per element, one e4m3 scale byte per 16
+    elements, one fp32 scale per matrix; norm gains fp32."""
+    H, qd, kvd = cfg.hidden, cfg.q_dim, cfg.kv_dim
+    mats = [qd * H, kvd * H, kvd * H, H * qd, cfg.ffn * H, cfg.ffn * H, H * cfg.ffn]
+    elems = cfg.n_layers * sum(mats) + cfg.vocab * H
+    n_mats = cfg.n_layers * len(mats) + 1
+    norms = 4 * H * (2 * cfg.n_layers + 1)
+    return elems // 2 + elems // 16 + 4 * n_mats + norms
 
 
 def step_bytes(cfg, kv_positions: int, batch: int = None) -> int:

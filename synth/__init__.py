@@ -12,6 +12,7 @@ from .gen import (  # noqa: F401
     normal_fp32,
     uniform_tokens,
     quantize_fp8_blocks,
+    quantize_nvfp4,
     make_weights,
     make_prompt,
     make_synthetic_kv,

@@ -58,8 +58,8 @@ class DecoderConfig:
     def with_(self, **kw) -> "DecoderConfig":
         return dataclasses.replace(self, **kw)
 
-    def weight_bytes_per_elem(self) -> int:
-        return 1 if self.weight_dtype == "fp8_e4m3" else 2
+    def weight_bytes_per_elem(self) -> float:
+        return {"fp8_e4m3": 1, "nvfp4": 0.5}.get(self.weight_dtype, 2)
 
 
 TINY = DecoderConfig(
@@ -76,12 +76,14 @@ LLAMA_8B = DecoderConfig(
 
 LLAMA_8B_FP8 = LLAMA_8B.with_(name="llama8b_fp8", weight_dtype="fp8_e4m3", kv_len=1024)
 
+LLAMA_8B_NVFP4 = LLAMA_8B.with_(name="llama8b_nvfp4", weight_dtype="nvfp4")
+
 MOE = DecoderConfig(
     name="moe", n_layers=24, hidden=2048, n_q_heads=16, n_kv_heads=4, head_dim=128,
     ffn=0, vocab=64000, kv_len=4096, steps=256, n_experts=64, top_k=8,
     n_shared_experts=1, expert_ffn=1408, prefill=False)
 
-CONFIGS = {c.name: c for c in (TINY, LLAMA_1B, LLAMA_8B, LLAMA_8B_FP8, MOE)}
+CONFIGS = {c.name: c for c in (TINY, LLAMA_1B, LLAMA_8B, LLAMA_8B_FP8, LLAMA_8B_NVFP4, MOE)}
 
 
 def fp8_kv(cfg: DecoderConfig) -> DecoderConfig:

@@ -148,12 +148,55 @@ def quantize_fp8_blocks(w: torch.Tensor, block: int = 128):
     return codes.contiguous(), scale.contiguous()
 
 
+FP4_E2M1_MAX = 6.0
+_E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)   # codes 0..7
+
+
+def quantize_nvfp4(w: torch.Tensor):
+    """NVFP4 quantisation of a [N][K] weight (input preparation only).
+
+    Tensor scale gs = max|w| / (448 * 6) (1 for an all-zero tensor); per 16
+    consecutive elements of a row, block scale = e4m3(max|block| / (6 gs))
+    (round to nearest even); codes = the E2M1 magnitude nearest to
+    |w| / (block scale * gs) (ties to the even code, saturated at 6) with w's
+    sign; an all-zero block gets scale 0 and codes 0.  Returns (codes uint8
+    [N][K/2] with element 2j in the low nibble, block scales uint8 e4m3 codes
+    [N][K/16], tensor scale fp32 [1]).
+    """
+    N, K = w.shape
+    assert K % 16 == 0
+    wf = w.float()
+    amax = float(wf.abs().max())
+    gs = amax / (FP8_E4M3_MAX * FP4_E2M1_MAX) if amax > 0 else 1.0
+    blocks = wf.view(N, K // 16, 16)
+    bmax = blocks.abs().amax(dim=-1)
+    sb = (bmax / (FP4_E2M1_MAX * gs)).clamp(max=FP8_E4M3_MAX).to(torch.float8_e4m3fn)
+    s = (sb.float() * gs)[..., None]
+    y = torch.where(s > 0, blocks / torch.where(s > 0, s, torch.ones_like(s)), torch.zeros_like(blocks))
+    mags = torch.tensor(_E2M1_MAGNITUDES, dtype=torch.float32, device=w.device)
+    a = y.abs().clamp(max=FP4_E2M1_MAX)
+    hi = torch.searchsorted(mags, a.contiguous()).clamp(max=7)
+    lo = (hi - 1).clamp(min=0)
+    d_hi, d_lo = mags[hi] - a, a - mags[lo]
+    take_lo = (d_lo < d_hi) | ((d_lo == d_hi) & (lo % 2 == 0) & (lo != hi))
+    code = torch.where(take_lo, lo, hi) | ((y < 0).to(torch.int64) << 3)
+    code = code.view(N, K // 2, 2)
+    packed = (code[..., 0] | (code[..., 1] << 4)).to(torch.uint8)
+    return packed.contiguous(), sb.view(torch.uint8).contiguous(), torch.tensor([gs], dtype=torch.float32,
+                                                                                 device=w.device)
+
+
 def _linear(cfg: DecoderConfig, name: str, n: int, k: int, device, out: Dict[str, torch.Tensor]):
     w = normal_bf16(cfg.seed, name, (n, k), cfg.init_std, device)
     if cfg.weight_dtype == "fp8_e4m3":
         codes, scales = quantize_fp8_blocks(w)
         out[name] = codes
         out[name + ".scale"] = scales
+    elif cfg.weight_dtype == "nvfp4":
+        codes, scales, gs = quantize_nvfp4(w)
+        out[name] = codes
+        out[name + ".scale"] = scales
+        out[name + ".gscale"] = gs
     else:
         out[name] = w
 

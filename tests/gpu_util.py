@@ -92,6 +92,7 @@ class MemoOracle(OracleDecoder):
             if isinstance(self.w, HostWeights):   # the fp32 copy replaces the stored bytes
                 self.w.pop(name, None)
                 self.w.pop(name + ".scale", None)
+                self.w.pop(name + ".gscale", None)
         return t
 
 

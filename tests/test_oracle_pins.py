@@ -510,3 +510,81 @@ def test_fp8_kv_round_is_code_times_a_power_of_two():
         assert bool((err <= best + 1e-7).all())
     with pytest.raises(AssertionError):
         kv_round(x, "fp8_e4m3", 0.3)                     # not a power of two
+
+
+# ----------------------------------------------------------- NVFP4 weights
+
+def test_e2m1_table_is_the_published_value_set():
+    # OCP MX v1.0 lists the FP4 (E2M1) magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 for
+    # codes 0..7; codes 8..15 are their negatives (sign bit 3)
+    from oracle import e2m1_decode_table
+    t = e2m1_decode_table()
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert t[:8].tolist() == mags
+    assert t[8:].tolist() == [-m for m in mags]
+    assert bool(torch.signbit(t[8]))
+
+
+def test_nvfp4_dequant_by_index():
+    # distinct codes and block scales on a 3 x 64 matrix (4 blocks per row): each
+    # element is the nibble of its byte (even element low) x its row's block scale
+    # x the tensor scale
+    from oracle import e2m1_decode_table, e4m3_decode_table, nvfp4_dequant
+    g = torch.Generator().manual_seed(11)
+    N, K = 3, 64
+    codes = torch.randint(0, 256, (N, K // 2), generator=g).to(torch.uint8)
+    scale_codes = torch.tensor([[0x30, 0x38, 0x40, 0x29], [0x31, 0x3F, 0x08, 0x50], [0x00, 0x44, 0x36, 0x3A]],
+                               dtype=torch.uint8)
+    gs = 0.375
+    got = nvfp4_dequant(codes, scale_codes, gs)
+    e2 = e2m1_decode_table().tolist()
+    e4 = e4m3_decode_table().tolist()
+    for r in range(N):
+        for k in range(K):
+            byte = int(codes[r, k // 2])
+            nib = byte & 0xF if k % 2 == 0 else byte >> 4
+            want = e2[nib] * e4[int(scale_codes[r, k // 16])] * gs
+            assert float(got[r, k]) == want, (r, k)
+
+
+def test_nvfp4_quantisation_picks_the_nearest_code():
+    # the synthetic quantiser (input preparation) against brute force: every
+    # element's value is, among the 16 codes times its block's scale, one nearest
+    # to the weight; the oracle's dequantisation of its output stays within half
+    # the largest code spacing (1 x scale) of the weight, below the saturation bound
+    import synth
+    from oracle import e4m3_decode_table, nvfp4_dequant
+    g = torch.Generator().manual_seed(3)
+    w = (torch.randn(8, 256, generator=g) * 0.02).to(torch.bfloat16)
+    w[0, :16] = 0                                          # an all-zero block
+    codes, sc, gs = synth.quantize_nvfp4(w)
+    deq = nvfp4_dequant(codes, sc, float(gs[0]))
+    s = e4m3_decode_table()[sc.long()].repeat_interleave(16, dim=1) * float(gs[0])
+    cand = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    wf = w.float()
+    assert bool((deq[0, :16] == 0).all())
+    for r in range(8):
+        for k in range(256):
+            if float(s[r, k]) == 0:
+                continue
+            opts = (torch.cat([cand, -cand]) * s[r, k] - wf[r, k]).abs()
+            assert abs(float(deq[r, k]) - float(wf[r, k])) <= float(opts.min()) + 1e-6 * abs(float(wf[r, k])) + 1e-9, (r, k)
+    # the block maximum maps to (about) 6: block scales are max|block| / 6 rounded to e4m3
+    assert float((deq - wf).abs().max()) <= float(s.max()) * 1.0
+
+
+def test_oracle_W_reads_nvfp4_weights():
+    # OracleDecoder.W dispatches on the tensor-scale companion and returns the
+    # dequantised matrix
+    import synth
+    from oracle import OracleDecoder, nvfp4_dequant
+    cfg = synth.get_config("tiny", n_layers=1, weight_dtype="nvfp4")
+    w = synth.make_weights(cfg)
+    o = OracleDecoder(cfg, w, cfg.batch, max_seq=cfg.max_seq)
+    name = "layers.0.wq"
+    assert w[name].dtype == torch.uint8 and w[name].shape == (cfg.q_dim, cfg.hidden // 2)
+    ref = nvfp4_dequant(w[name], w[name + ".scale"], float(w[name + ".gscale"][0]))
+    assert torch.equal(o.W(name), ref)
+    # and close to the bf16 weights it quantises (4-bit codes: ~10 % per element)
+    wb = synth.normal_bf16(cfg.seed, name, (cfg.q_dim, cfg.hidden), cfg.init_std, "cpu").float()
+    assert float((o.W(name) - wb).norm() / wb.norm()) < 0.15
