@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "xlpk.cu")
 KERNELS = os.path.join(HERE, "csrc", "kernels.cu")
-KERNEL_UNITS = 9   # kKernelUnits in csrc/kernels.h
+KERNEL_UNITS = 11   # kKernelUnits in csrc/kernels.h
 DEPS = [os.path.join(HERE, "csrc", f) for f in ("xlpk.cu", "kernels.cu", "kernels.h", "engine.cuh", "tcgen05.cuh",
                                                 "tc_tile.cuh", "params.h")] + \
     [os.path.join(ROOT, "include", "xlpk.h")]

@@ -1458,10 +1458,10 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
 
 // e4m3 and bf16 tiles are separate instantiations, so neither inner loop
 // carries the other's code.
-template <int B, class Epi>
+template <int B, bool W4, class Epi>
 __device__ __forceinline__ void consume_gemv(const Params& p, Ctx& cx, const Mat& m, RingPos& rp, int where,
                                              const float (&rn)[B], Epi& epi, int q0 = -1, int q1 = -1) {
-  if constexpr (B == 1) {   // NVFP4 weights are built for batch 1
+  if constexpr (W4) {   // NVFP4 kernels (batch 1): every projection's codes and scales
     if (m.fp4) {
       consume_gemv_t<B, 2>(p, cx, m, rp, where, rn, epi, q0, q1);
       return;
@@ -2403,9 +2403,11 @@ __device__ __forceinline__ const Mat& stage_mat(const LayerParams& L, int kind) 
 }
 
 // Consumers: one stage.  Returns false once the CTA is aborting.
-template <int B, int D, bool MOE, bool KV8>
+template <int B, int D, bool MOE, int VAR>
 __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, int l, int s,
                                            RingPos& rp, bool fused) {
+  constexpr bool KV8 = (VAR & 1) != 0;   // e4m3 KV cache
+  constexpr bool W4 = (VAR & 2) != 0;    // NVFP4 weights
   const unsigned G = static_cast<unsigned>(p.G);
   const unsigned S1 = static_cast<unsigned>(p.step_base + s + 1);
   const int where = where_code(kind, l, s);
@@ -2438,7 +2440,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
       load_act<B>(p, cx, p.H, p.resid_fixed ? SRC_FIXED : SRC_RESID, resid_src(p), p.final_norm, hid, SIDE_NONE, s, rn,
                   where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
-      consume_gemv<B>(p, cx, p.lm, rp, where, rn, epi);
+      consume_gemv<B, W4>(p, cx, p.lm, rp, where, rn, epi);
     }
     if (cx.lane < B) {
       cx.ctl->redv[cx.warp][cx.lane] = bv;
@@ -2573,7 +2575,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       }
       EpiQKV<B, KV8> epi{p, l, s, reinterpret_cast<const float2*>(cx.side + p.side_rope)};
-      consume_gemv<B>(p, cx, L.qkv, rp, where, rn, epi);
+      consume_gemv<B, W4>(p, cx, L.qkv, rp, where, rn, epi);
       break;
     }
     case ST_OPROJ: {
@@ -2583,7 +2585,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
                   rn, where);
       if (cx.tid == 0) trace_stamp(p, s, stage_index(p, kind, l), 2);
       EpiResid<B> epi{p, l == 0, cx.side, r0, p.ffn_fused ? p.y : nullptr};
-      consume_gemv<B>(p, cx, L.o, rp, where, rn, epi);
+      consume_gemv<B, W4>(p, cx, L.o, rp, where, rn, epi);
       break;
     }
     case ST_GATEUP: {
@@ -2595,7 +2597,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
           // router (all E logits in every CTA), routing, then this CTA's groups
           // of the virtual [slot][pair] gate/up space
           EpiRouter<B> er{cx.ctl->logits};
-          consume_gemv<B>(p, cx, L.router, rp, where, rn, er, 0, L.router.N >> 1);
+          consume_gemv<B, W4>(p, cx, L.router, rp, where, rn, er, 0, L.router.N >> 1);
           consumer_sync();
           if (cx.warp == 0) moe_route(p, cx, l, s);
           consumer_sync();
@@ -2603,7 +2605,7 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
           Mat v = L.egu;
           v.N = 2 * p.S * p.Fe;
           EpiMoeGU<B> eg{p, cx.ctl->route_w};
-          consume_gemv<B>(p, cx, v, rp, where, rn, eg, 8 * split_point(cx.c, ng, p.G),
+          consume_gemv<B, W4>(p, cx, v, rp, where, rn, eg, 8 * split_point(cx.c, ng, p.G),
                           8 * split_point(cx.c + 1, ng, p.G));
         }
       } else if (p.ffn_fused) {
@@ -2611,12 +2613,12 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         const int q0 = split_point(cx.c, p.F, p.G), q1 = split_point(cx.c + 1, p.F, p.G);
         float* hl = reinterpret_cast<float*>(cx.side + p.side_hloc);
         EpiSwiGLULocal<B> epi{hl, p.hloc, q0};
-        consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
+        consume_gemv<B, W4>(p, cx, L.gu, rp, where, rn, epi);
         consumer_sync();
         consume_downT<B>(p, cx, rp, where, q0, q1, hl);
       } else {
         EpiSwiGLU<B> epi{p};
-        consume_gemv<B>(p, cx, L.gu, rp, where, rn, epi);
+        consume_gemv<B, W4>(p, cx, L.gu, rp, where, rn, epi);
       }
       break;
     }
@@ -2641,9 +2643,9 @@ __device__ __noinline__ bool consume_stage(const Params& p, Ctx& cx, int kind, i
         // K runs over [slot][expert column]: the producer streams each slot's expert
         Mat v = L.edown;
         v.K = K;
-        consume_gemv<B>(p, cx, v, rp, where, rn, epi);
+        consume_gemv<B, W4>(p, cx, v, rp, where, rn, epi);
       } else {
-        consume_gemv<B>(p, cx, L.down, rp, where, rn, epi);
+        consume_gemv<B, W4>(p, cx, L.down, rp, where, rn, epi);
       }
       break;
     }
@@ -2806,8 +2808,9 @@ struct Run {
   int stage, layer, step;
 };
 
-template <int B, bool MOE, bool KV8>
+template <int B, bool MOE, int VAR>
 __device__ int cursor_next(const Params& p, int c, const SmemCtl* ctl, Cursor<B>& cu, Tile& t, Run* run) {
+  constexpr bool KV8 = (VAR & 1) != 0;   // e4m3 KV cache
   while (!cu.done) {
     if (p.serve && !cu.open && !cu.one_stage && cu.kind == ST_QKV && cu.l == 0) {
       // serve mode: a step's tiles are streamed once the step is requested
@@ -3057,8 +3060,9 @@ static __device__ __noinline__ bool route_wait(const Params& p, SmemCtl* ctl, in
 // `p.l2_prefetch_bytes` ahead.  Weights do not depend on activations, so both
 // run ahead of the consumers across stage boundaries; only attention chunks
 // wait for the previous step's KV write of their layer.
-template <int B, bool MOE, bool KV8>
+template <int B, bool MOE, int VAR>
 __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
+  constexpr bool KV8 = (VAR & 1) != 0;   // e4m3 KV cache
   RingPos rp;
   const uint64_t pol = evict_first_policy();
   Cursor<B> cc, pc;
@@ -3084,18 +3088,18 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
     bool t_attn = false;
     int t_stage, t_layer, t_step, t_y = 0;
     if (r_n1 + r_n2 == 0) {
-      int r = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, cc, t, &nr);
+      int r = cursor_next<B, MOE, VAR>(p, cx.c, cx.ctl, cc, t, &nr);
       while (r == CUR_REQ) {
         // serve mode: the next step is not requested yet (bounded wait)
         if (!serve_gate(p, cx.ctl, cc.s, false) && serve_state(p, cc.s) >= 0) break;
-        r = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, cc, t, &nr);
+        r = cursor_next<B, MOE, VAR>(p, cx.c, cx.ctl, cc, t, &nr);
       }
       if (r == CUR_REQ) break;
       if (r == CUR_BLOCKED) {
         // the next tile is an expert chosen by this CTA's own consumers: wait
         // (bounded) until they publish the layer's routing
         if (!route_wait(p, cx.ctl, route_want(p, cc.s, cc.l), where_code(cc.kind, cc.l, cc.s) | (1 << 15))) break;
-        r = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, cc, t, &nr);
+        r = cursor_next<B, MOE, VAR>(p, cx.c, cx.ctl, cc, t, &nr);
       }
       if (r == CUR_RUN) {
         r_src = nr.src;
@@ -3137,7 +3141,7 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
         ahead += nb;
         continue;
       }
-      const int pr = cursor_next<B, MOE, KV8>(p, cx.c, cx.ctl, pc, tp, &prun);
+      const int pr = cursor_next<B, MOE, VAR>(p, cx.c, cx.ctl, pc, tp, &prun);
       if (pr == CUR_BLOCKED || pr == CUR_REQ) break;   // resume once the routing / the request is known
       if (pr == CUR_RUN) {
         pf_src = prun.src;
@@ -3208,7 +3212,7 @@ __device__ void producer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
   drain_ring(p, cx, rp, p.nslot);
 }
 
-template <int B, int D, bool MOE, bool KV8>
+template <int B, int D, bool MOE, int VAR>
 __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s0, bool fused) {
   RingPos rp;
   if (fused) {
@@ -3220,11 +3224,11 @@ __device__ void consumer_main(const Params& p, Ctx& cx, int kind0, int l0, int s
       }
       for (int l = 0; l < p.L; ++l)
         for (int k = 0; k < ST_LAYER; ++k)
-          if (!consume_stage<B, D, MOE, KV8>(p, cx, k, l, s, rp, true)) return;
-      if (!consume_stage<B, D, MOE, KV8>(p, cx, ST_LM, 0, s, rp, true)) return;
+          if (!consume_stage<B, D, MOE, VAR>(p, cx, k, l, s, rp, true)) return;
+      if (!consume_stage<B, D, MOE, VAR>(p, cx, ST_LM, 0, s, rp, true)) return;
     }
   } else {
-    consume_stage<B, D, MOE, KV8>(p, cx, kind0, l0, s0, rp, false);
+    consume_stage<B, D, MOE, VAR>(p, cx, kind0, l0, s0, rp, false);
   }
 }
 
@@ -3264,23 +3268,23 @@ __device__ __forceinline__ void tc_close(const Params& p, Ctx& cx) {
   }
 }
 
-template <int B, int D, bool MOE, bool KV8>
+template <int B, int D, bool MOE, int VAR>
 __global__ void __launch_bounds__(kThreads, 1) engine_persistent(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Ctx cx = make_ctx(smem, p);
   init_ring(p, cx);
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<B, MOE, KV8>(p, cx, 0, 0, 0, true);
+    if (cx.lane == 0) producer_main<B, MOE, VAR>(p, cx, 0, 0, 0, true);
     __syncwarp();
   } else {
     tc_open<B>(p, cx);
-    consumer_main<B, D, MOE, KV8>(p, cx, 0, 0, 0, true);
+    consumer_main<B, D, MOE, VAR>(p, cx, 0, 0, 0, true);
     tc_close<B>(p, cx);
   }
 }
 
 // Kernel-per-op baseline: one launch runs one stage (same tiles, no waits).
-template <int B, int D, bool MOE, bool KV8>
+template <int B, int D, bool MOE, int VAR>
 __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constant__ Params p, int kind,
                                                             int layer, int step) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -3296,11 +3300,11 @@ __global__ void __launch_bounds__(kThreads, 1) engine_stage(const __grid_constan
     __syncthreads();
   }
   if (cx.warp == kConsumerWarps) {
-    if (cx.lane == 0) producer_main<B, MOE, KV8>(p, cx, kind, layer, step, false);
+    if (cx.lane == 0) producer_main<B, MOE, VAR>(p, cx, kind, layer, step, false);
     __syncwarp();
   } else {
     tc_open<B>(p, cx);
-    consumer_main<B, D, MOE, KV8>(p, cx, kind, layer, step, false);
+    consumer_main<B, D, MOE, VAR>(p, cx, kind, layer, step, false);
     tc_close<B>(p, cx);
   }
 }

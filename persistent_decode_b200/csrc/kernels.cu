@@ -10,16 +10,16 @@
 
 namespace xlpk {
 
-template <int B, int D, bool MOE, bool KV8>
+template <int B, int D, bool MOE, int VAR>
 void launch_stage_impl(const Params& p, int kind, int layer, int step, int grid, int smem, cudaStream_t st) {
-  engine_stage<B, D, MOE, KV8><<<grid, kThreads, smem, st>>>(p, kind, layer, step);
+  engine_stage<B, D, MOE, VAR><<<grid, kThreads, smem, st>>>(p, kind, layer, step);
 }
 
-template <int B, int D, bool MOE, bool KV8>
+template <int B, int D, bool MOE, int VAR>
 KernelSet kernel_set() {
-  return KernelSet{reinterpret_cast<const void*>(&engine_persistent<B, D, MOE, KV8>),
-                   reinterpret_cast<const void*>(&engine_stage<B, D, MOE, KV8>),
-                   &launch_stage_impl<B, D, MOE, KV8>};
+  return KernelSet{reinterpret_cast<const void*>(&engine_persistent<B, D, MOE, VAR>),
+                   reinterpret_cast<const void*>(&engine_stage<B, D, MOE, VAR>),
+                   &launch_stage_impl<B, D, MOE, VAR>};
 }
 
 #define XLPK_INST_SET(b, d, m, k) template KernelSet kernel_set<b, d, m, k>();
@@ -41,6 +41,10 @@ XLPK_UNIT6(XLPK_INST_SET)
 XLPK_UNIT7(XLPK_INST_SET)
 #elif XLPK_UNIT == 8
 XLPK_UNIT8(XLPK_INST_SET)
+#elif XLPK_UNIT == 9
+XLPK_UNIT9(XLPK_INST_SET)
+#elif XLPK_UNIT == 10
+XLPK_UNIT10(XLPK_INST_SET)
 #else
 #error "XLPK_UNIT out of range"
 #endif

@@ -292,25 +292,32 @@ namespace {
 // Dense and MoE models use separate kernel instantiations, so the dense
 // kernels carry none of the routing code; likewise bf16 and e4m3 caches, so
 // the bf16 kernels carry none of the e4m3 code (nor its register pressure).
-template <int B, int D, bool MOE = false, bool KV8 = false>
+template <int B, int D, bool MOE = false, int VAR = 0>
 void bind_kernels(xlpk_engine* e) {
-  const KernelSet k = kernel_set<B, D, MOE, KV8>();
+  const KernelSet k = kernel_set<B, D, MOE, VAR>();
   e->kern_persistent = k.persistent;
   e->kern_stage = k.stage;
   e->launch_stage = k.launch_stage;
 }
 
-bool bind_by_shape(xlpk_engine* e, int B, int D, bool moe, bool kv8) {
-  if (moe) {   // MoE is built for batch 1 with a bf16 cache
-    if (kv8) return false;
+// var: bit 0 an e4m3 KV cache, bit 1 NVFP4 weights (batch 1, dense).
+bool bind_by_shape(xlpk_engine* e, int B, int D, bool moe, int var) {
+  if (moe) {   // MoE is built for batch 1 with bf16 / e4m3 weights and a bf16 cache
+    if (var != 0) return false;
     if (B == 1 && D == 64) return bind_kernels<1, 64, true>(e), true;
     if (B == 1 && D == 128) return bind_kernels<1, 128, true>(e), true;
     return false;
   }
+  if (var & 2) {
+    if (B != 1) return false;
+    if (D == 64) return (var & 1 ? bind_kernels<1, 64, false, 3>(e) : bind_kernels<1, 64, false, 2>(e)), true;
+    if (D == 128) return (var & 1 ? bind_kernels<1, 128, false, 3>(e) : bind_kernels<1, 128, false, 2>(e)), true;
+    return false;
+  }
 #define XLPK_BIND(b, d)                     \
   if (B == b && D == d) {                   \
-    if (kv8)                                \
-      bind_kernels<b, d, false, true>(e);   \
+    if (var & 1)                            \
+      bind_kernels<b, d, false, 1>(e);      \
     else                                    \
       bind_kernels<b, d>(e);                \
     return true;                            \
@@ -807,7 +814,8 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
   e->smem = e->nslot * kSlotBytes + e->act_bytes + e->side_bytes + kMiscSmem;
-  if (!bind_by_shape(e, B, d, c.n_experts > 0, c.kv_dtype == XLPK_DTYPE_FP8_E4M3)) return XLPK_ERR_UNSUPPORTED;
+  const int var = (c.kv_dtype == XLPK_DTYPE_FP8_E4M3 ? 1 : 0) | (e->fp4 ? 2 : 0);
+  if (!bind_by_shape(e, B, d, c.n_experts > 0, var)) return XLPK_ERR_UNSUPPORTED;
 
   // The attribute is per kernel function, shared by every handle that uses the
   // same instantiation: allow the device maximum rather than this handle's size.
