@@ -195,7 +195,8 @@ typedef struct xlpk_decode_io {
                                          stages, totals of thread 0: [6] ns waiting for KV chunks,
                                          [7] ns of the combining CTA's wait for the partials,
                                          [8] q loads, [9] chunk math, [10] merge,
-                                         [11] arrive, [12] combine, [13] chunks processed; for the
+                                         [11] arrive, [12] combine, [13] the combining CTA's time to
+                                         its merged output (wait + arithmetic); for the
                                          other stages, thread 0's input staging: [6] copies issued,
                                          [7] landed, [8] converted, [9] RMSNorm factor ready.
                                          n_stages = 5 * n_layers + 1 */

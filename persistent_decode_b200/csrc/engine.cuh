@@ -2042,7 +2042,6 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
         __all_sync(0xffffffffu, cx.ctl->abort ? false : ring_wait(p, cx.ctl, fb, rp.phase, where));
     if (kTraceAttn && p.trace && cx.tid == 0) {
       ta[0] += globaltimer() - tw0;
-      ++ta[7];
     }
     const unsigned long long tc0 = (kTraceAttn && p.trace && cx.tid == 0) ? globaltimer() : 0;
     const uint32_t kt = ring_s + rp.slot * kSlotBytes;
@@ -2374,6 +2373,7 @@ __device__ __noinline__ void consume_attn(const Params& p, Ctx& cx, int l, int s
       *reinterpret_cast<float4*>(p.o + plane_index(seg_b, (seg_g * GQ + h) * D + dd, p.B, p.nq * D)) =
           make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
+    if (kTraceAttn && p.trace && cx.tid == 0) ta[7] += globaltimer() - tb0;
     fence_proxy_async_global();   // o is read by bulk copies
     consumer_sync();
     if (cx.tid == 0) {
