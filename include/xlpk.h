@@ -169,9 +169,9 @@ typedef struct xlpk_weights {
  * Source: the KV page planner that places each request's cache pages and the
  * decode worker that follows them ("XL-Persistent-Kernel", request lifecycle
  * steps 2-4 and the component table's KV row); a quantised (FP8) attention
- * cache read inside the persistent kernel, which the survey of persistent
- * execution names as an open combination ("持续执行范式：从 Kernel Boundary
- * Elimination 到 Ultra-Low-Latency Engine", section 7.5). */
+ * cache read inside the persistent kernel, which the page on the persistent
+ * execution paradigm names as an open combination ("持续执行范式：从 Kernel
+ * Boundary Elimination 到 Ultra-Low-Latency Engine", section 7.5). */
 typedef struct xlpk_kv {
   void* k_dev;
   void* v_dev;

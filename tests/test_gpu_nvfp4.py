@@ -49,3 +49,12 @@ def test_llama8b_nvfp4_full_size_prefix(cuda_device):
     m = workload.build(cfg, device=cuda_device)
     run = run_engine(m, cfg.steps)
     compare_with_oracle(m, run, oracle_for(m, memo=True), cfg.steps, tol=REL_L2_FP8)
+
+
+def test_nvfp4_with_e4m3_cache(cuda_device):
+    # both formats at once (their own kernel instantiation): NVFP4 weights, an e4m3 KV cache
+    cfg = synth.fp8_kv(synth.get_config("tiny", weight_dtype="nvfp4", steps=8))
+    m = workload.build(cfg, device=cuda_device)
+    assert m.k.dtype == torch.uint8
+    run = run_engine(m, cfg.steps)
+    compare_with_oracle(m, run, oracle_for(m), cfg.steps, tol=REL_L2_FP8)
