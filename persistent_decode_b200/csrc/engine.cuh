@@ -1339,6 +1339,11 @@ __device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t n) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(n) : "memory");
 }
 
+// Whether an epilogue is the LM head's (its running argmax is kept per lane in consume_tc).
+template <int B> struct EpiLM;
+template <class E> struct is_lm_epi { static constexpr bool value = false; };
+template <int B> struct is_lm_epi<EpiLM<B>> { static constexpr bool value = true; };
+
 // One batch-8 projection on the tensor cores: the CTA's 8-row units of `m`
 // (M-tiles of <= 128 rows, each with kTcAccCols accumulator columns in tensor
 // memory: columns b and 8 + b hold sequence b's high and low parts), the input
@@ -1433,6 +1438,20 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
   tc_fence_after();
   const bool aborting = consumer_sync_any(cx.ctl->abort != 0);   // uniform: tcgen05.ld is warp-collective
   if (cx.warp < 4 && !aborting) {
+    // The epilogue runs here after all of the stage's MMAs, so nothing hides
+    // its latency: every lane works on every pass (lane L: row pair L/8 of a
+    // group of four, sequence L%8, values fetched from the pair's rows with
+    // one shuffle per sequence), the functor is copied into registers, and the
+    // LM head's running argmax is kept per lane and reduced once at the end.
+    Epi e = epi;
+    constexpr bool kLm = is_lm_epi<Epi>::value;
+    const int bl = cx.lane & 7;                        // this lane's sequence
+    float rnb = rn[0];
+#pragma unroll
+    for (int b = 1; b < B; ++b)
+      if (b == bl) rnb = rn[b];
+    float lm_v = -INFINITY;
+    int lm_i = 0x7fffffff;
     for (int mt = 0; mt < nm; ++mt) {
       const int rv = min(128, R - 128 * mt);
       if (cx.warp * 32 >= rv) continue;               // warp-uniform
@@ -1441,16 +1460,52 @@ __device__ __noinline__ void consume_tc(const Params& p, Ctx& cx, const Mat& m, 
       float row[B];   // this lane's accumulator row: high + low part of each sequence
 #pragma unroll
       for (int b = 0; b < B; ++b) row[b] = __uint_as_float(v[b]) + __uint_as_float(v[8 + b]);
-      for (int i = 0; i < 16; ++i) {
-        if (cx.warp * 32 + 2 * i >= rv) break;         // warp-uniform
-        float a0[B], a1[B];
+      const int np = min(16, (rv - cx.warp * 32) >> 1);   // row pairs of this warp's 32 rows
+      for (int i0 = 0; i0 < np; i0 += 4) {             // warp-uniform
+        const int ip = i0 + (cx.lane >> 3);            // <= 15
+        float x0 = 0.f, x1 = 0.f;
 #pragma unroll
         for (int b = 0; b < B; ++b) {
-          a0[b] = __shfl_sync(0xffffffffu, row[b], 2 * i) * rn[b];
-          a1[b] = __shfl_sync(0xffffffffu, row[b], 2 * i + 1) * rn[b];
+          const float y0 = __shfl_sync(0xffffffffu, row[b], 2 * ip);
+          const float y1 = __shfl_sync(0xffffffffu, row[b], 2 * ip + 1);
+          if (b == bl) {
+            x0 = y0;
+            x1 = y1;
+          }
         }
-        epi(4 * u0 + 64 * mt + 16 * cx.warp + i, a0, a1, cx.lane);
+        if (ip >= np) continue;
+        x0 *= rnb;
+        x1 *= rnb;
+        const int pg = 4 * u0 + 64 * mt + 16 * cx.warp + ip;
+        if constexpr (kLm) {
+          argmax_merge(lm_v, lm_i, x0, 2 * pg);
+          argmax_merge(lm_v, lm_i, x1, 2 * pg + 1);
+          if (p.logits_out) {
+            float* lo = p.logits_out + (static_cast<size_t>(p.logits_overwrite ? 0 : e.s) * p.B + bl) * p.V + 2 * pg;
+            lo[0] = x0;
+            lo[1] = x1;
+          }
+        } else {
+          // the functor reads element bl of each array on lane bl
+          float a0[B], a1[B];
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            a0[b] = x0;
+            a1[b] = x1;
+          }
+          e(pg, a0, a1, bl);
+        }
       }
+    }
+    if constexpr (kLm) {
+      // lanes bl, bl + 8, bl + 16, bl + 24 hold sequence bl's candidates
+#pragma unroll
+      for (int o = 8; o < 32; o <<= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, lm_v, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, lm_i, o);
+        argmax_merge(lm_v, lm_i, v2, i2);
+      }
+      if (cx.lane < B) argmax_merge(*epi.best_v, *epi.best_i, lm_v, lm_i);
     }
   }
   tc_fence_before();
