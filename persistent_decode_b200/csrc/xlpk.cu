@@ -242,6 +242,7 @@ struct xlpk_engine {
   int device = 0;
   int G = 0;
   int nslot = 0;
+  bool shallow = false;         // dense batch 1: kShallowSlots ring slots, kShallowPrefetchBytes of L2 prefetch
   int smem = 0;
   int act_bytes = 0;
   int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, rows_side = 0, evb = 0;
@@ -811,7 +812,9 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       e->act_bytes = act_for(std::max(std::max(H, qd), win));
     }
   }
-  e->nslot = std::min(kMaxSlots, (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
+  e->shallow = B == 1 && c.n_experts == 0;
+  e->nslot = std::min(e->shallow ? kShallowSlots : kMaxSlots,
+                      (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
   e->smem = e->nslot * kSlotBytes + e->act_bytes + e->side_bytes + kMiscSmem;
   const int var = (c.kv_dtype == XLPK_DTYPE_FP8_E4M3 ? 1 : 0) | (e->fp4 ? 2 : 0);
@@ -1069,7 +1072,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
   p.evb = e->evb;
   p.attn_pos_per_tile = e->P;
   p.spin_limit_ns = 1000LL * (c.spin_limit_us > 0 ? c.spin_limit_us : 200000);
-  p.l2_prefetch_bytes = 256 * 1024;
+  p.l2_prefetch_bytes = e->shallow ? kShallowPrefetchBytes : kPrefetchBytes;
   p.wait_hint_ns = 20000;
   p.cl = cl;
   p.embed = embed_copy;
