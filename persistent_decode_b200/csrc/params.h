@@ -17,11 +17,12 @@ constexpr int kThreads = kConsumerThreads + 32;      // + one producer warp
 constexpr int kTileBytes = 32768;                     // data of one tile: weights, or a K and a V chunk
 constexpr int kSlotBytes = kTileBytes + 1024;         // ring slot stride: + FP8 tiles' per-row block scales
 constexpr int kMaxSlots = 8;
-// Ring depth and L2-prefetch distance of the dense batch-1 decode.  There the
-// short stages (QKV, attention, O-projection) wait on their input copy, and
-// every weight copy already queued on the SM (the ring's slots for the next
-// stage) and every prefetch in flight delay it: a ring of 4 slots and a 128 KB
-// prefetch distance decode 1-8 % faster than 5-6 slots and 256 KB.
+// Ring depth and L2-prefetch distance of the CUDA-core decode (batch <= 4,
+// dense or MoE).  There the short stages (QKV, attention, O-projection) wait on
+// their input copy, and every weight copy already queued on the SM (the ring's
+// slots for the next stage) and every prefetch in flight delay it: a ring of 4
+// slots and a 128 KB prefetch distance decode 0.5-9 % faster than 5-8 slots
+// and 256 KB.  (The batch-8 tensor-core decode keeps as many slots as fit.)
 constexpr int kShallowSlots = 4;
 constexpr long long kShallowPrefetchBytes = 128 * 1024;
 constexpr long long kPrefetchBytes = 256 * 1024;

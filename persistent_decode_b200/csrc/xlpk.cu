@@ -242,7 +242,7 @@ struct xlpk_engine {
   int device = 0;
   int G = 0;
   int nslot = 0;
-  bool shallow = false;         // dense batch 1: kShallowSlots ring slots, kShallowPrefetchBytes of L2 prefetch
+  bool shallow = false;         // batch <= 4: kShallowSlots ring slots, kShallowPrefetchBytes of L2 prefetch
   int smem = 0;
   int act_bytes = 0;
   int side_bytes = 0, side_rope = 0, side_resid = 0, side_embed = 0, nvr = 0, rows_side = 0, evb = 0;
@@ -812,7 +812,7 @@ xlpk_status create_impl(const xlpk_config* cfg, const xlpk_weights* w, const xlp
       e->act_bytes = act_for(std::max(std::max(H, qd), win));
     }
   }
-  e->shallow = B == 1 && c.n_experts == 0;
+  e->shallow = B <= 4;
   e->nslot = std::min(e->shallow ? kShallowSlots : kMaxSlots,
                       (max_smem - e->act_bytes - e->side_bytes - kMiscSmem) / kSlotBytes);
   if (e->nslot < 2) return XLPK_ERR_UNSUPPORTED;
