@@ -285,9 +285,8 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
 
 /* Allocation-free decode.  The pages have no counterpart to this entry point;
  * it exists for callers that must not allocate device memory while they
- * decode: code that records the decode into a CUDA graph during stream capture,
- * threads that must never enter the CUDA allocator, or processes whose device
- * memory is entirely owned by another framework's caching allocator.  It runs
+ * decode: threads that must never enter the CUDA allocator, or processes whose
+ * device memory is entirely owned by another framework's caching allocator.  It runs
  * the same persistent kernel as xlpk_decode, with the same arguments and
  * results, but every per-call scratch buffer of the kernel (activation vectors,
  * attention and LM-head partials, dependency counters) lives in one array
@@ -296,8 +295,7 @@ xlpk_status xlpk_decode_unfused(xlpk_handle h, int32_t n_steps, int32_t* tokens_
  * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
  *  - The array's device address is looked up (cudaGetSymbolAddress) with the
  *    device current at the first call on each device, and again if the
- *    device's context has been replaced since (after cudaDeviceReset); make
- *    the first call on a device before any stream capture.
+ *    device's context has been replaced since (after cudaDeviceReset).
  *  - Returns XLPK_ERR_UNSUPPORTED (with a message in xlpk_last_cuda_error) if
  *    the handle's scratch would exceed the array.
  *  - The counters in the array are cleared on `stream` at the start of each
