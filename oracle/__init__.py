@@ -6,8 +6,10 @@ path never calls it and has no CPU fallback.  It shares no code with the CUDA
 path: the two meet only in the seeded input generators of `synth`.
 
 Precision: fp32 throughout (a plain fp32 CPU decode forward), with the KV cache
-held as bf16 exactly like the device cache.  Weights keep their stored bytes
-(bf16, or e4m3 codes with fp32 block scales) and are widened to fp32 on use.
+held exactly like the device cache: bf16 entries, or e4m3 codes times one
+power-of-two scale per tensor.  Weights keep their stored bytes (bf16; e4m3
+codes with fp32 128x128 block scales; or NVFP4 e2m1 codes with an e4m3 scale
+per 16 columns and an fp32 matrix scale) and are widened to fp32 on use.
 
 Parity pins: every function here is pinned by a `-m "not gpu"` test to
 something other than itself (library routines, closed forms, invariants,
